@@ -1,0 +1,212 @@
+/*
+ * pkv.h -- C ABI of libpagedkv.so, a paged KV-cache data plane for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three explainer pages on KV caching in vLLM/Nano-vLLM-style
+ * inference engines; each entry point cites the passage that defines it:
+ *   "Nano-vLLM Part 2: model internals, KV cache and tensor parallelism"          (NV2)
+ *   "Inside the Nano-vLLM engine: KV cache, attention and tensor parallelism"     (ENG)
+ *   "LLM primer: from text to tokens, embeddings, QKV and Transformer"            (PRM)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every tensor argument is a DEVICE pointer owned by the caller, contiguous,
+ *           row-major in the shape given.  The library never allocates, frees or
+ *           synchronises on these calls (pkv_get_error is the one exception: it
+ *           synchronises the stream it is given).  Work is enqueued on `stream`
+ *           (a cudaStream_t; NULL = the legacy default stream) and runs asynchronously.
+ * Cache.    k_cache / v_cache are [num_blocks, block_size, n_kv_heads, head_dim]:
+ *           a physical block holds block_size consecutive tokens of one sequence, all kv
+ *           heads of a token are adjacent (ENG §2.2: fixed-size blocks; NV2 §5.2: block,
+ *           K/V and token dimensions).  Element type: bf16 (PKV_BF16) or OCP FP8 E4M3-FN
+ *           codes with one fp32 scale per kv head for K and for V (PKV_FP8_E4M3; value =
+ *           code_value * scale).  block_size must be 16, head_dim 64 or 128.
+ * Slots.    slot = physical_block * block_size + offset_in_block; slot -1 = padding token.
+ * Tables.   block_tables [num_seqs, max_blocks_per_seq] int32: logical block i of sequence
+ *           b lives in physical block block_tables[b][i] (ENG §2.2, PRM §17.7).  Entries
+ *           past ceil(context_lens[b] / block_size) are never read.
+ * Batches.  A call carries num_seqs sequences.  cu_seqlens [num_seqs+1] int32 (cu[0]=0)
+ *           splits the call's num_tokens new tokens by sequence; context_lens [num_seqs]
+ *           int32 is L_b, the number of cached tokens of sequence b INCLUDING this call's
+ *           new ones.  New token r of sequence b (0-based) sits at position
+ *           L_b - n_b + r, n_b = cu[b+1]-cu[b] (the new tokens are the last n_b).
+ * RoPE.     rope_cos_sin is a [max_pos, head_dim] fp32 table made by pkv_rope_build_table:
+ *           row p holds cos(p*theta_i) for i < head_dim/2, then sin(p*theta_i), with
+ *           theta_i = base^(-2i/head_dim) (rotate-half pairing (i, i+head_dim/2)).
+ *           A rotated value is computed in fp64 from the bf16 input and the fp32 table and
+ *           rounded once to bf16 (round to nearest even), so every entry point that
+ *           rotates produces the same bits (PRM §21.2; ENG §3.2).  NULL = no rotation.
+ * Errors.   Entry points return PKV_OK (0) or a negative PKV_E_* code; host-detected
+ *           problems (bad sizes, unsupported shapes, misalignment, a too-small workspace)
+ *           are reported before anything is enqueued.  Conditions only the device sees (a
+ *           slot, block id or position out of range; a bounded wait that ran out) never
+ *           trap: the kernel skips the access, records a flag in a per-device error word
+ *           and finishes; pkv_get_error() returns and clears it.
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pkv_stream_t; /* same type as cudaStream_t */
+
+enum pkv_dtype { PKV_BF16 = 0, PKV_FP8_E4M3 = 1 };
+
+enum pkv_status {
+    PKV_OK = 0,
+    PKV_E_INVALID = -1,     /* null pointer, negative size, inconsistent arguments       */
+    PKV_E_UNSUPPORTED = -2, /* shape/dtype outside the compiled set                      */
+    PKV_E_WORKSPACE = -3,   /* workspace missing or smaller than pkv_decode_workspace_bytes */
+    PKV_E_CUDA = -4,        /* a CUDA runtime call or launch failed                      */
+    PKV_E_TIMEOUT = -5,     /* (device) a bounded wait inside a kernel ran out            */
+    PKV_E_BOUNDS = -6,      /* (device) slot / block id / position outside its array      */
+    PKV_E_ALIGN = -7        /* a pointer is not 16-byte aligned                           */
+};
+
+/* Library version, (major << 16) | minor. */
+int pkv_version(void);
+
+/* Text for a status code (static storage). */
+const char *pkv_strerror(int code);
+
+/*
+ * pkv_rope_build_table -- fill a HOST array out[max_pos * head_dim] (fp32) with the RoPE
+ * table described above, evaluated in fp64 (cos/sin/pow of the C library) and rounded
+ * once to fp32.  Copy it to the device once and pass it as rope_cos_sin.
+ * (PRM §21.2: RoPE rotates Q/K inside attention; ENG §3.2: apply_rotary_pos_emb.)
+ * Returns PKV_E_INVALID for max_pos < 1, odd or non-positive head_dim, base <= 0.
+ */
+int pkv_rope_build_table(float *out, int max_pos, int head_dim, double base);
+
+/*
+ * pkv_cache_bytes -- bytes of ONE cache tensor pair (K and V) for num_layers layers of
+ * num_blocks blocks: 2 * num_layers * num_blocks * block_size * n_kv_heads * head_dim *
+ * element_bytes.  With cached_tokens = num_blocks * block_size this is the sizing formula
+ * of PRM §17.3 and §17.6.  Returns 0 for invalid arguments.
+ */
+size_t pkv_cache_bytes(int num_layers, long long num_blocks, int block_size, int n_kv_heads,
+                       int head_dim, int cache_dtype);
+
+/*
+ * pkv_kv_store -- slot-mapped scatter of new K/V into the paged cache
+ * (NV2 §5.1-5.3: the K and V of every token are cached, a kernel writes them into the
+ * block-structured cache; ENG §2.1: appended on every decode step; ENG §2.2: slots).
+ *   k, v          [num_tokens, n_kv_heads, head_dim] bf16
+ *   k_cache,
+ *   v_cache       cache tensors (see Cache); written only at the mapped slots
+ *   slot_mapping  [num_tokens] int32; -1 = skip the token
+ *   k_scale,
+ *   v_scale       [n_kv_heads] fp32, required for PKV_FP8_E4M3 (ignored for bf16):
+ *                 code = E4M3(value / scale), quotient in fp64, round to nearest even,
+ *                 saturated to +-448
+ *   rope_cos_sin  RoPE table or NULL; when given, K is rotated at its position before it
+ *                 is stored (V never is), and cu_seqlens/context_lens/num_seqs/max_pos
+ *                 must describe the batch; otherwise they are ignored and may be NULL/0
+ * Bit-exact: the stored bf16 (or E4M3) patterns are fully determined by the inputs.
+ * Device errors: slot >= num_blocks*block_size, position >= max_pos -> PKV_E_BOUNDS flag,
+ * that token is skipped.
+ */
+int pkv_kv_store(const void *k, const void *v, void *k_cache, void *v_cache,
+                 const int32_t *slot_mapping, int num_tokens, int n_kv_heads, int head_dim,
+                 int block_size, long long num_blocks, int cache_dtype, const float *k_scale,
+                 const float *v_scale, const float *rope_cos_sin, int max_pos,
+                 const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                 pkv_stream_t stream);
+
+/*
+ * pkv_rope_apply -- rotate q [num_tokens, n_q_heads, head_dim] and k [num_tokens,
+ * n_kv_heads, head_dim] (bf16) IN PLACE at each token's position (PRM §21.2, ENG §3.2).
+ * Either q or k may be NULL.  Device errors: position outside [0, max_pos) ->
+ * PKV_E_BOUNDS flag, that token is left unchanged.
+ */
+int pkv_rope_apply(void *q, void *k, const float *rope_cos_sin, int max_pos,
+                   const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                   int num_tokens, int n_q_heads, int n_kv_heads, int head_dim,
+                   pkv_stream_t stream);
+
+/*
+ * pkv_decode_workspace_bytes -- size of the device scratch buffer that
+ * pkv_paged_decode_attention needs for its split-context partial results, for the
+ * CURRENT device.  Depends only on the arguments and the device's SM count.
+ */
+size_t pkv_decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim);
+
+/*
+ * pkv_paged_decode_attention -- one query token per sequence against its whole paged
+ * cache (ENG §3: Q [batch, heads, 1, d] against cached K/V [batch, heads, seq_len, d];
+ * ENG §3.1 incremental decoding; ENG §3.2 max subtraction; PRM §17.1: decode is bound
+ * by memory bandwidth).  For sequence b and query head h (kv head g = h / (n_q_heads /
+ * n_kv_heads)):
+ *     s_j = scale * <q[b,h], K_b[j]>,  j < L_b = context_lens[b]
+ *     out[b,h] = sum_j exp(s_j - max s) V_b[j] / sum_j exp(s_j - max s)
+ * The query is the sequence's newest token, so every cached token is visible.
+ *   out           [num_seqs, n_q_heads, head_dim] bf16 (a row with L_b = 0 is zero)
+ *   q             [num_seqs, n_q_heads, head_dim] bf16
+ *   rope_cos_sin  NULL, or the RoPE table: q is then rotated at position L_b - 1 first
+ *   k_scale,
+ *   v_scale       [n_kv_heads] fp32 for PKV_FP8_E4M3, else ignored
+ *   workspace     device scratch of at least pkv_decode_workspace_bytes(...) bytes,
+ *                 16-byte aligned; its contents need no initialisation and are
+ *                 overwritten.  Calls that share a workspace must not overlap in time.
+ * Device errors: block id outside [0, num_blocks) or L_b > max_blocks_per_seq*block_size
+ * -> PKV_E_BOUNDS flag (the block reads as zeros / the context is clipped).
+ */
+int pkv_paged_decode_attention(void *out, const void *q, const void *k_cache,
+                               const void *v_cache, const int32_t *block_tables,
+                               int max_blocks_per_seq, const int32_t *context_lens,
+                               int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
+                               int block_size, long long num_blocks, float scale,
+                               int cache_dtype, const float *k_scale, const float *v_scale,
+                               const float *rope_cos_sin, int max_pos, void *workspace,
+                               size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * pkv_paged_prefill_attention -- causal attention of a chunk of new tokens per sequence
+ * over the paged cache, which must already hold those tokens' K/V (PRM §17.1 and ENG §2.1:
+ * prefill processes all prompt tokens in parallel and is compute-bound; ENG §3.2 causal
+ * mask; PRM §22 steps 6-8).  Row r of sequence b (position p = L_b - n_b + r) attends
+ * to the cached tokens j <= p (bottom-right alignment: a chunk appended to a cached
+ * prefix sees all of the prefix).
+ *   out           [num_tokens, n_q_heads, head_dim] bf16
+ *   q             [num_tokens, n_q_heads, head_dim] bf16, rows grouped by cu_seqlens
+ *   max_new_tokens host upper bound on every n_b (sizes the grid; no device read-back)
+ *   rope_cos_sin  NULL, or the RoPE table: q is rotated at its position on load
+ *   k_scale,
+ *   v_scale       [n_kv_heads] fp32 for PKV_FP8_E4M3, else ignored
+ * Device errors: as pkv_paged_decode_attention.
+ */
+int pkv_paged_prefill_attention(void *out, const void *q, const void *k_cache,
+                                const void *v_cache, const int32_t *cu_seqlens,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *context_lens, int num_seqs, int num_tokens,
+                                int n_q_heads, int n_kv_heads, int head_dim, int block_size,
+                                long long num_blocks, float scale, int cache_dtype,
+                                const float *k_scale, const float *v_scale,
+                                const float *rope_cos_sin, int max_pos, int max_new_tokens,
+                                pkv_stream_t stream);
+
+/*
+ * pkv_get_error -- synchronise `stream`, then return and clear the current device's error
+ * word: PKV_OK, PKV_E_TIMEOUT or PKV_E_BOUNDS (the first set wins if both are), or
+ * PKV_E_CUDA if the synchronisation itself failed.
+ */
+int pkv_get_error(pkv_stream_t stream);
+
+/*
+ * pkv_debug_wait_timeout -- failure-detection self test.  Launches one kernel whose
+ * mbarrier wait can never complete (nothing arrives on it); the wait gives up after
+ * timeout_ns nanoseconds (clamped to [1e3, 2e9]), sets the PKV_E_TIMEOUT flag and the
+ * kernel returns normally, so the context stays usable.  Read the result with
+ * pkv_get_error().
+ */
+int pkv_debug_wait_timeout(long long timeout_ns, pkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */
