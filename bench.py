@@ -1,0 +1,521 @@
+"""Benchmark of the paged KV-cache data plane on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-suite] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the hot path over one batch: kv_store of the step's new tokens
+(K rotated by RoPE on the way in), then attention over the paged cache (Q rotated on
+load): paged decode attention for decode rows, paged prefill attention for prefill rows.
+The default workload is the Qwen-7B-style MHA decode step (batch 64, 32 heads x 128,
+context lengths uniform in [128, 2048]); the headline value is the decode attention's
+KV bytes per step divided by the device-timed step time (GB/s).  ``--suite`` (on by
+default at N=1) also times the other workloads: GQA decode over 32 layers, the
+shared-prefix prefill (TFLOP/s of causal attention) and the continuous-batching mix
+(bf16 and FP8).
+
+Under torchrun (N > 1) every rank runs an independent replica of the workload on its
+own GPU (no data-path collective: the path shards by sequence); timing is the max over
+ranks, the value is the work of all ranks over that time.
+
+``--impl reference`` times the CPU oracle (plain fp64 C, OpenMP) on a bounded sample of
+the same workload, on this machine's host cores; it needs no GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_447_b200 import workloads as W  # noqa: E402
+
+METRIC = "paged decode attn KV GB/s (% of HBM peak); prefill TFLOP/s; decode tok/s/layer"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def timed_region(fn, steps, warmup, stream, dist=None, sampler_index=0, on_timed=None):
+    """Run fn() warmup times, then time `steps` calls with CUDA events on `stream`,
+    bracketed by a barrier and a device synchronisation; returns (ms total, clocks).
+    `on_timed` (if given) is called once between the warm-up and the timed calls."""
+    for _ in range(warmup):
+        fn()
+    if on_timed is not None:
+        on_timed()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(sampler_index) as cs:
+        time.sleep(0.25)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(steps):
+            fn()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return start.elapsed_time(end), cs.summary()
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def decode_kv_bytes(st: W.Step, hkv: int, d: int, esize: int) -> int:
+    L = st.context_lens[:st.decode_seqs].long()
+    return int(L.sum()) * hkv * d * esize * 2
+
+
+def decode_alg_bytes(st: W.Step, hq: int, hkv: int, d: int, esize: int) -> int:
+    """Bytes decode attention must move: K and V of every cached token of every kv head,
+    q and out (bf16), the context lengths and the block-table entries it reads."""
+    B = st.decode_seqs
+    L = st.context_lens[:B].long()
+    blocks = int(((L + 15) // 16).sum())
+    return decode_kv_bytes(st, hkv, d, esize) + 2 * B * hq * d * 2 + 4 * B + 4 * blocks
+
+
+def prefill_flops(st: W.Step, hq: int, d: int) -> float:
+    """4 * D flops (QK^T and PV multiply-adds) per visible (query, key) pair per q head."""
+    n = (st.cu_seqlens[1:] - st.cu_seqlens[:-1]).long()
+    L = st.context_lens.long()
+    first = st.decode_seqs
+    n, L = n[first:], L[first:]
+    pairs = (n * (L - n) + n * (n + 1) // 2).sum()
+    return float(4 * d * hq * int(pairs))
+
+
+# ----------------------------------------------------------------------------- runner
+
+class Runner:
+    """Device buffers of one workload and the step closure (ours)."""
+
+    def __init__(self, wl: W.Workload, layers: int = 1):
+        import paged_kv_cache_447_b200 as pkv
+        self.pkv = pkv
+        self.wl = wl
+        st = wl.steps[-1]
+        self.st = st
+        self.layers = layers
+        kc = wl.k_cache.cuda()
+        vc = wl.v_cache.cuda()
+        self.k_caches = [kc] + [kc.clone() for _ in range(layers - 1)]
+        self.v_caches = [vc] + [vc.clone() for _ in range(layers - 1)]
+        self.table = pkv.rope_build_table(wl.max_pos, wl.head_dim, wl.rope_base).cuda()
+        self.k_scale = wl.k_scale.cuda() if wl.k_scale is not None else None
+        self.v_scale = wl.v_scale.cuda() if wl.v_scale is not None else None
+        # per-step inputs (device copies) and pinned host copies for the end-to-end leg
+        names = ["q", "k", "v", "slot_mapping", "cu_seqlens", "context_lens", "block_tables"]
+        self.host = {n: getattr(st, n).contiguous().pin_memory() for n in names}
+        self.dev = {n: t.cuda() for n, t in self.host.items()}
+        B = st.decode_seqs
+        self.B = B
+        if B:
+            self.dec_bt = self.dev["block_tables"][:B].contiguous()
+            self.dec_ctx = self.dev["context_lens"][:B].contiguous()
+            self.ws = torch.empty(pkv.decode_workspace_bytes(B, wl.n_q_heads, wl.n_kv_heads,
+                                                             wl.head_dim),
+                                  dtype=torch.uint8, device="cuda")
+            self.dec_out = torch.empty((B, wl.n_q_heads, wl.head_dim), dtype=torch.bfloat16,
+                                       device="cuda")
+        P = st.num_seqs - B
+        self.P = P
+        if P:
+            tok0 = int(st.cu_seqlens[B])
+            self.pre_q = self.dev["q"][tok0:]
+            self.pre_cu = (self.dev["cu_seqlens"][B:] - tok0).contiguous()
+            self.pre_bt = self.dev["block_tables"][B:].contiguous()
+            self.pre_ctx = self.dev["context_lens"][B:].contiguous()
+            self.pre_out = torch.empty_like(self.pre_q)
+            self.max_new = int((st.cu_seqlens[B + 1:] - st.cu_seqlens[B:-1]).max())
+        self.host_out = torch.empty((st.num_tokens, wl.n_q_heads, wl.head_dim),
+                                    dtype=torch.bfloat16).pin_memory()
+        self.ev_attn = []  # (start, end) event pairs around the dominant kernel
+
+    def launches_per_step(self) -> int:
+        n = 1                      # kv_store
+        if self.B:
+            n += 2                 # decode + combine
+        if self.P:
+            n += 1                 # prefill
+        return n * self.layers
+
+    def step(self, record: bool = False, dominant: str = "decode"):
+        pkv, wl, d = self.pkv, self.wl, self.dev
+        s = torch.cuda.current_stream()
+        for layer in range(self.layers):
+            kc, vc = self.k_caches[layer], self.v_caches[layer]
+            pkv.kv_store(d["k"], d["v"], kc, vc, d["slot_mapping"], k_scale=self.k_scale,
+                         v_scale=self.v_scale, rope_cos_sin=self.table,
+                         cu_seqlens=d["cu_seqlens"], context_lens=d["context_lens"])
+            if self.B:
+                q = d["q"][:self.B]
+                if record and dominant == "decode":
+                    e0 = torch.cuda.Event(enable_timing=True); e0.record(s)
+                pkv.paged_decode_attention(q, kc, vc, self.dec_bt, self.dec_ctx, scale=wl.scale,
+                                           k_scale=self.k_scale, v_scale=self.v_scale,
+                                           rope_cos_sin=self.table, workspace=self.ws,
+                                           out=self.dec_out)
+                if record and dominant == "decode":
+                    e1 = torch.cuda.Event(enable_timing=True); e1.record(s)
+                    self.ev_attn.append((e0, e1))
+            if self.P:
+                if record and dominant == "prefill":
+                    e0 = torch.cuda.Event(enable_timing=True); e0.record(s)
+                pkv.paged_prefill_attention(self.pre_q, kc, vc, self.pre_cu, self.pre_bt,
+                                            self.pre_ctx, self.max_new, scale=wl.scale,
+                                            k_scale=self.k_scale, v_scale=self.v_scale,
+                                            rope_cos_sin=self.table, out=self.pre_out)
+                if record and dominant == "prefill":
+                    e1 = torch.cuda.Event(enable_timing=True); e1.record(s)
+                    self.ev_attn.append((e0, e1))
+
+    def e2e_step(self):
+        """Same step, with this step's inputs copied from pinned host memory first and the
+        attention output copied back (all on the current stream)."""
+        for n, h in self.host.items():
+            self.dev[n].copy_(h, non_blocking=True)
+        self.step()
+        parts = []
+        if self.B:
+            parts.append(self.dec_out)
+        if self.P:
+            parts.append(self.pre_out)
+        off = 0
+        for p in parts:
+            self.host_out[off:off + p.shape[0]].copy_(p, non_blocking=True)
+            off += p.shape[0]
+
+    def e2e_bytes(self):
+        h2d = sum(t.numel() * t.element_size() for t in self.host.values())
+        d2h = self.host_out.numel() * self.host_out.element_size()
+        return h2d, d2h
+
+    def attn_ms(self) -> float:
+        if not self.ev_attn:
+            return float("nan")
+        torch.cuda.synchronize()
+        ts = [a.elapsed_time(b) for a, b in self.ev_attn]
+        return sum(ts) / len(ts)
+
+
+def build_workload(name: str):
+    if name == "qwen_decode":
+        return W.qwen_decode(seed=2), 1
+    if name == "gqa_decode":
+        return W.gqa_decode(seed=3), 32
+    if name == "shared_prefix":
+        return W.shared_prefix(seed=4), 1
+    if name == "mix":
+        return W.mix(seed=5), 1
+    if name == "mix_fp8":
+        return W.mix(seed=5, fp8=True), 1
+    raise ValueError(name)
+
+
+def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=True):
+    wl, layers = build_workload(name)
+    r = Runner(wl, layers)
+    st = r.st
+    esize = 1 if wl.cache_dtype == "fp8" else 2
+    dominant = "decode" if r.B else "prefill"
+    ms, clocks = timed_region(lambda: r.step(record=True, dominant=dominant), steps, warmup,
+                              torch.cuda.current_stream(), dist, device_index,
+                              on_timed=r.ev_attn.clear)
+    code = r.pkv.get_error()
+    assert code == 0, f"device error flag set during the timed region: {code}"
+    ms = max_over_ranks(ms, dist)
+    world = dist.get_world_size() if dist is not None else 1
+    step_ms = ms / steps
+    attn_ms = r.attn_ms()
+    res = {"workload": name, "step_ms": step_ms, "layers": layers, "clocks": clocks,
+           "gpu_launches": r.launches_per_step() * steps}
+    hbm = (pk or FALLBACK_PEAKS)["hbm_gbs"]
+    if r.B:
+        kv_bytes = decode_kv_bytes(st, wl.n_kv_heads, wl.head_dim, esize) * layers
+        alg = decode_alg_bytes(st, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, esize)
+        res["decode_kv_bytes_per_step"] = kv_bytes
+        res["kv_gbs"] = world * kv_bytes / (step_ms * 1e-3) / 1e9
+        res["decode_tok_s_per_layer"] = world * r.B / (step_ms * 1e-3 / layers)
+        res["attn_kernel_ms"] = attn_ms
+        res["attn_alg_bytes"] = alg
+        res["attn_gbs"] = alg / (attn_ms * 1e-3) / 1e9
+        res["attn_hbm_frac"] = res["attn_gbs"] / hbm
+    if r.P:
+        fl = prefill_flops(st, wl.n_q_heads, wl.head_dim) * layers
+        res["prefill_flops_per_step"] = fl
+        if dominant == "prefill":
+            res["attn_kernel_ms"] = attn_ms
+            res["prefill_tflops"] = fl / (attn_ms * 1e-3) / 1e12
+        res["step_tflops"] = world * fl / (step_ms * 1e-3) / 1e12
+    if e2e:
+        ms_e, _ = timed_region(r.e2e_step, steps, warmup, torch.cuda.current_stream(), dist,
+                               device_index)
+        ms_e = max_over_ranks(ms_e, dist)
+        h2d, d2h = r.e2e_bytes()
+        res["e2e_step_ms"] = ms_e / steps
+        res["e2e_h2d"] = h2d
+        res["e2e_d2h"] = d2h
+    return res, r
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_step_rate(name: str, budget_s: float = 15.0):
+    """Time the CPU oracle on a bounded sample of the workload: the sample is the first
+    n decode sequences (or prefill requests), grown until it takes ~budget_s/4."""
+    import numpy as np
+    import oracle
+    wl, layers = build_workload(name)
+    st = wl.steps[-1]
+    fp8 = wl.cache_dtype == "fp8"
+    esize = 1 if fp8 else 2
+    kc0, vc0 = W.bits(wl.k_cache), W.bits(wl.v_cache)
+    tab = oracle.rope_table(wl.max_pos, wl.head_dim, wl.rope_base)
+    B = st.decode_seqs
+
+    def run(seqs):
+        sub = W.sub_step(st, seqs)
+        kc, vc = kc0.copy(), vc0.copy()
+        pos = oracle.positions(sub.cu_seqlens.numpy(), sub.context_lens.numpy())
+        t0 = time.perf_counter()
+        oracle.kv_store(W.bits(sub.k), W.bits(sub.v), kc, vc, sub.slot_mapping.numpy(), 16,
+                        fp8=fp8, k_scale=None if not fp8 else wl.k_scale.numpy(),
+                        v_scale=None if not fp8 else wl.v_scale.numpy(), table=tab, pos=pos)
+        oracle.attention(W.bits(sub.q), kc, vc, sub.cu_seqlens.numpy(),
+                         sub.block_tables.numpy(), sub.context_lens.numpy(), wl.scale, 16,
+                         wl.n_kv_heads, fp8=fp8,
+                         k_scale=None if not fp8 else wl.k_scale.numpy(),
+                         v_scale=None if not fp8 else wl.v_scale.numpy(), table=tab)
+        return time.perf_counter() - t0, sub
+
+    order = list(range(st.num_seqs)) if B == 0 else list(range(B))
+    n = 1
+    while True:
+        dt, sub = run(order[:n])
+        if dt > budget_s / 4 or n >= len(order):
+            break
+        n = min(len(order), max(n + 1, int(n * min(8.0, (budget_s / 4) / max(dt, 1e-3)))))
+    res = {"sample": f"{n} of {len(order)} sequences of one step (one layer)", "seconds": dt,
+           "cores": oracle.num_threads()}
+    if B:
+        kv = decode_kv_bytes(sub, wl.n_kv_heads, wl.head_dim, esize)
+        res["value"] = kv / dt / 1e9
+        res["unit"] = "GB/s"
+    else:
+        res["value"] = prefill_flops(sub, wl.n_q_heads, wl.head_dim) / dt / 1e12
+        res["unit"] = "TFLOP/s"
+    return res
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen_decode",
+                    choices=["qwen_decode", "gqa_decode", "shared_prefix", "mix", "mix_fp8"])
+    ap.add_argument("--no-suite", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pk, pk_kind = peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        r = oracle_step_rate(args.workload, budget_s=min(60.0, 6.0 * args.steps))
+        line = {"impl": "reference", "metric": METRIC, "value": r["value"], "unit": r["unit"],
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": r["seconds"] * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": args.workload, "sample": r["sample"]},
+                "cpu_baseline": {"value": r["value"], "unit": r["unit"], "cores": r["cores"],
+                                 "kind": "oracle", "sample": r["sample"]},
+                "e2e": {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(local)
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    else:
+        torch.cuda.set_device(0)
+
+    res, runner = measure_ours(args.workload, args.steps, args.warmup, dist, local, pk,
+                               e2e=not args.no_e2e)
+    wl = runner.wl
+    esize = 1 if wl.cache_dtype == "fp8" else 2
+    if runner.B:
+        value, unit = res["kv_gbs"], "GB/s"
+        bound, ach, peak, runit = "hbm", res["attn_gbs"], pk["hbm_gbs"], "GB/s"
+    else:
+        value, unit = res["step_tflops"], "TFLOP/s"
+        bound, ach, peak, runit = ("tensor", res.get("prefill_tflops", float("nan")),
+                                   pk["bf16_tflops"], "TFLOP/s")
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["step_ms"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if esize == 2 else "e4m3",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": runner.B or runner.P,
+                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
+                   "head_dim": wl.head_dim, "block_size": 16, "layers": res["layers"],
+                   "context": wl.notes.get("context", None),
+                   "l2": "inputs larger than L2 (KV bytes per step "
+                         f"{res.get('decode_kv_bytes_per_step', 0) / 1e9:.2f} GB), no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "decode_tok_s_per_layer": res.get("decode_tok_s_per_layer"),
+        "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": runit,
+                     "frac": ach / peak, "traffic": None,
+                     "kernel": "paged_decode_attention" if runner.B else "paged_prefill_attention",
+                     "peak_source": pk_kind, "kernel_ms": res.get("attn_kernel_ms")},
+        "clocks": res["clocks"],
+        "gpu_launches": res["gpu_launches"],
+    }
+    if not args.no_e2e:
+        if runner.B:
+            ev = world * res["decode_kv_bytes_per_step"] / (res["e2e_step_ms"] * 1e-3) / 1e9
+        else:
+            ev = world * res["prefill_flops_per_step"] / (res["e2e_step_ms"] * 1e-3) / 1e12
+        line["e2e"] = {"value": ev, "unit": unit, "h2d_bytes_per_step": res["e2e_h2d"],
+                       "d2h_bytes_per_step": res["e2e_d2h"], "ms_per_step": res["e2e_step_ms"]}
+    del runner
+    torch.cuda.empty_cache()
+
+    if world == 1 and not args.no_suite:
+        suite = {}
+        for name in ("gqa_decode", "shared_prefix", "mix", "mix_fp8"):
+            if name == args.workload:
+                continue
+            try:
+                r, rr = measure_ours(name, max(3, args.steps // 4), 3, None, 0, pk, e2e=False)
+                del rr
+                torch.cuda.empty_cache()
+                keep = {k: v for k, v in r.items() if k not in ("clocks",)}
+                if "attn_gbs" in r:
+                    keep["attn_hbm_frac"] = r["attn_gbs"] / pk["hbm_gbs"]
+                if "prefill_tflops" in r:
+                    keep["prefill_tensor_frac"] = r["prefill_tflops"] / pk["bf16_tflops"]
+                suite[name] = keep
+            except Exception as e:  # report, do not hide
+                suite[name] = {"error": f"{type(e).__name__}: {e}"}
+        line["suite"] = suite
+
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        try:
+            cb = oracle_step_rate(args.workload, budget_s=15.0)
+            line["cpu_baseline"] = {"value": cb["value"], "unit": cb["unit"], "cores": cb["cores"],
+                                    "kind": "oracle", "sample": cb["sample"]}
+        except Exception as e:
+            line["cpu_baseline"] = {"error": f"{type(e).__name__}: {e}"}
+
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -95,6 +95,8 @@ def _load():
         lib.orc_attention_weights.restype = None
         lib.orc_kv_cache_bytes.argtypes = [ctypes.c_int64] * 5
         lib.orc_kv_cache_bytes.restype = ctypes.c_int64
+        lib.orc_num_threads.argtypes = []
+        lib.orc_num_threads.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -247,3 +249,8 @@ def kv_cache_bytes(num_layers: int, n_kv_heads: int, head_dim: int, cached_token
                    bytes_per_element: int) -> int:
     return int(_load().orc_kv_cache_bytes(num_layers, n_kv_heads, head_dim, cached_tokens,
                                           bytes_per_element))
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle's parallel loops use."""
+    return int(_load().orc_num_threads())

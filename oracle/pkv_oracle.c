@@ -17,6 +17,7 @@
  * the docstrings of oracle/__init__.py and exercised by tests/test_oracle_pins.py.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -365,3 +366,6 @@ int64_t orc_kv_cache_bytes(int64_t num_layers, int64_t n_kv_heads, int64_t head_
 {
     return 2 * num_layers * n_kv_heads * head_dim * cached_tokens * bytes_per_element;
 }
+
+/* Threads the OpenMP loops above use (reported beside CPU timings). */
+int orc_num_threads(void) { return omp_get_max_threads(); }

@@ -1,0 +1,630 @@
+// decode.cu -- paged decode attention: one query token per sequence over its whole cache.
+//
+// "Inside the Nano-vLLM engine: KV cache, attention and tensor parallelism", §3 (Q of the
+// new token, [batch, heads, 1, d], against the cached K/V, [batch, heads, seq_len, d]),
+// §3.1 (incremental decoding; FlashAttention-style tiling with the softmax kept on chip),
+// §3.2 (subtract the maximum before the exponential).  "LLM primer", §17.1: decode is
+// bound by memory bandwidth, the cache keeps growing.
+//
+// Design (HBM-bound: every cached K/V byte is streamed from HBM exactly once):
+//  * Work unit = one 16-token block of one (sequence, kv head).  Units are numbered
+//    sequence-major; the whole unit space is cut into equal contiguous ranges, one per
+//    persistent CTA (grid = SMs x 2), so every CTA streams the same number of bytes
+//    whatever the length mix.  A CTA's range crosses sequence boundaries; each piece of a
+//    (sequence, kv head) it covers becomes one partial softmax state.
+//  * Warp 0 is the producer: it reads block-table entries 32 at a time and issues one TMA
+//    load per block for K and one for V into a ring of shared-memory stages (mbarrier
+//    full/empty pairs).  Warps 1-4 consume stages round robin.
+//  * A consumer warp handles all G = Hq/Hkv query heads of the kv head, so each K/V tile
+//    is read from shared memory once for the whole group.  q.k: two lanes per token (each
+//    half the head dim, chunk order rotated per token so shared-memory reads are
+//    conflict-free), packed fp32x2 FMAs.  p.v: each lane owns D/32 output dims.  Online
+//    softmax (running max m, sum l) per warp in exp2 space.
+//  * At the end of a piece the four consumer warps merge (m, l, acc) through shared
+//    memory.  A piece that covers its whole sequence writes the normalised bf16 output;
+//    otherwise its partial goes to the workspace and a small combine kernel merges the
+//    partials of that sequence:  M = max m_k,  o = sum e^(m_k-M) acc_k / sum e^(m_k-M) l_k.
+#include "common.cuh"
+#include "internal.h"
+
+#include <algorithm>
+
+namespace pkv {
+namespace {
+
+constexpr int kConsumers = 4;
+constexpr int kThreads = 32 * (1 + kConsumers);
+constexpr int kCtasPerSm = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMergeBar = 1;
+
+struct DecodeParams {
+    __nv_bfloat16 *out;
+    const uint16_t *q;
+    const int32_t *block_tables;
+    int max_blocks;
+    const int32_t *context_lens;
+    int B, Hq, Hkv;
+    long long num_blocks;
+    float scale_log2;
+    const float *k_scale, *v_scale;
+    const float *rope;
+    int max_pos;
+    int *prefix;      // [B+1] block prefix, written by CTA 0 for the combine kernel
+    float *partials;  // [(B*Hkv + nctas)][G][D+2]
+    int nctas;
+    int *err;
+};
+
+template <int D, bool FP8, int G>
+struct Geometry {
+    static constexpr int kElem = FP8 ? 1 : 2;
+    static constexpr int kRowBytes = D * kElem;
+    static constexpr int kTileBytes = kBlockSize * kRowBytes;          // one K (or V) block
+    static constexpr int kStageBytes = 2 * kTileBytes;                 // K + V
+    // q, probabilities and merge scratch, plus room for 1024 sequences' prefix
+    static constexpr int kExtraBytes = G * D * 4 + kConsumers * G * 16 * 4 +
+                                       kConsumers * G * (D + 2) * 4 + 4 * 1025;
+    // ring of ~100 KB in total so that two CTAs share an SM
+    // The stage count is a multiple of the consumer count, so that every fill of a given
+    // stage is consumed by the same warp: a warp then never waits on a barrier more than
+    // one phase ahead (a parity wait cannot tell phase n from phase n+2).
+    static constexpr int kStagesRaw = (100 * 1024 - kExtraBytes) / kStageBytes;
+    static constexpr int kStagesQ = (kStagesRaw / kConsumers) * kConsumers;
+    static constexpr int kStages = kStagesQ < kConsumers ? kConsumers : (kStagesQ > 64 ? 64 : kStagesQ);
+    static_assert(kStages % kConsumers == 0, "stage count must be a multiple of the consumers");
+    static constexpr int kChunkElems = 16 / kElem;                     // elements per 16 B
+    static constexpr int kChunks = kRowBytes / 16;                     // 16-B chunks per row
+    static constexpr int kHalf = kChunks / 2;                          // per lane of a pair
+    static constexpr int kQuads = kChunkElems / 4;                     // float4 per chunk
+    static constexpr int kDimsPerLane = D / 32;                        // p.v ownership
+};
+
+// Units of sequence b: ceil(min(L_b, max_blocks*16) / 16).
+__device__ __forceinline__ int seq_blocks(int L, int max_blocks, int *err) {
+    if (L < 0) L = 0;
+    int nb = (L + kBlockSize - 1) / kBlockSize;
+    if (nb > max_blocks) {
+        atomicOr(err, kErrBounds);
+        nb = max_blocks;
+    }
+    return nb;
+}
+
+// Exclusive prefix over sequences of their block counts, into pfx[0..B] (shared memory).
+__device__ void block_prefix(const DecodeParams &p, int *pfx) {
+    __shared__ int warp_tot[kThreads / 32];
+    __shared__ int carry_s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) carry_s = 0;
+    __syncthreads();
+    for (int base = 0; base < p.B; base += kThreads) {
+        const int b = base + threadIdx.x;
+        int v = (b < p.B) ? seq_blocks(__ldg(p.context_lens + b), p.max_blocks, p.err) : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        int before = carry_s;
+        for (int w = 0; w < warp; ++w) before += warp_tot[w];
+        if (b < p.B) pfx[b] = before + incl - v;
+        __syncthreads();
+        if (threadIdx.x == kThreads - 1) carry_s = before + incl;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) pfx[p.B] = carry_s;
+    __syncthreads();
+}
+
+// Last sequence b with Hkv*pfx[b] <= u (skips empty sequences).
+__device__ __forceinline__ int find_seq(const int *pfx, int B, int Hkv, long long u) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if ((long long)Hkv * pfx[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+struct UnitPos {
+    int b, kvh, blk, nb;
+};
+
+__device__ __forceinline__ UnitPos locate(const int *pfx, int B, int Hkv, long long u) {
+    UnitPos r;
+    r.b = find_seq(pfx, B, Hkv, u);
+    r.nb = pfx[r.b + 1] - pfx[r.b];
+    long long rel = u - (long long)Hkv * pfx[r.b];
+    r.kvh = (int)(rel / r.nb);
+    r.blk = (int)(rel % r.nb);
+    return r;
+}
+
+template <int D, bool FP8, int G>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const DecodeParams p) {
+    using Geo = Geometry<D, FP8, G>;
+    constexpr int NS = Geo::kStages;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *stages = smem;                                                  // NS x stage
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * Geo::kStageBytes);
+    uint64_t *empty = full + NS;
+    float *qs = reinterpret_cast<float *>(empty + NS);                      // [G][quads][chunks][4]
+    float *pbuf = qs + G * D;                                                // [consumers][G][16]
+    float *mrg = pbuf + kConsumers * G * 16;                                 // [consumers][G][D+2]
+    int *pfx = reinterpret_cast<int *>(mrg + kConsumers * G * (D + 2));      // [B+1]
+    __shared__ volatile int abort_s;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    block_prefix(p, pfx);
+    const long long total = (long long)p.Hkv * pfx[p.B];
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i <= p.B; i += kThreads) p.prefix[i] = pfx[i];
+    const long long U = total > 0 ? (total + p.nctas - 1) / p.nctas : 1;
+    const long long u0 = (long long)blockIdx.x * U;
+    const long long u1 = (u0 + U < total) ? u0 + U : total;
+    if (u0 >= u1) return;  // uniform across the CTA
+    const int nunits = (int)(u1 - u0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_u32(full + s), 1);
+            mbar_init(smem_u32(empty + s), 1);
+        }
+        abort_s = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+        uint64_t issued_mask = 0, issued_phase = 0;  // stage ever filled / parity of last fill
+        bool ok = true;
+        for (int k0 = 0; k0 < nunits; k0 += 32) {
+            const int k = k0 + lane;
+            int phys = 0, kvh = 0;
+            if (k < nunits) {
+                UnitPos up = locate(pfx, p.B, p.Hkv, u0 + k);
+                kvh = up.kvh;
+                phys = __ldg(p.block_tables + (size_t)up.b * p.max_blocks + up.blk);
+                if (phys < 0 || (long long)phys >= p.num_blocks) {
+                    atomicOr(p.err, kErrBounds);
+                    phys = (int)(p.num_blocks < 0x7fffffffLL / kBlockSize ? p.num_blocks : 0);
+                }
+            }
+            const int n = min(32, nunits - k0);
+            for (int j = 0; j < n; ++j) {
+                const int ph = __shfl_sync(0xffffffffu, phys, j);
+                const int hh = __shfl_sync(0xffffffffu, kvh, j);
+                if (lane == 0 && ok) {
+                    const int kk = k0 + j, s = kk % NS;
+                    const uint32_t parity = ((kk / NS) & 1) ^ 1;
+                    if (!mbar_wait_bounded(smem_u32(empty + s), parity, p.err) || abort_s) {
+                        ok = false;
+                        abort_s = 1;
+                    } else {
+                        const uint32_t fb = smem_u32(full + s);
+                        const uint32_t dst = smem_u32(stages + s * Geo::kStageBytes);
+                        mbar_arrive_expect_tx(fb, Geo::kStageBytes);
+                        tma_load_3d(dst, &tm_k, fb, 0, hh, ph * kBlockSize);
+                        tma_load_3d(dst + Geo::kTileBytes, &tm_v, fb, 0, hh, ph * kBlockSize);
+                        issued_mask |= 1ull << s;
+                        issued_phase = (issued_phase & ~(1ull << s)) | ((uint64_t)((kk / NS) & 1) << s);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        // Drain: never leave the CTA with a TMA copy still landing in its shared memory.
+        if (lane == 0) {
+            for (int s = 0; s < NS; ++s)
+                if ((issued_mask >> s) & 1)
+                    mbar_wait_bounded(smem_u32(full + s), (uint32_t)((issued_phase >> s) & 1), p.err);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------------- consumers
+    const int cw = warp - 1;          // consumer index 0..3
+    const int ct = threadIdx.x - 32;  // consumer thread 0..127
+    const int t = lane & 15, hpair = lane >> 4;
+
+    float m[G], l[G], acc[G][Geo::kDimsPerLane];
+    auto reset_state = [&]() {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            m[g] = -INFINITY;
+            l[g] = 0.f;
+#pragma unroll
+            for (int d = 0; d < Geo::kDimsPerLane; ++d) acc[g][d] = 0.f;
+        }
+    };
+    reset_state();
+
+    const uint32_t qs_a = smem_u32(qs);
+    const uint32_t pbuf_a = smem_u32(pbuf + cw * G * 16);
+
+    int k = 0;
+    UnitPos cur = locate(pfx, p.B, p.Hkv, u0);
+    bool dead = false;
+    while (k < nunits) {
+        // piece = the rest of the current (sequence, kv head) segment inside this range
+        const int piece_len = min(cur.nb - cur.blk, nunits - k);
+        const int b = cur.b, kvh = cur.kvh;
+        const int L = min(__ldg(p.context_lens + b), p.max_blocks * kBlockSize);
+        const bool whole = (cur.blk == 0) && (piece_len == cur.nb);
+
+        // ---- stage q for this (b, kv head): rotate (optional), scale, split layout
+        for (int e = ct; e < G * D / 2; e += kConsumers * 32) {
+            const int g = e / (D / 2), i = e % (D / 2);
+            const int h = kvh * G + g;
+            const uint16_t *qr = p.q + ((size_t)b * p.Hq + h) * D;
+            uint16_t x1 = __ldg(qr + i), x2 = __ldg(qr + i + D / 2);
+            if (p.rope) {
+                const int pos = L - 1;
+                if (pos >= 0 && pos < p.max_pos) {
+                    const float *row = p.rope + (size_t)pos * D;
+                    rope_pair(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
+                } else {
+                    atomicOr(p.err, kErrBounds);
+                }
+            }
+            const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
+            const int idx[2] = {i, i + D / 2};
+            const float val[2] = {__uint_as_float((uint32_t)x1 << 16) * sc,
+                                  __uint_as_float((uint32_t)x2 << 16) * sc};
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int dim = idx[r];
+                const int c = dim / Geo::kChunkElems, w = dim % Geo::kChunkElems;
+                const int quad = w / 4, comp = w % 4;
+                qs[((g * Geo::kQuads + quad) * Geo::kChunks + c) * 4 + comp] = val[r];
+            }
+        }
+        named_bar(kMergeBar, kConsumers * 32);
+
+        // ---- stream this piece's blocks
+        for (int j = 0; j < piece_len; ++j, ++k) {
+            if ((k % kConsumers) != cw) continue;
+            const int s = k % NS;
+            const uint32_t parity = (k / NS) & 1;
+            if (!dead) {
+                if (abort_s || !mbar_wait_bounded(smem_u32(full + s), parity, p.err)) {
+                    dead = true;
+                    abort_s = 1;
+                }
+            }
+            if (dead) continue;
+            const int blk = cur.blk + j;
+            const int valid = min(kBlockSize, L - blk * kBlockSize);
+            const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes);
+            const uint32_t vs_a = ks_a + Geo::kTileBytes;
+
+            // q.k: lane (t, hpair) covers half the dims of token t
+            float2 sacc[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) sacc[g] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < Geo::kHalf; ++i) {
+                const int c = hpair * Geo::kHalf + ((i + t) & (Geo::kHalf - 1));
+                const uint4 kr = lds128(ks_a + t * Geo::kRowBytes + c * 16);
+                float kf[Geo::kChunkElems];
+                if constexpr (FP8) {
+                    const uint32_t w4[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+                        for (int hb = 0; hb < 2; ++hb) {
+                            uint32_t h2;
+                            const uint16_t pair = (uint16_t)(w4[wi] >> (16 * hb));
+                            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+                            __half2 hv = *reinterpret_cast<__half2 *>(&h2);
+                            float2 f = __half22float2(hv);
+                            kf[wi * 4 + hb * 2 + 0] = f.x;
+                            kf[wi * 4 + hb * 2 + 1] = f.y;
+                        }
+                    }
+                } else {
+                    const uint32_t w4[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi) {
+                        kf[2 * wi] = bf16lo(w4[wi]);
+                        kf[2 * wi + 1] = bf16hi(w4[wi]);
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+#pragma unroll
+                    for (int qd = 0; qd < Geo::kQuads; ++qd) {
+                        const float4 qv = lds128f(qs_a + (((g * Geo::kQuads + qd) * Geo::kChunks + c) * 16));
+                        sacc[g] = __ffma2_rn(make_float2(kf[4 * qd + 0], kf[4 * qd + 1]),
+                                             make_float2(qv.x, qv.y), sacc[g]);
+                        sacc[g] = __ffma2_rn(make_float2(kf[4 * qd + 2], kf[4 * qd + 3]),
+                                             make_float2(qv.z, qv.w), sacc[g]);
+                    }
+                }
+            }
+            // softmax update for this block (all 32 lanes hold the scores of token t)
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float sc = sacc[g].x + sacc[g].y;
+                sc += __shfl_xor_sync(0xffffffffu, sc, 16);
+                if (t >= valid) sc = -INFINITY;
+                float mt = sc;
+#pragma unroll
+                for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+                const float mn = fmaxf(m[g], mt);
+                const float alpha = ex2(m[g] - mn);
+                const float pj = ex2(sc - mn);
+                l[g] = l[g] * alpha + (hpair == 0 ? pj : 0.f);
+                m[g] = mn;
+#pragma unroll
+                for (int d = 0; d < Geo::kDimsPerLane; ++d) acc[g][d] *= alpha;
+                if (hpair == 0) pbuf[cw * G * 16 + g * 16 + t] = pj;
+            }
+            __syncwarp();
+            // p.v: lane owns dims [lane*DPL, (lane+1)*DPL)
+            constexpr int DPL = Geo::kDimsPerLane;
+            auto pv_row = [&](int jj, const float *pw) {
+                float vf[DPL];
+                const uint32_t va = vs_a + jj * Geo::kRowBytes + lane * DPL * Geo::kElem;
+                if constexpr (FP8) {
+                    if constexpr (DPL == 4) {
+                        const uint32_t w = lds32(va);
+#pragma unroll
+                        for (int hb = 0; hb < 2; ++hb) {
+                            uint32_t h2;
+                            const uint16_t pair = (uint16_t)(w >> (16 * hb));
+                            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+                            float2 f = __half22float2(*reinterpret_cast<__half2 *>(&h2));
+                            vf[2 * hb] = f.x;
+                            vf[2 * hb + 1] = f.y;
+                        }
+                    } else {
+                        uint16_t pair;
+                        asm volatile("ld.shared.u16 %0, [%1];" : "=h"(pair) : "r"(va));
+                        uint32_t h2;
+                        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+                        float2 f = __half22float2(*reinterpret_cast<__half2 *>(&h2));
+                        vf[0] = f.x;
+                        vf[1] = f.y;
+                    }
+                } else {
+                    if constexpr (DPL == 4) {
+                        const uint2 w = lds64(va);
+                        vf[0] = bf16lo(w.x);
+                        vf[1] = bf16hi(w.x);
+                        vf[2] = bf16lo(w.y);
+                        vf[3] = bf16hi(w.y);
+                    } else {
+                        const uint32_t w = lds32(va);
+                        vf[0] = bf16lo(w);
+                        vf[1] = bf16hi(w);
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float pg = pw[g];
+#pragma unroll
+                    for (int d = 0; d < DPL; d += 2) {
+                        float2 r = __ffma2_rn(make_float2(pg, pg), make_float2(vf[d], vf[d + 1]),
+                                              make_float2(acc[g][d], acc[g][d + 1]));
+                        acc[g][d] = r.x;
+                        acc[g][d + 1] = r.y;
+                    }
+                }
+            };
+            if (valid == kBlockSize) {
+#pragma unroll
+                for (int j4 = 0; j4 < kBlockSize; j4 += 4) {
+                    float4 pq[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) pq[g] = lds128f(pbuf_a + (g * 16 + j4) * 4);
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        float pw[G];
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            pw[g] = jj == 0 ? pq[g].x : jj == 1 ? pq[g].y : jj == 2 ? pq[g].z : pq[g].w;
+                        pv_row(j4 + jj, pw);
+                    }
+                }
+            } else {
+                for (int jj = 0; jj < valid; ++jj) {
+                    float pw[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) pw[g] = pbuf[cw * G * 16 + g * 16 + jj];
+                    pv_row(jj, pw);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(empty + s));
+        }
+
+        // ---- merge the four consumer warps' states for this piece
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float lw = l[g];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+            float *mw = mrg + (cw * G + g) * (D + 2);
+            if (lane == 0) {
+                mw[D] = m[g];
+                mw[D + 1] = lw;
+            }
+#pragma unroll
+            for (int d = 0; d < Geo::kDimsPerLane; ++d) mw[lane * Geo::kDimsPerLane + d] = acc[g][d];
+        }
+        named_bar(kMergeBar, kConsumers * 32);
+        const int seg = b * p.Hkv + kvh;
+        for (int e = ct; e < G * D; e += kConsumers * 32) {
+            const int g = e / D, d = e % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, mrg[(w * G + g) * (D + 2) + D]);
+            float o = 0.f, lsum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumers; ++w) {
+                const float *mw = mrg + (w * G + g) * (D + 2);
+                const float f = (mw[D] == -INFINITY) ? 0.f : ex2(mw[D] - M);
+                o += f * mw[d];
+                lsum += f * mw[D + 1];
+            }
+            if (whole) {
+                const float vs = FP8 ? __ldg(p.v_scale + kvh) : 1.f;
+                const float r = (lsum > 0.f) ? o / lsum * vs : 0.f;
+                p.out[((size_t)b * p.Hq + kvh * G + g) * D + d] = __float2bfloat16_rn(r);
+            } else {
+                float *slot = p.partials + (size_t)(seg + blockIdx.x) * (G * (D + 2));
+                slot[g * D + d] = o;
+                if (d == 0) {
+                    slot[G * D + g] = M;
+                    slot[G * D + G + g] = lsum;
+                }
+            }
+        }
+        named_bar(kMergeBar, kConsumers * 32);
+        reset_state();
+        // advance to the next segment
+        cur.blk += piece_len;
+        if (cur.blk >= cur.nb && k < nunits) cur = locate(pfx, p.B, p.Hkv, u0 + k);
+    }
+}
+
+// Merge the partial states of every (sequence, kv head) that was split across CTAs, and
+// zero the rows of empty sequences.  One CTA per (sequence, kv head).
+template <int D, int G>
+__global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
+    const int seg = blockIdx.x;
+    const int b = seg / p.Hkv, kvh = seg % p.Hkv;
+    const int pb = p.prefix[b], nb = p.prefix[b + 1] - pb;
+    const long long total = (long long)p.Hkv * p.prefix[p.B];
+    if (nb == 0) {
+        for (int e = threadIdx.x; e < G * D; e += blockDim.x)
+            p.out[((size_t)b * p.Hq + kvh * G) * D + e] = __float2bfloat16_rn(0.f);
+        return;
+    }
+    const long long U = (total + p.nctas - 1) / p.nctas;
+    const long long start = (long long)p.Hkv * pb + (long long)kvh * nb;
+    const int c0 = (int)(start / U), c1 = (int)((start + nb - 1) / U);
+    if (c0 == c1) return;  // written directly by the decode kernel
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int g = e / D, d = e % D;
+        float M = -INFINITY;
+        for (int c = c0; c <= c1; ++c) {
+            const float *slot = p.partials + (size_t)(seg + c) * (G * (D + 2));
+            M = fmaxf(M, slot[G * D + g]);
+        }
+        float o = 0.f, lsum = 0.f;
+        for (int c = c0; c <= c1; ++c) {
+            const float *slot = p.partials + (size_t)(seg + c) * (G * (D + 2));
+            const float mk = slot[G * D + g];
+            const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
+            o += f * slot[g * D + d];
+            lsum += f * slot[G * D + G + g];
+        }
+        const float vsc = p.v_scale ? __ldg(p.v_scale + kvh) : 1.f;
+        p.out[((size_t)b * p.Hq + kvh * G + g) * D + d] =
+            __float2bfloat16_rn(lsum > 0.f ? o / lsum * vsc : 0.f);
+    }
+}
+
+template <int D, bool FP8, int G>
+size_t smem_bytes(int B) {
+    using Geo = Geometry<D, FP8, G>;
+    size_t s = (size_t)Geo::kStages * Geo::kStageBytes + 2 * Geo::kStages * sizeof(uint64_t);
+    s += (size_t)G * D * 4 + (size_t)kConsumers * G * 16 * 4 + (size_t)kConsumers * G * (D + 2) * 4;
+    s += (size_t)(B + 1) * 4;
+    return s;
+}
+
+template <int D, bool FP8, int G>
+cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t s) {
+    const size_t smem = smem_bytes<D, FP8, G>(a.num_seqs);
+    auto kern = decode_kernel<D, FP8, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) return cudaErrorInvalidConfiguration;
+    DecodeParams lp = prm;
+    lp.nctas = std::min(prm.nctas, occ * (prm.nctas / kCtasPerSm));
+    kern<<<lp.nctas, kThreads, smem, s>>>(*a.tm_k, *a.tm_v, lp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    DecodeParams cp = lp;
+    cp.v_scale = FP8 ? a.v_scale : nullptr;
+    combine_kernel<D, G><<<a.num_seqs * a.n_kv_heads, 128, 0, s>>>(cp);
+    return cudaGetLastError();
+}
+
+template <int D, bool FP8>
+cudaError_t launch_g(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t s) {
+    switch (a.n_q_heads / a.n_kv_heads) {
+        case 1: return launch_t<D, FP8, 1>(prm, a, s);
+        case 2: return launch_t<D, FP8, 2>(prm, a, s);
+        case 4: return launch_t<D, FP8, 4>(prm, a, s);
+        case 8: return launch_t<D, FP8, 8>(prm, a, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+
+}  // namespace
+
+int decode_grid_ctas(int num_sms) { return num_sms * kCtasPerSm; }
+
+size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
+                              int num_sms) {
+    const int G = n_q_heads / n_kv_heads;
+    const size_t slots = (size_t)num_seqs * n_kv_heads + (size_t)decode_grid_ctas(num_sms);
+    return align16((size_t)(num_seqs + 1) * sizeof(int)) +
+           slots * (size_t)G * (head_dim + 2) * sizeof(float);
+}
+
+cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t s) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t need = decode_workspace_bytes(a.num_seqs, a.n_q_heads, a.n_kv_heads, a.head_dim, sms);
+    if (a.workspace_bytes < need) return cudaErrorInvalidValue;
+    if (a.num_seqs == 0) return cudaSuccess;
+    DecodeParams prm;
+    prm.out = static_cast<__nv_bfloat16 *>(a.out);
+    prm.q = static_cast<const uint16_t *>(a.q);
+    prm.block_tables = a.block_tables;
+    prm.max_blocks = a.max_blocks_per_seq;
+    prm.context_lens = a.context_lens;
+    prm.B = a.num_seqs;
+    prm.Hq = a.n_q_heads;
+    prm.Hkv = a.n_kv_heads;
+    prm.num_blocks = a.num_blocks;
+    prm.scale_log2 = a.scale * kLog2e;
+    prm.k_scale = a.k_scale;
+    prm.v_scale = a.v_scale;
+    prm.rope = a.rope;
+    prm.max_pos = a.max_pos;
+    prm.prefix = static_cast<int *>(a.workspace);
+    prm.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(a.workspace) +
+                                             align16((size_t)(a.num_seqs + 1) * sizeof(int)));
+    prm.nctas = decode_grid_ctas(sms);
+    prm.err = a.err;
+    if (a.head_dim == 128) return a.fp8 ? launch_g<128, true>(prm, a, s) : launch_g<128, false>(prm, a, s);
+    if (a.head_dim == 64) return a.fp8 ? launch_g<64, true>(prm, a, s) : launch_g<64, false>(prm, a, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pkv
