@@ -64,8 +64,12 @@ enum pkv_status {
     PKV_E_CUDA = -4,        /* a CUDA runtime call or launch failed                      */
     PKV_E_TIMEOUT = -5,     /* (device) a bounded wait inside a kernel ran out            */
     PKV_E_BOUNDS = -6,      /* (device) slot / block id / position outside its array      */
-    PKV_E_ALIGN = -7        /* a pointer is not 16-byte aligned                           */
+    PKV_E_ALIGN = -7,       /* a pointer is not 16-byte aligned                           */
+    PKV_E_SCRATCH_LIMIT = -8 /* the call needs more than PKV_NOALLOC_SCRATCH_BYTES of scratch */
 };
+
+/* Size of the built-in decode scratch array used by pkv_paged_decode_attention_noalloc. */
+#define PKV_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 
 /* Library version, (major << 16) | minor. */
 int pkv_version(void);
@@ -188,6 +192,36 @@ int pkv_paged_prefill_attention(void *out, const void *q, const void *k_cache,
                                 const float *k_scale, const float *v_scale,
                                 const float *rope_cos_sin, int max_pos, int max_new_tokens,
                                 pkv_stream_t stream);
+
+/*
+ * pkv_paged_decode_attention_noalloc -- pkv_paged_decode_attention for callers that cannot
+ * allocate device memory.  (Not an operation of the pages: they have no counterpart.)
+ * Engines typically give nearly all HBM to the KV-block pool when they start, so a
+ * cudaMalloc from inside a decode step may fail, and on a latency-critical step a
+ * cudaMalloc/cudaFree pair can synchronise the device; framework plugins that must not
+ * allocate outside their host's allocator are in the same position.  This entry point
+ * takes the same arguments minus the workspace, allocates nothing, and uses instead a
+ * fixed array of PKV_NOALLOC_SCRATCH_BYTES (8 MiB) of device memory that is part of the
+ * library image: every GPU that loads the library holds it until the process exits.
+ *   - Calls needing more than PKV_NOALLOC_SCRATCH_BYTES (see pkv_decode_workspace_bytes)
+ *     return PKV_E_SCRATCH_LIMIT and enqueue nothing.
+ *   - All calls on a device share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race on it and must be serialised by the caller.  The
+ *     array keeps the last call's contents; none of them needs to start at zero, so
+ *     nothing is cleared.
+ *   - The first call on each device (with that device current) looks up the array's
+ *     device address with cudaGetSymbolAddress; make that first call before any stream
+ *     capture begins.
+ * Results equal pkv_paged_decode_attention's for the same inputs.
+ */
+int pkv_paged_decode_attention_noalloc(void *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       int max_blocks_per_seq, const int32_t *context_lens,
+                                       int num_seqs, int n_q_heads, int n_kv_heads,
+                                       int head_dim, int block_size, long long num_blocks,
+                                       float scale, int cache_dtype, const float *k_scale,
+                                       const float *v_scale, const float *rope_cos_sin,
+                                       int max_pos, pkv_stream_t stream);
 
 /*
  * pkv_get_error -- synchronise `stream`, then return and clear the current device's error

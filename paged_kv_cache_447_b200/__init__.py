@@ -16,6 +16,7 @@ import importlib
 
 _BINDING_NAMES = {
     "kv_store", "rope_apply", "paged_decode_attention", "paged_prefill_attention",
+    "paged_decode_attention_noalloc", "NOALLOC_SCRATCH_BYTES",
     "rope_build_table", "decode_workspace_bytes", "cache_bytes", "get_error", "strerror",
     "debug_wait_timeout", "version", "library_path", "load_library", "PagedKVError",
     "BF16", "FP8_E4M3",

@@ -19,11 +19,13 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 
 BF16 = 0
 FP8_E4M3 = 1
+NOALLOC_SCRATCH_BYTES = 8 << 20  # PKV_NOALLOC_SCRATCH_BYTES in include/pkv.h
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape or dtype",
            -3: "workspace missing or too small", -4: "CUDA runtime error",
            -5: "a bounded wait inside a kernel ran out",
-           -6: "slot, block id or position out of range", -7: "pointer not 16-byte aligned"}
+           -6: "slot, block id or position out of range", -7: "pointer not 16-byte aligned",
+           -8: "call needs more than the built-in decode scratch array"}
 
 
 class PagedKVError(RuntimeError):
@@ -62,6 +64,8 @@ def load_library():
                                         I, P, SZ, P], I),
         "pkv_paged_prefill_attention": ([P, P, P, P, P, P, I, P, I, I, I, I, I, I, LL, F, I,
                                          P, P, P, I, I, P], I),
+        "pkv_paged_decode_attention_noalloc": ([P, P, P, P, P, I, P, I, I, I, I, I, LL, F, I,
+                                                P, P, P, I, P], I),
         "pkv_get_error": ([P], I),
         "pkv_debug_wait_timeout": ([LL, P], I),
     }
@@ -213,6 +217,31 @@ def paged_prefill_attention(q, k_cache, v_cache, cu_seqlens, block_tables, conte
         _p(_i32(context_lens, "context_lens")), context_lens.shape[0], T, Hq, Hkv, D, bs, NB,
         float(scale), _cache_dtype(k_cache), _p(k_scale), _p(v_scale), _p(rope_cos_sin),
         max_pos, int(max_new_tokens), _stream(stream)))
+    return out
+
+
+def paged_decode_attention_noalloc(q, k_cache, v_cache, block_tables, context_lens, *,
+                                   scale=None, k_scale=None, v_scale=None, rope_cos_sin=None,
+                                   out=None, stream=None) -> torch.Tensor:
+    """Decode attention without a workspace argument, for callers that cannot allocate
+    device memory at decode time (for example an engine that gave nearly all HBM to its
+    KV-block pool).  The library uses its own fixed 8 MiB device array instead, shared by
+    every call on the device: calls must not overlap on the GPU.  Pass ``out`` to keep
+    the call itself free of allocations."""
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    _bf16(q, "q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    max_pos = rope_cos_sin.shape[0] if rope_cos_sin is not None else 0
+    _check("pkv_paged_decode_attention_noalloc",
+           load_library().pkv_paged_decode_attention_noalloc(
+               _p(out), _p(q), _p(k_cache), _p(v_cache), _p(_i32(block_tables, "block_tables")),
+               block_tables.shape[1], _p(_i32(context_lens, "context_lens")), B, Hq, Hkv, D, bs,
+               NB, float(scale), _cache_dtype(k_cache), _p(k_scale), _p(v_scale),
+               _p(rope_cos_sin), max_pos, _stream(stream)))
     return out
 
 

@@ -122,6 +122,7 @@ const char *pkv_strerror(int code) {
         case PKV_E_TIMEOUT: return "a bounded wait inside a kernel ran out";
         case PKV_E_BOUNDS: return "slot, block id or position out of range";
         case PKV_E_ALIGN: return "pointer not 16-byte aligned";
+        case PKV_E_SCRATCH_LIMIT: return "call needs more than the built-in decode scratch array";
         default: return "unknown status";
     }
 }
