@@ -1,7 +1,616 @@
-// prefill.cu -- paged causal prefill attention (placeholder until the tcgen05 kernel lands).
+// prefill.cu -- paged causal prefill attention on the 5th-generation tensor cores.
+//
+// "LLM primer: from text to tokens, embeddings, QKV and Transformer", §17.1: prefill
+// processes all prompt tokens at once and is compute-bound.  "Inside the Nano-vLLM engine:
+// KV cache, attention and tensor parallelism", §3 (softmax(QK^T/sqrt(d))V), §3.1 (tile the
+// computation on chip instead of materialising QK^T -- the FlashAttention idea), §3.2 (causal
+// mask, RoPE fused into the attention kernel, max subtraction), §2.2 (K/V read through the
+// block table).  The pages give no kernel design; this one is written for sm_100a.
+//
+// One CTA (384 threads, one per SM by shared memory) computes two 128-row query tiles that
+// share every K/V tile: two heads of one GQA group on the same rows, or (group 1) two
+// consecutive row tiles of one head.
+//   warp 0       TMA producer: Q tiles, then K and V tiles of 128 keys = 8 paged blocks, each
+//                block one 128-byte-swizzled box per 64 columns, addressed via the block table
+//   warp 1       TMEM owner and MMA issuer (one thread): S_i = Q_i K^T and O_i += P_i V with
+//                tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in tensor memory)
+//   warps 4-7    softmax for tile 0, warps 8-11 for tile 1: thread r owns row r; reads its S
+//                row from TMEM, masks (bottom-right causal), exp2 with the running max, writes
+//                P (bf16) back into the S columns, which the next MMA reads as its A operand
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).  The running max is
+// lazily updated: P is computed against a stale max unless the new one is more than 2^8
+// larger, so O needs a rescale (TMEM read-modify-write by the softmax thread) only rarely.
+// Keys past the sequence are masked; the one V tile holding the sequence's partial last
+// block has its tail rows zeroed in shared memory before use (0 * NaN would poison O).
 #include "common.cuh"
 #include "internal.h"
 
 namespace pkv {
-cudaError_t launch_paged_prefill(const PrefillArgs &, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kRows = 128;       // query rows per tile
+constexpr int kKeys = 128;       // keys per K/V tile (8 blocks)
+constexpr int kSoftmax0 = 4;     // first warp of softmax warpgroup 0
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+
+template <int D>
+struct PGeo {
+    static constexpr int kSlabs = D / 64;                    // 128-byte column slabs
+    static constexpr int kSlabBytes = kRows * 128;           // 16 KB (128 rows x 128 B)
+    static constexpr int kQBytes = kSlabs * kSlabBytes;      // one Q tile
+    static constexpr int kKVBytes = kSlabs * kSlabBytes;     // one K (or V) tile of 128 keys
+    static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = 2 * kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKVBytes;
+    static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+    static constexpr int kBarBytes = 8 * (16 + 3 * kStages) + 16;
+    static constexpr int kSmem = kOffBar + kBarBytes + 1024;  // + alignment slack
+};
+
+struct PrefillParams {
+    __nv_bfloat16 *out;
+    const int32_t *cu_seqlens, *block_tables, *context_lens;
+    int max_blocks, B, Hq, Hkv, n_qt;
+    long long num_blocks;
+    float scale_log2;
+    const float *k_scale, *v_scale;
+    const float *rope;
+    int max_pos;
+    int *err;
+};
+
+// ------------------------------------------------------------------ tcgen05 wrappers
+
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;  // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, A K-major.
+__host__ __device__ constexpr uint32_t mma_idesc(int M, int N, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                       uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum), "r"(0), "r"(0), "r"(0),
+        "r"(0));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+        "%27, %28, %29, %30, %31, %32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+        "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ------------------------------------------------------------------ work item
+
+struct Item {
+    int b, kvh, head[2], row0[2], n, L, t_base;
+    bool valid[2];
+    int n_kv;  // K/V tiles to visit
+};
+
+__device__ __forceinline__ Item decode_item(const PrefillParams &p, int idx) {
+    Item it;
+    const int G = p.Hq / p.Hkv;
+    int qt, h0, h1;
+    if (G >= 2) {
+        const int pairs = G / 2;
+        const int pair = idx % pairs;
+        int r = idx / pairs;
+        it.kvh = r % p.Hkv;
+        r /= p.Hkv;
+        it.b = r % p.B;
+        qt = p.n_qt - 1 - r / p.B;  // heaviest (last) row tiles first
+        h0 = it.kvh * G + 2 * pair;
+        h1 = h0 + 1;
+        it.row0[0] = it.row0[1] = qt * kRows;
+    } else {
+        const int nqt2 = (p.n_qt + 1) / 2;
+        int r = idx;
+        const int h = r % p.Hq;
+        r /= p.Hq;
+        it.b = r % p.B;
+        qt = nqt2 - 1 - r / p.B;
+        it.kvh = h;
+        h0 = h1 = h;
+        it.row0[0] = 2 * qt * kRows;
+        it.row0[1] = it.row0[0] + kRows;
+    }
+    it.head[0] = h0;
+    it.head[1] = h1;
+    it.t_base = __ldg(p.cu_seqlens + it.b);
+    it.n = __ldg(p.cu_seqlens + it.b + 1) - it.t_base;
+    it.L = __ldg(p.context_lens + it.b);
+    int ext = 0;
+    for (int i = 0; i < 2; ++i) {
+        it.valid[i] = it.row0[i] < it.n;
+        if (it.valid[i]) {
+            const int e = it.L - it.n + min(it.row0[i] + kRows, it.n);
+            ext = max(ext, e);
+        }
+    }
+    ext = min(ext, it.L);
+    it.n_kv = ext > 0 ? (ext + kKeys - 1) / kKeys : 0;
+    return it;
+}
+
+// ------------------------------------------------------------------ the kernel
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+    using Geo = PGeo<D>;
+    constexpr int NS = Geo::kStages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (sbase - smem_u32(smem_raw));
+
+    const uint32_t sQ = sbase + Geo::kOffQ;
+    const uint32_t sK = sbase + Geo::kOffK;
+    const uint32_t sV = sbase + Geo::kOffV;
+    const uint32_t bar0 = sbase + Geo::kOffBar;
+    // barrier addresses
+    const uint32_t b_qfull = bar0 + 0, b_qready = bar0 + 8, b_vraw = bar0 + 16, b_ofinal = bar0 + 24;
+    const uint32_t b_sfull = bar0 + 32;   // [2]
+    const uint32_t b_pfull = bar0 + 48;   // [2]
+    const uint32_t b_drain = bar0 + 64;
+    const uint32_t b_kfull = bar0 + 128;  // [NS]
+    const uint32_t b_vfull = b_kfull + 8 * NS;
+    const uint32_t b_empty = b_vfull + 8 * NS;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Geo::kOffBar + 72);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kOffBar + 76);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Item it = decode_item(p, blockIdx.x);
+    if (!it.valid[0]) return;  // no rows for this CTA (uniform)
+    const int Lc = min(it.L, p.max_blocks * kBlockSize);
+    if (Lc < it.L && threadIdx.x == 0) atomicOr(p.err, kErrBounds);
+
+    if (threadIdx.x == 0) {
+        mbar_init(b_qfull, 1);
+        mbar_init(b_qready, 256);
+        mbar_init(b_vraw, 1);
+        mbar_init(b_ofinal, 1);
+        mbar_init(b_drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(b_sfull + 8 * i, 1);
+            mbar_init(b_pfull + 8 * i, 128);
+        }
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(b_kfull + 8 * s, 1);
+            mbar_init(b_vfull + 8 * s, 1);
+            mbar_init(b_empty + 8 * s, 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
+                     ::"r"(smem_u32((const void *)tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int n_kv = it.n_kv;
+
+    const int nblk = (Lc + kBlockSize - 1) / kBlockSize;  // valid blocks of the sequence
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        uint32_t issued = 0;  // bitmask: stage s has an outstanding fill (bit s: K, bit 8+s: V)
+        uint32_t phase_bits = 0;
+        bool ok = true;
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            mbar_arrive_expect_tx(b_qfull, 2 * Geo::kQBytes);
+            for (int i = 0; i < 2; ++i)
+                for (int s = 0; s < Geo::kSlabs; ++s)
+                    tma_load_3d(sQ + i * Geo::kQBytes + s * Geo::kSlabBytes, &tm_q, b_qfull, 64 * s,
+                                it.head[i], it.t_base + it.row0[i]);
+        }
+        const int oob = (int)min(p.num_blocks, (long long)(0x7fffffff / kBlockSize));
+        for (int j = 0; j < n_kv && ok; ++j) {
+            const int st = j % NS;
+            const uint32_t par = ((j / NS) & 1) ^ 1;
+            int phys = oob;
+            if (lane < 8) {
+                const int lb = j * 8 + lane;
+                if (lb < nblk) {
+                    phys = __ldg(p.block_tables + (size_t)it.b * p.max_blocks + lb);
+                    if (phys < 0 || (long long)phys >= p.num_blocks) {
+                        atomicOr(p.err, kErrBounds);
+                        phys = oob;
+                    }
+                }
+            }
+            const bool fix = (Lc % kBlockSize) != 0 && j == (Lc - 1) / kKeys;
+            if (lane == 0) {
+                if (*abort_flag || !mbar_wait_bounded(b_empty + 8 * st, par, p.err)) {
+                    ok = false;
+                    *abort_flag = 1;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            int ph[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ph[i] = __shfl_sync(0xffffffffu, phys, i);
+            if (lane == 0) {
+                const uint32_t kb = b_kfull + 8 * st, vb = fix ? b_vraw : b_vfull + 8 * st;
+                mbar_arrive_expect_tx(kb, Geo::kKVBytes);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    for (int s = 0; s < Geo::kSlabs; ++s)
+                        tma_load_3d(sK + st * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_k, kb,
+                                    64 * s, it.kvh, ph[i] * kBlockSize);
+                mbar_arrive_expect_tx(vb, Geo::kKVBytes);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    for (int s = 0; s < Geo::kSlabs; ++s)
+                        tma_load_3d(sV + st * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_v, vb,
+                                    64 * s, it.kvh, ph[i] * kBlockSize);
+                issued |= (1u << st) | (fix ? 0u : (1u << (8 + st)));
+                phase_bits = (phase_bits & ~(1u << st)) | ((uint32_t)((j / NS) & 1) << st);
+            }
+            if (fix) {
+                // zero the rows past the sequence in the tile's partial block, then publish
+                bool landed = true;
+                if (lane == 0) landed = mbar_wait_bounded(b_vraw, 0, p.err);
+                landed = __shfl_sync(0xffffffffu, landed ? 1 : 0, 0) != 0;
+                if (landed) {
+                    const int blk_in_tile = ((Lc - 1) / kBlockSize) % 8;
+                    const int first = Lc % kBlockSize;
+                    const int rows = kBlockSize - first;
+                    for (int s = 0; s < Geo::kSlabs; ++s) {
+                        const uint32_t row0 = sV + st * Geo::kKVBytes + s * Geo::kSlabBytes +
+                                              blk_in_tile * 2048 + first * 128;
+                        for (int e = lane; e < rows * 8; e += 32)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + e * 16),
+                                         "r"(0)
+                                         : "memory");
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    if (landed) mbar_arrive(b_vfull + 8 * st);
+                    else *abort_flag = 1;
+                }
+                if (!landed) ok = false;
+            }
+        }
+        // drain outstanding TMA copies before the CTA can exit
+        if (lane == 0) {
+            mbar_wait_bounded(b_qfull, 0, p.err);
+            for (int s = 0; s < NS; ++s) {
+                const uint32_t par = (phase_bits >> s) & 1;
+                if ((issued >> s) & 1) mbar_wait_bounded(b_kfull + 8 * s, par, p.err);
+                if ((issued >> (8 + s)) & 1) mbar_wait_bounded(b_vfull + 8 * s, par, p.err);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0 && n_kv > 0) {
+            constexpr uint32_t idS = mma_idesc(kRows, kKeys, false);
+            constexpr uint32_t idO = mma_idesc(kRows, D, true);
+            const uint32_t tS[2] = {tmem + 0, tmem + 128};
+            const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+            bool ok = mbar_wait_bounded(b_qready, 0, p.err) && !*abort_flag;
+            auto issue_s = [&](int i, int st) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk / 4) * Geo::kSlabBytes + (kk % 4) * 32;
+                    mma_ss(tS[i], sw128_desc(sQ + i * Geo::kQBytes + off, 16, 1024),
+                           sw128_desc(sK + st * Geo::kKVBytes + off, 16, 1024), idS, kk > 0);
+                }
+                mma_commit(b_sfull + 8 * i);
+            };
+            auto issue_pv = [&](int i, int st, int j) {
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk)
+                    mma_ts(tO[i], tS[i] + 8 * kk,
+                           sw128_desc(sV + st * Geo::kKVBytes + kk * 2048, Geo::kSlabBytes, 1024), idO,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            if (ok) ok = mbar_wait_bounded(b_kfull, 0, p.err);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                issue_s(1, 0);
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int st = j % NS;
+                const uint32_t par = (j / NS) & 1;
+                const int st1 = (j + 1) % NS;
+                const uint32_t par1 = ((j + 1) / NS) & 1;
+                ok = mbar_wait_bounded(b_vfull + 8 * st, par, p.err) &&
+                     mbar_wait_bounded(b_pfull + 0, j & 1, p.err);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(0, st, j);
+                if (j + 1 < n_kv) {
+                    ok = mbar_wait_bounded(b_kfull + 8 * st1, par1, p.err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_s(0, st1);
+                }
+                ok = mbar_wait_bounded(b_pfull + 8, j & 1, p.err);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv(1, st, j);
+                mma_commit(b_empty + 8 * st);
+                if (j + 1 < n_kv) issue_s(1, st1);
+            }
+            mma_commit(b_ofinal);
+            if (!ok) *abort_flag = 1;
+            // every MMA issued above has finished before TMEM can be released
+            mma_commit(b_drain);
+            mbar_wait_bounded(b_drain, 0, p.err);
+        }
+    } else if (warp >= kSoftmax0) {
+        // ---------------------------------------------------------------- softmax
+        const int wg = (warp - kSoftmax0) / 4;       // tile index
+        const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const int row = it.row0[wg] + r;              // row within the sequence's new tokens
+        const bool row_valid = row < it.n;
+        const int pos = it.L - it.n + row;
+        const int limit = min(pos, Lc - 1);           // last visible key
+        const float c = p.scale_log2 * (p.k_scale ? __ldg(p.k_scale + it.kvh) : 1.f);
+
+        bool ok = mbar_wait_bounded(b_qfull, 0, p.err);
+        if (ok && p.rope && row_valid && it.valid[wg]) {
+            if (pos < 0 || pos >= p.max_pos) {
+                atomicOr(p.err, kErrBounds);
+            } else {
+                const float *cs = p.rope + (size_t)pos * D;
+                const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
+                const uint32_t sw = (uint32_t)(r & 7);
+#pragma unroll 1
+                for (int lc = 0; lc < D / 16; ++lc) {  // chunk pairs (lc, lc + D/16)
+                    const int lc2 = lc + D / 16;
+                    const uint32_t a1 = qrow + (lc / 8) * Geo::kSlabBytes + (((lc % 8) ^ sw) << 4);
+                    const uint32_t a2 = qrow + (lc2 / 8) * Geo::kSlabBytes + (((lc2 % 8) ^ sw) << 4);
+                    uint4 x1 = lds128(a1), x2 = lds128(a2);
+                    uint16_t *e1 = reinterpret_cast<uint16_t *>(&x1);
+                    uint16_t *e2 = reinterpret_cast<uint16_t *>(&x2);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int d = lc * 8 + e;
+                        rope_pair(e1[e], e2[e], __ldg(cs + d), __ldg(cs + D / 2 + d), e1[e], e2[e]);
+                    }
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(x1.x),
+                                 "r"(x1.y), "r"(x1.z), "r"(x1.w) : "memory");
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a2), "r"(x2.x),
+                                 "r"(x2.y), "r"(x2.z), "r"(x2.w) : "memory");
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(b_qready);
+
+        const uint32_t tS = tmem + lane_off + (uint32_t)(wg * 128);
+        const uint32_t tO = tmem + lane_off + (uint32_t)(256 + wg * D);
+        // Every tcgen05.ld/st below is executed by all 32 lanes of the warp together (the
+        // instructions are warp-aligned); per-row differences are data, not control flow.
+        float m_used = -INFINITY, l_sum = 0.f;
+        for (int j = 0; j < n_kv; ++j) {
+            bool got = !*abort_flag && mbar_wait_bounded(b_sfull + 8 * wg, j & 1, p.err);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            float s[kKeys];
+#pragma unroll
+            for (int q4 = 0; q4 < kKeys / 32; ++q4) {
+                uint32_t rr[32];
+                tmem_ld32(tS + q4 * 32, rr);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(rr[e]);
+            }
+            tc_wait_ld();
+            const int key0 = j * kKeys;
+            if (key0 + kKeys - 1 > limit) {  // diagonal / tail tile: mask keys past the limit
+#pragma unroll
+                for (int e = 0; e < kKeys; ++e)
+                    if (key0 + e > limit) s[e] = -INFINITY;
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < kKeys; ++e) mx = fmaxf(mx, s[e]);
+            const float m_tile = mx * c;  // c > 0; -inf when the row sees no key here
+            // a new running max only when it grew by more than 2^8 (lazy rescale)
+            float alpha = 1.f;
+            if (m_tile > m_used + kRescaleLog2) {
+                if (m_used != -INFINITY && j > 0) alpha = ex2(m_used - m_tile);
+                m_used = m_tile;
+            }
+            l_sum *= alpha;
+            const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;  // masked s: p = 0
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int h = 0; h < kKeys / 64; ++h) {  // 64 keys -> 32 packed columns
+                uint32_t rr[32];
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const float p0 = ex2(fmaf(s[h * 64 + e], c, neg_m));
+                    const float p1 = ex2(fmaf(s[h * 64 + e + 1], c, neg_m));
+                    acc0 += p0;
+                    acc1 += p1;
+                    rr[e / 2] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tS + h * 32, rr);
+            }
+            l_sum += acc0 + acc1;
+            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                // O_i <- alpha * O_i (alpha = 1 on rows that keep their max).  PV_i of the
+                // previous tile has completed: it was issued before this tile's S_i, whose
+                // completion we waited for.
+#pragma unroll 1
+                for (int q4 = 0; q4 < D / 32; ++q4) {
+                    uint32_t rr[32];
+                    tmem_ld32(tO + q4 * 32, rr);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+                    tmem_st32(tO + q4 * 32, rr);
+                }
+            }
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(b_pfull + 8 * wg);
+        }
+        // ---- epilogue: O / l -> bf16 -> global (valid rows only)
+        bool fin = n_kv > 0 && ok && mbar_wait_bounded(b_ofinal, 0, p.err);
+        const bool done = __all_sync(0xffffffffu, fin);
+        tc_fence_after();
+        const bool store = row_valid && it.valid[wg];
+        const float vs = p.v_scale ? __ldg(p.v_scale + it.kvh) : 1.f;
+        const float inv = (done && l_sum > 0.f) ? vs / l_sum : 0.f;
+        uint4 *dst = reinterpret_cast<uint4 *>(p.out + ((size_t)(it.t_base + (store ? row : 0)) * p.Hq + it.head[wg]) * D);
+#pragma unroll 1
+        for (int q4 = 0; q4 < D / 32; ++q4) {
+            uint32_t rr[32];
+            if (done) {
+                tmem_ld32(tO + q4 * 32, rr);
+                tc_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) rr[e] = 0u;
+            }
+            if (store) {
+#pragma unroll
+                for (int v8 = 0; v8 < 4; ++v8) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(rr[v8 * 8 + 0]) * inv, __uint_as_float(rr[v8 * 8 + 1]) * inv);
+                    w.y = pack_bf16x2(__uint_as_float(rr[v8 * 8 + 2]) * inv, __uint_as_float(rr[v8 * 8 + 3]) * inv);
+                    w.z = pack_bf16x2(__uint_as_float(rr[v8 * 8 + 4]) * inv, __uint_as_float(rr[v8 * 8 + 5]) * inv);
+                    w.w = pack_bf16x2(__uint_as_float(rr[v8 * 8 + 6]) * inv, __uint_as_float(rr[v8 * 8 + 7]) * inv);
+                    dst[q4 * 4 + v8] = w;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s) {
+    if (a.fp8) return cudaErrorNotSupported;  // FP8 prefill: not built yet
+    PrefillParams p;
+    p.out = static_cast<__nv_bfloat16 *>(a.out);
+    p.cu_seqlens = a.cu_seqlens;
+    p.block_tables = a.block_tables;
+    p.context_lens = a.context_lens;
+    p.max_blocks = a.max_blocks_per_seq;
+    p.B = a.num_seqs;
+    p.Hq = a.n_q_heads;
+    p.Hkv = a.n_kv_heads;
+    p.n_qt = (a.max_new_tokens + kRows - 1) / kRows;
+    p.num_blocks = a.num_blocks;
+    p.scale_log2 = a.scale * kLog2e;
+    p.k_scale = a.fp8 ? a.k_scale : nullptr;
+    p.v_scale = a.fp8 ? a.v_scale : nullptr;
+    p.rope = a.rope;
+    p.max_pos = a.max_pos;
+    p.err = a.err;
+    if (p.n_qt == 0) return cudaSuccess;
+    const int G = p.Hq / p.Hkv;
+    long long items = (G >= 2) ? (long long)p.n_qt * p.B * p.Hkv * (G / 2)
+                               : (long long)((p.n_qt + 1) / 2) * p.B * p.Hq;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (a.head_dim == 128) {
+        auto k = prefill_kernel<128>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<128>::kSmem);
+        if (e != cudaSuccess) return e;
+        k<<<(unsigned)items, kThreads, PGeo<128>::kSmem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+    } else if (a.head_dim == 64) {
+        auto k = prefill_kernel<64>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<64>::kSmem);
+        if (e != cudaSuccess) return e;
+        k<<<(unsigned)items, kThreads, PGeo<64>::kSmem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace pkv

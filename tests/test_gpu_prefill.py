@@ -1,0 +1,134 @@
+"""GPU parity of paged prefill attention (tcgen05/TMEM kernel) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_447_b200 as pkv
+from paged_kv_cache_447_b200 import workloads as W
+
+from helpers import (DeviceWorkload, cache_bits, compare, oracle_attention, oracle_caches,
+                     oracle_store)
+
+pytestmark = pytest.mark.gpu
+
+
+def _prefill_case(wl, rope=True, rows=None, steps=None):
+    """Store every step (GPU and oracle), then prefill the last one on both sides."""
+    d = DeviceWorkload(wl)
+    kc, vc = oracle_caches(wl)
+    steps = wl.steps if steps is None else steps
+    for st in steps:
+        d.store(st, rope=rope)
+        oracle_store(wl, st, kc, vc, rope=rope)
+    st = steps[-1]
+    out = d.prefill(st, rope=rope)
+    torch.cuda.synchronize()
+    assert pkv.get_error() == 0
+    assert np.array_equal(cache_bits(d.k_cache), kc)
+    ref = oracle_attention(wl, st, kc, vc, rope=rope, rows=rows)
+    return out, ref
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_prefill_tiny(rope):
+    wl = W.tiny(seed=1)
+    out, ref = _prefill_case(wl, rope, steps=wl.steps[:1])
+    compare(out, ref, what="tiny prefill")
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 4), (16, 4), (16, 2)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_groups_and_head_dims(hq, hkv, d):
+    """Every compiled GQA group (1, 2, 4, 8) and head_dim 64/128 on a ragged shared-prefix
+    batch: 3 requests, 48-token aliased prefix, 200 new tokens each (2 row tiles, the second
+    ragged; 2 key tiles, the last with a partial block)."""
+    wl = W.shared_prefix(seed=10 + hq + hkv + d, requests=3, prefix=48, new=200, hq=hq, hkv=hkv,
+                         d=d)
+    out, ref = _prefill_case(wl)
+    compare(out, ref, what=f"prefill hq={hq} hkv={hkv} d={d}")
+
+
+@pytest.mark.parametrize("prefix,new", [(0, 1), (0, 16), (0, 128), (0, 129), (16, 255),
+                                        (2048, 130), (96, 700)])
+def test_prefill_lengths(prefix, new):
+    """Row/key tile boundaries: one token, one block, exactly one tile, one past a tile,
+    a long cached prefix, several tiles."""
+    wl = W.shared_prefix(seed=7, requests=2, prefix=prefix, new=new, hq=8, hkv=2, d=128)
+    out, ref = _prefill_case(wl)
+    compare(out, ref, what=f"prefill prefix={prefix} new={new}")
+
+
+def test_prefill_shared_prefix_full_size_sampled():
+    """The 32-request shared-prefix workload at full size (2048-token aliased prefix + 2048
+    new tokens each, 32 q / 8 kv heads): the whole output is produced in the launch
+    configuration the benchmark times, and sampled rows are checked against the oracle."""
+    wl = W.shared_prefix(seed=4)
+    st = wl.steps[0]
+    rng = np.random.default_rng(0)
+    rows = []
+    for b in (0, 13, 31):
+        base = int(st.cu_seqlens[b])
+        for r in (0, 1, 127, 128, 1000, 2046, 2047) + tuple(rng.integers(0, 2048, 6)):
+            for h in (0, 3, 17, 31):
+                rows.append((base + int(r), h))
+    rows = np.array(rows, dtype=np.int32)
+    out, ref = _prefill_case(wl, rows=rows)
+    got = out[torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()]
+    compare(got, ref, what="shared prefix sampled")
+    assert torch.isfinite(out.float()).all()
+
+
+def test_prefill_mix_chunks_bf16():
+    """The four 512-token chunked prefills of the continuous-batching step (long lognormal
+    prior contexts), every row."""
+    full = W.mix(seed=5)
+    st = full.steps[0]
+    B = st.decode_seqs
+    chunks = W.sub_step(st, range(B, st.num_seqs))
+    wl = W.Workload(full.name, full.seed, 32, 8, 128, full.num_blocks, "bf16", full.k_cache,
+                    full.v_cache, [chunks], full.max_pos)
+    out, ref = _prefill_case(wl)
+    compare(out, ref, what="mix chunks")
+
+
+def test_prefill_unused_slots_hold_nan():
+    wl = W.tiny(seed=1, nan_fill=True)
+    out, ref = _prefill_case(wl, steps=wl.steps[:1])
+    compare(out, ref, what="prefill nan sentinels")
+
+
+def test_prefill_empty_and_single_token_sequences():
+    g = torch.Generator().manual_seed(3)
+    hq, hkv, d = 8, 2, 128
+    news = [0, 1, 130, 0, 17]
+    ctx = [0, 5, 130, 40, 17]      # seq 3 has cached context but no new tokens
+    counts = [W.blocks_needed(L) for L in ctx]
+    nb = sum(counts) + 2
+    perm = torch.randperm(nb, generator=g)
+    bt = W._assign_blocks(perm, counts, max_blocks=max(counts))
+    kc, vc = W._fill_cache(g, nb, hkv, d, False)
+    st = W._step("edge", g, hq, hkv, d, news, ctx, bt)
+    wl = W.Workload("edge", 0, hq, hkv, d, nb, "bf16", kc, vc, [st], max_pos=200)
+    out, ref = _prefill_case(wl)
+    compare(out, ref, what="edge prefill")
+
+
+def test_prefill_block_id_out_of_range_is_flagged():
+    wl = W.tiny(seed=1)
+    st = wl.steps[0]
+    bt = st.block_tables.clone()
+    bt[3, 2] = -5
+    d = DeviceWorkload(wl)
+    pkv.paged_prefill_attention(st.q.cuda(), d.k_cache, d.v_cache, st.cu_seqlens.cuda(),
+                                bt.cuda(), st.context_lens.cuda(), st.max_new_tokens)
+    assert pkv.get_error() == -6
+
+
+def test_prefill_fp8_cache_is_refused_cleanly():
+    full = W.mix(seed=5, decodes=4, chunks=1, chunk_len=64, fp8=True, max_context=512)
+    d = DeviceWorkload(full)
+    st = full.steps[0]
+    with pytest.raises(pkv.PagedKVError) as e:
+        d.prefill(st)
+    assert e.value.code == -2
