@@ -171,6 +171,26 @@ def prefill_flops(st: W.Step, hq: int, d: int) -> float:
     return float(4 * d * hq * int(pairs))
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (read + write) from the committed ncu record in profiles/, or
+    None if there is none for this kernel and workload or the kernel source has changed
+    since the counters were taken."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f).get(kernel)
+        if not rec or rec.get("workload") != workload:
+            return None
+        with open(os.path.join(ROOT, rec["src"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if not sha.startswith(rec["src_sha256_prefix"]):
+            return None
+        return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 # ----------------------------------------------------------------------------- runner
 
 class Runner:
@@ -467,7 +487,9 @@ def main():
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "decode_tok_s_per_layer": res.get("decode_tok_s_per_layer"),
         "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": runit,
-                     "frac": ach / peak, "traffic": None,
+                     "frac": ach / peak,
+                     "traffic": recorded_traffic("decode_kernel" if runner.B else "prefill_kernel",
+                                                 args.workload),
                      "kernel": "paged_decode_attention" if runner.B else "paged_prefill_attention",
                      "peak_source": pk_kind, "kernel_ms": res.get("attn_kernel_ms")},
         "clocks": res["clocks"],
