@@ -269,12 +269,13 @@ int pkv_paged_prefill_attention(void *out, const void *q, const void *k_cache,
     if (!err) return PKV_E_CUDA;
     const int esize = fp8 ? 1 : 2;
     const uint64_t slots = (uint64_t)num_blocks * block_size;
-    // 128-byte swizzled boxes: 64 bf16 (or 128 fp8) elements of a row per box.
-    const uint32_t inner = (uint32_t)(128 / esize) < (uint32_t)head_dim ? 128 / esize : head_dim;
+    // bf16: 128-byte swizzled boxes of 64 elements (the MMA operand layout);
+    // E4M3: plain boxes of a whole row (widened to f16 in shared memory by the kernel).
+    const uint32_t inner = fp8 ? (uint32_t)head_dim : 64u;
     CUtensorMap tq, tk, tv;
     if (!encode_3d(&tq, q, 2, head_dim, n_q_heads, num_tokens, 64, 1, 128, true) ||
-        !encode_3d(&tk, k_cache, esize, head_dim, n_kv_heads, slots, inner, 1, block_size, true) ||
-        !encode_3d(&tv, v_cache, esize, head_dim, n_kv_heads, slots, inner, 1, block_size, true))
+        !encode_3d(&tk, k_cache, esize, head_dim, n_kv_heads, slots, inner, 1, block_size, !fp8) ||
+        !encode_3d(&tv, v_cache, esize, head_dim, n_kv_heads, slots, inner, 1, block_size, !fp8))
         return PKV_E_CUDA;
     PrefillArgs a{out, q, cu_seqlens, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                   num_tokens, n_q_heads, n_kv_heads, head_dim, num_blocks, scale, fp8, k_scale,

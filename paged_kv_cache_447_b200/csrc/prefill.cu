@@ -35,19 +35,22 @@ constexpr int kSoftmax0 = 4;     // first warp of softmax warpgroup 0
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
-template <int D>
+template <int D, bool FP8>
 struct PGeo {
     static constexpr int kSlabs = D / 64;                    // 128-byte column slabs
     static constexpr int kSlabBytes = kRows * 128;           // 16 KB (128 rows x 128 B)
     static constexpr int kQBytes = kSlabs * kSlabBytes;      // one Q tile
     static constexpr int kKVBytes = kSlabs * kSlabBytes;     // one K (or V) tile of 128 keys
     static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr int kStgBytes = FP8 ? kKeys * D : 0;    // raw E4M3 tile (K or V)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = 2 * kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+    static constexpr int kOffStg = kOffV + kStages * kKVBytes;
+    static constexpr int kOffBar = kOffStg + 2 * kStgBytes;
     static constexpr int kBarBytes = 8 * (16 + 3 * kStages) + 16;
     static constexpr int kSmem = kOffBar + kBarBytes + 1024;  // + alignment slack
+    static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct PrefillParams {
@@ -74,9 +77,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
     return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, A K-major.
-__host__ __device__ constexpr uint32_t mma_idesc(int M, int N, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+// Instruction descriptor, kind::f16: A and B both bf16 (or both f16), fp32 accumulator,
+// A K-major.
+__host__ __device__ constexpr uint32_t mma_idesc(int M, int N, bool b_mn_major, bool f16) {
+    const uint32_t ab = f16 ? 0u : 1u;
+    return (1u << 4) | (ab << 7) | (ab << 10) | ((b_mn_major ? 1u : 0u) << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -139,10 +144,39 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)two));
+    return r;
+}
+
+// bf16 -> f16, exact for |x| in [2^-17, 65504] (8 significant bits fit in f16's 11).
+__device__ __forceinline__ uint16_t bf16_to_f16_bits(uint16_t b) {
+    __half h = __float2half_rn(__uint_as_float(((uint32_t)b) << 16));
+    return *reinterpret_cast<uint16_t *>(&h);
 }
 
 // ------------------------------------------------------------------ work item
@@ -200,11 +234,11 @@ __device__ __forceinline__ Item decode_item(const PrefillParams &p, int idx) {
 
 // ------------------------------------------------------------------ the kernel
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
-    using Geo = PGeo<D>;
+    using Geo = PGeo<D, FP8>;
     constexpr int NS = Geo::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -213,12 +247,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sQ = sbase + Geo::kOffQ;
     const uint32_t sK = sbase + Geo::kOffK;
     const uint32_t sV = sbase + Geo::kOffV;
+    const uint32_t sStg = sbase + Geo::kOffStg;  // FP8: raw K tile, then raw V tile
     const uint32_t bar0 = sbase + Geo::kOffBar;
     // barrier addresses
     const uint32_t b_qfull = bar0 + 0, b_qready = bar0 + 8, b_vraw = bar0 + 16, b_ofinal = bar0 + 24;
     const uint32_t b_sfull = bar0 + 32;   // [2]
     const uint32_t b_pfull = bar0 + 48;   // [2]
     const uint32_t b_drain = bar0 + 64;
+    const uint32_t b_stgfull = bar0 + 80, b_stgempty = bar0 + 88;  // FP8 staging
     const uint32_t b_kfull = bar0 + 128;  // [NS]
     const uint32_t b_vfull = b_kfull + 8 * NS;
     const uint32_t b_empty = b_vfull + 8 * NS;
@@ -242,10 +278,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(b_pfull + 8 * i, 128);
         }
         for (int s = 0; s < NS; ++s) {
-            mbar_init(b_kfull + 8 * s, 1);
-            mbar_init(b_vfull + 8 * s, 1);
+            // bf16: one arrival with the TMA byte count; FP8: the 64 converter threads
+            mbar_init(b_kfull + 8 * s, FP8 ? 64 : 1);
+            mbar_init(b_vfull + 8 * s, FP8 ? 64 : 1);
             mbar_init(b_empty + 8 * s, 1);
         }
+        mbar_init(b_stgfull, 1);
+        mbar_init(b_stgempty, 64);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -262,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int nblk = (Lc + kBlockSize - 1) / kBlockSize;  // valid blocks of the sequence
 
+    if (warp < kSoftmax0) {
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
         uint32_t issued = 0;  // bitmask: stage s has an outstanding fill (bit s: K, bit 8+s: V)
@@ -291,6 +331,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                         phys = oob;
                     }
                 }
+            }
+            if constexpr (FP8) {
+                // raw E4M3 tiles go to the single staging buffer; the converter warps
+                // widen them into the MMA operand stage
+                if (lane == 0) {
+                    if (*abort_flag || !mbar_wait_bounded(b_stgempty, (j & 1) ^ 1, p.err)) {
+                        ok = false;
+                        *abort_flag = 1;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                int ph[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ph[i] = __shfl_sync(0xffffffffu, phys, i);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(b_stgfull, 2 * Geo::kStgBytes);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        tma_load_3d(sStg + i * kBlockSize * D, &tm_k, b_stgfull, 0, it.kvh, ph[i] * kBlockSize);
+                        tma_load_3d(sStg + Geo::kStgBytes + i * kBlockSize * D, &tm_v, b_stgfull, 0, it.kvh,
+                                    ph[i] * kBlockSize);
+                    }
+                    issued |= 1u << 16;
+                    phase_bits = (phase_bits & ~(1u << 16)) | ((uint32_t)(j & 1) << 16);
+                }
+                continue;
             }
             const bool fix = (Lc % kBlockSize) != 0 && j == (Lc - 1) / kKeys;
             if (lane == 0) {
@@ -351,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // drain outstanding TMA copies before the CTA can exit
         if (lane == 0) {
             mbar_wait_bounded(b_qfull, 0, p.err);
+            if ((issued >> 16) & 1) mbar_wait_bounded(b_stgfull, (phase_bits >> 16) & 1, p.err);
             for (int s = 0; s < NS; ++s) {
                 const uint32_t par = (phase_bits >> s) & 1;
                 if ((issued >> s) & 1) mbar_wait_bounded(b_kfull + 8 * s, par, p.err);
@@ -360,8 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0 && n_kv > 0) {
-            constexpr uint32_t idS = mma_idesc(kRows, kKeys, false);
-            constexpr uint32_t idO = mma_idesc(kRows, D, true);
+            constexpr uint32_t idS = mma_idesc(kRows, kKeys, false, FP8);
+            constexpr uint32_t idO = mma_idesc(kRows, D, true, FP8);
             const uint32_t tS[2] = {tmem + 0, tmem + 128};
             const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
             bool ok = mbar_wait_bounded(b_qready, 0, p.err) && !*abort_flag;
@@ -416,7 +484,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(b_drain);
             mbar_wait_bounded(b_drain, 0, p.err);
         }
-    } else if (warp >= kSoftmax0) {
+    } else if (FP8 && warp >= 2) {
+        // ---------------------------------------------------------------- E4M3 -> f16
+        // Warps 2-3 widen each raw tile into the swizzled operand layout (the same
+        // 128-byte-swizzled K-major layout TMA produces for 16-bit caches).  V rows of keys
+        // past the sequence are written as zeros (0 * NaN would poison O).
+        const int ct = threadIdx.x - 64;
+        constexpr int CPR = D / 16;  // 16-byte E4M3 chunks per row
+        for (int j = 0; j < n_kv; ++j) {
+            const int st = j % NS;
+            const bool got = !*abort_flag && mbar_wait_bounded(b_stgfull, j & 1, p.err) &&
+                             mbar_wait_bounded(b_empty + 8 * st, ((j / NS) & 1) ^ 1, p.err);
+            if (!got) {
+                *abort_flag = 1;
+                break;
+            }
+            const int key0 = j * kKeys;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {  // K, then V
+                const uint32_t src = sStg + t * Geo::kStgBytes;
+                const uint32_t dst = (t == 0 ? sK : sV) + st * Geo::kKVBytes;
+#pragma unroll 2
+                for (int idx = ct; idx < kKeys * CPR; idx += 64) {
+                    const int row = idx / CPR, c = idx % CPR;
+                    uint4 raw = lds128(src + row * D + c * 16);
+                    if (t == 1 && key0 + row >= Lc) raw = make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                    uint32_t h[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        h[2 * q] = e4m3x2_to_f16x2(w[q] & 0xFFFFu);
+                        h[2 * q + 1] = e4m3x2_to_f16x2(w[q] >> 16);
+                    }
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int lc = 2 * c + hf;  // 8-element chunk of the 16-bit row
+                        const uint32_t a =
+                            dst + (lc / 8) * Geo::kSlabBytes + row * 128 + (((lc % 8) ^ (row & 7)) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(h[4 * hf]),
+                                     "r"(h[4 * hf + 1]), "r"(h[4 * hf + 2]), "r"(h[4 * hf + 3])
+                                     : "memory");
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(b_kfull + 8 * st);
+            mbar_arrive(b_vfull + 8 * st);
+            mbar_arrive(b_stgempty);
+        }
+    }
+    } else {
         // ---------------------------------------------------------------- softmax
         const int wg = (warp - kSoftmax0) / 4;       // tile index
         const int r = (warp & 3) * 32 + lane;         // row within the tile == TMEM lane
@@ -455,6 +572,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        if constexpr (FP8) {
+            // the FP8 path multiplies in f16: convert this row of Q (swizzle untouched)
+            if (ok) {
+                const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
+#pragma unroll 1
+                for (int ch = 0; ch < D / 8; ++ch) {
+                    const uint32_t a = qrow + (ch / 8) * Geo::kSlabBytes + (ch % 8) * 16;
+                    uint4 x = lds128(a);
+                    uint16_t *e = reinterpret_cast<uint16_t *>(&x);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) e[k] = bf16_to_f16_bits(e[k]);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x.x), "r"(x.y),
+                                 "r"(x.z), "r"(x.w) : "memory");
+                }
+            }
+        }
         fence_proxy_async_smem();
         mbar_arrive(b_qready);
 
@@ -486,9 +619,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < kKeys; ++e)
                     if (key0 + e > limit) s[e] = -INFINITY;
             }
-            float mx = -INFINITY;
+            float m8[8];  // eight independent max chains instead of one 128-long chain
 #pragma unroll
-            for (int e = 0; e < kKeys; ++e) mx = fmaxf(mx, s[e]);
+            for (int k = 0; k < 8; ++k) m8[k] = s[k];
+#pragma unroll
+            for (int e = 8; e < kKeys; e += 8)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[e + k]);
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             const float m_tile = mx * c;  // c > 0; -inf when the row sees no key here
             // a new running max only when it grew by more than 2^8 (lazy rescale)
             float alpha = 1.f;
@@ -498,21 +637,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             l_sum *= alpha;
             const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;  // masked s: p = 0
-            float acc0 = 0.f, acc1 = 0.f;
+            const float2 c2 = make_float2(c, c), nm2 = make_float2(neg_m, neg_m);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int h = 0; h < kKeys / 64; ++h) {  // 64 keys -> 32 packed columns
-                uint32_t rr[32];
+            for (int h = 0; h < kKeys / 32; ++h) {  // 32 keys -> 16 packed columns
+                uint32_t rr[16];
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float p0 = ex2(fmaf(s[h * 64 + e], c, neg_m));
-                    const float p1 = ex2(fmaf(s[h * 64 + e + 1], c, neg_m));
-                    acc0 += p0;
-                    acc1 += p1;
-                    rr[e / 2] = pack_bf16x2(p0, p1);
+                for (int e = 0; e < 32; e += 2) {
+                    const float2 x = __ffma2_rn(make_float2(s[h * 32 + e], s[h * 32 + e + 1]), c2, nm2);
+                    const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+                    acc[(e / 2) & 3] = __fadd2_rn(acc[(e / 2) & 3], pp);
+                    rr[e / 2] = FP8 ? pack_f16x2(pp.x, pp.y) : pack_bf16x2(pp.x, pp.y);
                 }
-                tmem_st32(tS + h * 32, rr);
+                tmem_st16(tS + h * 16, rr);
             }
-            l_sum += acc0 + acc1;
+            l_sum += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                     ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
             if (__any_sync(0xffffffffu, alpha != 1.f)) {
                 // O_i <- alpha * O_i (alpha = 1 on rows that keep their max).  PV_i of the
                 // previous tile has completed: it was issued before this tile's S_i, whose
@@ -571,10 +712,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+template <int D, bool FP8>
+cudaError_t run(const PrefillArgs &a, const PrefillParams &p, long long items, cudaStream_t s) {
+    auto k = prefill_kernel<D, FP8>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<D, FP8>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<(unsigned)items, kThreads, PGeo<D, FP8>::kSmem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s) {
-    if (a.fp8) return cudaErrorNotSupported;  // FP8 prefill: not built yet
     PrefillParams p;
     p.out = static_cast<__nv_bfloat16 *>(a.out);
     p.cu_seqlens = a.cu_seqlens;
@@ -597,19 +746,11 @@ cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s) {
     long long items = (G >= 2) ? (long long)p.n_qt * p.B * p.Hkv * (G / 2)
                                : (long long)((p.n_qt + 1) / 2) * p.B * p.Hq;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (a.head_dim == 128) {
-        auto k = prefill_kernel<128>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<128>::kSmem);
-        if (e != cudaSuccess) return e;
-        k<<<(unsigned)items, kThreads, PGeo<128>::kSmem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
-    } else if (a.head_dim == 64) {
-        auto k = prefill_kernel<64>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<64>::kSmem);
-        if (e != cudaSuccess) return e;
-        k<<<(unsigned)items, kThreads, PGeo<64>::kSmem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
-    } else {
-        return cudaErrorInvalidValue;
-    }
+    cudaError_t e;
+    if (a.head_dim == 128) e = a.fp8 ? run<128, true>(a, p, items, s) : run<128, false>(a, p, items, s);
+    else if (a.head_dim == 64) e = a.fp8 ? run<64, true>(a, p, items, s) : run<64, false>(a, p, items, s);
+    else return cudaErrorInvalidValue;
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -125,10 +125,34 @@ def test_prefill_block_id_out_of_range_is_flagged():
     assert pkv.get_error() == -6
 
 
-def test_prefill_fp8_cache_is_refused_cleanly():
-    full = W.mix(seed=5, decodes=4, chunks=1, chunk_len=64, fp8=True, max_context=512)
-    d = DeviceWorkload(full)
+def _fp8_workload(seed, news, ctx, hq, hkv, d):
+    """A prefill batch over an E4M3 cache with per-kv-head scales."""
+    g = torch.Generator().manual_seed(seed)
+    counts = [W.blocks_needed(L) for L in ctx]
+    nb = sum(counts) + 3
+    perm = torch.randperm(nb, generator=g)
+    bt = W._assign_blocks(perm, counts, max_blocks=max(counts) + 1)
+    st = W._step("fp8", g, hq, hkv, d, news, ctx, bt)
+    ks, vs = W._fp8_scales(st.k, st.v)
+    kc, vc = W._fill_cache(g, nb, hkv, d, True, ks, vs)
+    return W.Workload("fp8", seed, hq, hkv, d, nb, "fp8", kc, vc, [st], max_pos=max(ctx) + 1,
+                      k_scale=ks, v_scale=vs)
+
+
+def test_prefill_mix_chunks_fp8():
+    """The four 512-token chunks of the continuous-batching step over the E4M3 cache."""
+    full = W.mix(seed=5, fp8=True)
     st = full.steps[0]
-    with pytest.raises(pkv.PagedKVError) as e:
-        d.prefill(st)
-    assert e.value.code == -2
+    chunks = W.sub_step(st, range(st.decode_seqs, st.num_seqs))
+    wl = W.Workload(full.name, full.seed, 32, 8, 128, full.num_blocks, "fp8", full.k_cache,
+                    full.v_cache, [chunks], full.max_pos, full.k_scale, full.v_scale)
+    out, ref = _prefill_case(wl)
+    compare(out, ref, fp8=True, what="mix chunks fp8")
+
+
+@pytest.mark.parametrize("d,hq,hkv", [(128, 8, 8), (128, 16, 2), (64, 8, 4), (64, 4, 4)])
+def test_prefill_fp8_groups_and_head_dims(d, hq, hkv):
+    wl = _fp8_workload(40 + d + hq, news=[1, 200, 37, 300], ctx=[9, 233, 37, 900], hq=hq,
+                       hkv=hkv, d=d)
+    out, ref = _prefill_case(wl)
+    compare(out, ref, fp8=True, what=f"fp8 prefill d={d} hq={hq} hkv={hkv}")
