@@ -11,6 +11,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libpagedkv is written for sm_100a (B200) only"
 #endif
@@ -157,6 +159,15 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched so that it may
+// be scheduled while the previous kernel on the stream drains; it then waits for that
+// kernel's completion (and memory) before touching any global input, and lets the next
+// kernel be scheduled as early as possible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier among `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -211,6 +222,42 @@ __device__ __forceinline__ void rope_pair(uint16_t x1, uint16_t x2, float c, flo
     y2 = f64_to_bf16_rne(r2);
 }
 
+// Round r = fl(a*b - p) (one FMA; p = fl(c*d) is the other product) to bf16 into *out and
+// report whether that is guaranteed to equal rounding the exact a*b - c*d.
+// Error: |r - exact| <= ulp(p)/2 + ulp(r)/2 < (|p| + |r|) * 2^-23.
+// With y = bf16(r), r lies inside y's rounding interval, whose nearest boundary is at least
+// |y| * 2^-9 - |r - y| away (half a bf16 ulp is >= |y| * 2^-9 in every binade, and larger
+// than that for bf16 subnormals).  If that distance exceeds the error bound, the exact
+// value rounds to y as well.  NaN/inf make the comparison false (fp64 path).
+__device__ __forceinline__ bool bf16_round_checked(float r, float p, uint16_t *out) {
+    const __nv_bfloat16 yb = __float2bfloat16_rn(r);
+    const uint16_t bits = *reinterpret_cast<const uint16_t *>(&yb);
+    const float y = __uint_as_float((uint32_t)bits << 16);
+    *out = bits;
+    const float room = __fmaf_rn(fabsf(y), 0x1p-9f, -fabsf(r - y));
+    const float err = (fabsf(p) + fabsf(r)) * 0x1p-23f;
+    return room > err;
+}
+
+// rope_pair with the same result bits, computed in fp32 whenever the bound above proves
+// the fp32 value rounds like the exact one (nearly always), else in fp64.
+__device__ __forceinline__ void rope_pair_fast(uint16_t x1, uint16_t x2, float c, float s,
+                                               uint16_t &y1, uint16_t &y2) {
+    const float a = __uint_as_float((uint32_t)x1 << 16), b = __uint_as_float((uint32_t)x2 << 16);
+    const float p1 = __fmul_rn(b, s), p2 = __fmul_rn(a, s);
+    const float r1 = __fmaf_rn(a, c, -p1);  // x1 cos - x2 sin
+    const float r2 = __fmaf_rn(b, c, p2);   // x2 cos + x1 sin
+    uint16_t o1, o2;
+    const bool ok1 = bf16_round_checked(r1, p1, &o1);
+    const bool ok2 = bf16_round_checked(r2, p2, &o2);
+    if (ok1 && ok2) {
+        y1 = o1;
+        y2 = o2;
+    } else {
+        rope_pair(x1, x2, c, s, y1, y2);
+    }
+}
+
 // Sequence owning token row t: the b with cu[b] <= t < cu[b+1] (cu is non-decreasing).
 __device__ __forceinline__ int owner_seq(const int32_t *cu, int num_seqs, int t) {
     int lo = 0, hi = num_seqs - 1;
@@ -221,5 +268,24 @@ __device__ __forceinline__ int owner_seq(const int32_t *cu, int num_seqs, int t)
     }
     return lo;
 }
+
+#ifndef __CUDACC_RTC__
+// Launch `kern` on `stream` with programmatic stream serialisation allowed (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+#endif
 
 }  // namespace pkv

@@ -32,8 +32,10 @@
 namespace pkv {
 namespace {
 
-constexpr int kConsumers = 4;
-constexpr int kThreads = 32 * (1 + kConsumers);
+// Consumer warps per CTA: 4 for bf16 MHA (memory-bound: more warps do not help), 8 when a
+// tile feeds several query heads or must be widened from E4M3 (more arithmetic per byte).
+__host__ __device__ constexpr int consumers_for(int G, bool fp8) { return (G > 1 || fp8) ? 8 : 4; }
+constexpr int kMaxThreads = 32 * (1 + 8);
 constexpr int kCtasPerSm = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMergeBar = 1;
@@ -58,6 +60,8 @@ struct DecodeParams {
 
 template <int D, bool FP8, int G>
 struct Geometry {
+    static constexpr int kConsumers = consumers_for(G, FP8);
+    static constexpr int kThreads = 32 * (1 + kConsumers);
     static constexpr int kElem = FP8 ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
     static constexpr int kTileBytes = kBlockSize * kRowBytes;          // one K (or V) block
@@ -92,8 +96,9 @@ __device__ __forceinline__ int seq_blocks(int L, int max_blocks, int *err) {
 }
 
 // Exclusive prefix over sequences of their block counts, into pfx[0..B] (shared memory).
+template <int kThreads>
 __device__ void block_prefix(const DecodeParams &p, int *pfx) {
-    __shared__ int warp_tot[kThreads / 32];
+    __shared__ int warp_tot[kMaxThreads / 32];
     __shared__ int carry_s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (threadIdx.x == 0) carry_s = 0;
@@ -146,11 +151,13 @@ __device__ __forceinline__ UnitPos locate(const int *pfx, int B, int Hkv, long l
 }
 
 template <int D, bool FP8, int G>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecodeParams p) {
     using Geo = Geometry<D, FP8, G>;
     constexpr int NS = Geo::kStages;
+    constexpr int kConsumers = Geo::kConsumers;
+    constexpr int kThreads = Geo::kThreads;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;                                                  // NS x stage
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * Geo::kStageBytes);
@@ -163,10 +170,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    block_prefix(p, pfx);
+    pdl_wait();
+    pdl_trigger();
+    block_prefix<kThreads>(p, pfx);
     const long long total = (long long)p.Hkv * pfx[p.B];
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i <= p.B; i += kThreads) p.prefix[i] = pfx[i];
+    // sequences with an empty context get zero rows (strided over the CTAs)
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x)
+        if (pfx[b + 1] == pfx[b])
+            for (int e = threadIdx.x; e < p.Hq * D; e += kThreads)
+                p.out[(size_t)b * p.Hq * D + e] = __float2bfloat16_rn(0.f);
     const long long U = total > 0 ? (total + p.nctas - 1) / p.nctas : 1;
     const long long u0 = (long long)blockIdx.x * U;
     const long long u1 = (u0 + U < total) ? u0 + U : total;
@@ -275,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int pos = L - 1;
                 if (pos >= 0 && pos < p.max_pos) {
                     const float *row = p.rope + (size_t)pos * D;
-                    rope_pair(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
+                    rope_pair_fast(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
                 } else {
                     atomicOr(p.err, kErrBounds);
                 }
@@ -502,33 +516,47 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 }
 
-// Merge the partial states of every (sequence, kv head) that was split across CTAs, and
-// zero the rows of empty sequences.  One CTA per (sequence, kv head).
+// Merge the partial states of every (sequence, kv head) that was split across CTAs.
+// A segment is split iff some CTA boundary c*U falls strictly inside it; the CTA of the
+// first such boundary merges it (one CTA per decode CTA, most have nothing to do).
+__device__ __forceinline__ int find_seq_global(const int *pfx, int B, int Hkv, long long u) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if ((long long)Hkv * __ldg(pfx + mid) <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
-    const int seg = blockIdx.x;
-    const int b = seg / p.Hkv, kvh = seg % p.Hkv;
-    const int pb = p.prefix[b], nb = p.prefix[b + 1] - pb;
-    const long long total = (long long)p.Hkv * p.prefix[p.B];
-    if (nb == 0) {
-        for (int e = threadIdx.x; e < G * D; e += blockDim.x)
-            p.out[((size_t)b * p.Hq + kvh * G) * D + e] = __float2bfloat16_rn(0.f);
-        return;
-    }
+    pdl_wait();
+    pdl_trigger();
+    const int c = blockIdx.x;
+    const long long total = (long long)p.Hkv * __ldg(p.prefix + p.B);
+    if (c == 0 || total == 0) return;
     const long long U = (total + p.nctas - 1) / p.nctas;
+    const long long x = (long long)c * U;
+    if (x >= total) return;
+    const int b = find_seq_global(p.prefix, p.B, p.Hkv, x);
+    const int pb = __ldg(p.prefix + b), nb = __ldg(p.prefix + b + 1) - pb;
+    const int kvh = (int)((x - (long long)p.Hkv * pb) / nb);
     const long long start = (long long)p.Hkv * pb + (long long)kvh * nb;
+    if (start == x) return;                          // boundary at a segment start: no split
     const int c0 = (int)(start / U), c1 = (int)((start + nb - 1) / U);
-    if (c0 == c1) return;  // written directly by the decode kernel
+    if (c0 != c - 1) return;                         // an earlier boundary's CTA merges it
+    const int seg = b * p.Hkv + kvh;
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
         const int g = e / D, d = e % D;
         float M = -INFINITY;
-        for (int c = c0; c <= c1; ++c) {
-            const float *slot = p.partials + (size_t)(seg + c) * (G * (D + 2));
+        for (int cc = c0; cc <= c1; ++cc) {
+            const float *slot = p.partials + (size_t)(seg + cc) * (G * (D + 2));
             M = fmaxf(M, slot[G * D + g]);
         }
         float o = 0.f, lsum = 0.f;
-        for (int c = c0; c <= c1; ++c) {
-            const float *slot = p.partials + (size_t)(seg + c) * (G * (D + 2));
+        for (int cc = c0; cc <= c1; ++cc) {
+            const float *slot = p.partials + (size_t)(seg + cc) * (G * (D + 2));
             const float mk = slot[G * D + g];
             const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
             o += f * slot[g * D + d];
@@ -543,6 +571,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
 template <int D, bool FP8, int G>
 size_t smem_bytes(int B) {
     using Geo = Geometry<D, FP8, G>;
+    constexpr int kConsumers = Geo::kConsumers;
     size_t s = (size_t)Geo::kStages * Geo::kStageBytes + 2 * Geo::kStages * sizeof(uint64_t);
     s += (size_t)G * D * 4 + (size_t)kConsumers * G * 16 * 4 + (size_t)kConsumers * G * (D + 2) * 4;
     s += (size_t)(B + 1) * 4;
@@ -556,18 +585,17 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
+    constexpr int kThreads = Geometry<D, FP8, G>::kThreads;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
     DecodeParams lp = prm;
     lp.nctas = std::min(prm.nctas, occ * (prm.nctas / kCtasPerSm));
-    kern<<<lp.nctas, kThreads, smem, s>>>(*a.tm_k, *a.tm_v, lp);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3(lp.nctas), dim3(kThreads), smem, s, *a.tm_k, *a.tm_v, lp);
     if (e != cudaSuccess) return e;
     DecodeParams cp = lp;
     cp.v_scale = FP8 ? a.v_scale : nullptr;
-    combine_kernel<D, G><<<a.num_seqs * a.n_kv_heads, 128, 0, s>>>(cp);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel<D, G>, dim3(lp.nctas), dim3(128), 0, s, cp);
 }
 
 template <int D, bool FP8>

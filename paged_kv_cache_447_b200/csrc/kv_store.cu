@@ -32,7 +32,7 @@ __device__ __forceinline__ void rotate_chunk(Chunk &x, const float *cos_row, con
     const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
     const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) rope_pair(a[e], b[e], cs[e], sn[e], ra[e], rb[e]);
+    for (int e = 0; e < 8; ++e) rope_pair_fast(a[e], b[e], cs[e], sn[e], ra[e], rb[e]);
     x.lo = *reinterpret_cast<uint4 *>(ra);
     x.hi = *reinterpret_cast<uint4 *>(rb);
 }
@@ -50,6 +50,8 @@ __device__ __forceinline__ uint2 quantize_chunk(uint4 v, double s) {
 
 template <bool FP8, bool ROPE>
 __global__ void __launch_bounds__(256) kv_store_kernel(StoreArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int D = a.head_dim, H = a.n_kv_heads;
     const int cpr = D / 16;                      // chunk pairs per head row
     const long long items = (long long)a.num_tokens * H * cpr;
@@ -102,6 +104,8 @@ __global__ void __launch_bounds__(256) kv_store_kernel(StoreArgs a) {
 }
 
 __global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int D = a.head_dim, H = a.n_q_heads + a.n_kv_heads;
     const int cpr = D / 16;
     const long long items = (long long)a.num_tokens * H * cpr;
@@ -151,22 +155,16 @@ cudaError_t launch_kv_store(const StoreArgs &a, cudaStream_t s) {
     const long long items = (long long)a.num_tokens * a.n_kv_heads * (a.head_dim / 16);
     if (items == 0) return cudaSuccess;
     const int grid = grid_for(items, 256);
-    if (a.fp8) {
-        if (a.rope) kv_store_kernel<true, true><<<grid, 256, 0, s>>>(a);
-        else kv_store_kernel<true, false><<<grid, 256, 0, s>>>(a);
-    } else {
-        if (a.rope) kv_store_kernel<false, true><<<grid, 256, 0, s>>>(a);
-        else kv_store_kernel<false, false><<<grid, 256, 0, s>>>(a);
-    }
-    return cudaGetLastError();
+    auto k = a.fp8 ? (a.rope ? kv_store_kernel<true, true> : kv_store_kernel<true, false>)
+                   : (a.rope ? kv_store_kernel<false, true> : kv_store_kernel<false, false>);
+    return launch_pdl(k, dim3(grid), dim3(256), 0, s, a);
 }
 
 cudaError_t launch_rope_apply(const RopeArgs &a, cudaStream_t s) {
     const long long items =
         (long long)a.num_tokens * (a.n_q_heads + a.n_kv_heads) * (a.head_dim / 16);
     if (items == 0) return cudaSuccess;
-    rope_apply_kernel<<<grid_for(items, 256), 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(rope_apply_kernel, dim3(grid_for(items, 256)), dim3(256), 0, s, a);
 }
 
 }  // namespace pkv

@@ -262,6 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kOffBar + 76);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     const Item it = decode_item(p, blockIdx.x);
     if (!it.valid[0]) return;  // no rows for this CTA (uniform)
     const int Lc = min(it.L, p.max_blocks * kBlockSize);
@@ -544,31 +546,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int limit = min(pos, Lc - 1);           // last visible key
         const float c = p.scale_log2 * (p.k_scale ? __ldg(p.k_scale + it.kvh) : 1.f);
 
+        // Q-RoPE on load: this thread rotates its row in shared memory.  In fp32: one
+        // product, one FMA and one rounding to bf16 per value, i.e. within one bf16 ulp of
+        // the exact rotation (which pkv_rope_apply and the K rotation of pkv_kv_store
+        // produce bit for bit); the difference stays far inside the attention tolerance and
+        // keeps this prologue off the critical path of the tensor pipe.
         bool ok = mbar_wait_bounded(b_qfull, 0, p.err);
         if (ok && p.rope && row_valid && it.valid[wg]) {
             if (pos < 0 || pos >= p.max_pos) {
                 atomicOr(p.err, kErrBounds);
             } else {
-                const float *cs = p.rope + (size_t)pos * D;
+                const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope + (size_t)pos * D);
                 const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
                 const uint32_t sw = (uint32_t)(r & 7);
 #pragma unroll 1
-                for (int lc = 0; lc < D / 16; ++lc) {  // chunk pairs (lc, lc + D/16)
-                    const int lc2 = lc + D / 16;
-                    const uint32_t a1 = qrow + (lc / 8) * Geo::kSlabBytes + (((lc % 8) ^ sw) << 4);
-                    const uint32_t a2 = qrow + (lc2 / 8) * Geo::kSlabBytes + (((lc2 % 8) ^ sw) << 4);
-                    uint4 x1 = lds128(a1), x2 = lds128(a2);
-                    uint16_t *e1 = reinterpret_cast<uint16_t *>(&x1);
-                    uint16_t *e2 = reinterpret_cast<uint16_t *>(&x2);
+                for (int g4 = 0; g4 < D / 16; g4 += 4) {
+                    float4 cv[8], sv[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int d = lc * 8 + e;
-                        rope_pair(e1[e], e2[e], __ldg(cs + d), __ldg(cs + D / 2 + d), e1[e], e2[e]);
+                    for (int k = 0; k < 8; ++k) {
+                        cv[k] = __ldg(cs4 + g4 * 2 + k);
+                        sv[k] = __ldg(cs4 + D / 8 + g4 * 2 + k);
                     }
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(x1.x),
-                                 "r"(x1.y), "r"(x1.z), "r"(x1.w) : "memory");
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a2), "r"(x2.x),
-                                 "r"(x2.y), "r"(x2.z), "r"(x2.w) : "memory");
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int lc = g4 + k4, lc2 = lc + D / 16;  // chunk pair (lc, lc + D/16)
+                        const uint32_t a1 = qrow + (lc / 8) * Geo::kSlabBytes + (((lc % 8) ^ sw) << 4);
+                        const uint32_t a2 = qrow + (lc2 / 8) * Geo::kSlabBytes + (((lc2 % 8) ^ sw) << 4);
+                        uint4 x1 = lds128(a1), x2 = lds128(a2);
+                        const uint32_t w1[4] = {x1.x, x1.y, x1.z, x1.w};
+                        const uint32_t w2[4] = {x2.x, x2.y, x2.z, x2.w};
+                        const float cc[8] = {cv[2 * k4].x, cv[2 * k4].y, cv[2 * k4].z, cv[2 * k4].w,
+                                             cv[2 * k4 + 1].x, cv[2 * k4 + 1].y, cv[2 * k4 + 1].z,
+                                             cv[2 * k4 + 1].w};
+                        const float ss[8] = {sv[2 * k4].x, sv[2 * k4].y, sv[2 * k4].z, sv[2 * k4].w,
+                                             sv[2 * k4 + 1].x, sv[2 * k4 + 1].y, sv[2 * k4 + 1].z,
+                                             sv[2 * k4 + 1].w};
+                        uint32_t o1[4], o2[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float a0 = bf16lo(w1[q]), a1v = bf16hi(w1[q]);
+                            const float b0 = bf16lo(w2[q]), b1v = bf16hi(w2[q]);
+                            const float c0 = cc[2 * q], c1 = cc[2 * q + 1], s0 = ss[2 * q], s1 = ss[2 * q + 1];
+                            o1[q] = pack_bf16x2(__fmaf_rn(a0, c0, -__fmul_rn(b0, s0)),
+                                                __fmaf_rn(a1v, c1, -__fmul_rn(b1v, s1)));
+                            o2[q] = pack_bf16x2(__fmaf_rn(b0, c0, __fmul_rn(a0, s0)),
+                                                __fmaf_rn(b1v, c1, __fmul_rn(a1v, s1)));
+                        }
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(o1[0]),
+                                     "r"(o1[1]), "r"(o1[2]), "r"(o1[3]) : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a2), "r"(o2[0]),
+                                     "r"(o2[1]), "r"(o2[2]), "r"(o2[3]) : "memory");
+                    }
                 }
             }
         }
@@ -717,8 +745,8 @@ cudaError_t run(const PrefillArgs &a, const PrefillParams &p, long long items, c
     auto k = prefill_kernel<D, FP8>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<D, FP8>::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<(unsigned)items, kThreads, PGeo<D, FP8>::kSmem, s>>>(*a.tm_q, *a.tm_k, *a.tm_v, p);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3((unsigned)items), dim3(kThreads), PGeo<D, FP8>::kSmem, s, *a.tm_q,
+                      *a.tm_k, *a.tm_v, p);
 }
 
 }  // namespace
