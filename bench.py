@@ -305,11 +305,11 @@ class Runner:
         return sum(ts) / len(ts)
 
 
-def build_workload(name: str):
+def build_workload(name: str, layers=None):
     if name == "qwen_decode":
         return W.qwen_decode(seed=2), 1
     if name == "gqa_decode":
-        return W.gqa_decode(seed=3), 32
+        return W.gqa_decode(seed=3), (32 if layers is None else layers)
     if name == "shared_prefix":
         return W.shared_prefix(seed=4), 1
     if name == "mix":
@@ -319,10 +319,15 @@ def build_workload(name: str):
     raise ValueError(name)
 
 
-def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=True):
-    wl, layers = build_workload(name)
+def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=True, layers=None):
+    wl, layers = build_workload(name, layers)
     r = Runner(wl, layers)
     st = r.st
+    # one checked step first: a device error (bounds, a bounded wait that ran out) stops here
+    r.step()
+    code = r.pkv.get_error()
+    if code != 0:
+        raise RuntimeError(f"{name}: device error {code} ({r.pkv.strerror(code)}) on the first step")
     esize = 1 if wl.cache_dtype == "fp8" else 2
     dominant = "decode" if r.B else "prefill"
     ms, clocks = timed_region(lambda: r.step(record=True, dominant=dominant), steps, warmup,
@@ -427,6 +432,8 @@ def main():
     ap.add_argument("--no-suite", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers of the GQA decode workload (default 32; fewer for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -463,7 +470,7 @@ def main():
         torch.cuda.set_device(0)
 
     res, runner = measure_ours(args.workload, args.steps, args.warmup, dist, local, pk,
-                               e2e=not args.no_e2e)
+                               e2e=not args.no_e2e, layers=args.layers)
     wl = runner.wl
     esize = 1 if wl.cache_dtype == "fp8" else 2
     if runner.B:

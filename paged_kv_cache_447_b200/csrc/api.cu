@@ -50,22 +50,6 @@ bool encoder() {
     return g_encode != nullptr;
 }
 
-// 3-D tiled map over a row-major [d2, d1, d0] tensor of `esize`-byte elements.
-bool encode_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128) {
-    if (!encoder()) return false;
-    const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
-    const cuuint32_t box[3] = {b0, b1, b2};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                          3, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_E_CUDA; }
@@ -98,6 +82,22 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns, int *err) {
 }
 
 }  // namespace
+
+// 3-D tiled map over a row-major [d2, d1, d0] tensor of `esize`-byte elements.
+bool encode_tensor_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128) {
+    if (!encoder()) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+    const cuuint32_t box[3] = {b0, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                          3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 cudaError_t launch_wait_timeout(unsigned long long limit_ns, int *err, cudaStream_t s) {
     wait_timeout_kernel<<<1, 32, 0, s>>>(limit_ns, err);
@@ -229,15 +229,9 @@ int pkv_paged_decode_attention(void *out, const void *q, const void *k_cache,
         return PKV_E_WORKSPACE;
     int *err = error_word();
     if (!err) return PKV_E_CUDA;
-    const int esize = fp8 ? 1 : 2;
-    CUtensorMap tk, tv;
-    const uint64_t slots = (uint64_t)num_blocks * block_size;
-    if (!encode_3d(&tk, k_cache, esize, head_dim, n_kv_heads, slots, head_dim, 1, block_size, false) ||
-        !encode_3d(&tv, v_cache, esize, head_dim, n_kv_heads, slots, head_dim, 1, block_size, false))
-        return PKV_E_CUDA;
-    DecodeArgs a{out, q, block_tables, max_blocks_per_seq, context_lens, num_seqs, n_q_heads,
-                 n_kv_heads, head_dim, num_blocks, scale, fp8, k_scale, v_scale, rope_cos_sin,
-                 max_pos, workspace, workspace_bytes, err, &tk, &tv};
+    DecodeArgs a{out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                 num_seqs, n_q_heads, n_kv_heads, head_dim, num_blocks, scale, fp8, k_scale,
+                 v_scale, rope_cos_sin, max_pos, workspace, workspace_bytes, err};
     cudaError_t e = launch_paged_decode(a, reinterpret_cast<cudaStream_t>(stream));
     if (e == cudaErrorInvalidValue) return PKV_E_WORKSPACE;
     return status_of(e);
@@ -267,19 +261,9 @@ int pkv_paged_prefill_attention(void *out, const void *q, const void *k_cache,
     if (rope_cos_sin && max_pos < 1) return PKV_E_INVALID;
     int *err = error_word();
     if (!err) return PKV_E_CUDA;
-    const int esize = fp8 ? 1 : 2;
-    const uint64_t slots = (uint64_t)num_blocks * block_size;
-    // bf16: 128-byte swizzled boxes of 64 elements (the MMA operand layout);
-    // E4M3: plain boxes of a whole row (widened to f16 in shared memory by the kernel).
-    const uint32_t inner = fp8 ? (uint32_t)head_dim : 64u;
-    CUtensorMap tq, tk, tv;
-    if (!encode_3d(&tq, q, 2, head_dim, n_q_heads, num_tokens, 64, 1, 128, true) ||
-        !encode_3d(&tk, k_cache, esize, head_dim, n_kv_heads, slots, inner, 1, block_size, !fp8) ||
-        !encode_3d(&tv, v_cache, esize, head_dim, n_kv_heads, slots, inner, 1, block_size, !fp8))
-        return PKV_E_CUDA;
-    PrefillArgs a{out, q, cu_seqlens, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                  num_tokens, n_q_heads, n_kv_heads, head_dim, num_blocks, scale, fp8, k_scale,
-                  v_scale, rope_cos_sin, max_pos, max_new_tokens, err, &tq, &tk, &tv};
+    PrefillArgs a{out, q, k_cache, v_cache, cu_seqlens, block_tables, max_blocks_per_seq,
+                  context_lens, num_seqs, num_tokens, n_q_heads, n_kv_heads, head_dim, num_blocks,
+                  scale, fp8, k_scale, v_scale, rope_cos_sin, max_pos, max_new_tokens, err};
     cudaError_t e = launch_paged_prefill(a, reinterpret_cast<cudaStream_t>(stream));
     if (e == cudaErrorNotSupported) return PKV_E_UNSUPPORTED;
     return status_of(e);

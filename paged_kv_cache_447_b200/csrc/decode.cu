@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, kCtasPerSm)
     constexpr int NS = Geo::kStages;
     constexpr int kConsumers = Geo::kConsumers;
     constexpr int kThreads = Geo::kThreads;
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;                                                  // NS x stage
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * Geo::kStageBytes);
     uint64_t *empty = full + NS;
@@ -575,7 +576,7 @@ size_t smem_bytes(int B) {
     size_t s = (size_t)Geo::kStages * Geo::kStageBytes + 2 * Geo::kStages * sizeof(uint64_t);
     s += (size_t)G * D * 4 + (size_t)kConsumers * G * 16 * 4 + (size_t)kConsumers * G * (D + 2) * 4;
     s += (size_t)(B + 1) * 4;
-    return s;
+    return s + 1024;  // alignment slack for the swizzled stages
 }
 
 template <int D, bool FP8, int G>
@@ -591,7 +592,16 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
     if (occ < 1) return cudaErrorInvalidConfiguration;
     DecodeParams lp = prm;
     lp.nctas = std::min(prm.nctas, occ * (prm.nctas / kCtasPerSm));
-    e = launch_pdl(kern, dim3(lp.nctas), dim3(kThreads), smem, s, *a.tm_k, *a.tm_v, lp);
+    // K/V maps with exactly the boxes the kernel's producer issues
+    using Geo = Geometry<D, FP8, G>;
+    CUtensorMap tk, tv;
+    const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
+    // one box per tile: a whole 16-token block of one kv head (16 rows of D elements)
+    if (!encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, D, 1, kBlockSize, false) ||
+        !encode_tensor_map_3d(&tv, a.v_cache, Geo::kElem, D, a.n_kv_heads, slots, D, 1, kBlockSize, false))
+        return cudaErrorUnknown;  // (cudaErrorInvalidValue means a short workspace)
+    static_assert(kBlockSize * D * Geo::kElem == Geo::kTileBytes, "one TMA box fills one tile");
+    e = launch_pdl(kern, dim3(lp.nctas), dim3(kThreads), smem, s, tk, tv, lp);
     if (e != cudaSuccess) return e;
     DecodeParams cp = lp;
     cp.v_scale = FP8 ? a.v_scale : nullptr;

@@ -35,6 +35,7 @@ struct RopeArgs {
 struct DecodeArgs {
     void *out;
     const void *q;
+    const void *k_cache, *v_cache;
     const int32_t *block_tables;
     int max_blocks_per_seq;
     const int32_t *context_lens;
@@ -48,12 +49,12 @@ struct DecodeArgs {
     void *workspace;
     size_t workspace_bytes;
     int *err;
-    const CUtensorMap *tm_k, *tm_v;  // host copies, passed by value to the kernel
 };
 
 struct PrefillArgs {
     void *out;
     const void *q;
+    const void *k_cache, *v_cache;
     const int32_t *cu_seqlens;
     const int32_t *block_tables;
     int max_blocks_per_seq;
@@ -66,8 +67,13 @@ struct PrefillArgs {
     const float *rope;
     int max_pos, max_new_tokens;
     int *err;
-    const CUtensorMap *tm_q, *tm_k, *tm_v;
 };
+
+// 3-D tiled TMA descriptor over a row-major [d2][d1][d0] tensor of `esize`-byte elements
+// (bf16 or bytes), box b0 x b1 x b2, optionally 128-byte swizzled.  Each launcher encodes
+// the maps its kernel reads, from the same compile-time geometry the kernel uses.
+bool encode_tensor_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
+                          uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128);
 
 cudaError_t launch_kv_store(const StoreArgs &a, cudaStream_t s);
 cudaError_t launch_rope_apply(const RopeArgs &a, cudaStream_t s);

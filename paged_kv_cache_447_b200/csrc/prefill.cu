@@ -742,11 +742,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool FP8>
 cudaError_t run(const PrefillArgs &a, const PrefillParams &p, long long items, cudaStream_t s) {
+    // Q: 128-byte swizzled boxes of 64 bf16 x 128 rows (one operand slab each).  K/V: for
+    // bf16 the same 128-byte swizzled 64-column boxes of one block (16 rows); for E4M3 one
+    // plain box of a whole block row range (widened in shared memory by the kernel).
+    constexpr int esize = FP8 ? 1 : 2;
+    CUtensorMap tq, tk, tv;
+    const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
+    const uint32_t inner = FP8 ? (uint32_t)D : 64u;
+    if (!encode_tensor_map_3d(&tq, a.q, 2, D, a.n_q_heads, a.num_tokens, 64, 1, kRows, true) ||
+        !encode_tensor_map_3d(&tk, a.k_cache, esize, D, a.n_kv_heads, slots, inner, 1, kBlockSize, !FP8) ||
+        !encode_tensor_map_3d(&tv, a.v_cache, esize, D, a.n_kv_heads, slots, inner, 1, kBlockSize, !FP8))
+        return cudaErrorInvalidValue;
     auto k = prefill_kernel<D, FP8>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<D, FP8>::kSmem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k, dim3((unsigned)items), dim3(kThreads), PGeo<D, FP8>::kSmem, s, *a.tm_q,
-                      *a.tm_k, *a.tm_v, p);
+    return launch_pdl(k, dim3((unsigned)items), dim3(kThreads), PGeo<D, FP8>::kSmem, s, tq, tk, tv, p);
 }
 
 }  // namespace
