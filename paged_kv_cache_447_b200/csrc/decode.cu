@@ -253,7 +253,12 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, kCtasPerSm)
     // ---------------------------------------------------------------------- consumers
     const int cw = warp - 1;          // consumer index 0..3
     const int ct = threadIdx.x - 32;  // consumer thread 0..127
-    const int t = lane & 15, hpair = lane >> 4;
+    // q.k lane mapping (see the q.k loop): kTPL tokens per lane group of kLPG lanes
+    constexpr int kTPL = (G == 2 || G == 4) ? 2 : 1;
+    constexpr int kLPG = 2 * kTPL;
+    constexpr int kCPL = Geo::kChunks / kLPG;  // 16-byte chunks per lane per row
+    static_assert(kCPL >= 1 && (kCPL & (kCPL - 1)) == 0, "chunks per lane: a power of two");
+    const int grp = lane / kLPG, sub = lane % kLPG;
 
     float m[G], l[G], acc[G][Geo::kDimsPerLane];
     auto reset_state = [&]() {
@@ -326,36 +331,43 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, kCtasPerSm)
             const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes);
             const uint32_t vs_a = ks_a + Geo::kTileBytes;
 
-            // q.k: lane (t, hpair) covers half the dims of token t
-            float2 sacc[G];
+            // q.k: the 16 tokens form groups of kTPL, each served by kLPG = 2*kTPL lanes; lane
+            // `sub` of a group owns chunks sub, sub + kLPG, ... of the row, so one q load
+            // feeds kTPL tokens.  Groups start at different chunks (rotation by group), which
+            // keeps every 8-lane phase of the shared-memory loads conflict-free.
+            float2 sacc[G][kTPL];
 #pragma unroll
-            for (int g = 0; g < G; ++g) sacc[g] = make_float2(0.f, 0.f);
+            for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int i = 0; i < Geo::kHalf; ++i) {
-                const int c = hpair * Geo::kHalf + ((i + t) & (Geo::kHalf - 1));
-                const uint4 kr = lds128(ks_a + t * Geo::kRowBytes + c * 16);
-                float kf[Geo::kChunkElems];
-                if constexpr (FP8) {
+                for (int u = 0; u < kTPL; ++u) sacc[g][u] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int mi = 0; mi < kCPL; ++mi) {
+                const int mm = (mi + grp) & (kCPL - 1);
+                const int c = sub + kLPG * mm;
+                float kf[kTPL][Geo::kChunkElems];
+#pragma unroll
+                for (int u = 0; u < kTPL; ++u) {
+                    const uint4 kr = lds128(ks_a + (grp * kTPL + u) * Geo::kRowBytes + c * 16);
                     const uint32_t w4[4] = {kr.x, kr.y, kr.z, kr.w};
+                    if constexpr (FP8) {
 #pragma unroll
-                    for (int wi = 0; wi < 4; ++wi) {
+                        for (int wi = 0; wi < 4; ++wi) {
 #pragma unroll
-                        for (int hb = 0; hb < 2; ++hb) {
-                            uint32_t h2;
-                            const uint16_t pair = (uint16_t)(w4[wi] >> (16 * hb));
-                            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-                            __half2 hv = *reinterpret_cast<__half2 *>(&h2);
-                            float2 f = __half22float2(hv);
-                            kf[wi * 4 + hb * 2 + 0] = f.x;
-                            kf[wi * 4 + hb * 2 + 1] = f.y;
+                            for (int hb = 0; hb < 2; ++hb) {
+                                uint32_t h2;
+                                const uint16_t pair = (uint16_t)(w4[wi] >> (16 * hb));
+                                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+                                const float2 f = __half22float2(*reinterpret_cast<__half2 *>(&h2));
+                                kf[u][wi * 4 + hb * 2 + 0] = f.x;
+                                kf[u][wi * 4 + hb * 2 + 1] = f.y;
+                            }
                         }
-                    }
-                } else {
-                    const uint32_t w4[4] = {kr.x, kr.y, kr.z, kr.w};
+                    } else {
 #pragma unroll
-                    for (int wi = 0; wi < 4; ++wi) {
-                        kf[2 * wi] = bf16lo(w4[wi]);
-                        kf[2 * wi + 1] = bf16hi(w4[wi]);
+                        for (int wi = 0; wi < 4; ++wi) {
+                            kf[u][2 * wi] = bf16lo(w4[wi]);
+                            kf[u][2 * wi + 1] = bf16hi(w4[wi]);
+                        }
                     }
                 }
 #pragma unroll
@@ -363,30 +375,47 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, kCtasPerSm)
 #pragma unroll
                     for (int qd = 0; qd < Geo::kQuads; ++qd) {
                         const float4 qv = lds128f(qs_a + (((g * Geo::kQuads + qd) * Geo::kChunks + c) * 16));
-                        sacc[g] = __ffma2_rn(make_float2(kf[4 * qd + 0], kf[4 * qd + 1]),
-                                             make_float2(qv.x, qv.y), sacc[g]);
-                        sacc[g] = __ffma2_rn(make_float2(kf[4 * qd + 2], kf[4 * qd + 3]),
-                                             make_float2(qv.z, qv.w), sacc[g]);
+#pragma unroll
+                        for (int u = 0; u < kTPL; ++u) {
+                            sacc[g][u] = __ffma2_rn(make_float2(kf[u][4 * qd + 0], kf[u][4 * qd + 1]),
+                                                    make_float2(qv.x, qv.y), sacc[g][u]);
+                            sacc[g][u] = __ffma2_rn(make_float2(kf[u][4 * qd + 2], kf[u][4 * qd + 3]),
+                                                    make_float2(qv.z, qv.w), sacc[g][u]);
+                        }
                     }
                 }
             }
-            // softmax update for this block (all 32 lanes hold the scores of token t)
+            // softmax update for this block: after the group reduction every lane of a group
+            // holds its kTPL tokens' scores
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float sc = sacc[g].x + sacc[g].y;
-                sc += __shfl_xor_sync(0xffffffffu, sc, 16);
-                if (t >= valid) sc = -INFINITY;
-                float mt = sc;
+                float sc[kTPL];
+                float mt = -INFINITY;
 #pragma unroll
-                for (int o = 1; o < 16; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+                for (int u = 0; u < kTPL; ++u) {
+                    float v = sacc[g][u].x + sacc[g][u].y;
+#pragma unroll
+                    for (int o = 1; o < kLPG; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    sc[u] = (grp * kTPL + u < valid) ? v : -INFINITY;
+                    mt = fmaxf(mt, sc[u]);
+                }
+#pragma unroll
+                for (int o = kLPG; o < 32; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
                 const float mn = fmaxf(m[g], mt);
                 const float alpha = ex2(m[g] - mn);
-                const float pj = ex2(sc - mn);
-                l[g] = l[g] * alpha + (hpair == 0 ? pj : 0.f);
+                float ls = 0.f;
+#pragma unroll
+                for (int u = 0; u < kTPL; ++u) {
+                    const float pj = ex2(sc[u] - mn);
+                    if (sub == 0) {
+                        pbuf[cw * G * 16 + g * 16 + grp * kTPL + u] = pj;
+                        ls += pj;
+                    }
+                }
+                l[g] = l[g] * alpha + ls;
                 m[g] = mn;
 #pragma unroll
                 for (int d = 0; d < Geo::kDimsPerLane; ++d) acc[g][d] *= alpha;
-                if (hpair == 0) pbuf[cw * G * 16 + g * 16 + t] = pj;
             }
             __syncwarp();
             // p.v: lane owns dims [lane*DPL, (lane+1)*DPL)
