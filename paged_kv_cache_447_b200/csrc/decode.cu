@@ -32,11 +32,20 @@
 namespace pkv {
 namespace {
 
-// Consumer warps per CTA: 4 for bf16 MHA (memory-bound: more warps do not help), 8 when a
-// tile feeds several query heads or must be widened from E4M3 (more arithmetic per byte).
-__host__ __device__ constexpr int consumers_for(int G, bool fp8) { return (G > 1 || fp8) ? 8 : 4; }
+// Launch geometry per instantiation (measured on B200): several small CTAs per SM beat
+// one large one -- each CTA brings its own TMA producer, and the SM overlaps their rings.
+//   bf16 MHA:     4 consumer warps, 3 CTAs per SM, ~72 KB each (8-stage ring)
+//   bf16 grouped: 4 consumer warps, 3 CTAs per SM, ~60 KB each (q, merge scratch grow with G)
+//   E4M3:         4 consumer warps, 4 CTAs per SM, ~48 KB each (4 KB stages)
+struct DecodeCfg {
+    int consumers, ctas_per_sm, smem_budget;
+};
+__host__ __device__ constexpr DecodeCfg decode_cfg(int G, bool fp8) {
+    return fp8 ? DecodeCfg{4, 4, 48 * 1024}
+               : (G > 1 ? DecodeCfg{4, 3, 60 * 1024} : DecodeCfg{4, 3, 72 * 1024});
+}
 constexpr int kMaxThreads = 32 * (1 + 8);
-constexpr int kCtasPerSm = 2;
+constexpr int kMaxCtasPerSm = 4;  // sizes the workspace for any instantiation
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMergeBar = 1;
 
@@ -60,8 +69,10 @@ struct DecodeParams {
 
 template <int D, bool FP8, int G>
 struct Geometry {
-    static constexpr int kConsumers = consumers_for(G, FP8);
+    static constexpr DecodeCfg kCfg = decode_cfg(G, FP8);
+    static constexpr int kConsumers = kCfg.consumers;
     static constexpr int kThreads = 32 * (1 + kConsumers);
+    static constexpr int kCtasPerSm = kCfg.ctas_per_sm;
     static constexpr int kElem = FP8 ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
     static constexpr int kTileBytes = kBlockSize * kRowBytes;          // one K (or V) block
@@ -73,7 +84,7 @@ struct Geometry {
     // The stage count is a multiple of the consumer count, so that every fill of a given
     // stage is consumed by the same warp: a warp then never waits on a barrier more than
     // one phase ahead (a parity wait cannot tell phase n from phase n+2).
-    static constexpr int kStagesRaw = (100 * 1024 - kExtraBytes) / kStageBytes;
+    static constexpr int kStagesRaw = (kCfg.smem_budget - kExtraBytes) / kStageBytes;
     static constexpr int kStagesQ = (kStagesRaw / kConsumers) * kConsumers;
     static constexpr int kStages = kStagesQ < kConsumers ? kConsumers : (kStagesQ > 64 ? 64 : kStagesQ);
     static_assert(kStages % kConsumers == 0, "stage count must be a multiple of the consumers");
@@ -151,7 +162,7 @@ __device__ __forceinline__ UnitPos locate(const int *pfx, int B, int Hkv, long l
 }
 
 template <int D, bool FP8, int G>
-__global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8, G>::kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecodeParams p) {
     using Geo = Geometry<D, FP8, G>;
@@ -620,7 +631,8 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
     DecodeParams lp = prm;
-    lp.nctas = std::min(prm.nctas, occ * (prm.nctas / kCtasPerSm));
+    lp.nctas = std::min(prm.nctas / kMaxCtasPerSm * Geometry<D, FP8, G>::kCtasPerSm,
+                        occ * (prm.nctas / kMaxCtasPerSm));
     // K/V maps with exactly the boxes the kernel's producer issues
     using Geo = Geometry<D, FP8, G>;
     CUtensorMap tk, tv;
@@ -652,7 +664,7 @@ size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
 }  // namespace
 
-int decode_grid_ctas(int num_sms) { return num_sms * kCtasPerSm; }
+int decode_grid_ctas(int num_sms) { return num_sms * kMaxCtasPerSm; }
 
 size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
                               int num_sms) {
