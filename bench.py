@@ -70,7 +70,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -140,11 +140,21 @@ def timed_region(fn, steps, warmup, stream, dist=None, sampler_index=0, on_timed
 
 
 def max_over_ranks(x: float, dist) -> float:
+    """Largest value over the ranks (timing: the job ends when its slowest rank ends)."""
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ms_local: float, dist=None) -> tuple:
+    """Replicas: every rank processes `units_per_rank`; the job's time is the slowest
+    rank's.  Returns (units per second of the whole job, job milliseconds)."""
+    world = dist.get_world_size() if dist is not None else 1
+    ms = max_over_ranks(ms_local, dist)
+    return world * units_per_rank / (ms * 1e-3), ms
 
 
 def decode_kv_bytes(st: W.Step, hkv: int, d: int, esize: int) -> int:
@@ -335,7 +345,7 @@ def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=Tr
                               on_timed=r.ev_attn.clear)
     code = r.pkv.get_error()
     assert code == 0, f"device error flag set during the timed region: {code}"
-    ms = max_over_ranks(ms, dist)
+    _, ms = job_throughput(steps, ms, dist)
     world = dist.get_world_size() if dist is not None else 1
     step_ms = ms / steps
     attn_ms = r.attn_ms()
@@ -372,10 +382,10 @@ def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=Tr
 
 # ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_step_rate(name: str, budget_s: float = 15.0):
-    """Time the CPU oracle on a bounded sample of the workload: the sample is the first
-    n decode sequences (or prefill requests), grown until it takes ~budget_s/4."""
-    import numpy as np
+def oracle_sample(name: str, step_budget_s: float):
+    """A bounded sample of the workload for the CPU oracle: the first n decode sequences
+    (or prefill requests), n grown until one oracle pass takes about step_budget_s.
+    Returns a closure running one pass and a description."""
     import oracle
     wl, layers = build_workload(name)
     st = wl.steps[-1]
@@ -384,39 +394,55 @@ def oracle_step_rate(name: str, budget_s: float = 15.0):
     kc0, vc0 = W.bits(wl.k_cache), W.bits(wl.v_cache)
     tab = oracle.rope_table(wl.max_pos, wl.head_dim, wl.rope_base)
     B = st.decode_seqs
+    ks = None if not fp8 else wl.k_scale.numpy()
+    vs = None if not fp8 else wl.v_scale.numpy()
 
-    def run(seqs):
+    def make(seqs):
         sub = W.sub_step(st, seqs)
-        kc, vc = kc0.copy(), vc0.copy()
         pos = oracle.positions(sub.cu_seqlens.numpy(), sub.context_lens.numpy())
-        t0 = time.perf_counter()
-        oracle.kv_store(W.bits(sub.k), W.bits(sub.v), kc, vc, sub.slot_mapping.numpy(), 16,
-                        fp8=fp8, k_scale=None if not fp8 else wl.k_scale.numpy(),
-                        v_scale=None if not fp8 else wl.v_scale.numpy(), table=tab, pos=pos)
-        oracle.attention(W.bits(sub.q), kc, vc, sub.cu_seqlens.numpy(),
-                         sub.block_tables.numpy(), sub.context_lens.numpy(), wl.scale, 16,
-                         wl.n_kv_heads, fp8=fp8,
-                         k_scale=None if not fp8 else wl.k_scale.numpy(),
-                         v_scale=None if not fp8 else wl.v_scale.numpy(), table=tab)
-        return time.perf_counter() - t0, sub
 
-    order = list(range(st.num_seqs)) if B == 0 else list(range(B))
+        kc, vc = kc0.copy(), vc0.copy()  # the store rewrites the same slots every pass
+
+        def one_pass():
+            oracle.kv_store(W.bits(sub.k), W.bits(sub.v), kc, vc, sub.slot_mapping.numpy(), 16,
+                            fp8=fp8, k_scale=ks, v_scale=vs, table=tab, pos=pos)
+            oracle.attention(W.bits(sub.q), kc, vc, sub.cu_seqlens.numpy(),
+                             sub.block_tables.numpy(), sub.context_lens.numpy(), wl.scale, 16,
+                             wl.n_kv_heads, fp8=fp8, k_scale=ks, v_scale=vs, table=tab)
+        return sub, one_pass
+
+    order = list(range(B)) if B else list(range(st.num_seqs))
     n = 1
     while True:
-        dt, sub = run(order[:n])
-        if dt > budget_s / 4 or n >= len(order):
+        sub, one = make(order[:n])
+        t0 = time.perf_counter()
+        one()
+        dt = time.perf_counter() - t0
+        if dt >= step_budget_s / 2 or n >= len(order):
             break
-        n = min(len(order), max(n + 1, int(n * min(8.0, (budget_s / 4) / max(dt, 1e-3)))))
-    res = {"sample": f"{n} of {len(order)} sequences of one step (one layer)", "seconds": dt,
-           "cores": oracle.num_threads()}
+        n = min(len(order), max(n + 1, int(n * min(8.0, step_budget_s / max(dt, 1e-4)))))
     if B:
-        kv = decode_kv_bytes(sub, wl.n_kv_heads, wl.head_dim, esize)
-        res["value"] = kv / dt / 1e9
-        res["unit"] = "GB/s"
+        work, unit = decode_kv_bytes(sub, wl.n_kv_heads, wl.head_dim, esize) / 1e9, "GB/s"
     else:
-        res["value"] = prefill_flops(sub, wl.n_q_heads, wl.head_dim) / dt / 1e12
-        res["unit"] = "TFLOP/s"
-    return res
+        work, unit = prefill_flops(sub, wl.n_q_heads, wl.head_dim) / 1e12, "TFLOP/s"
+    desc = f"{n} of {len(order)} sequences of one step (one layer), kv_store + attention"
+    return one, work, unit, desc
+
+
+def oracle_step_rate(name: str, budget_s: float = 15.0, steps: int = 3, warmup: int = 1):
+    """Time the CPU oracle on a bounded sample of the workload (warm-up passes, then
+    `steps` timed passes; each pass sized to about budget_s / (steps + warmup))."""
+    import oracle
+    per = max(0.05, budget_s / max(1, steps + warmup))
+    one, work, unit, desc = oracle_sample(name, per)
+    for _ in range(warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one()
+    dt = (time.perf_counter() - t0) / steps
+    return {"value": work / dt, "unit": unit, "seconds": dt, "sample": desc,
+            "cores": oracle.num_threads()}
 
 
 # ----------------------------------------------------------------------------- main
@@ -445,7 +471,9 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        r = oracle_step_rate(args.workload, budget_s=min(60.0, 6.0 * args.steps))
+        # the whole --steps/--warmup run of the oracle stays within about two minutes
+        r = oracle_step_rate(args.workload, budget_s=120.0, steps=args.steps,
+                             warmup=args.warmup)
         line = {"impl": "reference", "metric": METRIC, "value": r["value"], "unit": r["unit"],
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": r["seconds"] * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -533,7 +561,7 @@ def main():
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         try:
-            cb = oracle_step_rate(args.workload, budget_s=15.0)
+            cb = oracle_step_rate(args.workload, budget_s=15.0, steps=3, warmup=1)
             line["cpu_baseline"] = {"value": cb["value"], "unit": cb["unit"], "cores": cb["cores"],
                                     "kind": "oracle", "sample": cb["sample"]}
         except Exception as e:
