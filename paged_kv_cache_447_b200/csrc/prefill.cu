@@ -555,6 +555,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && p.rope && row_valid && it.valid[wg]) {
             if (pos < 0 || pos >= p.max_pos) {
                 atomicOr(p.err, kErrBounds);
+            } else if (it.row0[0] == it.row0[1]) {
+                // Both tiles hold the same rows (two heads of a group): warpgroup wg rotates
+                // its half of the pairs of row r in both tiles, so each thread fetches half
+                // a table row, in one round.
+                constexpr int NP = D / 32;  // chunk pairs per warpgroup
+                const int lc0 = wg * NP;
+                const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope + (size_t)pos * D);
+                float4 cv[2 * NP], sv[2 * NP];
+#pragma unroll
+                for (int k = 0; k < 2 * NP; ++k) {
+                    cv[k] = __ldg(cs4 + lc0 * 2 + k);
+                    sv[k] = __ldg(cs4 + D / 8 + lc0 * 2 + k);
+                }
+                const uint32_t sw = (uint32_t)(r & 7);
+#pragma unroll
+                for (int tile = 0; tile < 2; ++tile) {
+                    const uint32_t qrow = sQ + tile * Geo::kQBytes + r * 128;
+#pragma unroll
+                    for (int k4 = 0; k4 < NP; ++k4) {
+                        const int lc = lc0 + k4, lc2 = lc + D / 16;
+                        const uint32_t a1 = qrow + (lc / 8) * Geo::kSlabBytes + (((lc % 8) ^ sw) << 4);
+                        const uint32_t a2 = qrow + (lc2 / 8) * Geo::kSlabBytes + (((lc2 % 8) ^ sw) << 4);
+                        const uint4 x1 = lds128(a1), x2 = lds128(a2);
+                        const uint32_t w1[4] = {x1.x, x1.y, x1.z, x1.w};
+                        const uint32_t w2[4] = {x2.x, x2.y, x2.z, x2.w};
+                        const float cc[8] = {cv[2 * k4].x, cv[2 * k4].y, cv[2 * k4].z, cv[2 * k4].w,
+                                             cv[2 * k4 + 1].x, cv[2 * k4 + 1].y, cv[2 * k4 + 1].z,
+                                             cv[2 * k4 + 1].w};
+                        const float ss[8] = {sv[2 * k4].x, sv[2 * k4].y, sv[2 * k4].z, sv[2 * k4].w,
+                                             sv[2 * k4 + 1].x, sv[2 * k4 + 1].y, sv[2 * k4 + 1].z,
+                                             sv[2 * k4 + 1].w};
+                        uint32_t o1[4], o2[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float a0 = bf16lo(w1[q]), a1v = bf16hi(w1[q]);
+                            const float b0 = bf16lo(w2[q]), b1v = bf16hi(w2[q]);
+                            const float c0 = cc[2 * q], c1 = cc[2 * q + 1], s0 = ss[2 * q], s1 = ss[2 * q + 1];
+                            o1[q] = pack_bf16x2(__fmaf_rn(a0, c0, -__fmul_rn(b0, s0)),
+                                                __fmaf_rn(a1v, c1, -__fmul_rn(b1v, s1)));
+                            o2[q] = pack_bf16x2(__fmaf_rn(b0, c0, __fmul_rn(a0, s0)),
+                                                __fmaf_rn(b1v, c1, __fmul_rn(a1v, s1)));
+                        }
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a1), "r"(o1[0]),
+                                     "r"(o1[1]), "r"(o1[2]), "r"(o1[3]) : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a2), "r"(o2[0]),
+                                     "r"(o2[1]), "r"(o2[2]), "r"(o2[3]) : "memory");
+                    }
+                }
             } else {
                 const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope + (size_t)pos * D);
                 const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
@@ -601,7 +649,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if constexpr (FP8) {
-            // the FP8 path multiplies in f16: convert this row of Q (swizzle untouched)
+            // the FP8 path multiplies in f16: convert this row of Q (swizzle untouched), after
+            // both warpgroups finished rotating (they may share rows)
+            named_bar(2, 256);
             if (ok) {
                 const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
 #pragma unroll 1
