@@ -16,10 +16,15 @@
 //    load per block for K and one for V into a ring of shared-memory stages (mbarrier
 //    full/empty pairs).  Warps 1-4 consume stages round robin.
 //  * A consumer warp handles all G = Hq/Hkv query heads of the kv head, so each K/V tile
-//    is read from shared memory once for the whole group.  q.k: two lanes per token (each
-//    half the head dim, chunk order rotated per token so shared-memory reads are
-//    conflict-free), packed fp32x2 FMAs.  p.v: each lane owns D/32 output dims.  Online
-//    softmax (running max m, sum l) per warp in exp2 space.
+//    is read from shared memory once for the whole group.  Online softmax (running max m,
+//    sum l) per warp in exp2 space.
+//      - one head per kv head, and E4M3 caches: CUDA cores.  q.k: two lanes per token
+//        (each half the head dim, chunk order rotated per token so shared-memory reads are
+//        conflict-free), packed fp32x2 FMAs.  p.v: each lane owns D/32 output dims.
+//      - grouped bf16 heads (G = 2, 4, 8): tensor cores, mma.sync m16n8k16.  S = Q K^T with
+//        the G heads as rows of A (q held in registers for the whole piece, K fragments by
+//        ldmatrix); P stays in registers and feeds O^T = V^T P^T as the B operand (V^T
+//        fragments by ldmatrix.trans), so O needs D/16 accumulator tiles and no shuffles.
 //  * At the end of a piece the four consumer warps merge (m, l, acc) through shared
 //    memory.  A piece that covers its whole sequence writes the normalised bf16 output;
 //    otherwise its partial goes to the workspace and a small combine kernel merges the
@@ -161,6 +166,55 @@ __device__ __forceinline__ UnitPos locate(const int *pfx, int B, int Hkv, long l
     return r;
 }
 
+// ---- grouped heads on the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate)
+// The G query heads of a kv head are the rows of the A operand (rows G..15 are zero), a
+// 16-token block is the N (q.k) or K (p.v) extent.  K and V tiles arrive 128-byte swizzled
+// (16-byte chunk index XOR row & 7), so the eight 16-byte rows one ldmatrix phase reads
+// fall in eight different bank groups.
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+// c += A * B for one 16x8 tile; A rows 8..15 are zero (a2a3 = a6a7 = 0), so c[2], c[3]
+// stay zero.
+__device__ __forceinline__ void mma_rows8(float (&c)[4], uint32_t a01, uint32_t a45, uint32_t b01,
+                                          uint32_t b23) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a01), "r"(0u), "r"(a45), "r"(0u), "r"(b01), "r"(b23));
+}
+
+// c += A * B for one 16x8 tile with a full 16x16 A fragment.
+__device__ __forceinline__ void mma_full(float (&c)[4], const uint32_t (&a)[4], uint32_t b01,
+                                         uint32_t b23) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b01), "r"(b23));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Offset of the 16-byte chunk c (0 .. D/8-1) of row t (0..15) in a swizzled tile: 64-column
+// slabs of 16 rows x 128 bytes, 2 KB apart.
+__device__ __forceinline__ uint32_t swz(int t, int c) {
+    return (uint32_t)((c >> 3) * 2048 + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+}
+
 template <int D, bool FP8, int G>
 __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8, G>::kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -169,6 +223,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     constexpr int NS = Geo::kStages;
     constexpr int kConsumers = Geo::kConsumers;
     constexpr int kThreads = Geo::kThreads;
+    constexpr bool kMma = !FP8 && G >= 2;  // grouped bf16 heads: tensor-core consumers
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;                                                  // NS x stage
@@ -243,8 +298,18 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                         const uint32_t fb = smem_u32(full + s);
                         const uint32_t dst = smem_u32(stages + s * Geo::kStageBytes);
                         mbar_arrive_expect_tx(fb, Geo::kStageBytes);
-                        tma_load_3d(dst, &tm_k, fb, 0, hh, ph * kBlockSize);
-                        tma_load_3d(dst + Geo::kTileBytes, &tm_v, fb, 0, hh, ph * kBlockSize);
+                        if constexpr (kMma) {
+                            // one swizzled box per 64-column slab
+#pragma unroll
+                            for (int h = 0; h < D / 64; ++h) {
+                                tma_load_3d(dst + h * 2048, &tm_k, fb, 64 * h, hh, ph * kBlockSize);
+                                tma_load_3d(dst + Geo::kTileBytes + h * 2048, &tm_v, fb, 64 * h, hh,
+                                            ph * kBlockSize);
+                            }
+                        } else {
+                            tma_load_3d(dst, &tm_k, fb, 0, hh, ph * kBlockSize);
+                            tma_load_3d(dst + Geo::kTileBytes, &tm_v, fb, 0, hh, ph * kBlockSize);
+                        }
                         issued_mask |= 1ull << s;
                         issued_phase = (issued_phase & ~(1ull << s)) | ((uint64_t)((kk / NS) & 1) << s);
                     }
@@ -272,13 +337,30 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     const int grp = lane / kLPG, sub = lane % kLPG;
 
     float m[G], l[G], acc[G][Geo::kDimsPerLane];
+    // tensor-core path: lane = 4 * row + q4.  The lane's S fragment holds head `row` (valid
+    // when row < G) against tokens 2*q4, 2*q4+1, 8+2*q4, 9+2*q4 of the block; its O^T
+    // fragment of tile mt holds dims 16*mt+row and 16*mt+8+row of heads 2*q4 and 2*q4+1.
+    constexpr int kMT = kMma ? D / 16 : 1;
+    const int row = lane >> 2, q4 = lane & 3;
+    float mr = -INFINITY, lr = 0.f;
+    float o[kMT][4];
+    uint32_t qa[kMT][2];
     auto reset_state = [&]() {
+        if constexpr (kMma) {
+            mr = -INFINITY;
+            lr = 0.f;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            m[g] = -INFINITY;
-            l[g] = 0.f;
+            for (int mt = 0; mt < kMT; ++mt)
 #pragma unroll
-            for (int d = 0; d < Geo::kDimsPerLane; ++d) acc[g][d] = 0.f;
+                for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
+        } else {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                m[g] = -INFINITY;
+                l[g] = 0.f;
+#pragma unroll
+                for (int d = 0; d < Geo::kDimsPerLane; ++d) acc[g][d] = 0.f;
+            }
         }
     };
     reset_state();
@@ -311,6 +393,13 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                     atomicOr(p.err, kErrBounds);
                 }
             }
+            if constexpr (kMma) {
+                // rotated bf16 q, [G][D]; the scale is applied to the fp32 scores
+                uint16_t *qh = reinterpret_cast<uint16_t *>(qs);
+                qh[g * D + i] = x1;
+                qh[g * D + i + D / 2] = x2;
+                continue;
+            }
             const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
             const int idx[2] = {i, i + D / 2};
             const float val[2] = {__uint_as_float((uint32_t)x1 << 16) * sc,
@@ -324,6 +413,15 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             }
         }
         named_bar(kMergeBar, kConsumers * 32);
+        if constexpr (kMma) {
+            // A fragments of Q for every 16-dim k step (zero for rows past the group)
+#pragma unroll
+            for (int ks = 0; ks < kMT; ++ks) {
+                const uint32_t a = qs_a + (uint32_t)((row * D + 16 * ks + 2 * q4) * 2);
+                qa[ks][0] = row < G ? lds32(a) : 0u;
+                qa[ks][1] = row < G ? lds32(a + 16) : 0u;
+            }
+        }
 
         // ---- stream this piece's blocks
         for (int j = 0; j < piece_len; ++j, ++k) {
@@ -341,6 +439,70 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             const int valid = min(kBlockSize, L - blk * kBlockSize);
             const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes);
             const uint32_t vs_a = ks_a + Geo::kTileBytes;
+            if constexpr (kMma) {
+                // S = Q K^T: n tile 0 = tokens 0-7, n tile 1 = tokens 8-15.  ldmatrix x4
+                // matrices: (tokens 0-7 | 8-15) x (first | second 8 dims of the k step).
+                float sa[2][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) sa[0][i] = sa[1][i] = 0.f;
+                const int tk = ((lane >> 4) << 3) | (lane & 7), hk = (lane >> 3) & 1;
+#pragma unroll
+                for (int ks = 0; ks < kMT; ++ks) {
+                    uint32_t b[4];
+                    ldsm_x4(ks_a + swz(tk, 2 * ks + hk), b);
+                    mma_rows8(sa[0], qa[ks][0], qa[ks][1], b[0], b[1]);
+                    mma_rows8(sa[1], qa[ks][0], qa[ks][1], b[2], b[3]);
+                }
+                // online softmax of row `row` over this block (the quad holds its 16 tokens)
+                const float sc = p.scale_log2;
+                const int t0 = 2 * q4;
+                float sv[4] = {sa[0][0] * sc, sa[0][1] * sc, sa[1][0] * sc, sa[1][1] * sc};
+                if (valid < kBlockSize) {
+                    if (t0 >= valid) sv[0] = -INFINITY;
+                    if (t0 + 1 >= valid) sv[1] = -INFINITY;
+                    if (t0 + 8 >= valid) sv[2] = -INFINITY;
+                    if (t0 + 9 >= valid) sv[3] = -INFINITY;
+                    // V rows past the sequence are zeroed (0 * NaN would poison O)
+                    for (int e = lane; e < (kBlockSize - valid) * (D / 8); e += 32) {
+                        const int t = valid + e / (D / 8), c = e % (D / 8);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vs_a + swz(t, c)),
+                                     "r"(0u) : "memory");
+                    }
+                    fence_proxy_async_smem();  // before the stage is refilled by TMA
+                    __syncwarp();
+                }
+                float mt = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+                const float mn = fmaxf(mr, mt);  // finite: token 0 of a block is always valid
+                const float alpha = ex2(mr - mn);
+                float pr[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) pr[i] = ex2(sv[i] - mn);
+                lr = lr * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+                mr = mn;
+                // O^T columns are heads 2*q4 and 2*q4+1, whose alphas live in lanes 8*q4, 8*q4+4
+                const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * q4);
+                const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * q4 + 4);
+                const uint32_t pb01 = pack_bf16x2(pr[0], pr[1]), pb23 = pack_bf16x2(pr[2], pr[3]);
+                // O^T += V^T P^T: ldmatrix.trans matrices (tokens 0-7 | 8-15) x (dims 16mt..+7 |
+                // 16mt+8..+15) give the A fragment; P^T is the S fragment just computed.
+                const int tv = ((lane >> 4) << 3) | (lane & 7), hv = (lane >> 3) & 1;
+#pragma unroll
+                for (int mt2 = 0; mt2 < kMT; ++mt2) {
+                    o[mt2][0] *= al0;
+                    o[mt2][1] *= al1;
+                    o[mt2][2] *= al0;
+                    o[mt2][3] *= al1;
+                    uint32_t a[4];
+                    ldsm_x4_trans(vs_a + swz(tv, 2 * mt2 + hv), a);
+                    const uint32_t af[4] = {a[0], a[1], a[2], a[3]};
+                    mma_full(o[mt2], af, pb01, pb23);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(empty + s));
+                continue;
+            }
 
             // q.k: the 16 tokens form groups of kTPL, each served by kLPG = 2*kTPL lanes; lane
             // `sub` of a group owns chunks sub, sub + kLPG, ... of the row, so one q load
@@ -508,8 +670,30 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
         }
 
         // ---- merge the four consumer warps' states for this piece
+        if constexpr (kMma) {
+            float lw = lr;
+            lw += __shfl_xor_sync(0xffffffffu, lw, 1);
+            lw += __shfl_xor_sync(0xffffffffu, lw, 2);
+            if (row < G && q4 == 0) {
+                float *mw = mrg + (cw * G + row) * (D + 2);
+                mw[D] = mr;
+                mw[D + 1] = lw;
+            }
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
+            for (int hh = 0; hh < 2; ++hh) {
+                const int g = 2 * q4 + hh;
+                if (g < G) {
+                    float *mw = mrg + (cw * G + g) * (D + 2);
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        mw[16 * mt + row] = o[mt][hh];
+                        mw[16 * mt + 8 + row] = o[mt][2 + hh];
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G && !kMma; ++g) {
             float lw = l[g];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
@@ -637,9 +821,12 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
     using Geo = Geometry<D, FP8, G>;
     CUtensorMap tk, tv;
     const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
-    // one box per tile: a whole 16-token block of one kv head (16 rows of D elements)
-    if (!encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, D, 1, kBlockSize, false) ||
-        !encode_tensor_map_3d(&tv, a.v_cache, Geo::kElem, D, a.n_kv_heads, slots, D, 1, kBlockSize, false))
+    // CUDA-core consumers: one box per tile, a whole 16-token block of one kv head (16 rows of
+    // D elements).  Tensor-core consumers: one 128-byte-swizzled box per 64-column slab.
+    constexpr bool kMma = !FP8 && G >= 2;
+    const uint32_t box0 = kMma ? 64u : (uint32_t)D;
+    if (!encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma) ||
+        !encode_tensor_map_3d(&tv, a.v_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma))
         return cudaErrorUnknown;  // (cudaErrorInvalidValue means a short workspace)
     static_assert(kBlockSize * D * Geo::kElem == Geo::kTileBytes, "one TMA box fills one tile");
     e = launch_pdl(kern, dim3(lp.nctas), dim3(kThreads), smem, s, tk, tv, lp);

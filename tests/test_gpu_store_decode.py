@@ -201,6 +201,41 @@ def test_decode_unused_slots_hold_nan():
     compare(out, ref, what="nan sentinels")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("group", [2, 4, 8])
+def test_decode_grouped_nan_sentinels(group, d):
+    """Grouped heads: NaN in every K and V slot no sequence owns (the tails of last blocks
+    included) never reaches the output, whatever the group size and head dim."""
+    g = torch.Generator().manual_seed(300 + group + d)
+    lens = [1, 15, 17, 250, 16 * 5, 1000]
+    hkv = 2
+    hq = hkv * group
+    counts = [W.blocks_needed(L) for L in lens]
+    nb = sum(counts) + 4
+    perm = torch.randperm(nb, generator=g)
+    bt = W._assign_blocks(perm, counts, max_blocks=max(counts))
+    kc, vc = W._fill_cache(g, nb, hkv, d, False)
+    owned = torch.zeros(nb * 16, dtype=torch.bool)
+    for b, L in enumerate(lens):
+        for j in range(L):
+            owned[int(bt[b, j // 16]) * 16 + j % 16] = True
+    kc.view(nb * 16, hkv, d)[~owned] = float("nan")
+    vc.view(nb * 16, hkv, d)[~owned] = float("nan")
+    B = len(lens)
+    st = W.Step("nan-grouped", W._randn_bf16(g, B, hq, d), W._randn_bf16(g, B, hkv, d),
+                W._randn_bf16(g, B, hkv, d), torch.full((B,), -1, dtype=torch.int32),
+                torch.arange(B + 1, dtype=torch.int32), torch.tensor(lens, dtype=torch.int32),
+                bt, B)
+    wl = W.Workload("nan-grouped", 0, hq, hkv, d, nb, "bf16", kc, vc, [st], max_pos=max(lens) + 1)
+    dw = DeviceWorkload(wl)
+    out = dw.decode(st, rope=False)
+    torch.cuda.synchronize()
+    _assert_no_device_error()
+    assert torch.isfinite(out.float()).all()
+    ref = oracle_attention(wl, st, W.bits(kc), W.bits(vc), rope=False)
+    compare(out, ref, what=f"nan sentinels G={group} D={d}")
+
+
 def test_decode_block_id_out_of_range_is_flagged():
     wl = W.tiny(seed=1)
     st = wl.steps[1]
