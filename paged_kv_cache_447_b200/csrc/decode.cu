@@ -41,12 +41,14 @@ namespace {
 // one large one -- each CTA brings its own TMA producer, and the SM overlaps their rings.
 //   bf16 MHA:     4 consumer warps, 3 CTAs per SM, ~72 KB each (8-stage ring)
 //   bf16 grouped: 4 consumer warps, 3 CTAs per SM, ~60 KB each (q, merge scratch grow with G)
-//   E4M3:         4 consumer warps, 4 CTAs per SM, ~48 KB each (4 KB stages)
+//   E4M3 MHA:     4 consumer warps, 4 CTAs per SM, ~48 KB each (4 KB stages)
+//   E4M3 grouped: 4 consumer warps, 3 CTAs per SM, ~64 KB each (tensor-core consumers need
+//                 the registers of 3 CTAs per SM)
 struct DecodeCfg {
     int consumers, ctas_per_sm, smem_budget;
 };
 __host__ __device__ constexpr DecodeCfg decode_cfg(int G, bool fp8) {
-    return fp8 ? DecodeCfg{4, 4, 48 * 1024}
+    return fp8 ? (G > 1 ? DecodeCfg{4, 3, 64 * 1024} : DecodeCfg{4, 4, 48 * 1024})
                : (G > 1 ? DecodeCfg{4, 3, 60 * 1024} : DecodeCfg{4, 3, 72 * 1024});
 }
 constexpr int kMaxThreads = 32 * (1 + 8);
@@ -203,14 +205,52 @@ __device__ __forceinline__ void mma_full(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b01), "r"(b23));
 }
 
+// The same two tiles in f16 (E4M3 caches: K/V widened exactly to f16, q and P rounded).
+__device__ __forceinline__ void mma_rows8_f16(float (&c)[4], uint32_t a01, uint32_t a45,
+                                              uint32_t b01, uint32_t b23) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a01), "r"(0u), "r"(a45), "r"(0u), "r"(b01), "r"(b23));
+}
+
+__device__ __forceinline__ void mma_full_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b01,
+                                             uint32_t b23) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b01), "r"(b23));
+}
+
+// Two E4M3 codes (bits 0-7 and 8-15 of `two`) -> f16x2, low code in the low half (exact).
+__device__ __forceinline__ uint32_t e4m3x2_f16x2(uint32_t two) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)two));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
-// Offset of the 16-byte chunk c (0 .. D/8-1) of row t (0..15) in a swizzled tile: 64-column
-// slabs of 16 rows x 128 bytes, 2 KB apart.
+// Offset of the 16-byte chunk c of row t (0..15) in a swizzled tile: slabs of 16 rows x
+// 128 bytes (64 bf16 columns, or a whole 128-byte E4M3 row), 2 KB apart.
 __device__ __forceinline__ uint32_t swz(int t, int c) {
     return (uint32_t)((c >> 3) * 2048 + t * 128 + (((c & 7) ^ (t & 7)) << 4));
 }
@@ -223,7 +263,9 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     constexpr int NS = Geo::kStages;
     constexpr int kConsumers = Geo::kConsumers;
     constexpr int kThreads = Geo::kThreads;
-    constexpr bool kMma = !FP8 && G >= 2;  // grouped bf16 heads: tensor-core consumers
+    // grouped heads on the tensor cores: bf16 caches, and E4M3 caches at head dim 128
+    constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
+    constexpr int kSlabs = Geo::kRowBytes / 128;  // swizzled boxes per tile (kMma)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;                                                  // NS x stage
@@ -301,9 +343,10 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                         if constexpr (kMma) {
                             // one swizzled box per 64-column slab
 #pragma unroll
-                            for (int h = 0; h < D / 64; ++h) {
-                                tma_load_3d(dst + h * 2048, &tm_k, fb, 64 * h, hh, ph * kBlockSize);
-                                tma_load_3d(dst + Geo::kTileBytes + h * 2048, &tm_v, fb, 64 * h, hh,
+                            for (int h = 0; h < kSlabs; ++h) {
+                                const int x = h * (128 / Geo::kElem);
+                                tma_load_3d(dst + h * 2048, &tm_k, fb, x, hh, ph * kBlockSize);
+                                tma_load_3d(dst + Geo::kTileBytes + h * 2048, &tm_v, fb, x, hh,
                                             ph * kBlockSize);
                             }
                         } else {
@@ -339,7 +382,11 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     float m[G], l[G], acc[G][Geo::kDimsPerLane];
     // tensor-core path: lane = 4 * row + q4.  The lane's S fragment holds head `row` (valid
     // when row < G) against tokens 2*q4, 2*q4+1, 8+2*q4, 9+2*q4 of the block; its O^T
-    // fragment of tile mt holds dims 16*mt+row and 16*mt+8+row of heads 2*q4 and 2*q4+1.
+    // fragment of tile mt holds, for heads 2*q4 and 2*q4+1, dims odim(mt, row) and
+    // odim(mt, row + 8):  bf16: 16*mt + r;  E4M3: 16*row + 8*(r >= 8) + mt, so that a lane's
+    // V bytes are one contiguous 16-byte chunk of each token row.  (Any permutation of the
+    // contracted dims, applied to q and K alike, and of the output dims, undone at the merge,
+    // leaves the result unchanged.)
     constexpr int kMT = kMma ? D / 16 : 1;
     const int row = lane >> 2, q4 = lane & 3;
     float mr = -INFINITY, lr = 0.f;
@@ -417,9 +464,18 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             // A fragments of Q for every 16-dim k step (zero for rows past the group)
 #pragma unroll
             for (int ks = 0; ks < kMT; ++ks) {
-                const uint32_t a = qs_a + (uint32_t)((row * D + 16 * ks + 2 * q4) * 2);
-                qa[ks][0] = row < G ? lds32(a) : 0u;
-                qa[ks][1] = row < G ? lds32(a + 16) : 0u;
+                if constexpr (FP8) {
+                    // k step ks, quad lane q4: dims 32*q4 + 4*ks + {0,1 | 2,3}, in f16
+                    const uint32_t a = qs_a + (uint32_t)((row * D + 32 * q4 + 4 * ks) * 2);
+                    const uint2 w = row < G ? lds64(a) : make_uint2(0u, 0u);
+                    qa[ks][0] = pack_f16x2(bf16lo(w.x), bf16hi(w.x));
+                    qa[ks][1] = pack_f16x2(bf16lo(w.y), bf16hi(w.y));
+                } else {
+                    // k step ks, quad lane q4: dims 16*ks + 2*q4 + {0,1 | 8,9}
+                    const uint32_t a = qs_a + (uint32_t)((row * D + 16 * ks + 2 * q4) * 2);
+                    qa[ks][0] = row < G ? lds32(a) : 0u;
+                    qa[ks][1] = row < G ? lds32(a + 16) : 0u;
+                }
             }
         }
 
@@ -445,16 +501,32 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                 float sa[2][4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) sa[0][i] = sa[1][i] = 0.f;
-                const int tk = ((lane >> 4) << 3) | (lane & 7), hk = (lane >> 3) & 1;
+                if constexpr (FP8) {
+                    // B fragment of n tile nt: token 8*nt + row, bytes [32*q4, 32*q4 + 32) of
+                    // its row (two swizzled chunks), widened to f16 per k step
 #pragma unroll
-                for (int ks = 0; ks < kMT; ++ks) {
-                    uint32_t b[4];
-                    ldsm_x4(ks_a + swz(tk, 2 * ks + hk), b);
-                    mma_rows8(sa[0], qa[ks][0], qa[ks][1], b[0], b[1]);
-                    mma_rows8(sa[1], qa[ks][0], qa[ks][1], b[2], b[3]);
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int t = 8 * nt + row;
+                        const uint4 k0 = lds128(ks_a + swz(t, 2 * q4));
+                        const uint4 k1 = lds128(ks_a + swz(t, 2 * q4 + 1));
+                        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+                        for (int ks = 0; ks < kMT; ++ks)
+                            mma_rows8_f16(sa[nt], qa[ks][0], qa[ks][1], e4m3x2_f16x2(kw[ks]),
+                                          e4m3x2_f16x2(kw[ks] >> 16));
+                    }
+                } else {
+                    const int tk = ((lane >> 4) << 3) | (lane & 7), hk = (lane >> 3) & 1;
+#pragma unroll
+                    for (int ks = 0; ks < kMT; ++ks) {
+                        uint32_t b[4];
+                        ldsm_x4(ks_a + swz(tk, 2 * ks + hk), b);
+                        mma_rows8(sa[0], qa[ks][0], qa[ks][1], b[0], b[1]);
+                        mma_rows8(sa[1], qa[ks][0], qa[ks][1], b[2], b[3]);
+                    }
                 }
                 // online softmax of row `row` over this block (the quad holds its 16 tokens)
-                const float sc = p.scale_log2;
+                const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
                 const int t0 = 2 * q4;
                 float sv[4] = {sa[0][0] * sc, sa[0][1] * sc, sa[1][0] * sc, sa[1][1] * sc};
                 if (valid < kBlockSize) {
@@ -463,8 +535,9 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                     if (t0 + 8 >= valid) sv[2] = -INFINITY;
                     if (t0 + 9 >= valid) sv[3] = -INFINITY;
                     // V rows past the sequence are zeroed (0 * NaN would poison O)
-                    for (int e = lane; e < (kBlockSize - valid) * (D / 8); e += 32) {
-                        const int t = valid + e / (D / 8), c = e % (D / 8);
+                    constexpr int kRowChunks = Geo::kRowBytes / 16;
+                    for (int e = lane; e < (kBlockSize - valid) * kRowChunks; e += 32) {
+                        const int t = valid + e / kRowChunks, c = e % kRowChunks;
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vs_a + swz(t, c)),
                                      "r"(0u) : "memory");
                     }
@@ -484,20 +557,50 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                 // O^T columns are heads 2*q4 and 2*q4+1, whose alphas live in lanes 8*q4, 8*q4+4
                 const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * q4);
                 const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * q4 + 4);
-                const uint32_t pb01 = pack_bf16x2(pr[0], pr[1]), pb23 = pack_bf16x2(pr[2], pr[3]);
-                // O^T += V^T P^T: ldmatrix.trans matrices (tokens 0-7 | 8-15) x (dims 16mt..+7 |
-                // 16mt+8..+15) give the A fragment; P^T is the S fragment just computed.
-                const int tv = ((lane >> 4) << 3) | (lane & 7), hv = (lane >> 3) & 1;
 #pragma unroll
                 for (int mt2 = 0; mt2 < kMT; ++mt2) {
                     o[mt2][0] *= al0;
                     o[mt2][1] *= al1;
                     o[mt2][2] *= al0;
                     o[mt2][3] *= al1;
-                    uint32_t a[4];
-                    ldsm_x4_trans(vs_a + swz(tv, 2 * mt2 + hv), a);
-                    const uint32_t af[4] = {a[0], a[1], a[2], a[3]};
-                    mma_full(o[mt2], af, pb01, pb23);
+                }
+                if constexpr (FP8) {
+                    // O^T += V^T P^T in f16.  The A fragment of tile mt needs, at dims
+                    // 16*row + mt and 16*row + 8 + mt, tokens 2q4, 2q4+1 (a0a1, a2a3) and
+                    // 8+2q4, 9+2q4 (a4a5, a6a7): one 16-byte chunk of each of the four token
+                    // rows, regrouped into token pairs by byte permutes, then widened.
+                    const uint32_t pb01 = pack_f16x2(pr[0], pr[1]), pb23 = pack_f16x2(pr[2], pr[3]);
+                    const int tA = 2 * q4;
+                    const uint4 vA = lds128(vs_a + swz(tA, row)), vB = lds128(vs_a + swz(tA + 1, row));
+                    const uint4 vC = lds128(vs_a + swz(tA + 8, row)), vD = lds128(vs_a + swz(tA + 9, row));
+                    const uint32_t wA[4] = {vA.x, vA.y, vA.z, vA.w}, wB[4] = {vB.x, vB.y, vB.z, vB.w};
+                    const uint32_t wC[4] = {vC.x, vC.y, vC.z, vC.w}, wD[4] = {vD.x, vD.y, vD.z, vD.w};
+#pragma unroll
+                    for (int mp = 0; mp < 4; ++mp) {  // m tiles 2mp, 2mp+1 = bytes 2mp, 2mp+1
+                        const uint32_t sel = (mp & 1) ? 0x7362u : 0x5140u;  // [x_b, y_b, x_b+1, y_b+1]
+                        const uint32_t lo01 = prmt(wA[mp >> 1], wB[mp >> 1], sel);
+                        const uint32_t hi01 = prmt(wA[2 + (mp >> 1)], wB[2 + (mp >> 1)], sel);
+                        const uint32_t lo23 = prmt(wC[mp >> 1], wD[mp >> 1], sel);
+                        const uint32_t hi23 = prmt(wC[2 + (mp >> 1)], wD[2 + (mp >> 1)], sel);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const uint32_t af[4] = {e4m3x2_f16x2(lo01 >> (16 * e)), e4m3x2_f16x2(hi01 >> (16 * e)),
+                                                    e4m3x2_f16x2(lo23 >> (16 * e)), e4m3x2_f16x2(hi23 >> (16 * e))};
+                            mma_full_f16(o[2 * mp + e], af, pb01, pb23);
+                        }
+                    }
+                } else {
+                    const uint32_t pb01 = pack_bf16x2(pr[0], pr[1]), pb23 = pack_bf16x2(pr[2], pr[3]);
+                    // O^T += V^T P^T: ldmatrix.trans matrices (tokens 0-7 | 8-15) x (dims
+                    // 16mt..+7 | 16mt+8..+15) give the A fragment; P^T is the S fragment.
+                    const int tv = ((lane >> 4) << 3) | (lane & 7), hv = (lane >> 3) & 1;
+#pragma unroll
+                    for (int mt2 = 0; mt2 < kMT; ++mt2) {
+                        uint32_t a[4];
+                        ldsm_x4_trans(vs_a + swz(tv, 2 * mt2 + hv), a);
+                        const uint32_t af[4] = {a[0], a[1], a[2], a[3]};
+                        mma_full(o[mt2], af, pb01, pb23);
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(empty + s));
@@ -686,8 +789,9 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                     float *mw = mrg + (cw * G + g) * (D + 2);
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt) {
-                        mw[16 * mt + row] = o[mt][hh];
-                        mw[16 * mt + 8 + row] = o[mt][2 + hh];
+                        const int d0 = FP8 ? 16 * row + mt : 16 * mt + row;
+                        mw[d0] = o[mt][hh];
+                        mw[d0 + 8] = o[mt][2 + hh];
                     }
                 }
             }
@@ -823,8 +927,8 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
     const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
     // CUDA-core consumers: one box per tile, a whole 16-token block of one kv head (16 rows of
     // D elements).  Tensor-core consumers: one 128-byte-swizzled box per 64-column slab.
-    constexpr bool kMma = !FP8 && G >= 2;
-    const uint32_t box0 = kMma ? 64u : (uint32_t)D;
+    constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
+    const uint32_t box0 = kMma ? 128u / Geo::kElem : (uint32_t)D;
     if (!encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma) ||
         !encode_tensor_map_3d(&tv, a.v_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma))
         return cudaErrorUnknown;  // (cudaErrorInvalidValue means a short workspace)

@@ -201,39 +201,64 @@ def test_decode_unused_slots_hold_nan():
     compare(out, ref, what="nan sentinels")
 
 
-@pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("group", [2, 4, 8])
-def test_decode_grouped_nan_sentinels(group, d):
-    """Grouped heads: NaN in every K and V slot no sequence owns (the tails of last blocks
-    included) never reaches the output, whatever the group size and head dim."""
-    g = torch.Generator().manual_seed(300 + group + d)
-    lens = [1, 15, 17, 250, 16 * 5, 1000]
-    hkv = 2
+def _grouped_case(seed, lens, group, d, fp8, hkv=2, nan_unowned=False):
+    """A decode step over a random cache with ragged lengths; optionally every K and V slot
+    no sequence owns (the tails of last blocks included) holds NaN (E4M3: code 0x7F)."""
+    g = torch.Generator().manual_seed(seed)
     hq = hkv * group
     counts = [W.blocks_needed(L) for L in lens]
     nb = sum(counts) + 4
     perm = torch.randperm(nb, generator=g)
-    bt = W._assign_blocks(perm, counts, max_blocks=max(counts))
-    kc, vc = W._fill_cache(g, nb, hkv, d, False)
-    owned = torch.zeros(nb * 16, dtype=torch.bool)
-    for b, L in enumerate(lens):
-        for j in range(L):
-            owned[int(bt[b, j // 16]) * 16 + j % 16] = True
-    kc.view(nb * 16, hkv, d)[~owned] = float("nan")
-    vc.view(nb * 16, hkv, d)[~owned] = float("nan")
+    bt = W._assign_blocks(perm, counts, max_blocks=max(max(counts), 1) + 1)
+    ks = vs = None
+    if fp8:
+        ks = (0.5 + torch.rand(hkv, generator=g)) / 100.0
+        vs = (0.5 + torch.rand(hkv, generator=g)) / 100.0
+    kc, vc = W._fill_cache(g, nb, hkv, d, fp8, ks, vs)
+    if nan_unowned:
+        owned = torch.zeros(nb * 16, dtype=torch.bool)
+        for b, L in enumerate(lens):
+            for j in range(L):
+                owned[int(bt[b, j // 16]) * 16 + j % 16] = True
+        fill = 0x7F if fp8 else float("nan")
+        kc.view(nb * 16, hkv, d)[~owned] = fill
+        vc.view(nb * 16, hkv, d)[~owned] = fill
     B = len(lens)
-    st = W.Step("nan-grouped", W._randn_bf16(g, B, hq, d), W._randn_bf16(g, B, hkv, d),
+    st = W.Step("grouped", W._randn_bf16(g, B, hq, d), W._randn_bf16(g, B, hkv, d),
                 W._randn_bf16(g, B, hkv, d), torch.full((B,), -1, dtype=torch.int32),
                 torch.arange(B + 1, dtype=torch.int32), torch.tensor(lens, dtype=torch.int32),
                 bt, B)
-    wl = W.Workload("nan-grouped", 0, hq, hkv, d, nb, "bf16", kc, vc, [st], max_pos=max(lens) + 1)
+    wl = W.Workload("grouped", seed, hq, hkv, d, nb, "fp8" if fp8 else "bf16", kc, vc, [st],
+                    max_pos=max(lens) + 1, k_scale=ks, v_scale=vs)
     dw = DeviceWorkload(wl)
     out = dw.decode(st, rope=False)
     torch.cuda.synchronize()
     _assert_no_device_error()
-    assert torch.isfinite(out.float()).all()
     ref = oracle_attention(wl, st, W.bits(kc), W.bits(vc), rope=False)
-    compare(out, ref, what=f"nan sentinels G={group} D={d}")
+    return out, ref
+
+
+@pytest.mark.parametrize("d,fp8", [(64, False), (128, False), (64, True), (128, True)])
+@pytest.mark.parametrize("group", [2, 4, 8])
+def test_decode_grouped_nan_sentinels(group, d, fp8):
+    """Grouped heads: NaN in every K and V slot no sequence owns (the tails of last blocks
+    included) never reaches the output, whatever the group size, head dim and cache type."""
+    out, ref = _grouped_case(300 + group + d, [1, 15, 17, 250, 16 * 5, 1000], group, d, fp8,
+                             nan_unowned=True)
+    assert torch.isfinite(out.float()).all()
+    compare(out, ref, fp8=fp8, what=f"nan sentinels G={group} D={d} fp8={fp8}")
+
+
+@pytest.mark.parametrize("lens", [[1, 16, 17, 0, 33], [5000, 1, 2, 3], [16 * 7] * 9])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+def test_decode_fp8_edge_lengths_and_groups(lens, group):
+    """E4M3 caches with per-head scales: empty, single-token, block-multiple and ragged
+    contexts for every compiled group size (head dim 128)."""
+    out, ref = _grouped_case(500 + group, lens, group, 128, True)
+    compare(out, ref, fp8=True, what=f"fp8 edge {lens} G={group}")
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert torch.all(out[b] == 0)
 
 
 def test_decode_block_id_out_of_range_is_flagged():
