@@ -91,11 +91,17 @@ bool encode_tensor_map_3d(CUtensorMap *map, const void *base, int esize, uint64_
     const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
     const cuuint32_t box[3] = {b0, b1, b2};
     const cuuint32_t estr[3] = {1, 1, 1};
+    // L2 fetch granularity no larger than one contiguous row: a wider promotion would drag in
+    // the next head's row of the same slot, which the paged layout does not read next.
+    const uint64_t row = d0 * esize;
+    const CUtensorMapL2promotion promo = row >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                         : row >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                      : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
     CUresult r = g_encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                           3, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 

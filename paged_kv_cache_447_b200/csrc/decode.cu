@@ -54,6 +54,7 @@ __host__ __device__ constexpr DecodeCfg decode_cfg(int G, bool fp8) {
 constexpr int kMaxThreads = 32 * (1 + 8);
 constexpr int kMaxCtasPerSm = 4;  // sizes the workspace for any instantiation
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;  // tensor-core path: lazy max update threshold (log2)
 constexpr int kMergeBar = 1;
 
 struct DecodeParams {
@@ -547,22 +548,29 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                 float mt = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
                 mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-                const float mn = fmaxf(mr, mt);  // finite: token 0 of a block is always valid
-                const float alpha = ex2(mr - mn);
+                // Lazy rescale: the reference max mr moves only when the block's max exceeds
+                // it by more than 2^8 (mt is finite: token 0 of a block is always valid), so
+                // P <= 2^8 and O is rescaled only on the rare blocks that move it.
+                float alpha = 1.f;
+                if (mt > mr + kRescaleLog2) {
+                    alpha = ex2(mr - mt);  // 0 on the first block (mr = -inf; O, l are 0)
+                    mr = mt;
+                }
                 float pr[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) pr[i] = ex2(sv[i] - mn);
+                for (int i = 0; i < 4; ++i) pr[i] = ex2(sv[i] - mr);
                 lr = lr * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-                mr = mn;
-                // O^T columns are heads 2*q4 and 2*q4+1, whose alphas live in lanes 8*q4, 8*q4+4
-                const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * q4);
-                const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * q4 + 4);
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O^T columns are heads 2*q4, 2*q4+1: their alphas live in lanes 8*q4, 8*q4+4
+                    const float al0 = __shfl_sync(0xffffffffu, alpha, 8 * q4);
+                    const float al1 = __shfl_sync(0xffffffffu, alpha, 8 * q4 + 4);
 #pragma unroll
-                for (int mt2 = 0; mt2 < kMT; ++mt2) {
-                    o[mt2][0] *= al0;
-                    o[mt2][1] *= al1;
-                    o[mt2][2] *= al0;
-                    o[mt2][3] *= al1;
+                    for (int mt2 = 0; mt2 < kMT; ++mt2) {
+                        o[mt2][0] *= al0;
+                        o[mt2][1] *= al1;
+                        o[mt2][2] *= al0;
+                        o[mt2][3] *= al1;
+                    }
                 }
                 if constexpr (FP8) {
                     // O^T += V^T P^T in f16.  The A fragment of tile mt needs, at dims
