@@ -83,26 +83,36 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns, int *err) {
 
 }  // namespace
 
-// 3-D tiled map over a row-major [d2, d1, d0] tensor of `esize`-byte elements.
-bool encode_tensor_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
-               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128) {
+// 3-D tiled map with explicit byte strides for dims 1 and 2 (the dims need not be listed in
+// address order) and an L2 promotion of `promo_bytes` (64, 128 or 256).
+bool encode_tensor_map_3d_strided(CUtensorMap *map, const void *base, int esize, uint64_t d0,
+                                  uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2,
+                                  uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128,
+                                  int promo_bytes) {
     if (!encoder()) return false;
     const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+    const cuuint64_t strides[2] = {stride1, stride2};
     const cuuint32_t box[3] = {b0, b1, b2};
     const cuuint32_t estr[3] = {1, 1, 1};
-    // L2 fetch granularity no larger than one contiguous row: a wider promotion would drag in
-    // the next head's row of the same slot, which the paged layout does not read next.
-    const uint64_t row = d0 * esize;
-    const CUtensorMapL2promotion promo = row >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
-                                         : row >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
-                                                      : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+    const CUtensorMapL2promotion promo = promo_bytes >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                         : promo_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                              : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
     CUresult r = g_encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                           3, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                           promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// 3-D tiled map over a row-major [d2, d1, d0] tensor of `esize`-byte elements.  L2 fetches
+// are promoted to one contiguous row at most: a wider promotion would drag in the next
+// head's row of the same slot, which the paged layout does not read next.
+bool encode_tensor_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128) {
+    const uint64_t row = d0 * esize;
+    return encode_tensor_map_3d_strided(map, base, esize, d0, d1, d2, row, row * d1, b0, b1, b2,
+                                        swizzle128, (int)(row >= 256 ? 256 : row));
 }
 
 cudaError_t launch_wait_timeout(unsigned long long limit_ns, int *err, cudaStream_t s) {

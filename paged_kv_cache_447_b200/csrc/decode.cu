@@ -7,14 +7,18 @@
 // bound by memory bandwidth, the cache keeps growing.
 //
 // Design (HBM-bound: every cached K/V byte is streamed from HBM exactly once):
-//  * Work unit = one 16-token block of one (sequence, kv head).  Units are numbered
-//    sequence-major; the whole unit space is cut into equal contiguous ranges, one per
-//    persistent CTA (grid = SMs x 2), so every CTA streams the same number of bytes
-//    whatever the length mix.  A CTA's range crosses sequence boundaries; each piece of a
-//    (sequence, kv head) it covers becomes one partial softmax state.
-//  * Warp 0 is the producer: it reads block-table entries 32 at a time and issues one TMA
-//    load per block for K and one for V into a ring of shared-memory stages (mbarrier
-//    full/empty pairs).  Warps 1-4 consume stages round robin.
+//  * Work unit = one 16-token block of one (sequence, kv-head group) -- the group is one kv
+//    head, or for E4M3 caches with grouped heads two adjacent kv heads, so that every cache
+//    row fetched is 256 contiguous bytes (128-byte rows measured at ~60 % of the DRAM
+//    bandwidth 256-byte rows reach).  Units are numbered sequence-major; the whole unit space
+//    is cut into equal contiguous ranges, one per persistent CTA, so every CTA streams the
+//    same number of bytes whatever the length mix.  A CTA's range crosses sequence
+//    boundaries; each piece of a (sequence, kv-head group) it covers becomes one partial
+//    softmax state per kv head.
+//  * Warp 0 is the producer: it reads block-table entries 32 at a time and issues TMA loads
+//    of K and V into a ring of shared-memory stages (mbarrier full/empty pairs).  Warps 1-4
+//    consume stages round robin; with two kv heads per unit they form two pairs, one warp
+//    per head, each pair taking every other unit.
 //  * A consumer warp handles all G = Hq/Hkv query heads of the kv head, so each K/V tile
 //    is read from shared memory once for the whole group.  Online softmax (running max m,
 //    sum l) per warp in exp2 space.
@@ -70,12 +74,12 @@ struct DecodeParams {
     const float *rope;
     int max_pos;
     int *prefix;      // [B+1] block prefix, written by CTA 0 for the combine kernel
-    float *partials;  // [(B*Hkv + nctas)][G][D+2]
+    float *partials;  // [(B*Hkv + 2*nctas)][G][D+2]
     int nctas;
     int *err;
 };
 
-template <int D, bool FP8, int G>
+template <int D, bool FP8, int G, int HPU>
 struct Geometry {
     static constexpr DecodeCfg kCfg = decode_cfg(G, FP8);
     static constexpr int kConsumers = kCfg.consumers;
@@ -83,19 +87,21 @@ struct Geometry {
     static constexpr int kCtasPerSm = kCfg.ctas_per_sm;
     static constexpr int kElem = FP8 ? 1 : 2;
     static constexpr int kRowBytes = D * kElem;
-    static constexpr int kTileBytes = kBlockSize * kRowBytes;          // one K (or V) block
-    static constexpr int kStageBytes = 2 * kTileBytes;                 // K + V
+    static constexpr int kTileBytes = kBlockSize * kRowBytes;          // one K (or V) block, one head
+    static constexpr int kStageBytes = 2 * HPU * kTileBytes;           // K + V of the unit's heads
+    static constexpr int kGroups = kConsumers / HPU;                   // consumer groups (warp per head)
     // q, probabilities and merge scratch, plus room for 1024 sequences' prefix
     static constexpr int kExtraBytes = G * D * 4 + kConsumers * G * 16 * 4 +
                                        kConsumers * G * (D + 2) * 4 + 4 * 1025;
     // ring of ~100 KB in total so that two CTAs share an SM
-    // The stage count is a multiple of the consumer count, so that every fill of a given
-    // stage is consumed by the same warp: a warp then never waits on a barrier more than
-    // one phase ahead (a parity wait cannot tell phase n from phase n+2).
+    // The stage count is a multiple of the consumer-group count, so that every fill of a
+    // given stage is consumed by the same warp(s): a warp then never waits on a barrier more
+    // than one phase ahead (a parity wait cannot tell phase n from phase n+2).
     static constexpr int kStagesRaw = (kCfg.smem_budget - kExtraBytes) / kStageBytes;
-    static constexpr int kStagesQ = (kStagesRaw / kConsumers) * kConsumers;
-    static constexpr int kStages = kStagesQ < kConsumers ? kConsumers : (kStagesQ > 64 ? 64 : kStagesQ);
-    static_assert(kStages % kConsumers == 0, "stage count must be a multiple of the consumers");
+    static constexpr int kStagesQ = (kStagesRaw / kGroups) * kGroups;
+    static constexpr int kStages = kStagesQ < kGroups ? kGroups : (kStagesQ > 64 ? 64 : kStagesQ);
+    static_assert(kStages % kGroups == 0, "stage count must be a multiple of the consumer groups");
+    static_assert(kConsumers % HPU == 0, "one consumer warp per head of a unit");
     static constexpr int kChunkElems = 16 / kElem;                     // elements per 16 B
     static constexpr int kChunks = kRowBytes / 16;                     // 16-B chunks per row
     static constexpr int kHalf = kChunks / 2;                          // per lane of a pair
@@ -256,17 +262,19 @@ __device__ __forceinline__ uint32_t swz(int t, int c) {
     return (uint32_t)((c >> 3) * 2048 + t * 128 + (((c & 7) ^ (t & 7)) << 4));
 }
 
-template <int D, bool FP8, int G>
-__global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8, G>::kCtasPerSm)
+template <int D, bool FP8, int G, int HPU>
+__global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
+                                  Geometry<D, FP8, G, HPU>::kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                   const DecodeParams p) {
-    using Geo = Geometry<D, FP8, G>;
+    using Geo = Geometry<D, FP8, G, HPU>;
     constexpr int NS = Geo::kStages;
     constexpr int kConsumers = Geo::kConsumers;
     constexpr int kThreads = Geo::kThreads;
     // grouped heads on the tensor cores: bf16 caches, and E4M3 caches at head dim 128
     constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
     constexpr int kSlabs = Geo::kRowBytes / 128;  // swizzled boxes per tile (kMma)
+    static_assert(HPU == 1 || (kMma && kSlabs == 1), "two heads per unit: one-slab tiles only");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;                                                  // NS x stage
@@ -283,7 +291,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     pdl_wait();
     pdl_trigger();
     block_prefix<kThreads>(p, pfx);
-    const long long total = (long long)p.Hkv * pfx[p.B];
+    const int Hu = p.Hkv / HPU;  // kv-head groups (units per block of a sequence)
+    const long long total = (long long)Hu * pfx[p.B];
     if (blockIdx.x == 0)
         for (int i = threadIdx.x; i <= p.B; i += kThreads) p.prefix[i] = pfx[i];
     // sequences with an empty context get zero rows (strided over the CTAs)
@@ -300,7 +309,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_u32(full + s), 1);
-            mbar_init(smem_u32(empty + s), 1);
+            mbar_init(smem_u32(empty + s), HPU);  // one arrival per head's warp
         }
         abort_s = 0;
         fence_mbar_init();
@@ -319,7 +328,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             const int k = k0 + lane;
             int phys = 0, kvh = 0;
             if (k < nunits) {
-                UnitPos up = locate(pfx, p.B, p.Hkv, u0 + k);
+                UnitPos up = locate(pfx, p.B, Hu, u0 + k);
                 kvh = up.kvh;
                 phys = __ldg(p.block_tables + (size_t)up.b * p.max_blocks + up.blk);
                 if (phys < 0 || (long long)phys >= p.num_blocks) {
@@ -341,7 +350,12 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                         const uint32_t fb = smem_u32(full + s);
                         const uint32_t dst = smem_u32(stages + s * Geo::kStageBytes);
                         mbar_arrive_expect_tx(fb, Geo::kStageBytes);
-                        if constexpr (kMma) {
+                        if constexpr (HPU == 2) {
+                            // one box per tensor: 16 slots x 2 adjacent heads (256 contiguous
+                            // bytes per slot), landing as the two heads' swizzled tiles
+                            tma_load_3d(dst, &tm_k, fb, 0, ph * kBlockSize, 2 * hh);
+                            tma_load_3d(dst + 2 * Geo::kTileBytes, &tm_v, fb, 0, ph * kBlockSize, 2 * hh);
+                        } else if constexpr (kMma) {
                             // one swizzled box per 64-column slab
 #pragma unroll
                             for (int h = 0; h < kSlabs; ++h) {
@@ -373,6 +387,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     // ---------------------------------------------------------------------- consumers
     const int cw = warp - 1;          // consumer index 0..3
     const int ct = threadIdx.x - 32;  // consumer thread 0..127
+    const int cgrp = cw / HPU, hsel = cw % HPU;  // consumer group; head of the unit it serves
     // q.k lane mapping (see the q.k loop): kTPL tokens per lane group of kLPG lanes
     constexpr int kTPL = (G == 2 || G == 4) ? 2 : 1;
     constexpr int kLPG = 2 * kTPL;
@@ -417,19 +432,20 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
     const uint32_t pbuf_a = smem_u32(pbuf + cw * G * 16);
 
     int k = 0;
-    UnitPos cur = locate(pfx, p.B, p.Hkv, u0);
+    UnitPos cur = locate(pfx, p.B, Hu, u0);
     bool dead = false;
     while (k < nunits) {
-        // piece = the rest of the current (sequence, kv head) segment inside this range
+        // piece = the rest of the current (sequence, kv-head group) segment inside this range
         const int piece_len = min(cur.nb - cur.blk, nunits - k);
-        const int b = cur.b, kvh = cur.kvh;
+        const int b = cur.b, kvg = cur.kvh;
+        const int kvh = kvg * HPU + hsel;  // this warp's kv head
         const int L = min(__ldg(p.context_lens + b), p.max_blocks * kBlockSize);
         const bool whole = (cur.blk == 0) && (piece_len == cur.nb);
 
-        // ---- stage q for this (b, kv head): rotate (optional), scale, split layout
-        for (int e = ct; e < G * D / 2; e += kConsumers * 32) {
-            const int g = e / (D / 2), i = e % (D / 2);
-            const int h = kvh * G + g;
+        // ---- stage q for this (b, kv-head group): rotate (optional), scale, split layout
+        for (int e = ct; e < HPU * G * D / 2; e += kConsumers * 32) {
+            const int hh = e / (G * D / 2), g = (e / (D / 2)) % G, i = e % (D / 2);
+            const int h = (kvg * HPU + hh) * G + g;
             const uint16_t *qr = p.q + ((size_t)b * p.Hq + h) * D;
             uint16_t x1 = __ldg(qr + i), x2 = __ldg(qr + i + D / 2);
             if (p.rope) {
@@ -442,10 +458,10 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
                 }
             }
             if constexpr (kMma) {
-                // rotated bf16 q, [G][D]; the scale is applied to the fp32 scores
-                uint16_t *qh = reinterpret_cast<uint16_t *>(qs);
-                qh[g * D + i] = x1;
-                qh[g * D + i + D / 2] = x2;
+                // rotated bf16 q, [HPU][G][D]; the scale is applied to the fp32 scores
+                uint16_t *qh = reinterpret_cast<uint16_t *>(qs) + (hh * G + g) * D;
+                qh[i] = x1;
+                qh[i + D / 2] = x2;
                 continue;
             }
             const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
@@ -467,13 +483,13 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             for (int ks = 0; ks < kMT; ++ks) {
                 if constexpr (FP8) {
                     // k step ks, quad lane q4: dims 32*q4 + 4*ks + {0,1 | 2,3}, in f16
-                    const uint32_t a = qs_a + (uint32_t)((row * D + 32 * q4 + 4 * ks) * 2);
+                    const uint32_t a = qs_a + (uint32_t)(((hsel * G + row) * D + 32 * q4 + 4 * ks) * 2);
                     const uint2 w = row < G ? lds64(a) : make_uint2(0u, 0u);
                     qa[ks][0] = pack_f16x2(bf16lo(w.x), bf16hi(w.x));
                     qa[ks][1] = pack_f16x2(bf16lo(w.y), bf16hi(w.y));
                 } else {
                     // k step ks, quad lane q4: dims 16*ks + 2*q4 + {0,1 | 8,9}
-                    const uint32_t a = qs_a + (uint32_t)((row * D + 16 * ks + 2 * q4) * 2);
+                    const uint32_t a = qs_a + (uint32_t)(((hsel * G + row) * D + 16 * ks + 2 * q4) * 2);
                     qa[ks][0] = row < G ? lds32(a) : 0u;
                     qa[ks][1] = row < G ? lds32(a + 16) : 0u;
                 }
@@ -482,7 +498,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
 
         // ---- stream this piece's blocks
         for (int j = 0; j < piece_len; ++j, ++k) {
-            if ((k % kConsumers) != cw) continue;
+            if ((k % Geo::kGroups) != cgrp) continue;
             const int s = k % NS;
             const uint32_t parity = (k / NS) & 1;
             if (!dead) {
@@ -494,8 +510,9 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             if (dead) continue;
             const int blk = cur.blk + j;
             const int valid = min(kBlockSize, L - blk * kBlockSize);
-            const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes);
-            const uint32_t vs_a = ks_a + Geo::kTileBytes;
+            // this warp's head: K tile hsel, then V tile hsel after the HPU K tiles
+            const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes) + hsel * Geo::kTileBytes;
+            const uint32_t vs_a = ks_a + HPU * Geo::kTileBytes;
             if constexpr (kMma) {
                 // S = Q K^T: n tile 0 = tokens 0-7, n tile 1 = tokens 8-15.  ldmatrix x4
                 // matrices: (tokens 0-7 | 8-15) x (first | second 8 dims of the k step).
@@ -818,26 +835,29 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
             for (int d = 0; d < Geo::kDimsPerLane; ++d) mw[lane * Geo::kDimsPerLane + d] = acc[g][d];
         }
         named_bar(kMergeBar, kConsumers * 32);
-        const int seg = b * p.Hkv + kvh;
-        for (int e = ct; e < G * D; e += kConsumers * 32) {
-            const int g = e / D, d = e % D;
+        // warps w with w % HPU == hd hold head hd of the group; partial slots are
+        // HPU * (segment + CTA) + hd, distinct for every (segment, CTA, head)
+        const int segu = b * Hu + kvg;
+        for (int e = ct; e < HPU * G * D; e += kConsumers * 32) {
+            const int hd = e / (G * D), g = (e / D) % G, d = e % D;
+            const int kvo = kvg * HPU + hd;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, mrg[(w * G + g) * (D + 2) + D]);
+            for (int w = hd; w < kConsumers; w += HPU) M = fmaxf(M, mrg[(w * G + g) * (D + 2) + D]);
             float o = 0.f, lsum = 0.f;
 #pragma unroll
-            for (int w = 0; w < kConsumers; ++w) {
+            for (int w = hd; w < kConsumers; w += HPU) {
                 const float *mw = mrg + (w * G + g) * (D + 2);
                 const float f = (mw[D] == -INFINITY) ? 0.f : ex2(mw[D] - M);
                 o += f * mw[d];
                 lsum += f * mw[D + 1];
             }
             if (whole) {
-                const float vs = FP8 ? __ldg(p.v_scale + kvh) : 1.f;
+                const float vs = FP8 ? __ldg(p.v_scale + kvo) : 1.f;
                 const float r = (lsum > 0.f) ? o / lsum * vs : 0.f;
-                p.out[((size_t)b * p.Hq + kvh * G + g) * D + d] = __float2bfloat16_rn(r);
+                p.out[((size_t)b * p.Hq + kvo * G + g) * D + d] = __float2bfloat16_rn(r);
             } else {
-                float *slot = p.partials + (size_t)(seg + blockIdx.x) * (G * (D + 2));
+                float *slot = p.partials + (size_t)(HPU * (segu + blockIdx.x) + hd) * (G * (D + 2));
                 slot[g * D + d] = o;
                 if (d == 0) {
                     slot[G * D + g] = M;
@@ -849,7 +869,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G>::kThreads, Geometry<D, FP8
         reset_state();
         // advance to the next segment
         cur.blk += piece_len;
-        if (cur.blk >= cur.nb && k < nunits) cur = locate(pfx, p.B, p.Hkv, u0 + k);
+        if (cur.blk >= cur.nb && k < nunits) cur = locate(pfx, p.B, Hu, u0 + k);
     }
 }
 
@@ -866,48 +886,50 @@ __device__ __forceinline__ int find_seq_global(const int *pfx, int B, int Hkv, l
     return lo;
 }
 
-template <int D, int G>
+template <int D, int G, int HPU>
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     pdl_wait();
     pdl_trigger();
     const int c = blockIdx.x;
-    const long long total = (long long)p.Hkv * __ldg(p.prefix + p.B);
+    const int Hu = p.Hkv / HPU;
+    const long long total = (long long)Hu * __ldg(p.prefix + p.B);
     if (c == 0 || total == 0) return;
     const long long U = (total + p.nctas - 1) / p.nctas;
     const long long x = (long long)c * U;
     if (x >= total) return;
-    const int b = find_seq_global(p.prefix, p.B, p.Hkv, x);
+    const int b = find_seq_global(p.prefix, p.B, Hu, x);
     const int pb = __ldg(p.prefix + b), nb = __ldg(p.prefix + b + 1) - pb;
-    const int kvh = (int)((x - (long long)p.Hkv * pb) / nb);
-    const long long start = (long long)p.Hkv * pb + (long long)kvh * nb;
+    const int kvg = (int)((x - (long long)Hu * pb) / nb);
+    const long long start = (long long)Hu * pb + (long long)kvg * nb;
     if (start == x) return;                          // boundary at a segment start: no split
     const int c0 = (int)(start / U), c1 = (int)((start + nb - 1) / U);
     if (c0 != c - 1) return;                         // an earlier boundary's CTA merges it
-    const int seg = b * p.Hkv + kvh;
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int g = e / D, d = e % D;
+    const int segu = b * Hu + kvg;
+    for (int e = threadIdx.x; e < HPU * G * D; e += blockDim.x) {
+        const int hd = e / (G * D), g = (e / D) % G, d = e % D;
+        const int kvo = kvg * HPU + hd;
         float M = -INFINITY;
         for (int cc = c0; cc <= c1; ++cc) {
-            const float *slot = p.partials + (size_t)(seg + cc) * (G * (D + 2));
+            const float *slot = p.partials + (size_t)(HPU * (segu + cc) + hd) * (G * (D + 2));
             M = fmaxf(M, slot[G * D + g]);
         }
         float o = 0.f, lsum = 0.f;
         for (int cc = c0; cc <= c1; ++cc) {
-            const float *slot = p.partials + (size_t)(seg + cc) * (G * (D + 2));
+            const float *slot = p.partials + (size_t)(HPU * (segu + cc) + hd) * (G * (D + 2));
             const float mk = slot[G * D + g];
             const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
             o += f * slot[g * D + d];
             lsum += f * slot[G * D + G + g];
         }
-        const float vsc = p.v_scale ? __ldg(p.v_scale + kvh) : 1.f;
-        p.out[((size_t)b * p.Hq + kvh * G + g) * D + d] =
+        const float vsc = p.v_scale ? __ldg(p.v_scale + kvo) : 1.f;
+        p.out[((size_t)b * p.Hq + kvo * G + g) * D + d] =
             __float2bfloat16_rn(lsum > 0.f ? o / lsum * vsc : 0.f);
     }
 }
 
-template <int D, bool FP8, int G>
+template <int D, bool FP8, int G, int HPU>
 size_t smem_bytes(int B) {
-    using Geo = Geometry<D, FP8, G>;
+    using Geo = Geometry<D, FP8, G, HPU>;
     constexpr int kConsumers = Geo::kConsumers;
     size_t s = (size_t)Geo::kStages * Geo::kStageBytes + 2 * Geo::kStages * sizeof(uint64_t);
     s += (size_t)G * D * 4 + (size_t)kConsumers * G * 16 * 4 + (size_t)kConsumers * G * (D + 2) * 4;
@@ -915,46 +937,64 @@ size_t smem_bytes(int B) {
     return s + 1024;  // alignment slack for the swizzled stages
 }
 
-template <int D, bool FP8, int G>
+template <int D, bool FP8, int G, int HPU>
 cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t s) {
-    const size_t smem = smem_bytes<D, FP8, G>(a.num_seqs);
-    auto kern = decode_kernel<D, FP8, G>;
+    using Geo = Geometry<D, FP8, G, HPU>;
+    const size_t smem = smem_bytes<D, FP8, G, HPU>(a.num_seqs);
+    auto kern = decode_kernel<D, FP8, G, HPU>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int occ = 0;
-    constexpr int kThreads = Geometry<D, FP8, G>::kThreads;
+    constexpr int kThreads = Geo::kThreads;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (occ < 1) return cudaErrorInvalidConfiguration;
     DecodeParams lp = prm;
-    lp.nctas = std::min(prm.nctas / kMaxCtasPerSm * Geometry<D, FP8, G>::kCtasPerSm,
-                        occ * (prm.nctas / kMaxCtasPerSm));
-    // K/V maps with exactly the boxes the kernel's producer issues
-    using Geo = Geometry<D, FP8, G>;
+    lp.nctas = std::min(prm.nctas / kMaxCtasPerSm * Geo::kCtasPerSm, occ * (prm.nctas / kMaxCtasPerSm));
+    // K/V maps with exactly the boxes the kernel's producer issues.
+    //   CUDA-core consumers: one box per tile, a whole 16-token block of one kv head.
+    //   Tensor-core consumers: one 128-byte-swizzled box per 64-column slab.
+    //   Two heads per unit: dims listed (column, slot, head) so that one box of 16 slots x 2
+    //   heads lands as the two heads' tiles back to back, fetched 256 bytes at a time.
     CUtensorMap tk, tv;
     const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
-    // CUDA-core consumers: one box per tile, a whole 16-token block of one kv head (16 rows of
-    // D elements).  Tensor-core consumers: one 128-byte-swizzled box per 64-column slab.
     constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
-    const uint32_t box0 = kMma ? 128u / Geo::kElem : (uint32_t)D;
-    if (!encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma) ||
-        !encode_tensor_map_3d(&tv, a.v_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma))
-        return cudaErrorUnknown;  // (cudaErrorInvalidValue means a short workspace)
-    static_assert(kBlockSize * D * Geo::kElem == Geo::kTileBytes, "one TMA box fills one tile");
+    bool ok;
+    if constexpr (HPU == 2) {
+        const uint64_t row = (uint64_t)a.n_kv_heads * D * Geo::kElem, head = (uint64_t)D * Geo::kElem;
+        ok = encode_tensor_map_3d_strided(&tk, a.k_cache, Geo::kElem, D, slots, a.n_kv_heads, row, head,
+                                          D, kBlockSize, 2, true, 256) &&
+             encode_tensor_map_3d_strided(&tv, a.v_cache, Geo::kElem, D, slots, a.n_kv_heads, row, head,
+                                          D, kBlockSize, 2, true, 256);
+    } else {
+        const uint32_t box0 = kMma ? 128u / Geo::kElem : (uint32_t)D;
+        ok = encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma) &&
+             encode_tensor_map_3d(&tv, a.v_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma);
+    }
+    if (!ok) return cudaErrorUnknown;  // (cudaErrorInvalidValue means a short workspace)
+    static_assert(kBlockSize * D * Geo::kElem == Geo::kTileBytes, "one head's box fills one tile");
     e = launch_pdl(kern, dim3(lp.nctas), dim3(kThreads), smem, s, tk, tv, lp);
     if (e != cudaSuccess) return e;
     DecodeParams cp = lp;
     cp.v_scale = FP8 ? a.v_scale : nullptr;
-    return launch_pdl(combine_kernel<D, G>, dim3(lp.nctas), dim3(128), 0, s, cp);
+    return launch_pdl(combine_kernel<D, G, HPU>, dim3(lp.nctas), dim3(128), 0, s, cp);
+}
+
+template <int D, bool FP8, int G>
+cudaError_t launch_h(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t s) {
+    // E4M3 rows of one head are 128 bytes: grouped heads fetch two heads per unit
+    if constexpr (FP8 && D == 128 && G >= 2)
+        if (a.n_kv_heads % 2 == 0) return launch_t<D, FP8, G, 2>(prm, a, s);
+    return launch_t<D, FP8, G, 1>(prm, a, s);
 }
 
 template <int D, bool FP8>
 cudaError_t launch_g(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t s) {
     switch (a.n_q_heads / a.n_kv_heads) {
-        case 1: return launch_t<D, FP8, 1>(prm, a, s);
-        case 2: return launch_t<D, FP8, 2>(prm, a, s);
-        case 4: return launch_t<D, FP8, 4>(prm, a, s);
-        case 8: return launch_t<D, FP8, 8>(prm, a, s);
+        case 1: return launch_h<D, FP8, 1>(prm, a, s);
+        case 2: return launch_h<D, FP8, 2>(prm, a, s);
+        case 4: return launch_h<D, FP8, 4>(prm, a, s);
+        case 8: return launch_h<D, FP8, 8>(prm, a, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -968,7 +1008,9 @@ int decode_grid_ctas(int num_sms) { return num_sms * kMaxCtasPerSm; }
 size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
                               int num_sms) {
     const int G = n_q_heads / n_kv_heads;
-    const size_t slots = (size_t)num_seqs * n_kv_heads + (size_t)decode_grid_ctas(num_sms);
+    // one slot per (sequence, kv head), plus up to two per CTA (a CTA's range splits at most
+    // two segments, and a segment may carry two kv heads)
+    const size_t slots = (size_t)num_seqs * n_kv_heads + 2 * (size_t)decode_grid_ctas(num_sms);
     return align16((size_t)(num_seqs + 1) * sizeof(int)) +
            slots * (size_t)G * (head_dim + 2) * sizeof(float);
 }

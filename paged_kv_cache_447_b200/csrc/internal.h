@@ -74,6 +74,11 @@ struct PrefillArgs {
 // the maps its kernel reads, from the same compile-time geometry the kernel uses.
 bool encode_tensor_map_3d(CUtensorMap *map, const void *base, int esize, uint64_t d0, uint64_t d1,
                           uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128);
+// The same with explicit byte strides of dims 1 and 2 (dims in any order) and L2 promotion.
+bool encode_tensor_map_3d_strided(CUtensorMap *map, const void *base, int esize, uint64_t d0,
+                                  uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2,
+                                  uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128,
+                                  int promo_bytes);
 
 cudaError_t launch_kv_store(const StoreArgs &a, cudaStream_t s);
 cudaError_t launch_rope_apply(const RopeArgs &a, cudaStream_t s);

@@ -261,6 +261,13 @@ def test_decode_fp8_edge_lengths_and_groups(lens, group):
             assert torch.all(out[b] == 0)
 
 
+@pytest.mark.parametrize("group", [2, 4])
+def test_decode_fp8_odd_kv_heads(group):
+    """E4M3 with an odd kv-head count: units hold one kv head (two-head units need pairs)."""
+    out, ref = _grouped_case(700 + group, [5000, 1, 17, 250], group, 128, True, hkv=3)
+    compare(out, ref, fp8=True, what=f"fp8 odd kv heads G={group}")
+
+
 def test_decode_block_id_out_of_range_is_flagged():
     wl = W.tiny(seed=1)
     st = wl.steps[1]
