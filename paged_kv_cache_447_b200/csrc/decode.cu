@@ -104,7 +104,6 @@ struct Geometry {
     static_assert(kConsumers % HPU == 0, "one consumer warp per head of a unit");
     static constexpr int kChunkElems = 16 / kElem;                     // elements per 16 B
     static constexpr int kChunks = kRowBytes / 16;                     // 16-B chunks per row
-    static constexpr int kHalf = kChunks / 2;                          // per lane of a pair
     static constexpr int kQuads = kChunkElems / 4;                     // float4 per chunk
     static constexpr int kDimsPerLane = D / 32;                        // p.v ownership
 };
@@ -439,6 +438,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
         const int piece_len = min(cur.nb - cur.blk, nunits - k);
         const int b = cur.b, kvg = cur.kvh;
         const int kvh = kvg * HPU + hsel;  // this warp's kv head
+        // score scale in exp2 units (E4M3: with the head's K scale folded in)
+        const float sc_piece = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
         const int L = min(__ldg(p.context_lens + b), p.max_blocks * kBlockSize);
         const bool whole = (cur.blk == 0) && (piece_len == cur.nb);
 
@@ -544,7 +545,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                     }
                 }
                 // online softmax of row `row` over this block (the quad holds its 16 tokens)
-                const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
+                const float sc = sc_piece;
                 const int t0 = 2 * q4;
                 float sv[4] = {sa[0][0] * sc, sa[0][1] * sc, sa[1][0] * sc, sa[1][1] * sc};
                 if (valid < kBlockSize) {
@@ -821,18 +822,20 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                 }
             }
         }
+        if constexpr (!kMma) {
 #pragma unroll
-        for (int g = 0; g < G && !kMma; ++g) {
-            float lw = l[g];
+            for (int g = 0; g < G; ++g) {
+                float lw = l[g];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-            float *mw = mrg + (cw * G + g) * (D + 2);
-            if (lane == 0) {
-                mw[D] = m[g];
-                mw[D + 1] = lw;
+                for (int o = 1; o < 32; o <<= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+                float *mw = mrg + (cw * G + g) * (D + 2);
+                if (lane == 0) {
+                    mw[D] = m[g];
+                    mw[D + 1] = lw;
+                }
+#pragma unroll
+                for (int d = 0; d < Geo::kDimsPerLane; ++d) mw[lane * Geo::kDimsPerLane + d] = acc[g][d];
             }
-#pragma unroll
-            for (int d = 0; d < Geo::kDimsPerLane; ++d) mw[lane * Geo::kDimsPerLane + d] = acc[g][d];
         }
         named_bar(kMergeBar, kConsumers * 32);
         // warps w with w % HPU == hd hold head hd of the group; partial slots are

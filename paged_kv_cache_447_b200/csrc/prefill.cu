@@ -41,14 +41,18 @@ struct PGeo {
     static constexpr int kSlabBytes = kRows * 128;           // 16 KB (128 rows x 128 B)
     static constexpr int kQBytes = kSlabs * kSlabBytes;      // one Q tile
     static constexpr int kKVBytes = kSlabs * kSlabBytes;     // one K (or V) tile of 128 keys
-    static constexpr int kStages = D == 128 ? 2 : 4;
+    // Separate K and V rings: K(j) is released as soon as S1(j) completes, V(j) after PV1(j),
+    // so the K load that gates S(j+2) gets five MMAs of slack instead of two.  (A third K
+    // stage fits at D 128 in bf16 but measured 1-2 % slower than two.)
+    static constexpr int kKStages = D == 128 ? 2 : 4;
+    static constexpr int kVStages = D == 128 ? 2 : 4;
     static constexpr int kStgBytes = FP8 ? kKeys * D : 0;    // raw E4M3 tile (K or V)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = 2 * kQBytes;
-    static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffStg = kOffV + kStages * kKVBytes;
+    static constexpr int kOffV = kOffK + kKStages * kKVBytes;
+    static constexpr int kOffStg = kOffV + kVStages * kKVBytes;
     static constexpr int kOffBar = kOffStg + 2 * kStgBytes;
-    static constexpr int kBarBytes = 8 * (16 + 3 * kStages) + 16;
+    static constexpr int kBarBytes = 8 * (16 + 2 * kKStages + 2 * kVStages) + 16;
     static constexpr int kSmem = kOffBar + kBarBytes + 1024;  // + alignment slack
     static_assert(kSmem <= 232448, "shared memory budget");
 };
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
     using Geo = PGeo<D, FP8>;
-    constexpr int NS = Geo::kStages;
+    constexpr int KS = Geo::kKStages, VS = Geo::kVStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t *smem = smem_raw + (sbase - smem_u32(smem_raw));
@@ -255,9 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t b_pfull = bar0 + 48;   // [2]
     const uint32_t b_drain = bar0 + 64;
     const uint32_t b_stgfull = bar0 + 80, b_stgempty = bar0 + 88;  // FP8 staging
-    const uint32_t b_kfull = bar0 + 128;  // [NS]
-    const uint32_t b_vfull = b_kfull + 8 * NS;
-    const uint32_t b_empty = b_vfull + 8 * NS;
+    const uint32_t b_kfull = bar0 + 128;  // [KS]
+    const uint32_t b_kempty = b_kfull + 8 * KS;
+    const uint32_t b_vfull = b_kempty + 8 * KS;  // [VS]
+    const uint32_t b_vempty = b_vfull + 8 * VS;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Geo::kOffBar + 72);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kOffBar + 76);
 
@@ -279,11 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(b_sfull + 8 * i, 1);
             mbar_init(b_pfull + 8 * i, 128);
         }
-        for (int s = 0; s < NS; ++s) {
-            // bf16: one arrival with the TMA byte count; FP8: the 64 converter threads
+        // bf16: one arrival with the TMA byte count; FP8: the 64 converter threads
+        for (int s = 0; s < KS; ++s) {
             mbar_init(b_kfull + 8 * s, FP8 ? 64 : 1);
+            mbar_init(b_kempty + 8 * s, 1);
+        }
+        for (int s = 0; s < VS; ++s) {
             mbar_init(b_vfull + 8 * s, FP8 ? 64 : 1);
-            mbar_init(b_empty + 8 * s, 1);
+            mbar_init(b_vempty + 8 * s, 1);
         }
         mbar_init(b_stgfull, 1);
         mbar_init(b_stgempty, 64);
@@ -306,7 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kSoftmax0) {
     if (warp == 0) {
         // ---------------------------------------------------------------- producer
-        uint32_t issued = 0;  // bitmask: stage s has an outstanding fill (bit s: K, bit 8+s: V)
+        // outstanding fills: bit s = K stage s, bit 8+s = V stage s, bit 16 = E4M3 staging,
+        // bit 17 = the V fill of the partial last block (completes on b_vraw)
+        uint32_t issued = 0;
         uint32_t phase_bits = 0;
         bool ok = true;
         if (lane == 0) {
@@ -321,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int oob = (int)min(p.num_blocks, (long long)(0x7fffffff / kBlockSize));
         for (int j = 0; j < n_kv && ok; ++j) {
-            const int st = j % NS;
-            const uint32_t par = ((j / NS) & 1) ^ 1;
+            const int ks = j % KS, vs = j % VS;
+            const uint32_t kpar = ((j / KS) & 1) ^ 1, vpar = ((j / VS) & 1) ^ 1;
             int phys = oob;
             if (lane < 8) {
                 const int lb = j * 8 + lane;
@@ -363,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const bool fix = (Lc % kBlockSize) != 0 && j == (Lc - 1) / kKeys;
             if (lane == 0) {
-                if (*abort_flag || !mbar_wait_bounded(b_empty + 8 * st, par, p.err)) {
+                if (*abort_flag || !mbar_wait_bounded(b_kempty + 8 * ks, kpar, p.err)) {
                     ok = false;
                     *abort_flag = 1;
                 }
@@ -374,22 +384,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) ph[i] = __shfl_sync(0xffffffffu, phys, i);
             if (lane == 0) {
-                const uint32_t kb = b_kfull + 8 * st, vb = fix ? b_vraw : b_vfull + 8 * st;
+                const uint32_t kb = b_kfull + 8 * ks;
                 mbar_arrive_expect_tx(kb, Geo::kKVBytes);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     for (int s = 0; s < Geo::kSlabs; ++s)
-                        tma_load_3d(sK + st * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_k, kb,
+                        tma_load_3d(sK + ks * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_k, kb,
                                     64 * s, it.kvh, ph[i] * kBlockSize);
-                mbar_arrive_expect_tx(vb, Geo::kKVBytes);
+                issued |= 1u << ks;
+                phase_bits = (phase_bits & ~(1u << ks)) | ((uint32_t)((j / KS) & 1) << ks);
+                // V of the same tile: its stage frees later (after PV1 of tile j - VS)
+                if (*abort_flag || !mbar_wait_bounded(b_vempty + 8 * vs, vpar, p.err)) {
+                    ok = false;
+                    *abort_flag = 1;
+                } else {
+                    const uint32_t vb = fix ? b_vraw : b_vfull + 8 * vs;
+                    mbar_arrive_expect_tx(vb, Geo::kKVBytes);
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    for (int s = 0; s < Geo::kSlabs; ++s)
-                        tma_load_3d(sV + st * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_v, vb,
-                                    64 * s, it.kvh, ph[i] * kBlockSize);
-                issued |= (1u << st) | (fix ? 0u : (1u << (8 + st)));
-                phase_bits = (phase_bits & ~(1u << st)) | ((uint32_t)((j / NS) & 1) << st);
+                    for (int i = 0; i < 8; ++i)
+                        for (int s = 0; s < Geo::kSlabs; ++s)
+                            tma_load_3d(sV + vs * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_v, vb,
+                                        64 * s, it.kvh, ph[i] * kBlockSize);
+                    if (!fix) {
+                        issued |= 1u << (8 + vs);
+                        phase_bits = (phase_bits & ~(1u << (8 + vs))) | ((uint32_t)((j / VS) & 1) << (8 + vs));
+                    } else {
+                        // this fill completes on b_vraw (drained below); the stage's earlier
+                        // fill has landed (its PV1 freed the stage), so its bit is retired
+                        issued = (issued & ~(1u << (8 + vs))) | (1u << 17);
+                    }
+                }
             }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
             if (fix) {
                 // zero the rows past the sequence in the tile's partial block, then publish
                 bool landed = true;
@@ -400,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int first = Lc % kBlockSize;
                     const int rows = kBlockSize - first;
                     for (int s = 0; s < Geo::kSlabs; ++s) {
-                        const uint32_t row0 = sV + st * Geo::kKVBytes + s * Geo::kSlabBytes +
+                        const uint32_t row0 = sV + vs * Geo::kKVBytes + s * Geo::kSlabBytes +
                                               blk_in_tile * 2048 + first * 128;
                         for (int e = lane; e < rows * 8; e += 32)
                             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + e * 16),
@@ -411,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    if (landed) mbar_arrive(b_vfull + 8 * st);
+                    if (landed) mbar_arrive(b_vfull + 8 * vs);
                     else *abort_flag = 1;
                 }
                 if (!landed) ok = false;
@@ -421,11 +448,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             mbar_wait_bounded(b_qfull, 0, p.err);
             if ((issued >> 16) & 1) mbar_wait_bounded(b_stgfull, (phase_bits >> 16) & 1, p.err);
-            for (int s = 0; s < NS; ++s) {
-                const uint32_t par = (phase_bits >> s) & 1;
-                if ((issued >> s) & 1) mbar_wait_bounded(b_kfull + 8 * s, par, p.err);
-                if ((issued >> (8 + s)) & 1) mbar_wait_bounded(b_vfull + 8 * s, par, p.err);
-            }
+            if ((issued >> 17) & 1) mbar_wait_bounded(b_vraw, 0, p.err);
+            for (int s = 0; s < KS; ++s)
+                if ((issued >> s) & 1) mbar_wait_bounded(b_kfull + 8 * s, (phase_bits >> s) & 1, p.err);
+            for (int s = 0; s < VS; ++s)
+                if ((issued >> (8 + s)) & 1)
+                    mbar_wait_bounded(b_vfull + 8 * s, (phase_bits >> (8 + s)) & 1, p.err);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
@@ -435,20 +463,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tS[2] = {tmem + 0, tmem + 128};
             const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
             bool ok = mbar_wait_bounded(b_qready, 0, p.err) && !*abort_flag;
-            auto issue_s = [&](int i, int st) {
+            auto issue_s = [&](int i, int kst) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk / 4) * Geo::kSlabBytes + (kk % 4) * 32;
                     mma_ss(tS[i], sw128_desc(sQ + i * Geo::kQBytes + off, 16, 1024),
-                           sw128_desc(sK + st * Geo::kKVBytes + off, 16, 1024), idS, kk > 0);
+                           sw128_desc(sK + kst * Geo::kKVBytes + off, 16, 1024), idS, kk > 0);
                 }
                 mma_commit(b_sfull + 8 * i);
+                if (i == 1) mma_commit(b_kempty + 8 * kst);  // both S MMAs of this K tile issued
             };
-            auto issue_pv = [&](int i, int st, int j) {
+            auto issue_pv = [&](int i, int vst, int j) {
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk)
                     mma_ts(tO[i], tS[i] + 8 * kk,
-                           sw128_desc(sV + st * Geo::kKVBytes + kk * 2048, Geo::kSlabBytes, 1024), idO,
+                           sw128_desc(sV + vst * Geo::kKVBytes + kk * 2048, Geo::kSlabBytes, 1024), idO,
                            (j > 0 || kk > 0) ? 1u : 0u);
             };
             if (ok) ok = mbar_wait_bounded(b_kfull, 0, p.err);
@@ -458,27 +487,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 issue_s(1, 0);
             }
             for (int j = 0; j < n_kv && ok; ++j) {
-                const int st = j % NS;
-                const uint32_t par = (j / NS) & 1;
-                const int st1 = (j + 1) % NS;
-                const uint32_t par1 = ((j + 1) / NS) & 1;
-                ok = mbar_wait_bounded(b_vfull + 8 * st, par, p.err) &&
+                const int vst = j % VS;
+                const uint32_t vpar = (j / VS) & 1;
+                const int kst1 = (j + 1) % KS;
+                const uint32_t kpar1 = ((j + 1) / KS) & 1;
+                ok = mbar_wait_bounded(b_vfull + 8 * vst, vpar, p.err) &&
                      mbar_wait_bounded(b_pfull + 0, j & 1, p.err);
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv(0, st, j);
+                issue_pv(0, vst, j);
                 if (j + 1 < n_kv) {
-                    ok = mbar_wait_bounded(b_kfull + 8 * st1, par1, p.err);
+                    ok = mbar_wait_bounded(b_kfull + 8 * kst1, kpar1, p.err);
                     if (!ok) break;
                     tc_fence_after();
-                    issue_s(0, st1);
+                    issue_s(0, kst1);
                 }
                 ok = mbar_wait_bounded(b_pfull + 8, j & 1, p.err);
                 if (!ok) break;
                 tc_fence_after();
-                issue_pv(1, st, j);
-                mma_commit(b_empty + 8 * st);
-                if (j + 1 < n_kv) issue_s(1, st1);
+                issue_pv(1, vst, j);
+                mma_commit(b_vempty + 8 * vst);
+                if (j + 1 < n_kv) issue_s(1, kst1);
             }
             mma_commit(b_ofinal);
             if (!ok) *abort_flag = 1;
@@ -494,18 +523,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ct = threadIdx.x - 64;
         constexpr int CPR = D / 16;  // 16-byte E4M3 chunks per row
         for (int j = 0; j < n_kv; ++j) {
-            const int st = j % NS;
-            const bool got = !*abort_flag && mbar_wait_bounded(b_stgfull, j & 1, p.err) &&
-                             mbar_wait_bounded(b_empty + 8 * st, ((j / NS) & 1) ^ 1, p.err);
-            if (!got) {
+            const int ks = j % KS, vs = j % VS;
+            if (*abort_flag || !mbar_wait_bounded(b_stgfull, j & 1, p.err)) {
                 *abort_flag = 1;
                 break;
             }
             const int key0 = j * kKeys;
+            bool got = true;
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {  // K, then V
+            for (int t = 0; t < 2; ++t) {  // K, then V (each into its own ring)
+                const uint32_t empty_b = t == 0 ? b_kempty + 8 * ks : b_vempty + 8 * vs;
+                const uint32_t par = t == 0 ? (((j / KS) & 1) ^ 1) : (((j / VS) & 1) ^ 1);
+                if (*abort_flag || !mbar_wait_bounded(empty_b, par, p.err)) {
+                    got = false;
+                    break;
+                }
                 const uint32_t src = sStg + t * Geo::kStgBytes;
-                const uint32_t dst = (t == 0 ? sK : sV) + st * Geo::kKVBytes;
+                const uint32_t dst = t == 0 ? sK + ks * Geo::kKVBytes : sV + vs * Geo::kKVBytes;
 #pragma unroll 2
                 for (int idx = ct; idx < kKeys * CPR; idx += 64) {
                     const int row = idx / CPR, c = idx % CPR;
@@ -528,10 +562,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      : "memory");
                     }
                 }
+                fence_proxy_async_smem();
+                mbar_arrive(t == 0 ? b_kfull + 8 * ks : b_vfull + 8 * vs);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(b_kfull + 8 * st);
-            mbar_arrive(b_vfull + 8 * st);
+            if (!got) {
+                *abort_flag = 1;
+                break;
+            }
             mbar_arrive(b_stgempty);
         }
     }
