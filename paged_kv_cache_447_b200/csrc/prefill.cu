@@ -191,6 +191,10 @@ struct Item {
     int n_kv;  // K/V tiles to visit
 };
 
+// Item order: (sequence, kv head) major, so the 2 x 16 items that read one (sequence, kv head)
+// K/V run on neighbouring SMs at the same time and share its tiles in L2 (row-tile-major
+// order spread them over waves, and the concurrent working set overflowed L2); inside a
+// group the heaviest (last) row tiles come first, so the light ones fill the tail.
 __device__ __forceinline__ Item decode_item(const PrefillParams &p, int idx) {
     Item it;
     const int G = p.Hq / p.Hkv;
@@ -199,20 +203,20 @@ __device__ __forceinline__ Item decode_item(const PrefillParams &p, int idx) {
         const int pairs = G / 2;
         const int pair = idx % pairs;
         int r = idx / pairs;
+        qt = p.n_qt - 1 - r % p.n_qt;
+        r /= p.n_qt;
         it.kvh = r % p.Hkv;
-        r /= p.Hkv;
-        it.b = r % p.B;
-        qt = p.n_qt - 1 - r / p.B;  // heaviest (last) row tiles first
+        it.b = r / p.Hkv;
         h0 = it.kvh * G + 2 * pair;
         h1 = h0 + 1;
         it.row0[0] = it.row0[1] = qt * kRows;
     } else {
         const int nqt2 = (p.n_qt + 1) / 2;
         int r = idx;
+        qt = nqt2 - 1 - r % nqt2;
+        r /= nqt2;
         const int h = r % p.Hq;
-        r /= p.Hq;
-        it.b = r % p.B;
-        qt = nqt2 - 1 - r / p.B;
+        it.b = r / p.Hq;
         it.kvh = h;
         h0 = h1 = h;
         it.row0[0] = 2 * qt * kRows;
@@ -588,23 +592,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the exact rotation (which pkv_rope_apply and the K rotation of pkv_kv_store
         // produce bit for bit); the difference stays far inside the attention tolerance and
         // keeps this prologue off the critical path of the tensor pipe.
+        const bool rope_row = p.rope && row_valid && it.valid[wg];
+        const bool pos_ok = pos >= 0 && pos < p.max_pos;
+        const bool same_rows = it.row0[0] == it.row0[1];
+        constexpr int NP = D / 32;  // chunk pairs per warpgroup (same-rows split)
+        const int lc0 = wg * NP;
+        float4 cv[2 * NP], sv[2 * NP];
+        if (rope_row && pos_ok && same_rows) {
+            // the table row depends only on the position: fetch it while Q is in flight
+            const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope + (size_t)pos * D);
+#pragma unroll
+            for (int k = 0; k < 2 * NP; ++k) {
+                cv[k] = __ldg(cs4 + lc0 * 2 + k);
+                sv[k] = __ldg(cs4 + D / 8 + lc0 * 2 + k);
+            }
+        }
         bool ok = mbar_wait_bounded(b_qfull, 0, p.err);
-        if (ok && p.rope && row_valid && it.valid[wg]) {
-            if (pos < 0 || pos >= p.max_pos) {
+        if (ok && rope_row) {
+            if (!pos_ok) {
                 atomicOr(p.err, kErrBounds);
-            } else if (it.row0[0] == it.row0[1]) {
+            } else if (same_rows) {
                 // Both tiles hold the same rows (two heads of a group): warpgroup wg rotates
                 // its half of the pairs of row r in both tiles, so each thread fetches half
                 // a table row, in one round.
-                constexpr int NP = D / 32;  // chunk pairs per warpgroup
-                const int lc0 = wg * NP;
-                const float4 *cs4 = reinterpret_cast<const float4 *>(p.rope + (size_t)pos * D);
-                float4 cv[2 * NP], sv[2 * NP];
-#pragma unroll
-                for (int k = 0; k < 2 * NP; ++k) {
-                    cv[k] = __ldg(cs4 + lc0 * 2 + k);
-                    sv[k] = __ldg(cs4 + D / 8 + lc0 * 2 + k);
-                }
                 const uint32_t sw = (uint32_t)(r & 7);
 #pragma unroll
                 for (int tile = 0; tile < 2; ++tile) {
