@@ -7,10 +7,11 @@
 // bound by memory bandwidth, the cache keeps growing.
 //
 // Design (HBM-bound: every cached K/V byte is streamed from HBM exactly once):
-//  * Work unit = one 16-token block of one (sequence, kv-head group) -- the group is one kv
-//    head, or for E4M3 caches with grouped heads two adjacent kv heads, so that every cache
-//    row fetched is 256 contiguous bytes (128-byte rows measured at ~60 % of the DRAM
-//    bandwidth 256-byte rows reach).  Units are numbered sequence-major; the whole unit space
+//  * Work unit = one 16-token block of one (sequence, kv-head group) -- the group is two
+//    adjacent kv heads when the kv-head count is even (else one), so that each cache slot
+//    row fetched is 2 x D x esize contiguous bytes: short rows measured far below the DRAM
+//    bandwidth long ones reach (E4M3 at D 128, idle consumers: 3.8 TB/s with 128-byte rows,
+//    5.0-5.2 TB/s with 256-byte rows).  Units are numbered sequence-major; the whole unit space
 //    is cut into equal contiguous ranges, one per persistent CTA, so every CTA streams the
 //    same number of bytes whatever the length mix.  A CTA's range crosses sequence
 //    boundaries; each piece of a (sequence, kv-head group) it covers becomes one partial
@@ -91,7 +92,10 @@ struct Geometry {
     static constexpr int kStageBytes = 2 * HPU * kTileBytes;           // K + V of the unit's heads
     static constexpr int kGroups = kConsumers / HPU;                   // consumer groups (warp per head)
     // q, probabilities and merge scratch, plus room for 1024 sequences' prefix
-    static constexpr int kExtraBytes = G * D * 4 + kConsumers * G * 16 * 4 +
+    // grouped heads on the tensor cores (bf16 caches, and E4M3 at head dim 128) keep q as bf16
+    static constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
+    static constexpr int kQFloats = kMma ? HPU * G * D / 2 : HPU * G * D;  // q scratch
+    static constexpr int kExtraBytes = kQFloats * 4 + kConsumers * G * 16 * 4 +
                                        kConsumers * G * (D + 2) * 4 + 4 * 1025;
     // ring of ~100 KB in total so that two CTAs share an SM
     // The stage count is a multiple of the consumer-group count, so that every fill of a
@@ -256,9 +260,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Offset of the 16-byte chunk c of row t (0..15) in a swizzled tile: slabs of 16 rows x
-// 128 bytes (64 bf16 columns, or a whole 128-byte E4M3 row), 2 KB apart.
+// 128 bytes (64 bf16 columns, or a whole 128-byte E4M3 row), kSlabStride bytes apart (the
+// heads of a unit interleave by slab: 2 KB x heads per unit).
+template <int kSlabStride>
 __device__ __forceinline__ uint32_t swz(int t, int c) {
-    return (uint32_t)((c >> 3) * 2048 + t * 128 + (((c & 7) ^ (t & 7)) << 4));
+    return (uint32_t)((c >> 3) * kSlabStride + t * 128 + (((c & 7) ^ (t & 7)) << 4));
 }
 
 template <int D, bool FP8, int G, int HPU>
@@ -270,17 +276,18 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
     constexpr int NS = Geo::kStages;
     constexpr int kConsumers = Geo::kConsumers;
     constexpr int kThreads = Geo::kThreads;
-    // grouped heads on the tensor cores: bf16 caches, and E4M3 caches at head dim 128
-    constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
+    constexpr bool kMma = Geo::kMma;  // grouped heads on the tensor cores
     constexpr int kSlabs = Geo::kRowBytes / 128;  // swizzled boxes per tile (kMma)
-    static_assert(HPU == 1 || (kMma && kSlabs == 1), "two heads per unit: one-slab tiles only");
+    constexpr int kSlabStride = HPU * 2048;       // swizzled slabs of a unit's heads interleave
+    // a head's tile inside a stage (K tiles, then V tiles): swizzled tiles interleave by slab
+    constexpr int kHeadStride = kMma ? 2048 : Geo::kTileBytes;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *stages = smem;                                                  // NS x stage
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + NS * Geo::kStageBytes);
     uint64_t *empty = full + NS;
-    float *qs = reinterpret_cast<float *>(empty + NS);                      // [G][quads][chunks][4]
-    float *pbuf = qs + G * D;                                                // [consumers][G][16]
+    float *qs = reinterpret_cast<float *>(empty + NS);                      // [HPU][G][quads][chunks][4]
+    float *pbuf = qs + Geo::kQFloats;                                        // [consumers][G][16]
     float *mrg = pbuf + kConsumers * G * 16;                                 // [consumers][G][D+2]
     int *pfx = reinterpret_cast<int *>(mrg + kConsumers * G * (D + 2));      // [B+1]
     __shared__ volatile int abort_s;
@@ -350,10 +357,15 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                         const uint32_t dst = smem_u32(stages + s * Geo::kStageBytes);
                         mbar_arrive_expect_tx(fb, Geo::kStageBytes);
                         if constexpr (HPU == 2) {
-                            // one box per tensor: 16 slots x 2 adjacent heads (256 contiguous
-                            // bytes per slot), landing as the two heads' swizzled tiles
-                            tma_load_3d(dst, &tm_k, fb, 0, ph * kBlockSize, 2 * hh);
-                            tma_load_3d(dst + 2 * Geo::kTileBytes, &tm_v, fb, 0, ph * kBlockSize, 2 * hh);
+                            // one box per tensor (per slab when swizzled): 16 slots x 2 adjacent
+                            // heads, landing as the two heads' tiles (slab-interleaved)
+#pragma unroll
+                            for (int h = 0; h < (kMma ? kSlabs : 1); ++h) {
+                                const int x = kMma ? h * (128 / Geo::kElem) : 0;
+                                tma_load_3d(dst + h * kSlabStride, &tm_k, fb, x, ph * kBlockSize, 2 * hh);
+                                tma_load_3d(dst + 2 * Geo::kTileBytes + h * kSlabStride, &tm_v, fb, x,
+                                            ph * kBlockSize, 2 * hh);
+                            }
                         } else if constexpr (kMma) {
                             // one swizzled box per 64-column slab
 #pragma unroll
@@ -465,7 +477,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                 qh[i + D / 2] = x2;
                 continue;
             }
-            const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvh) : 1.f);
+            const float sc = p.scale_log2 * (FP8 ? __ldg(p.k_scale + kvg * HPU + hh) : 1.f);
             const int idx[2] = {i, i + D / 2};
             const float val[2] = {__uint_as_float((uint32_t)x1 << 16) * sc,
                                   __uint_as_float((uint32_t)x2 << 16) * sc};
@@ -474,7 +486,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                 const int dim = idx[r];
                 const int c = dim / Geo::kChunkElems, w = dim % Geo::kChunkElems;
                 const int quad = w / 4, comp = w % 4;
-                qs[((g * Geo::kQuads + quad) * Geo::kChunks + c) * 4 + comp] = val[r];
+                qs[hh * G * D + ((g * Geo::kQuads + quad) * Geo::kChunks + c) * 4 + comp] = val[r];
             }
         }
         named_bar(kMergeBar, kConsumers * 32);
@@ -512,7 +524,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
             const int blk = cur.blk + j;
             const int valid = min(kBlockSize, L - blk * kBlockSize);
             // this warp's head: K tile hsel, then V tile hsel after the HPU K tiles
-            const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes) + hsel * Geo::kTileBytes;
+            const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes) + hsel * kHeadStride;
             const uint32_t vs_a = ks_a + HPU * Geo::kTileBytes;
             if constexpr (kMma) {
                 // S = Q K^T: n tile 0 = tokens 0-7, n tile 1 = tokens 8-15.  ldmatrix x4
@@ -526,8 +538,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         const int t = 8 * nt + row;
-                        const uint4 k0 = lds128(ks_a + swz(t, 2 * q4));
-                        const uint4 k1 = lds128(ks_a + swz(t, 2 * q4 + 1));
+                        const uint4 k0 = lds128(ks_a + swz<kSlabStride>(t, 2 * q4));
+                        const uint4 k1 = lds128(ks_a + swz<kSlabStride>(t, 2 * q4 + 1));
                         const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
                         for (int ks = 0; ks < kMT; ++ks)
@@ -539,7 +551,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
 #pragma unroll
                     for (int ks = 0; ks < kMT; ++ks) {
                         uint32_t b[4];
-                        ldsm_x4(ks_a + swz(tk, 2 * ks + hk), b);
+                        ldsm_x4(ks_a + swz<kSlabStride>(tk, 2 * ks + hk), b);
                         mma_rows8(sa[0], qa[ks][0], qa[ks][1], b[0], b[1]);
                         mma_rows8(sa[1], qa[ks][0], qa[ks][1], b[2], b[3]);
                     }
@@ -557,7 +569,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                     constexpr int kRowChunks = Geo::kRowBytes / 16;
                     for (int e = lane; e < (kBlockSize - valid) * kRowChunks; e += 32) {
                         const int t = valid + e / kRowChunks, c = e % kRowChunks;
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vs_a + swz(t, c)),
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vs_a + swz<kSlabStride>(t, c)),
                                      "r"(0u) : "memory");
                     }
                     fence_proxy_async_smem();  // before the stage is refilled by TMA
@@ -597,8 +609,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                     // rows, regrouped into token pairs by byte permutes, then widened.
                     const uint32_t pb01 = pack_f16x2(pr[0], pr[1]), pb23 = pack_f16x2(pr[2], pr[3]);
                     const int tA = 2 * q4;
-                    const uint4 vA = lds128(vs_a + swz(tA, row)), vB = lds128(vs_a + swz(tA + 1, row));
-                    const uint4 vC = lds128(vs_a + swz(tA + 8, row)), vD = lds128(vs_a + swz(tA + 9, row));
+                    const uint4 vA = lds128(vs_a + swz<kSlabStride>(tA, row)), vB = lds128(vs_a + swz<kSlabStride>(tA + 1, row));
+                    const uint4 vC = lds128(vs_a + swz<kSlabStride>(tA + 8, row)), vD = lds128(vs_a + swz<kSlabStride>(tA + 9, row));
                     const uint32_t wA[4] = {vA.x, vA.y, vA.z, vA.w}, wB[4] = {vB.x, vB.y, vB.z, vB.w};
                     const uint32_t wC[4] = {vC.x, vC.y, vC.z, vC.w}, wD[4] = {vD.x, vD.y, vD.z, vD.w};
 #pragma unroll
@@ -623,7 +635,7 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
 #pragma unroll
                     for (int mt2 = 0; mt2 < kMT; ++mt2) {
                         uint32_t a[4];
-                        ldsm_x4_trans(vs_a + swz(tv, 2 * mt2 + hv), a);
+                        ldsm_x4_trans(vs_a + swz<kSlabStride>(tv, 2 * mt2 + hv), a);
                         const uint32_t af[4] = {a[0], a[1], a[2], a[3]};
                         mma_full(o[mt2], af, pb01, pb23);
                     }
@@ -676,7 +688,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                 for (int g = 0; g < G; ++g) {
 #pragma unroll
                     for (int qd = 0; qd < Geo::kQuads; ++qd) {
-                        const float4 qv = lds128f(qs_a + (((g * Geo::kQuads + qd) * Geo::kChunks + c) * 16));
+                        const float4 qv = lds128f(qs_a + hsel * G * D * 4 +
+                                                  (((g * Geo::kQuads + qd) * Geo::kChunks + c) * 16));
 #pragma unroll
                         for (int u = 0; u < kTPL; ++u) {
                             sacc[g][u] = __ffma2_rn(make_float2(kf[u][4 * qd + 0], kf[u][4 * qd + 1]),
@@ -935,7 +948,7 @@ size_t smem_bytes(int B) {
     using Geo = Geometry<D, FP8, G, HPU>;
     constexpr int kConsumers = Geo::kConsumers;
     size_t s = (size_t)Geo::kStages * Geo::kStageBytes + 2 * Geo::kStages * sizeof(uint64_t);
-    s += (size_t)G * D * 4 + (size_t)kConsumers * G * 16 * 4 + (size_t)kConsumers * G * (D + 2) * 4;
+    s += (size_t)Geo::kQFloats * 4 + (size_t)kConsumers * G * 16 * 4 + (size_t)kConsumers * G * (D + 2) * 4;
     s += (size_t)(B + 1) * 4;
     return s + 1024;  // alignment slack for the swizzled stages
 }
@@ -961,14 +974,15 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
     //   heads lands as the two heads' tiles back to back, fetched 256 bytes at a time.
     CUtensorMap tk, tv;
     const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
-    constexpr bool kMma = G >= 2 && (!FP8 || D == 128);
+    constexpr bool kMma = Geo::kMma;
     bool ok;
     if constexpr (HPU == 2) {
         const uint64_t row = (uint64_t)a.n_kv_heads * D * Geo::kElem, head = (uint64_t)D * Geo::kElem;
+        const uint32_t box0 = kMma ? 128u / Geo::kElem : (uint32_t)D;
         ok = encode_tensor_map_3d_strided(&tk, a.k_cache, Geo::kElem, D, slots, a.n_kv_heads, row, head,
-                                          D, kBlockSize, 2, true, 256) &&
+                                          box0, kBlockSize, 2, kMma, 256) &&
              encode_tensor_map_3d_strided(&tv, a.v_cache, Geo::kElem, D, slots, a.n_kv_heads, row, head,
-                                          D, kBlockSize, 2, true, 256);
+                                          box0, kBlockSize, 2, kMma, 256);
     } else {
         const uint32_t box0 = kMma ? 128u / Geo::kElem : (uint32_t)D;
         ok = encode_tensor_map_3d(&tk, a.k_cache, Geo::kElem, D, a.n_kv_heads, slots, box0, 1, kBlockSize, kMma) &&
@@ -985,8 +999,12 @@ cudaError_t launch_t(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t 
 
 template <int D, bool FP8, int G>
 cudaError_t launch_h(const DecodeParams &prm, const DecodeArgs &a, cudaStream_t s) {
-    // E4M3 rows of one head are 128 bytes: grouped heads fetch two heads per unit
-    if constexpr (FP8 && D == 128 && G >= 2)
+    // Two adjacent kv heads per unit (longer contiguous rows) when the kv-head count is even,
+    // for the CUDA-core consumers and for tensor-core tiles of one 128-byte slab.  Measured:
+    // MHA bf16 D 128 5.90 -> 6.12 TB/s, E4M3 grouped 3.8 -> 4.1 TB/s; bf16 grouped D 128
+    // (two slabs per row) loses ring depth and ran 15 % slower, so it keeps one head.
+    constexpr bool kTwo = !Geometry<D, FP8, G, 1>::kMma || D * (FP8 ? 1 : 2) <= 128;
+    if constexpr (kTwo)
         if (a.n_kv_heads % 2 == 0) return launch_t<D, FP8, G, 2>(prm, a, s);
     return launch_t<D, FP8, G, 1>(prm, a, s);
 }
