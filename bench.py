@@ -315,6 +315,20 @@ class Runner:
         return sum(ts) / len(ts)
 
 
+def workload_config(name: str, wl, layers: int, world: int) -> dict:
+    """The `config` object of the JSON line (both arms): the workload and its shape."""
+    st = wl.steps[-1]
+    B = st.decode_seqs
+    esize = 1 if wl.cache_dtype == "fp8" else 2
+    kv = decode_kv_bytes(st, wl.n_kv_heads, wl.head_dim, esize) * layers if B else 0
+    return {"workload": name, "batch": B or (st.num_seqs - B),
+            "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
+            "head_dim": wl.head_dim, "block_size": 16, "layers": layers,
+            "context": wl.notes.get("context", None),
+            "l2": f"inputs larger than L2 (KV bytes per step {kv / 1e9:.2f} GB), no flush",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 def build_workload(name: str, layers=None):
     if name == "qwen_decode":
         return W.qwen_decode(seed=2), 1
@@ -478,7 +492,8 @@ def main():
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": r["seconds"] * 1e3, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": args.workload, "sample": r["sample"]},
+                "config": dict(workload_config(args.workload, *build_workload(args.workload, args.layers),
+                                               world), sample=r["sample"]),
                 "cpu_baseline": {"value": r["value"], "unit": r["unit"], "cores": r["cores"],
                                  "kind": "oracle", "sample": r["sample"]},
                 "e2e": {"value": r["value"], "unit": r["unit"], "h2d_bytes_per_step": 0,
@@ -513,13 +528,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": res["step_ms"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if esize == 2 else "e4m3",
         "data": "synthetic",
-        "config": {"workload": args.workload, "batch": runner.B or runner.P,
-                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads,
-                   "head_dim": wl.head_dim, "block_size": 16, "layers": res["layers"],
-                   "context": wl.notes.get("context", None),
-                   "l2": "inputs larger than L2 (KV bytes per step "
-                         f"{res.get('decode_kv_bytes_per_step', 0) / 1e9:.2f} GB), no flush",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": workload_config(args.workload, wl, res["layers"], world),
         "decode_tok_s_per_layer": res.get("decode_tok_s_per_layer"),
         "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": runit,
                      "frac": ach / peak,
