@@ -32,6 +32,12 @@ function               passage                                               pin
                                                                              prefix invariance
 ``kv_cache_bytes``     2 x layers x kv_heads x head_dim x tokens x bytes     printed sizes ("LLM primer",
                        ("LLM primer", §17.3, §17.6)                          §17.3, §17.6, §23.2 exp. 2)
+``slot_mapping``       block table lists a sequence's physical blocks, 16    hand-worked example
+                       tokens each ("Inside the Nano-vLLM engine", §2.2)     (tests/golden); brute-force
+                                                                             enumeration of each table's
+                                                                             slots; -1 past the table
+``copy_blocks``        shared prefix blocks, copy on write ("Inside the      numpy block slicing: dst
+                       Nano-vLLM engine", §2.2; "LLM primer", §17.7)         equals old src, rest unchanged
 =====================  ====================================================  ===========================
 """
 from __future__ import annotations
@@ -94,6 +100,10 @@ def _load():
         lib.orc_attention_weights.argtypes = [P, P, P, P, I, P, I, I, I, I, I, I, D, P, I, I, P]
         lib.orc_attention_weights.restype = None
         lib.orc_kv_cache_bytes.argtypes = [ctypes.c_int64] * 5
+        lib.orc_slot_mapping.argtypes = [P, P, I, P, P, I, I, ctypes.c_int64]
+        lib.orc_slot_mapping.restype = None
+        lib.orc_copy_blocks.argtypes = [P, P, P, I, ctypes.c_int64, ctypes.c_int64]
+        lib.orc_copy_blocks.restype = None
         lib.orc_kv_cache_bytes.restype = ctypes.c_int64
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = ctypes.c_int
@@ -249,6 +259,27 @@ def kv_cache_bytes(num_layers: int, n_kv_heads: int, head_dim: int, cached_token
                    bytes_per_element: int) -> int:
     return int(_load().orc_kv_cache_bytes(num_layers, n_kv_heads, head_dim, cached_tokens,
                                           bytes_per_element))
+
+
+def slot_mapping(block_tables, cu_seqlens, context_lens, block_size: int,
+                 num_blocks: int) -> np.ndarray:
+    """int32 slot of every new token of the batch (-1 past the table / bad block id)."""
+    bt = _c(block_tables, np.int32)
+    cu = _c(cu_seqlens, np.int32)
+    cl = _c(context_lens, np.int32)
+    out = np.full(int(cu[-1]), -1, dtype=np.int32)
+    _load().orc_slot_mapping(_ptr(out), _ptr(bt), bt.shape[1], _ptr(cu), _ptr(cl), len(cl),
+                             block_size, num_blocks)
+    return out
+
+
+def copy_blocks(k_cache, v_cache, pairs) -> None:
+    """In place: block dst of both caches (numpy, [NB, ...]) becomes a copy of block src."""
+    pr = _c(np.asarray(pairs).reshape(-1, 2), np.int32)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    nb = k_cache.shape[0]
+    block_bytes = k_cache.nbytes // nb
+    _load().orc_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pr), pr.shape[0], block_bytes, nb)
 
 
 def num_threads() -> int:

@@ -211,6 +211,54 @@ void orc_kv_store(const uint16_t *k, const uint16_t *v, void *k_cache, void *v_c
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Block bookkeeping: slots of new tokens, copy-on-write block copies                   */
+/* ------------------------------------------------------------------------------------ */
+
+/* [ENG] §2.2: a sequence's block table lists the physical blocks that hold its tokens,
+ * in order, block_size tokens per block.  The token at position p of sequence b is
+ * therefore the (p mod block_size)-th slot of the (p div block_size)-th block of its
+ * table, i.e. slot = table[p / block_size] * block_size + p % block_size.  New token r of
+ * sequence b is at p = L_b - n_b + r.  A position past the table or a table entry outside
+ * [0, num_blocks) gives slot -1 (and no store). */
+void orc_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables, int max_blocks,
+                      const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                      int block_size, int64_t num_blocks)
+{
+    for (int b = 0; b < num_seqs; ++b) {
+        int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        for (int r = 0; r < n; ++r) {
+            int64_t p = (int64_t)context_lens[b] - n + r;
+            int32_t slot = -1;
+            if (p >= 0 && p < (int64_t)max_blocks * block_size) {
+                int32_t blk = block_tables[(size_t)b * max_blocks + (size_t)(p / block_size)];
+                if (blk >= 0 && blk < num_blocks)
+                    slot = (int32_t)((int64_t)blk * block_size + p % block_size);
+            }
+            slot_mapping[cu_seqlens[b] + r] = slot;
+        }
+    }
+}
+
+/* [ENG] §2.2 (requests that share a prefix point at the same physical blocks; a shared
+ * block is copied when one of them writes to it: copy on write) and [PRM] §17.7.  For each
+ * pair (src, dst): block dst of both caches becomes a byte copy of block src.  Pairs are
+ * applied in order; ids outside [0, num_blocks) skip the pair.  block_bytes is the size of
+ * one block of one cache (block_size * n_kv_heads * head_dim * element size). */
+void orc_copy_blocks(uint8_t *k_cache, uint8_t *v_cache, const int32_t *pairs, int num_pairs,
+                     int64_t block_bytes, int64_t num_blocks)
+{
+    for (int i = 0; i < num_pairs; ++i) {
+        int32_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks || src == dst)
+            continue;
+        for (int64_t j = 0; j < block_bytes; ++j) {
+            k_cache[(int64_t)dst * block_bytes + j] = k_cache[(int64_t)src * block_bytes + j];
+            v_cache[(int64_t)dst * block_bytes + j] = v_cache[(int64_t)src * block_bytes + j];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Attention over the paged cache                                                       */
 /* ------------------------------------------------------------------------------------ */
 

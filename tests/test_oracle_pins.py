@@ -496,3 +496,105 @@ def test_planted_mistakes_are_caught():
     short = oracle.attention(W.bits(pre.q), kc, vc, pre.cu_seqlens.numpy(), bt,
                              pre.context_lens.numpy() - 1, wl.scale, 16, 2)
     assert np.max(np.abs(short - ref)) > 1e-3
+
+
+# ----------------------------------------------------------------------------- block bookkeeping
+
+SLOT_EXAMPLE = dict(tables=[[7, 2, 9], [5, -1, -1], [4, 0, -1], [6, 3, -1]],
+                    ctx=[20, 1, 32, 17], new=[3, 1, 2, 17])
+
+
+def _cu(new):
+    return np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+
+
+def test_slot_mapping_hand_worked_example():
+    rows = _golden_rows("slot_mapping.txt")
+    got = oracle.slot_mapping(np.array(SLOT_EXAMPLE["tables"], np.int32), _cu(SLOT_EXAMPLE["new"]),
+                              np.array(SLOT_EXAMPLE["ctx"], np.int32), 16, 10)
+    assert [int(x) for x in got] == [int(r[1]) for r in rows]
+
+
+def test_slot_mapping_brute_force_enumeration():
+    """Enumerate each sequence's slots block by block in table order (the p-th entry is
+    the slot of position p) and take the last n_b: no division or modulo involved."""
+    g = np.random.default_rng(5)
+    bs, nb = 16, 64
+    for _ in range(30):
+        B = int(g.integers(1, 6))
+        lens = g.integers(1, 120, B)
+        new = [int(g.integers(1, L + 1)) for L in lens]
+        maxb = int((lens.max() + bs - 1) // bs) + 1
+        perm = g.permutation(nb)
+        tables = np.full((B, maxb), -1, np.int32)
+        cur = 0
+        for b in range(B):
+            k = int((lens[b] + bs - 1) // bs)
+            tables[b, :k] = perm[cur:cur + k]
+            cur += k
+        got = oracle.slot_mapping(tables, _cu(new), lens.astype(np.int32), bs, nb)
+        exp = []
+        for b in range(B):
+            enum = [int(blk) * bs + o for blk in tables[b] if blk >= 0 for o in range(bs)]
+            exp += enum[int(lens[b]) - new[b]:int(lens[b])]
+        assert got.tolist() == exp
+
+
+def test_slot_mapping_out_of_table_is_minus_one():
+    bt = np.array([[3, -1]], np.int32)
+    assert oracle.slot_mapping(bt, [0, 1], [17], 16, 8).tolist() == [-1]   # entry -1
+    assert oracle.slot_mapping(bt, [0, 1], [33], 16, 8).tolist() == [-1]   # past the table
+    assert oracle.slot_mapping(np.array([[9]], np.int32), [0, 1], [1], 16, 8).tolist() == [-1]
+    assert oracle.slot_mapping(bt, [0, 2], [1], 16, 8).tolist() == [-1, 48]  # position -1, 0
+
+
+def test_copy_blocks_copies_whole_blocks_only():
+    g = np.random.default_rng(7)
+    for dtype, hi in ((np.uint16, 2 ** 16), (np.uint8, 256)):
+        kc = g.integers(0, hi, size=(12, 16, 2, 64)).astype(dtype)
+        vc = g.integers(0, hi, size=(12, 16, 2, 64)).astype(dtype)
+        k0, v0 = kc.copy(), vc.copy()
+        oracle.copy_blocks(kc, vc, [(3, 7), (0, 11), (5, 5), (2, 99), (-1, 4)])
+        ek, ev = k0.copy(), v0.copy()
+        ek[7], ev[7] = k0[3], v0[3]
+        ek[11], ev[11] = k0[0], v0[0]
+        assert np.array_equal(kc, ek) and np.array_equal(vc, ev)
+
+
+def test_copy_on_write_divergence_equals_private_copy():
+    """Two sequences share the blocks of a 24-token prefix (the second block half full).
+    Before either appends, sequence 1 takes a private copy of the shared partial block
+    (copy on write) and points its table there; then each stores its own next token through
+    its slots.  Attention for both must equal the result on fully private caches, and the
+    shared full block must be untouched."""
+    g = torch.Generator().manual_seed(11)
+    hq, hkv, d, bs, nb = 4, 2, 64, 16, 8
+    prefix = W._randn_bf16(g, 24, hkv, d), W._randn_bf16(g, 24, hkv, d)
+    tails = [(W._randn_bf16(g, 1, hkv, d), W._randn_bf16(g, 1, hkv, d)) for _ in range(2)]
+    q = W._randn_bf16(g, 2, hq, d)
+
+    def store(kc, vc, bt, b, ctx, rows):
+        slots = oracle.slot_mapping(bt[b:b + 1], [0, rows[0].shape[0]], [ctx], bs, nb)
+        oracle.kv_store(W.bits(rows[0]), W.bits(rows[1]), kc, vc, slots, bs)
+
+    kc = np.zeros((nb, bs, hkv, d), np.uint16)
+    vc = np.zeros((nb, bs, hkv, d), np.uint16)
+    shared = np.array([[0, 1, -1], [0, 1, -1]], np.int32)
+    store(kc, vc, shared, 0, 24, prefix)                 # the prefix, once, in blocks 0-1
+    before = kc[0].copy()
+    oracle.copy_blocks(kc, vc, [(1, 5)])                 # copy on write for sequence 1
+    bt = np.array([[0, 1, -1], [0, 5, -1]], np.int32)
+    for b in range(2):
+        store(kc, vc, bt, b, 25, tails[b])
+    kp = np.zeros_like(kc)
+    vp = np.zeros_like(vc)
+    private = np.array([[0, 1, -1], [2, 3, -1]], np.int32)
+    for b in range(2):
+        store(kp, vp, private, b, 24, prefix)
+        store(kp, vp, private, b, 25, tails[b])
+    cu = np.array([0, 1, 2], np.int32)
+    ctx = np.array([25, 25], np.int32)
+    got = oracle.attention(W.bits(q), kc, vc, cu, bt, ctx, d ** -0.5, bs, hkv)
+    ref = oracle.attention(W.bits(q), kp, vp, cu, private, ctx, d ** -0.5, bs, hkv)
+    assert np.array_equal(got, ref)
+    assert np.array_equal(kc[0], before)
