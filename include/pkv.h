@@ -122,6 +122,42 @@ int pkv_kv_store(const void *k, const void *v, void *k_cache, void *v_cache,
                  pkv_stream_t stream);
 
 /*
+ * pkv_slot_mapping -- the cache slot of every new token of a batch, from the block tables
+ * (ENG §2.2: a sequence's block table lists the physical blocks holding its tokens, in
+ * order, block_size tokens each).  New token r of sequence b sits at position
+ * p = L_b - n_b + r (see Batches), i.e. at offset p % block_size of physical block
+ * block_tables[b][p / block_size]:
+ *     slot_mapping[t] = block_tables[b][p / block_size] * block_size + p % block_size
+ * This is the slot_mapping that pkv_kv_store takes.
+ *   slot_mapping  [num_tokens] int32, written; num_tokens = cu_seqlens[num_seqs]
+ *   block_tables, max_blocks_per_seq, cu_seqlens, context_lens, num_seqs: see Tables and
+ *                 Batches; num_blocks: physical blocks of the cache (bounds check only)
+ * Bit-exact (integer arithmetic).  Device errors: a position outside
+ * [0, max_blocks_per_seq * block_size) or a table entry outside [0, num_blocks) ->
+ * PKV_E_BOUNDS flag, that token's slot is -1 (so a following store skips it).
+ */
+int pkv_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                     int num_tokens, int block_size, long long num_blocks, pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks -- copy whole physical blocks of the K and V caches, src -> dst, for
+ * every pair: the copy-on-write step when sequences that share the blocks of a common
+ * prefix diverge (ENG §2.2: requests with a common prefix point at the same physical
+ * blocks, copied on write; PRM §17.7).
+ *   k_cache,
+ *   v_cache       cache tensors (see Cache); blocks dst are overwritten
+ *   block_pairs   [num_pairs, 2] int32: (src, dst) physical block ids
+ * Every slot and head of the block is copied byte for byte (bf16 values or E4M3 codes; the
+ * per-head scales are shared, so codes stay valid).  No dst may appear as a src or dst of
+ * another pair of the same call (the copies run concurrently); src == dst is a no-op.
+ * Device errors: an id outside [0, num_blocks) -> PKV_E_BOUNDS flag, that pair is skipped.
+ */
+int pkv_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, int num_pairs,
+                    int n_kv_heads, int head_dim, int block_size, long long num_blocks,
+                    int cache_dtype, pkv_stream_t stream);
+
+/*
  * pkv_rope_apply -- rotate q [num_tokens, n_q_heads, head_dim] and k [num_tokens,
  * n_kv_heads, head_dim] (bf16) IN PLACE at each token's position (PRM §21.2, ENG §3.2).
  * Either q or k may be NULL.  Device errors: position outside [0, max_pos) ->

@@ -66,6 +66,8 @@ def load_library():
                                          P, P, P, I, I, P], I),
         "pkv_paged_decode_attention_noalloc": ([P, P, P, P, P, I, P, I, I, I, I, I, LL, F, I,
                                                 P, P, P, I, P], I),
+        "pkv_slot_mapping": ([P, P, I, P, P, I, I, I, LL, P], I),
+        "pkv_copy_blocks": ([P, P, P, I, I, I, I, LL, I, P], I),
         "pkv_get_error": ([P], I),
         "pkv_debug_wait_timeout": ([LL, P], I),
     }
@@ -157,6 +159,31 @@ def kv_store(k, v, k_cache, v_cache, slot_mapping, *, k_scale=None, v_scale=None
         _cache_dtype(k_cache), _p(k_scale), _p(v_scale), _p(rope_cos_sin), max_pos,
         _p(_i32(cu_seqlens, "cu_seqlens")), _p(_i32(context_lens, "context_lens")), B,
         _stream(stream)))
+
+
+def slot_mapping(block_tables, cu_seqlens, context_lens, num_tokens: int, num_blocks: int, *,
+                 block_size: int = 16, out=None, stream=None) -> torch.Tensor:
+    """int32 [num_tokens] cache slot of every new token (num_tokens = cu_seqlens[-1])."""
+    _i32(block_tables, "block_tables"); _i32(cu_seqlens, "cu_seqlens")
+    _i32(context_lens, "context_lens")
+    if out is None:
+        out = torch.empty(num_tokens, dtype=torch.int32, device=block_tables.device)
+    _i32(out, "out")
+    _check("pkv_slot_mapping", load_library().pkv_slot_mapping(
+        _p(out), _p(block_tables), block_tables.shape[1], _p(cu_seqlens), _p(context_lens),
+        context_lens.shape[0], num_tokens, block_size, num_blocks, _stream(stream)))
+    return out
+
+
+def copy_blocks(k_cache, v_cache, block_pairs, *, stream=None) -> None:
+    """Copy physical blocks src -> dst of both caches for every (src, dst) row of the int32
+    [n, 2] block_pairs (copy on write)."""
+    _i32(block_pairs, "block_pairs")
+    NB, bs, H, D = k_cache.shape
+    n = block_pairs.shape[0] if block_pairs.numel() else 0
+    _check("pkv_copy_blocks", load_library().pkv_copy_blocks(
+        _p(k_cache), _p(v_cache), _p(block_pairs) if n else None, n, H, D, bs, NB,
+        _cache_dtype(k_cache), _stream(stream)))
 
 
 def rope_apply(q, k, rope_cos_sin, cu_seqlens, context_lens, *, stream=None) -> None:

@@ -194,6 +194,41 @@ int pkv_kv_store(const void *k, const void *v, void *k_cache, void *v_cache,
     return status_of(launch_kv_store(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int pkv_slot_mapping(int32_t *slot_mapping, const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                     int num_tokens, int block_size, long long num_blocks, pkv_stream_t stream) {
+    if (block_size != kBlockSize) return PKV_E_UNSUPPORTED;
+    if (num_tokens < 0 || num_seqs < 0 || max_blocks_per_seq < 0 || num_blocks < 0)
+        return PKV_E_INVALID;
+    if (num_blocks * (long long)block_size >= (1LL << 31)) return PKV_E_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!slot_mapping || !block_tables || !cu_seqlens || !context_lens || num_seqs == 0 ||
+        max_blocks_per_seq == 0)
+        return PKV_E_INVALID;
+    int *err = error_word();
+    if (!err) return PKV_E_CUDA;
+    SlotArgs a{slot_mapping, block_tables, max_blocks_per_seq, cu_seqlens, context_lens,
+               num_seqs, num_tokens, num_blocks, err};
+    return status_of(launch_slot_mapping(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int pkv_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, int num_pairs,
+                    int n_kv_heads, int head_dim, int block_size, long long num_blocks,
+                    int cache_dtype, pkv_stream_t stream) {
+    int st = check_cache_shape(n_kv_heads, head_dim, block_size, num_blocks, cache_dtype);
+    if (st) return st;
+    if (num_pairs < 0) return PKV_E_INVALID;
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !block_pairs) return PKV_E_INVALID;
+    if (!aligned16(k_cache) || !aligned16(v_cache)) return PKV_E_ALIGN;
+    int *err = error_word();
+    if (!err) return PKV_E_CUDA;
+    const long long esize = cache_dtype == PKV_FP8_E4M3 ? 1 : 2;
+    CopyArgs a{k_cache, v_cache, block_pairs, num_pairs,
+               (long long)block_size * n_kv_heads * head_dim * esize, num_blocks, err};
+    return status_of(launch_copy_blocks(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int pkv_rope_apply(void *q, void *k, const float *rope_cos_sin, int max_pos,
                    const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
                    int num_tokens, int n_q_heads, int n_kv_heads, int head_dim,

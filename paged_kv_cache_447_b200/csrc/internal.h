@@ -69,6 +69,25 @@ struct PrefillArgs {
     int *err;
 };
 
+struct SlotArgs {
+    int32_t *slot_mapping;
+    const int32_t *block_tables;
+    int max_blocks;
+    const int32_t *cu_seqlens, *context_lens;
+    int num_seqs, num_tokens;
+    long long num_blocks;
+    int *err;
+};
+
+struct CopyArgs {
+    void *k_cache, *v_cache;
+    const int32_t *pairs;  // [num_pairs][2] (src, dst)
+    int num_pairs;
+    long long block_bytes;  // one block of one cache
+    long long num_blocks;
+    int *err;
+};
+
 // 3-D tiled TMA descriptor over a row-major [d2][d1][d0] tensor of `esize`-byte elements
 // (bf16 or bytes), box b0 x b1 x b2, optionally 128-byte swizzled.  Each launcher encodes
 // the maps its kernel reads, from the same compile-time geometry the kernel uses.
@@ -88,6 +107,8 @@ size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int h
                               int num_sms);
 cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_wait_timeout(unsigned long long limit_ns, int *err, cudaStream_t s);
+cudaError_t launch_slot_mapping(const SlotArgs &a, cudaStream_t s);
+cudaError_t launch_copy_blocks(const CopyArgs &a, cudaStream_t s);
 
 // Number of persistent decode CTAs the library launches on a device with `num_sms` SMs.
 int decode_grid_ctas(int num_sms);

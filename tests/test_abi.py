@@ -83,6 +83,27 @@ def test_host_argument_checks_need_no_device():
     assert lib.pkv_rope_build_table(p, 4, 63, 1e4) == -1
 
 
+def test_block_helpers_host_checks_need_no_device():
+    lib = binding.load_library()
+    n = None
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
+    # slot mapping: block size 8 not compiled; negative sizes; null pointers; empty is a no-op
+    assert lib.pkv_slot_mapping(p, p, 4, p, p, 2, 5, 8, 32, n) == -2
+    assert lib.pkv_slot_mapping(p, p, 4, p, p, -1, 5, 16, 32, n) == -1
+    assert lib.pkv_slot_mapping(n, p, 4, p, p, 2, 5, 16, 32, n) == -1
+    assert lib.pkv_slot_mapping(p, p, 0, p, p, 2, 5, 16, 32, n) == -1
+    assert lib.pkv_slot_mapping(n, n, 4, n, n, 2, 0, 16, 32, n) == 0
+    # slots are int32: num_blocks * block_size must stay below 2^31
+    assert lib.pkv_slot_mapping(p, p, 4, p, p, 2, 5, 16, 1 << 27, n) == -2
+    # block copies: shape checks, null pairs, misaligned cache, empty is a no-op
+    assert lib.pkv_copy_blocks(p, p, p, 1, 2, 96, 16, 32, 0, n) == -2
+    assert lib.pkv_copy_blocks(p, p, n, 1, 2, 64, 16, 32, 0, n) == -1
+    assert lib.pkv_copy_blocks(p, p, p, -1, 2, 64, 16, 32, 0, n) == -1
+    assert lib.pkv_copy_blocks(ctypes.c_void_p(p.value + 4), p, p, 1, 2, 64, 16, 32, 0, n) == -7
+    assert lib.pkv_copy_blocks(n, n, n, 0, 2, 64, 16, 32, 0, n) == 0
+
+
 def test_workspace_size_is_positive_and_monotone():
     a = pkv.decode_workspace_bytes(64, 32, 32, 128)
     b = pkv.decode_workspace_bytes(128, 32, 32, 128)
