@@ -181,20 +181,29 @@ def prefill_flops(st: W.Step, hq: int, d: int) -> float:
     return float(4 * d * hq * int(pairs))
 
 
+def code_sha256(path: str) -> str:
+    """sha256 of a C/CUDA source with comments and whitespace removed: it changes when the
+    code changes, not when only its comments do."""
+    import hashlib
+    import re
+    src = open(path, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    src = re.sub(r"\s+", "", src)
+    return hashlib.sha256(src.encode()).hexdigest()
+
+
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch (read + write) from the committed ncu record in profiles/, or
-    None if there is none for this kernel and workload or the kernel source has changed
+    None if there is none for this kernel and workload or the kernel's code has changed
     since the counters were taken."""
-    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f).get(kernel)
         if not rec or rec.get("workload") != workload:
             return None
-        with open(os.path.join(ROOT, rec["src"]), "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        if not sha.startswith(rec["src_sha256_prefix"]):
+        if not code_sha256(os.path.join(ROOT, rec["src"])).startswith(rec["code_sha256_prefix"]):
             return None
         return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
     except (OSError, ValueError, KeyError):

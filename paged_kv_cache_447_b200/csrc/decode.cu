@@ -8,7 +8,8 @@
 //
 // Design (HBM-bound: every cached K/V byte is streamed from HBM exactly once):
 //  * Work unit = one 16-token block of one (sequence, kv-head group) -- the group is two
-//    adjacent kv heads when the kv-head count is even (else one), so that each cache slot
+//    adjacent kv heads when the kv-head count is even (else one; and one for bf16 grouped
+//    heads at D 128, whose two-slab tiles would halve the ring), so that each cache slot
 //    row fetched is 2 x D x esize contiguous bytes: short rows measured far below the DRAM
 //    bandwidth long ones reach (E4M3 at D 128, idle consumers: 3.8 TB/s with 128-byte rows,
 //    5.0-5.2 TB/s with 256-byte rows).  Units are numbered sequence-major; the whole unit space
@@ -23,14 +24,17 @@
 //  * A consumer warp handles all G = Hq/Hkv query heads of the kv head, so each K/V tile
 //    is read from shared memory once for the whole group.  Online softmax (running max m,
 //    sum l) per warp in exp2 space.
-//      - one head per kv head, and E4M3 caches: CUDA cores.  q.k: two lanes per token
-//        (each half the head dim, chunk order rotated per token so shared-memory reads are
-//        conflict-free), packed fp32x2 FMAs.  p.v: each lane owns D/32 output dims.
-//      - grouped bf16 heads (G = 2, 4, 8): tensor cores, mma.sync m16n8k16.  S = Q K^T with
-//        the G heads as rows of A (q held in registers for the whole piece, K fragments by
-//        ldmatrix); P stays in registers and feeds O^T = V^T P^T as the B operand (V^T
-//        fragments by ldmatrix.trans), so O needs D/16 accumulator tiles and no shuffles.
-//  * At the end of a piece the four consumer warps merge (m, l, acc) through shared
+//      - one q head per kv head, and E4M3 grouped heads at D 64: CUDA cores.  q.k: two
+//        lanes per token (each half the head dim, chunk order rotated per token so
+//        shared-memory reads are conflict-free), packed fp32x2 FMAs.  p.v: each lane owns
+//        D/32 output dims.
+//      - grouped heads (G = 2, 4, 8), bf16, and E4M3 at D 128: tensor cores, mma.sync
+//        m16n8k16.  S = Q K^T with the G heads as rows of A (q held in registers for the
+//        whole piece; K fragments by ldmatrix, or E4M3 bytes widened to f16); P stays in
+//        registers and feeds O^T = V^T P^T as the B operand (V^T fragments by
+//        ldmatrix.trans, or E4M3 bytes regrouped by byte permutes and widened), so O needs
+//        D/16 accumulator tiles and no shuffles.
+//  * At the end of a piece the consumer warps of each head merge (m, l, acc) through shared
 //    memory.  A piece that covers its whole sequence writes the normalised bf16 output;
 //    otherwise its partial goes to the workspace and a small combine kernel merges the
 //    partials of that sequence:  M = max m_k,  o = sum e^(m_k-M) acc_k / sum e^(m_k-M) l_k.
@@ -97,7 +101,7 @@ struct Geometry {
     static constexpr int kQFloats = kMma ? HPU * G * D / 2 : HPU * G * D;  // q scratch
     static constexpr int kExtraBytes = kQFloats * 4 + kConsumers * G * 16 * 4 +
                                        kConsumers * G * (D + 2) * 4 + 4 * 1025;
-    // ring of ~100 KB in total so that two CTAs share an SM
+    // the ring takes what the instantiation's shared-memory budget leaves
     // The stage count is a multiple of the consumer-group count, so that every fill of a
     // given stage is consumed by the same warp(s): a warp then never waits on a barrier more
     // than one phase ahead (a parity wait cannot tell phase n from phase n+2).
