@@ -18,6 +18,8 @@
 //                into separate K and V rings
 //   warp 1       TMEM owner and MMA issuer (one thread): S_i = Q_i K^T and O_i += P_i V with
 //                tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in tensor memory)
+//   warps 2-3    E4M3 caches only: widen each raw E4M3 tile (staged by plain TMA boxes) into
+//                the swizzled f16 operand layout; the MMAs then run on f16 (Q converted too)
 //   warps 4-7    softmax for tile 0, warps 8-11 for tile 1: thread r owns row r; reads its S
 //                row from TMEM, masks (bottom-right causal), exp2 with the running max, writes
 //                P (bf16) back into the S columns, which the next MMA reads as its A operand
