@@ -29,7 +29,9 @@ function               passage                                               pin
                                                                              K/V; L=1 returns V; rows sum
                                                                              to 1; x1e4 logits finite;
                                                                              block-permutation and shared-
-                                                                             prefix invariance
+                                                                             prefix invariance; E4M3 caches:
+                                                                             SDPA on torch-dequantised
+                                                                             codes x scales
 ``kv_cache_bytes``     2 x layers x kv_heads x head_dim x tokens x bytes     printed sizes ("LLM primer",
                        ("LLM primer", §17.3, §17.6)                          §17.3, §17.6, §23.2 exp. 2)
 ``slot_mapping``       block table lists a sequence's physical blocks, 16    hand-worked example

@@ -324,15 +324,18 @@ def test_worked_example_i_eat_fish():
     assert np.allclose(o, w[0] * vv[0] + w[1] * vv[1], atol=1e-12)
 
 
-def _sdpa_reference(wl, st, table=None):
+def _sdpa_reference(wl, st, table=None, kv=None):
     """torch's CPU SDPA (fp64) on K/V gathered with numpy fancy indexing and an explicit
-    boolean bottom-right causal mask -- an independent statement of the definition."""
+    boolean bottom-right causal mask -- an independent statement of the definition.
+    kv: optional fp64 caches [NB, 16, Hkv, D] (default: the workload's bf16 caches)."""
     q = oracle.bf16_to_f64(W.bits(st.q))
     if table is not None:
         pos = oracle.positions(st.cu_seqlens.numpy(), st.context_lens.numpy())
         q = oracle.bf16_to_f64(oracle.rope(W.bits(st.q), pos, table))
-    kc = oracle.bf16_to_f64(W.bits(wl.k_cache)).reshape(-1, wl.n_kv_heads, wl.head_dim)
-    vc = oracle.bf16_to_f64(W.bits(wl.v_cache)).reshape(-1, wl.n_kv_heads, wl.head_dim)
+    if kv is None:
+        kv = (oracle.bf16_to_f64(W.bits(wl.k_cache)), oracle.bf16_to_f64(W.bits(wl.v_cache)))
+    kc = kv[0].reshape(-1, wl.n_kv_heads, wl.head_dim)
+    vc = kv[1].reshape(-1, wl.n_kv_heads, wl.head_dim)
     G = wl.n_q_heads // wl.n_kv_heads
     out = np.zeros_like(q)
     for b in range(st.num_seqs):
@@ -371,6 +374,27 @@ def test_attention_matches_torch_sdpa(which):
                                wl.n_kv_heads, table=table)
         ref = _sdpa_reference(wl2, st, table)
         assert np.max(np.abs(got - ref)) < 1e-12
+
+
+def test_fp8_attention_matches_sdpa_on_torch_dequantised_cache():
+    """E4M3 caches: the oracle's attention (its own code decoder, times the head's scale)
+    equals SDPA on the cache dequantised by torch's float8_e4m3fn with the same scales."""
+    wl = W.mix(seed=5, decodes=6, chunks=1, chunk_len=24, fp8=True, max_context=300)
+    st = wl.steps[0]
+    kc = W.bits(wl.k_cache).copy()
+    vc = W.bits(wl.v_cache).copy()
+    ks, vs = wl.k_scale.double(), wl.v_scale.double()
+
+    def deq(codes, scale):
+        x = torch.from_numpy(codes).view(torch.float8_e4m3fn).double()
+        return (x * scale.view(1, 1, -1, 1)).numpy()
+
+    kv = (deq(kc, ks), deq(vc, vs))
+    got = oracle.attention(W.bits(st.q), kc, vc, st.cu_seqlens.numpy(), st.block_tables.numpy(),
+                           st.context_lens.numpy(), wl.scale, 16, wl.n_kv_heads, fp8=True,
+                           k_scale=wl.k_scale.numpy(), v_scale=wl.v_scale.numpy())
+    ref = _sdpa_reference(wl, st, None, kv)
+    assert np.max(np.abs(got - ref)) < 1e-12
 
 
 def test_context_len_one_returns_v_and_rows_sum_to_one():
