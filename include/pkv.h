@@ -192,6 +192,8 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, i
  *   workspace     device scratch of at least pkv_decode_workspace_bytes(...) bytes,
  *                 16-byte aligned; its contents need no initialisation and are
  *                 overwritten.  Calls that share a workspace must not overlap in time.
+ * Sizes: num_seqs up to about 39,000 per call (each CTA keeps the prefix of the sequences'
+ * block counts in shared memory; a call past the limit fails to launch: PKV_E_CUDA).
  * Device errors: block id outside [0, num_blocks) or L_b > max_blocks_per_seq*block_size
  * -> PKV_E_BOUNDS flag (the block reads as zeros / the context is clipped).
  */
