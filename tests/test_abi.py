@@ -109,3 +109,15 @@ def test_workspace_size_is_positive_and_monotone():
     b = pkv.decode_workspace_bytes(128, 32, 32, 128)
     assert 0 < a < b
     assert pkv.decode_workspace_bytes(64, 32, 5, 128) == 0
+
+
+def test_missing_library_fails_loudly():
+    """No CPU fallback: without the CUDA library every entry point raises at first use."""
+    import subprocess
+    import sys
+    code = ("import paged_kv_cache_447_b200 as pkv\n"
+            "try:\n    pkv.version()\nexcept ImportError as e:\n    print('raised', e)\n")
+    env = dict(os.environ, PKV_LIBRARY=os.path.join(ROOT, "no_such_libpagedkv.so"))
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.startswith("raised") and "missing" in r.stdout
