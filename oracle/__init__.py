@@ -17,7 +17,13 @@ function               passage                                               pin
                                                                              monotonicity, saturation
 ``rope_table/rope``    RoPE rotates Q/K inside attention ("LLM primer",      pos 0 = identity, pairwise
                        §21.2; "Inside the Nano-vLLM engine", §3.2)           norm kept, relative-position
-                                                                             property, quarter turn
+                                                                             property, quarter turn, direct
+                                                                             fp64 rotation at position p
+``positions``          new token r of sequence b at L_b - n_b + r (the new   hand-worked positions
+                       tokens are the newest; "Inside the Nano-vLLM          (tests/golden); attention on q
+                       engine", §2.1, §3.1)                                  rotated at hand-written
+                                                                             positions; prefix + chunk
+                                                                             shift invariance
 ``kv_store``           K/V cached per token, written by a cache kernel       round trip through the block
                        ("Nano-vLLM Part 2", §5.1-5.3); fixed 16-token        table equals the source rows;
                        blocks + block table ("Inside the Nano-vLLM engine",  slot -1 writes nothing

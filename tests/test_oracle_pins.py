@@ -227,6 +227,127 @@ def test_rope_relative_position_property():
         assert abs(dot(10 + shift, 3 + shift) - ref) < 0.15
 
 
+# ---- where new tokens sit when part of the sequence is cached
+
+POS_EXAMPLE = dict(ctx=[20, 1, 32, 17, 41], new=[3, 1, 2, 17, 1])
+
+
+def test_positions_hand_worked_example():
+    """Positions of new tokens after a cached prefix (chunked prefill and decode rows),
+    worked by hand in tests/golden/positions.txt."""
+    rows = _golden_rows("positions.txt")
+    cu = np.concatenate([[0], np.cumsum(POS_EXAMPLE["new"])]).astype(np.int32)
+    got = oracle.positions(cu, np.array(POS_EXAMPLE["ctx"], np.int32))
+    assert [int(x) for x in got] == [int(r[1]) for r in rows]
+
+
+def test_rope_at_position_is_direct_rotation():
+    """One vector rotated by the oracle at position p equals a direct fp64 cos/sin rotation
+    by p * theta_i (within the bf16 output rounding), for p where p - 1 and p + 1 differ:
+    a position off by one, or read from another row, fails."""
+    D = 64
+    tab = oracle.rope_table(512, D)
+    x = _rand_bits((1, 1, D), 11)
+    xf = oracle.bf16_to_f64(x)[0, 0]
+    theta = 10000.0 ** (-(2.0 * np.arange(D // 2)) / D)
+    for p in (1, 17, 36, 40, 300):
+        y = oracle.bf16_to_f64(oracle.rope(x, np.array([p]), tab))[0, 0]
+        c, s = np.cos(p * theta), np.sin(p * theta)
+        ref = np.concatenate([xf[:D // 2] * c - xf[D // 2:] * s, xf[D // 2:] * c + xf[:D // 2] * s])
+        tol = 2.0 ** -8 * np.abs(ref) + 1e-6
+        assert np.all(np.abs(y - ref) <= tol), p
+        for wrong in (p - 1, p + 1):
+            yw = oracle.bf16_to_f64(oracle.rope(x, np.array([wrong]), tab))[0, 0]
+            assert np.any(np.abs(yw - ref) > tol)
+
+
+def _mixed_batch(seed, lens_new, lens_ctx, hq=4, hkv=2, d=64, nb=16):
+    """Random bf16 caches, a permuted block table per sequence and q for the new tokens."""
+    g = torch.Generator().manual_seed(seed)
+    kc = W.bits(torch.randn(nb, 16, hkv, d, generator=g).to(torch.bfloat16)).copy()
+    vc = W.bits(torch.randn(nb, 16, hkv, d, generator=g).to(torch.bfloat16)).copy()
+    perm = torch.randperm(nb, generator=g).numpy()
+    bt = np.full((len(lens_ctx), nb), -1, np.int32)
+    used = 0
+    for b, L in enumerate(lens_ctx):
+        k = W.blocks_needed(L)
+        bt[b, :k] = perm[used:used + k]
+        used += k
+    cu = np.concatenate([[0], np.cumsum(lens_new)]).astype(np.int32)
+    q = W.bits(torch.randn(int(cu[-1]), hq, d, generator=g).to(torch.bfloat16))
+    return kc, vc, bt, cu, np.array(lens_ctx, np.int32), q
+
+
+def test_attention_rotates_q_at_cached_offset():
+    """attention(table=...) on a decode row (L = 37) and on a 5-token chunk after 35 cached
+    tokens equals attention on q rotated beforehand at positions written out by hand
+    (36; then 35 .. 39).  The slips a position rule can make (the row's index inside the
+    chunk, or one off either way) give outputs far outside rounding."""
+    kc, vc, bt, cu, cl, q = _mixed_batch(21, [1, 5], [37, 40])
+    tab = oracle.rope_table(64, 64)
+    scale = 0.125
+    args = (kc, vc, cu, bt, cl, scale, 16, 2)
+    got = oracle.attention(q, *args, table=tab)
+    by_hand = np.array([36, 35, 36, 37, 38, 39])
+    ref = oracle.attention(oracle.rope(q, by_hand, tab), *args)
+    assert np.array_equal(got, ref)
+    for wrong in (np.array([0, 0, 1, 2, 3, 4]), by_hand - 1, by_hand + 1):
+        alt = oracle.attention(oracle.rope(q, wrong, tab), *args)
+        assert np.max(np.abs(alt - ref)) > 1e-2
+
+
+def _prefix_then_chunk(q, k, v, P, n, nb, tab, pos_rule):
+    """Store a P-token prefix, then an n-token chunk, into empty caches (K rotated on the
+    way in), then attend with the chunk's queries.  pos_rule None: the oracle's own
+    positions/slot rules drive both calls and q is rotated by attention(table=...);
+    otherwise pos_rule is the explicit position array of all P + n tokens, slots are
+    enumerated from the table and q is rotated beforehand at pos_rule[P:]."""
+    hkv, d = k.shape[1], k.shape[2]
+    kc = np.zeros((nb, 16, hkv, d), np.uint16)
+    vc = np.zeros_like(kc)
+    bt = np.arange(nb, dtype=np.int32)[::-1].copy()[None, :]   # blocks in reverse order
+    L = P + n
+    if pos_rule is None:
+        for lo, hi in ((0, P), (P, L)):
+            cu = np.array([0, hi - lo], np.int32)
+            cl = np.array([hi], np.int32)
+            slots = oracle.slot_mapping(bt, cu, cl, 16, nb)
+            oracle.kv_store(k[lo:hi], v[lo:hi], kc, vc, slots, 16, table=tab,
+                            pos=oracle.positions(cu, cl))
+        return oracle.attention(q, kc, vc, np.array([0, n], np.int32), bt,
+                                np.array([L], np.int32), 0.125, 16, hkv, table=tab)
+    slots = np.array([bt[0, j // 16] * 16 + j % 16 for j in range(L)], np.int32)
+    oracle.kv_store(k, v, kc, vc, slots, 16, table=tab, pos=pos_rule)
+    return oracle.attention(oracle.rope(q, pos_rule[P:], tab), kc, vc,
+                            np.array([0, n], np.int32), bt, np.array([L], np.int32), 0.125, 16,
+                            hkv)
+
+
+def test_prefix_and_chunk_positions_are_relative():
+    """RoPE makes attention depend on q and k positions only through their difference.
+    A 21-token prefix stored by one call and a 7-token chunk by the next, attended through
+    the oracle's own position rule, equals the same tokens placed explicitly at 0..27 (bit
+    for bit) and at s..s+27 for shifts s (within bf16 rounding of the rotated values).  A
+    rule that placed the chunk at its local indices 0..6 is far off."""
+    g = torch.Generator().manual_seed(23)
+    P, n, hq, hkv, d = 21, 7, 4, 2, 64
+    k = W.bits(torch.randn(P + n, hkv, d, generator=g).to(torch.bfloat16))
+    v = W.bits(torch.randn(P + n, hkv, d, generator=g).to(torch.bfloat16))
+    q = W.bits(torch.randn(n, hq, d, generator=g).to(torch.bfloat16))
+    tab = oracle.rope_table(4096, d)
+    got = _prefix_then_chunk(q, k, v, P, n, 4, tab, None)
+    explicit = np.arange(P + n)
+    assert np.array_equal(got, _prefix_then_chunk(q, k, v, P, n, 4, tab, explicit))
+    for s in (1, 100, 3000):
+        shifted = _prefix_then_chunk(q, k, v, P, n, 4, tab, explicit + s)
+        assert np.max(np.abs(shifted - got)) < 2e-2, s
+    local = np.concatenate([np.arange(P), np.arange(n)])
+    assert np.max(np.abs(_prefix_then_chunk(q, k, v, P, n, 4, tab, local) - got)) > 5e-2
+    one_short = explicit.copy()
+    one_short[P:] -= 1
+    assert np.max(np.abs(_prefix_then_chunk(q, k, v, P, n, 4, tab, one_short) - got)) > 5e-2
+
+
 # ----------------------------------------------------------------------------- store
 
 def test_kv_store_round_trip_and_padding():
