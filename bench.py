@@ -3,9 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-suite] [--no-e2e] [--no-cpu-baseline]
 
-A step is one pass of the hot path over one batch: kv_store of the step's new tokens
-(K rotated by RoPE on the way in), then attention over the paged cache (Q rotated on
-load): paged decode attention for decode rows, paged prefill attention for prefill rows.
+A step is one pass of the hot path over one batch: the step's new tokens are stored into
+the paged cache (K rotated by RoPE on the way in) and attention runs over the cache (Q
+rotated on load).  Decode rows go through the one-launch decode step (store + attention +
+split merge in one kernel); prefill rows through kv_store and paged prefill attention.
+``--unfused`` runs decode rows as kv_store + paged decode attention (+ its merge kernel)
+instead.
 The default workload is the Qwen-7B-style MHA decode step (batch 64, 32 heads x 128,
 context lengths uniform in [128, 2048]); the headline value is the decode attention's
 KV bytes per step divided by the device-timed step time (GB/s).  ``--suite`` (on by
@@ -215,7 +218,7 @@ def recorded_traffic(kernel: str, workload: str):
 class Runner:
     """Device buffers of one workload and the step closure (ours)."""
 
-    def __init__(self, wl: W.Workload, layers: int = 1):
+    def __init__(self, wl: W.Workload, layers: int = 1, fused: bool = True):
         import paged_kv_cache_447_b200 as pkv
         self.pkv = pkv
         self.wl = wl
@@ -235,7 +238,12 @@ class Runner:
         self.dev = {n: t.cuda() for n, t in self.host.items()}
         B = st.decode_seqs
         self.B = B
+        self.fused = fused
         if B:
+            self.dec_k = self.dev["k"][:B]
+            self.dec_v = self.dev["v"][:B]
+            # zero-filled once; every decode step leaves its counters at zero
+            self.ws_step = pkv.decode_step_workspace(B, wl.n_q_heads, wl.n_kv_heads, wl.head_dim)
             self.dec_bt = self.dev["block_tables"][:B].contiguous()
             self.dec_ctx = self.dev["context_lens"][:B].contiguous()
             self.ws = torch.empty(pkv.decode_workspace_bytes(B, wl.n_q_heads, wl.n_kv_heads,
@@ -248,6 +256,9 @@ class Runner:
         if P:
             tok0 = int(st.cu_seqlens[B])
             self.pre_q = self.dev["q"][tok0:]
+            self.pre_k = self.dev["k"][tok0:]
+            self.pre_v = self.dev["v"][tok0:]
+            self.pre_slots = self.dev["slot_mapping"][tok0:]
             self.pre_cu = (self.dev["cu_seqlens"][B:] - tok0).contiguous()
             self.pre_bt = self.dev["block_tables"][B:].contiguous()
             self.pre_ctx = self.dev["context_lens"][B:].contiguous()
@@ -258,11 +269,10 @@ class Runner:
         self.ev_attn = []  # (start, end) event pairs around the dominant kernel
 
     def launches_per_step(self) -> int:
-        n = 1                      # kv_store
-        if self.B:
-            n += 2                 # decode + combine
-        if self.P:
-            n += 1                 # prefill
+        if self.fused:
+            n = (1 if self.B else 0) + (2 if self.P else 0)  # decode step; store + prefill
+        else:
+            n = 1 + (2 if self.B else 0) + (1 if self.P else 0)  # store, decode + merge, prefill
         return n * self.layers
 
     def step(self, record: bool = False, dominant: str = "decode"):
@@ -270,17 +280,28 @@ class Runner:
         s = torch.cuda.current_stream()
         for layer in range(self.layers):
             kc, vc = self.k_caches[layer], self.v_caches[layer]
-            pkv.kv_store(d["k"], d["v"], kc, vc, d["slot_mapping"], k_scale=self.k_scale,
-                         v_scale=self.v_scale, rope_cos_sin=self.table,
-                         cu_seqlens=d["cu_seqlens"], context_lens=d["context_lens"])
+            if not self.fused:
+                pkv.kv_store(d["k"], d["v"], kc, vc, d["slot_mapping"], k_scale=self.k_scale,
+                             v_scale=self.v_scale, rope_cos_sin=self.table,
+                             cu_seqlens=d["cu_seqlens"], context_lens=d["context_lens"])
+            elif self.P:
+                pkv.kv_store(self.pre_k, self.pre_v, kc, vc, self.pre_slots, k_scale=self.k_scale,
+                             v_scale=self.v_scale, rope_cos_sin=self.table,
+                             cu_seqlens=self.pre_cu, context_lens=self.pre_ctx)
             if self.B:
                 q = d["q"][:self.B]
                 if record and dominant == "decode":
                     e0 = torch.cuda.Event(enable_timing=True); e0.record(s)
-                pkv.paged_decode_attention(q, kc, vc, self.dec_bt, self.dec_ctx, scale=wl.scale,
-                                           k_scale=self.k_scale, v_scale=self.v_scale,
-                                           rope_cos_sin=self.table, workspace=self.ws,
-                                           out=self.dec_out)
+                if self.fused:
+                    pkv.paged_decode_step(q, self.dec_k, self.dec_v, kc, vc, self.dec_bt,
+                                          self.dec_ctx, self.ws_step, scale=wl.scale,
+                                          k_scale=self.k_scale, v_scale=self.v_scale,
+                                          rope_cos_sin=self.table, out=self.dec_out)
+                else:
+                    pkv.paged_decode_attention(q, kc, vc, self.dec_bt, self.dec_ctx, scale=wl.scale,
+                                               k_scale=self.k_scale, v_scale=self.v_scale,
+                                               rope_cos_sin=self.table, workspace=self.ws,
+                                               out=self.dec_out)
                 if record and dominant == "decode":
                     e1 = torch.cuda.Event(enable_timing=True); e1.record(s)
                     self.ev_attn.append((e0, e1))
@@ -339,6 +360,8 @@ def workload_config(name: str, wl, layers: int, world: int) -> dict:
 
 
 def build_workload(name: str, layers=None):
+    if name == "small_batch":
+        return W.gqa_decode(seed=6, batch=4, context=4096), 1
     if name == "qwen_decode":
         return W.qwen_decode(seed=2), 1
     if name == "gqa_decode":
@@ -352,9 +375,10 @@ def build_workload(name: str, layers=None):
     raise ValueError(name)
 
 
-def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=True, layers=None):
+def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=True, layers=None,
+                 fused=True):
     wl, layers = build_workload(name, layers)
-    r = Runner(wl, layers)
+    r = Runner(wl, layers, fused=fused)
     st = r.st
     # one checked step first: a device error (bounds, a bounded wait that ran out) stops here
     r.step()
@@ -372,8 +396,9 @@ def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=Tr
     world = dist.get_world_size() if dist is not None else 1
     step_ms = ms / steps
     attn_ms = r.attn_ms()
-    res = {"workload": name, "step_ms": step_ms, "layers": layers, "clocks": clocks,
-           "gpu_launches": r.launches_per_step() * steps}
+    res = {"workload": name, "step_ms": step_ms, "step_us": step_ms * 1e3, "layers": layers,
+           "clocks": clocks, "gpu_launches": r.launches_per_step() * steps,
+           "decode_path": "fused step" if fused else "store + attention + merge"}
     hbm = (pk or FALLBACK_PEAKS)["hbm_gbs"]
     if r.B:
         kv_bytes = decode_kv_bytes(st, wl.n_kv_heads, wl.head_dim, esize) * layers
@@ -477,7 +502,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen_decode",
-                    choices=["qwen_decode", "gqa_decode", "shared_prefix", "mix", "mix_fp8"])
+                    choices=["qwen_decode", "gqa_decode", "shared_prefix", "mix", "mix_fp8",
+                             "small_batch"])
+    ap.add_argument("--unfused", action="store_true",
+                    help="decode rows as kv_store + paged decode attention (+ merge kernel)")
     ap.add_argument("--no-suite", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -522,7 +550,7 @@ def main():
         torch.cuda.set_device(0)
 
     res, runner = measure_ours(args.workload, args.steps, args.warmup, dist, local, pk,
-                               e2e=not args.no_e2e, layers=args.layers)
+                               e2e=not args.no_e2e, layers=args.layers, fused=not args.unfused)
     wl = runner.wl
     esize = 1 if wl.cache_dtype == "fp8" else 2
     if runner.B:
@@ -560,11 +588,17 @@ def main():
 
     if world == 1 and not args.no_suite:
         suite = {}
-        for name in ("gqa_decode", "shared_prefix", "mix", "mix_fp8"):
-            if name == args.workload:
+        runs = [(n, True) for n in ("gqa_decode", "shared_prefix", "mix", "mix_fp8", "small_batch")
+                if n != args.workload]
+        # the same decode workloads through the three-launch path, for comparison
+        runs += [("qwen_decode", False), ("small_batch", False), ("mix_fp8", False)]
+        for name, fused in runs:
+            key = name if fused else name + "_unfused"
+            if name == args.workload and fused != args.unfused:
                 continue
             try:
-                r, rr = measure_ours(name, max(3, args.steps // 4), 3, None, 0, pk, e2e=False)
+                r, rr = measure_ours(name, max(3, args.steps // 4), 3, None, 0, pk, e2e=False,
+                                     fused=fused)
                 del rr
                 torch.cuda.empty_cache()
                 keep = {k: v for k, v in r.items() if k not in ("clocks",)}
@@ -572,9 +606,9 @@ def main():
                     keep["attn_hbm_frac"] = r["attn_gbs"] / pk["hbm_gbs"]
                 if "prefill_tflops" in r:
                     keep["prefill_tensor_frac"] = r["prefill_tflops"] / pk["bf16_tflops"]
-                suite[name] = keep
+                suite[key] = keep
             except Exception as e:  # report, do not hide
-                suite[name] = {"error": f"{type(e).__name__}: {e}"}
+                suite[key] = {"error": f"{type(e).__name__}: {e}"}
         line["suite"] = suite
 
     if world == 1 and rank == 0 and not args.no_cpu_baseline:

@@ -19,7 +19,9 @@
  *           heads of a token are adjacent (ENG §2.2: fixed-size blocks; NV2 §5.2: block,
  *           K/V and token dimensions).  Element type: bf16 (PKV_BF16) or OCP FP8 E4M3-FN
  *           codes with one fp32 scale per kv head for K and for V (PKV_FP8_E4M3; value =
- *           code_value * scale).  block_size must be 16, head_dim 64 or 128.
+ *           code_value * scale).  block_size 8, 16 or 32 (ENG §2.2 uses 16 as an example);
+ *           head_dim 64 or 128 everywhere, and 256 for the store, RoPE and decode entry
+ *           points (pkv_paged_prefill_attention returns PKV_E_UNSUPPORTED for 256).
  * Slots.    slot = physical_block * block_size + offset_in_block; slot -1 = padding token.
  * Tables.   block_tables [num_seqs, max_blocks_per_seq] int32: logical block i of sequence
  *           b lives in physical block block_tables[b][i] (ENG §2.2, PRM §17.7).  Entries
@@ -65,7 +67,8 @@ enum pkv_status {
     PKV_E_TIMEOUT = -5,     /* (device) a bounded wait inside a kernel ran out            */
     PKV_E_BOUNDS = -6,      /* (device) slot / block id / position outside its array      */
     PKV_E_ALIGN = -7,       /* a pointer is not 16-byte aligned                           */
-    PKV_E_SCRATCH_LIMIT = -8 /* the call needs more than PKV_NOALLOC_SCRATCH_BYTES of scratch */
+    PKV_E_SCRATCH_LIMIT = -8, /* the call needs more than PKV_NOALLOC_SCRATCH_BYTES of scratch */
+    PKV_E_POOL = -9          /* (device) a block-pool allocation the pool could not cover    */
 };
 
 /* Size of the built-in decode scratch array used by pkv_paged_decode_attention_noalloc. */
@@ -158,6 +161,40 @@ int pkv_copy_blocks(void *k_cache, void *v_cache, const int32_t *block_pairs, in
                     int cache_dtype, pkv_stream_t stream);
 
 /*
+ * Block pool on the device (ENG §2.2: physical blocks come from a pool, a sequence receives
+ * a new block only when its tokens outgrow the blocks it holds, and a finished request
+ * returns its blocks; PRM §17.7: the block table works like a page table).
+ * The pool is a caller-allocated device buffer of pkv_block_pool_bytes(num_blocks) bytes:
+ * int32 [0] = number of free blocks (readable by the caller), then the stack of free ids and
+ * one free flag per block.  Calls on one pool must not overlap in time; each runs as one
+ * small kernel on `stream`, so the results are in stream order with the other entry points.
+ *
+ * pkv_block_pool_init -- every block free; the first allocations hand out 0, 1, 2, ...
+ *
+ * pkv_block_pool_alloc -- for every sequence b (cu_seqlens / context_lens as in Batches:
+ * n_b new tokens, L_b cached tokens including them) the blocks its new tokens need beyond
+ * the ceil((L_b - n_b) / block_size) it holds: ceil(L_b / block_size) - that many, taken in
+ * sequence order from the top of the free stack and written to block_tables[b] right after
+ * its held entries.  All or nothing: if the pool cannot cover the whole request the call
+ * takes nothing and sets the PKV_E_POOL flag; a table too short for L_b (or a negative
+ * count) takes nothing and sets PKV_E_BOUNDS.  Follow it with pkv_slot_mapping and
+ * pkv_kv_store.
+ *
+ * pkv_block_pool_free -- push block_ids[0 .. num_ids) back in that order (last freed, first
+ * reused).  An id outside the pool, not allocated, or repeated within the call is skipped and
+ * sets the PKV_E_BOUNDS flag.  (Reference counts for blocks shared by several sequences are
+ * the caller's: free a shared block once, when its last user finishes.)
+ */
+size_t pkv_block_pool_bytes(long long num_blocks);
+int pkv_block_pool_init(void *pool, long long num_blocks, pkv_stream_t stream);
+int pkv_block_pool_alloc(void *pool, long long num_blocks, int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *cu_seqlens,
+                         const int32_t *context_lens, int num_seqs, int block_size,
+                         pkv_stream_t stream);
+int pkv_block_pool_free(void *pool, long long num_blocks, const int32_t *block_ids, int num_ids,
+                        pkv_stream_t stream);
+
+/*
  * pkv_rope_apply -- rotate q [num_tokens, n_q_heads, head_dim] and k [num_tokens,
  * n_kv_heads, head_dim] (bf16) IN PLACE at each token's position (PRM §21.2, ENG §3.2).
  * Either q or k may be NULL.  Device errors: position outside [0, max_pos) ->
@@ -193,7 +230,8 @@ size_t pkv_decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, i
  *                 16-byte aligned; its contents need no initialisation and are
  *                 overwritten.  Calls that share a workspace must not overlap in time.
  * Sizes: num_seqs up to about 39,000 per call (each CTA keeps the prefix of the sequences'
- * block counts in shared memory; a call past the limit fails to launch: PKV_E_CUDA).
+ * block counts in shared memory); a larger call returns PKV_E_UNSUPPORTED and enqueues
+ * nothing.
  * Device errors: block id outside [0, num_blocks) or L_b > max_blocks_per_seq*block_size
  * -> PKV_E_BOUNDS flag (the block reads as zeros / the context is clipped).
  */
@@ -205,6 +243,48 @@ int pkv_paged_decode_attention(void *out, const void *q, const void *k_cache,
                                int cache_dtype, const float *k_scale, const float *v_scale,
                                const float *rope_cos_sin, int max_pos, void *workspace,
                                size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * pkv_decode_step_workspace_bytes -- size of the device buffer pkv_paged_decode_step needs,
+ * for the CURRENT device: the decode attention workspace followed by one int counter per
+ * (sequence, kv head).
+ */
+size_t pkv_decode_step_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads,
+                                       int head_dim);
+
+/*
+ * pkv_paged_decode_step -- one whole decode step in one launch: store each sequence's new
+ * token into the paged cache and run decode attention over the cache including it
+ * (ENG §2.1: every decode step appends the new token's K/V to the cache and attends over
+ * all of it; PRM §17.1: decode is one token per sequence per step and its latency is the
+ * time per output token; ENG §6.3: fusing kernels).  The result is that of
+ *     pkv_kv_store(k, v, ..., slot of position L_b - 1, K rotated at L_b - 1)
+ *     pkv_paged_decode_attention(out, q, ...)
+ * with the same cache bytes and bit-identical outputs.
+ *   k, v          [num_seqs, n_kv_heads, head_dim] bf16: the new token of each sequence.
+ *                 Its slot follows from the block table: position p = L_b - 1 is offset
+ *                 p % block_size of block block_tables[b][p / block_size] (ENG §2.2), so
+ *                 no slot mapping is taken; a sequence with L_b = 0 has no new token.
+ *   k_cache,
+ *   v_cache       written at those slots (E4M3 codes for PKV_FP8_E4M3, from the fp64 quotient
+ *                 by the head's scale, as in pkv_kv_store)
+ *   other arguments as pkv_paged_decode_attention (rope_cos_sin rotates both the new K and q
+ *   at L_b - 1)
+ *   workspace     at least pkv_decode_step_workspace_bytes(...) bytes, 16-byte aligned,
+ *                 FILLED WITH ZEROS before its first use (cudaMemset); every call that
+ *                 completes leaves its counters at zero again.  A call that ran into a
+ *                 PKV_E_TIMEOUT may not: zero the workspace again after one.  Calls that share
+ *                 a workspace must not overlap in time.
+ * Device errors: as pkv_paged_decode_attention and pkv_kv_store (a table entry outside the
+ * pool or a position past the RoPE table stores nothing and sets PKV_E_BOUNDS).
+ */
+int pkv_paged_decode_step(void *out, const void *q, const void *k, const void *v, void *k_cache,
+                          void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *context_lens, int num_seqs, int n_q_heads,
+                          int n_kv_heads, int head_dim, int block_size, long long num_blocks,
+                          float scale, int cache_dtype, const float *k_scale,
+                          const float *v_scale, const float *rope_cos_sin, int max_pos,
+                          void *workspace, size_t workspace_bytes, pkv_stream_t stream);
 
 /*
  * pkv_paged_prefill_attention -- causal attention of a chunk of new tokens per sequence
@@ -248,7 +328,8 @@ int pkv_paged_prefill_attention(void *out, const void *q, const void *k_cache,
  *     array keeps the last call's contents; none of them needs to start at zero, so
  *     nothing is cleared.
  *   - The first call on each device (with that device current) looks up the array's
- *     device address with cudaGetSymbolAddress; make that first call before any stream
+ *     device address with cudaGetSymbolAddress, and so does the first call after that
+ *     device's context was replaced (cudaDeviceReset); make such a call before any stream
  *     capture begins.
  * Results equal pkv_paged_decode_attention's for the same inputs.
  */
@@ -263,7 +344,7 @@ int pkv_paged_decode_attention_noalloc(void *out, const void *q, const void *k_c
 
 /*
  * pkv_get_error -- synchronise `stream`, then return and clear the current device's error
- * word: PKV_OK, PKV_E_TIMEOUT or PKV_E_BOUNDS (the first set wins if both are), or
+ * word: PKV_OK, PKV_E_TIMEOUT, PKV_E_BOUNDS or PKV_E_POOL (in that order of precedence), or
  * PKV_E_CUDA if the synchronisation itself failed.
  */
 int pkv_get_error(pkv_stream_t stream);

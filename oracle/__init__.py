@@ -46,6 +46,12 @@ function               passage                                               pin
                                                                              slots; -1 past the table
 ``copy_blocks``        shared prefix blocks, copy on write ("Inside the      numpy block slicing: dst
                        Nano-vLLM engine", §2.2; "LLM primer", §17.7)         equals old src, rest unchanged
+``pool_*``             blocks come from a pool on demand and go back when   hand-worked sequence
+                       a request finishes ("Inside the Nano-vLLM engine",    (tests/golden); invariants
+                       §2.2; "LLM primer", §17.7)                            (no id held twice, ids
+                                                                             conserved, tables cover every
+                                                                             token); random alloc/free runs
+                                                                             against a set-based model
 =====================  ====================================================  ===========================
 """
 from __future__ import annotations
@@ -113,6 +119,12 @@ def _load():
         lib.orc_copy_blocks.argtypes = [P, P, P, I, ctypes.c_int64, ctypes.c_int64]
         lib.orc_copy_blocks.restype = None
         lib.orc_kv_cache_bytes.restype = ctypes.c_int64
+        lib.orc_pool_init.argtypes = [P, ctypes.c_int32]
+        lib.orc_pool_init.restype = None
+        lib.orc_pool_alloc.argtypes = [P, ctypes.c_int32, P, I, P, P, I, I]
+        lib.orc_pool_alloc.restype = I
+        lib.orc_pool_free.argtypes = [P, ctypes.c_int32, P, I]
+        lib.orc_pool_free.restype = I
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -288,6 +300,31 @@ def copy_blocks(k_cache, v_cache, pairs) -> None:
     nb = k_cache.shape[0]
     block_bytes = k_cache.nbytes // nb
     _load().orc_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pr), pr.shape[0], block_bytes, nb)
+
+
+def pool_init(num_blocks: int) -> np.ndarray:
+    """Block pool state (int32): [free count, stack of free ids bottom first, free flags]."""
+    pool = np.zeros(1 + 2 * num_blocks, dtype=np.int32)
+    _load().orc_pool_init(_ptr(pool), num_blocks)
+    return pool
+
+
+def pool_alloc(pool, block_tables, cu_seqlens, context_lens, block_size: int = 16) -> int:
+    """Give every sequence the blocks its new tokens need (written into block_tables in
+    place); 0, or -1 (nothing taken) when the pool or a table is too small."""
+    nb = (pool.shape[0] - 1) // 2
+    assert block_tables.flags.c_contiguous and block_tables.dtype == np.int32
+    cu = _c(cu_seqlens, np.int32)
+    cl = _c(context_lens, np.int32)
+    return int(_load().orc_pool_alloc(_ptr(pool), nb, _ptr(block_tables), block_tables.shape[1],
+                                      _ptr(cu), _ptr(cl), len(cl), block_size))
+
+
+def pool_free(pool, ids) -> int:
+    """Return ids to the pool; the number of ids rejected (outside the pool or already free)."""
+    nb = (pool.shape[0] - 1) // 2
+    ids = _c(np.asarray(ids).reshape(-1), np.int32)
+    return int(_load().orc_pool_free(_ptr(pool), nb, _ptr(ids), len(ids)))
 
 
 def num_threads() -> int:

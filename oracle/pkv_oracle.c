@@ -258,6 +258,71 @@ void orc_copy_blocks(uint8_t *k_cache, uint8_t *v_cache, const int32_t *pairs, i
     }
 }
 
+/* [ENG] §2.2: physical blocks come from a pool; a sequence gets a new block when its
+ * tokens outgrow the blocks it has, and a finished request returns its blocks to the pool
+ * ([PRM] §17.7 likens the block table to an operating system's page table).  The pool here
+ * is a stack of free ids plus a free flag per block:
+ *   init   : every block free, stacked so that the first allocations hand out 0, 1, 2, ...
+ *   alloc  : sequence by sequence, the blocks its new tokens need beyond those its cached
+ *            tokens already fill, taken one by one from the top of the stack and written to
+ *            the sequence's table after its existing entries.  If the pool cannot cover the
+ *            whole request, nothing is taken and -1 is returned.
+ *   free   : ids pushed back one by one; an id outside the pool or already free is skipped
+ *            and counted.
+ * State layout (int32): [0] = number of free ids, [1 .. num_blocks] = the stack (bottom first),
+ * then num_blocks free flags. */
+void orc_pool_init(int32_t *pool, int32_t num_blocks)
+{
+    pool[0] = num_blocks;
+    for (int32_t i = 0; i < num_blocks; ++i) {
+        pool[1 + i] = num_blocks - 1 - i;          /* top of the stack = block 0 */
+        pool[1 + num_blocks + i] = 1;
+    }
+}
+
+int orc_pool_alloc(int32_t *pool, int32_t num_blocks, int32_t *block_tables, int max_blocks,
+                   const int32_t *cu_seqlens, const int32_t *context_lens, int num_seqs,
+                   int block_size)
+{
+    int64_t total = 0;
+    for (int b = 0; b < num_seqs; ++b) {
+        int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        int have = (context_lens[b] - n + block_size - 1) / block_size;
+        int need = (context_lens[b] + block_size - 1) / block_size;
+        if (need > max_blocks) return -1;
+        total += need - have;
+    }
+    if (total > pool[0]) return -1;
+    for (int b = 0; b < num_seqs; ++b) {
+        int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        int have = (context_lens[b] - n + block_size - 1) / block_size;
+        int need = (context_lens[b] + block_size - 1) / block_size;
+        for (int j = have; j < need; ++j) {
+            int32_t id = pool[pool[0]];              /* top of the stack */
+            pool[0] -= 1;
+            pool[1 + num_blocks + id] = 0;
+            block_tables[(size_t)b * max_blocks + j] = id;
+        }
+    }
+    return 0;
+}
+
+int orc_pool_free(int32_t *pool, int32_t num_blocks, const int32_t *ids, int num_ids)
+{
+    int rejected = 0;
+    for (int i = 0; i < num_ids; ++i) {
+        int32_t id = ids[i];
+        if (id < 0 || id >= num_blocks || pool[1 + num_blocks + id]) {
+            ++rejected;
+            continue;
+        }
+        pool[0] += 1;
+        pool[pool[0]] = id;
+        pool[1 + num_blocks + id] = 1;
+    }
+    return rejected;
+}
+
 /* ------------------------------------------------------------------------------------ */
 /* Attention over the paged cache                                                       */
 /* ------------------------------------------------------------------------------------ */

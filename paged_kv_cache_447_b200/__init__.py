@@ -2,7 +2,8 @@
 
 The compute lives in ``libpagedkv.so`` (hand-written CUDA behind the C ABI declared in
 ``include/pkv.h``).  This package is its thin Python binding: ``kv_store``, ``rope_apply``,
-``paged_decode_attention``, ``paged_prefill_attention``, ``slot_mapping``, ``copy_blocks``
+``paged_decode_attention``, ``paged_decode_step``, ``paged_prefill_attention``,
+``slot_mapping``, ``copy_blocks``
 and helpers take torch tensors,
 pass their device pointers and sizes across the C ABI and raise on a non-zero status.
 PyTorch only provides device memory and streams.
@@ -18,6 +19,8 @@ import importlib
 _BINDING_NAMES = {
     "kv_store", "rope_apply", "paged_decode_attention", "paged_prefill_attention",
     "paged_decode_attention_noalloc", "NOALLOC_SCRATCH_BYTES", "slot_mapping", "copy_blocks",
+    "paged_decode_step", "decode_step_workspace_bytes", "decode_step_workspace",
+    "block_pool", "block_pool_alloc", "block_pool_free",
     "rope_build_table", "decode_workspace_bytes", "cache_bytes", "get_error", "strerror",
     "debug_wait_timeout", "version", "library_path", "load_library", "PagedKVError",
     "BF16", "FP8_E4M3",

@@ -25,7 +25,8 @@ _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape or dtype",
            -3: "workspace missing or too small", -4: "CUDA runtime error",
            -5: "a bounded wait inside a kernel ran out",
            -6: "slot, block id or position out of range", -7: "pointer not 16-byte aligned",
-           -8: "call needs more than the built-in decode scratch array"}
+           -8: "call needs more than the built-in decode scratch array",
+           -9: "block pool cannot cover the allocation"}
 
 
 class PagedKVError(RuntimeError):
@@ -66,7 +67,14 @@ def load_library():
                                          P, P, P, I, I, P], I),
         "pkv_paged_decode_attention_noalloc": ([P, P, P, P, P, I, P, I, I, I, I, I, LL, F, I,
                                                 P, P, P, I, P], I),
+        "pkv_decode_step_workspace_bytes": ([I, I, I, I], SZ),
+        "pkv_paged_decode_step": ([P, P, P, P, P, P, P, I, P, I, I, I, I, I, LL, F, I, P, P, P, I,
+                                   P, SZ, P], I),
         "pkv_slot_mapping": ([P, P, I, P, P, I, I, I, LL, P], I),
+        "pkv_block_pool_bytes": ([LL], SZ),
+        "pkv_block_pool_init": ([P, LL, P], I),
+        "pkv_block_pool_alloc": ([P, LL, P, I, P, P, I, I, P], I),
+        "pkv_block_pool_free": ([P, LL, P, I, P], I),
         "pkv_copy_blocks": ([P, P, P, I, I, I, I, LL, I, P], I),
         "pkv_get_error": ([P], I),
         "pkv_debug_wait_timeout": ([LL, P], I),
@@ -175,6 +183,40 @@ def slot_mapping(block_tables, cu_seqlens, context_lens, num_tokens: int, num_bl
     return out
 
 
+def block_pool(num_blocks: int, device=None, stream=None) -> torch.Tensor:
+    """A device block pool of num_blocks blocks, all free (int32 tensor; element 0 is the
+    number of free blocks)."""
+    n = int(load_library().pkv_block_pool_bytes(num_blocks))
+    if n == 0:
+        raise PagedKVError("pkv_block_pool_bytes", -1)
+    pool = torch.empty(n // 4, dtype=torch.int32, device=device or "cuda")
+    _check("pkv_block_pool_init", load_library().pkv_block_pool_init(_p(pool), num_blocks,
+                                                                      _stream(stream)))
+    return pool
+
+
+def _pool_blocks(pool: torch.Tensor) -> int:
+    return (pool.numel() - 4) // 2
+
+
+def block_pool_alloc(pool, block_tables, cu_seqlens, context_lens, *, block_size: int = 16,
+                     stream=None) -> None:
+    """Write into block_tables the blocks each sequence's new tokens need (in place)."""
+    _i32(pool, "pool"); _i32(block_tables, "block_tables"); _i32(cu_seqlens, "cu_seqlens")
+    _i32(context_lens, "context_lens")
+    _check("pkv_block_pool_alloc", load_library().pkv_block_pool_alloc(
+        _p(pool), _pool_blocks(pool), _p(block_tables), block_tables.shape[1], _p(cu_seqlens),
+        _p(context_lens), context_lens.shape[0], block_size, _stream(stream)))
+
+
+def block_pool_free(pool, block_ids, *, stream=None) -> None:
+    """Return the int32 block ids to the pool, in order."""
+    _i32(pool, "pool"); _i32(block_ids, "block_ids")
+    n = block_ids.numel()
+    _check("pkv_block_pool_free", load_library().pkv_block_pool_free(
+        _p(pool), _pool_blocks(pool), _p(block_ids) if n else None, n, _stream(stream)))
+
+
 def copy_blocks(k_cache, v_cache, block_pairs, *, stream=None) -> None:
     """Copy physical blocks src -> dst of both caches for every (src, dst) row of the int32
     [n, 2] block_pairs (copy on write)."""
@@ -223,6 +265,42 @@ def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, *, s
         block_tables.shape[1], _p(_i32(context_lens, "context_lens")), B, Hq, Hkv, D, bs, NB,
         float(scale), _cache_dtype(k_cache), _p(k_scale), _p(v_scale), _p(rope_cos_sin),
         max_pos, _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def decode_step_workspace_bytes(num_seqs: int, n_q_heads: int, n_kv_heads: int,
+                                head_dim: int) -> int:
+    return int(load_library().pkv_decode_step_workspace_bytes(num_seqs, n_q_heads, n_kv_heads,
+                                                              head_dim))
+
+
+def decode_step_workspace(num_seqs: int, n_q_heads: int, n_kv_heads: int, head_dim: int,
+                          device=None) -> torch.Tensor:
+    """A zero-filled workspace for paged_decode_step (reusable: every call leaves it zero)."""
+    return torch.zeros(decode_step_workspace_bytes(num_seqs, n_q_heads, n_kv_heads, head_dim),
+                       dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_decode_step(q, k, v, k_cache, v_cache, block_tables, context_lens, workspace, *,
+                      scale=None, k_scale=None, v_scale=None, rope_cos_sin=None, out=None,
+                      stream=None) -> torch.Tensor:
+    """One decode step in one launch: store k/v [B, Hkv, D] (each sequence's new token, at
+    position context_lens[b] - 1) into the paged cache and attend with q [B, Hq, D].
+    ``workspace`` comes from decode_step_workspace (zero-filled)."""
+    B, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    _bf16(q, "q"); _bf16(k, "k"); _bf16(v, "v")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    max_pos = rope_cos_sin.shape[0] if rope_cos_sin is not None else 0
+    _check("pkv_paged_decode_step", load_library().pkv_paged_decode_step(
+        _p(out), _p(q), _p(k), _p(v), _p(k_cache), _p(v_cache),
+        _p(_i32(block_tables, "block_tables")), block_tables.shape[1],
+        _p(_i32(context_lens, "context_lens")), B, Hq, Hkv, D, bs, NB, float(scale),
+        _cache_dtype(k_cache), _p(k_scale), _p(v_scale), _p(rope_cos_sin), max_pos,
+        _p(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
 
 

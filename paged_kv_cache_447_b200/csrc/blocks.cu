@@ -3,7 +3,8 @@
 //
 // "Inside the Nano-vLLM engine: KV cache, attention and tensor parallelism", §2.2: a
 // sequence's block table lists the physical blocks that hold its tokens, in order, 16
-// tokens per block, so position p lives at offset p % 16 of block table[p / 16]; requests
+// tokens per block (block_size here), so position p lives at offset p % block_size of block
+// table[p / block_size]; requests
 // that share a prefix point at the same physical blocks, and a shared block is copied when
 // one of them writes into it (copy on write; "LLM primer", §17.7 lists the same idea).
 // Both kernels are small: the slot kernel is latency-bound (one int per token), the copy
@@ -24,14 +25,15 @@ __global__ void __launch_bounds__(256) slot_mapping_kernel(SlotArgs a) {
         const int n = __ldg(a.cu_seqlens + b + 1) - c0;
         const long long p = (long long)__ldg(a.context_lens + b) - n + (t - c0);
         int slot = -1;
-        if (p < 0 || p >= (long long)a.max_blocks * kBlockSize) {
+        const int bs = a.block_size;
+        if (p < 0 || p >= (long long)a.max_blocks * bs) {
             atomicOr(a.err, kErrBounds);
         } else {
-            const int blk = __ldg(a.block_tables + (size_t)b * a.max_blocks + (size_t)(p / kBlockSize));
+            const int blk = __ldg(a.block_tables + (size_t)b * a.max_blocks + (size_t)(p / bs));
             if (blk < 0 || (long long)blk >= a.num_blocks)
                 atomicOr(a.err, kErrBounds);
             else
-                slot = blk * kBlockSize + (int)(p % kBlockSize);
+                slot = blk * bs + (int)(p % bs);
         }
         a.slot_mapping[t] = slot;
     }
@@ -65,9 +67,7 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(CopyArgs a) {
 }
 
 int grid_cap(long long items) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = current_sm_count();
     long long blocks = (items + 255) / 256;
     const long long cap = (long long)sms * 8;
     if (blocks > cap) blocks = cap;

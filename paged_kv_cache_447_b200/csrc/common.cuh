@@ -22,12 +22,15 @@ namespace pkv {
 // Error-word bits (see pkv_get_error).
 constexpr int kErrTimeout = 1;
 constexpr int kErrBounds = 2;
+constexpr int kErrPool = 4;  // a block-pool allocation the pool could not cover
 
 // A bounded wait gives up after this long (ns).  Legitimate waits in these kernels last
 // microseconds; a second means the pipeline is broken.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
-constexpr int kBlockSize = 16;  // tokens per physical cache block
+// Cache rows per TMA piece: the attention kernels stream the cache in 16-token tiles of a
+// sequence, whatever its physical block size (8, 16 or 32 tokens per block).
+constexpr int kPiece = 16;
 
 // ------------------------------------------------------------------------------ formats
 

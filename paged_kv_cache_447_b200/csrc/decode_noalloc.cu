@@ -11,9 +11,13 @@
 //
 // The array is file-scope device memory.  Its name in host code is only a host-side
 // stand-in for the symbol, not a device address, so host code never passes it to a
-// kernel; instead the per-device set-up below asks the runtime for the device address
-// with cudaGetSymbolAddress (with that device current) and hands that pointer on.
+// kernel; instead the set-up below asks the runtime for the device address with
+// cudaGetSymbolAddress (with the device current) and hands that pointer on.  The set-up
+// runs on the first call on each device, and again if that device's context has been
+// replaced (after cudaDeviceReset the library's module is loaded again and the array may
+// sit at another address).
 #include "../../include/pkv.h"
+#include "internal.h"
 
 #include <cuda_runtime.h>
 #include <mutex>
@@ -27,20 +31,15 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
+pkv::CachedSymbol g_scratch_cache[kMaxDevices];
 
-// Device address of the scratch array on the current device (looked up once per device).
+// Device address of the scratch array in the current device's context.
 int scratch_for_current_device(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKV_E_CUDA;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr)
-            return PKV_E_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void *p = pkv::cached_symbol_address(
+        g_scratch_cache, kMaxDevices, g_scratch_mu,
+        [](void **o) { return cudaGetSymbolAddress(o, g_decode_scratch); });
+    if (!p) return PKV_E_CUDA;
+    *out = p;
     return PKV_OK;
 }
 

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace pkv {
 
 struct StoreArgs {
@@ -49,6 +51,11 @@ struct DecodeArgs {
     void *workspace;
     size_t workspace_bytes;
     int *err;
+    // pkv_paged_decode_step only: the step's new K and V ([num_seqs, n_kv_heads, head_dim]
+    // bf16) and the same caches, writable
+    const void *k_new = nullptr, *v_new = nullptr;
+    void *k_cache_w = nullptr, *v_cache_w = nullptr;
+    int block_size = 16;
 };
 
 struct PrefillArgs {
@@ -67,6 +74,7 @@ struct PrefillArgs {
     const float *rope;
     int max_pos, max_new_tokens;
     int *err;
+    int block_size = 16;
 };
 
 struct SlotArgs {
@@ -77,6 +85,7 @@ struct SlotArgs {
     int num_seqs, num_tokens;
     long long num_blocks;
     int *err;
+    int block_size;
 };
 
 struct CopyArgs {
@@ -85,6 +94,25 @@ struct CopyArgs {
     int num_pairs;
     long long block_bytes;  // one block of one cache
     long long num_blocks;
+    int *err;
+};
+
+struct PoolArgs {
+    int32_t *pool;  // [4 + 2 * num_blocks]: free count, (3 unused), stack, free flags
+    long long num_blocks;
+    int32_t *block_tables;
+    int max_blocks;
+    const int32_t *cu_seqlens, *context_lens;
+    int num_seqs;
+    int *err;
+    int block_size;
+};
+
+struct PoolFreeArgs {
+    int32_t *pool;
+    long long num_blocks;
+    const int32_t *ids;
+    int num_ids;
     int *err;
 };
 
@@ -105,10 +133,43 @@ cudaError_t launch_rope_apply(const RopeArgs &a, cudaStream_t s);
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t s);
 size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
                               int num_sms);
+// The decode step: store each sequence's new token, attend, merge split partials in-kernel.
+// Its workspace is decode_workspace_bytes(...) followed by num_seqs * n_kv_heads int
+// counters that must be zero before the first call (every call leaves them zero).
+cudaError_t launch_paged_decode_step(const DecodeArgs &a, cudaStream_t s);
+size_t decode_step_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
+                                   int num_sms);
 cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s);
 cudaError_t launch_wait_timeout(unsigned long long limit_ns, int *err, cudaStream_t s);
 cudaError_t launch_slot_mapping(const SlotArgs &a, cudaStream_t s);
 cudaError_t launch_copy_blocks(const CopyArgs &a, cudaStream_t s);
+size_t block_pool_bytes(long long num_blocks);
+cudaError_t launch_pool_init(int32_t *pool, long long num_blocks, cudaStream_t s);
+cudaError_t launch_pool_alloc(const PoolArgs &a, cudaStream_t s);
+cudaError_t launch_pool_free(const PoolFreeArgs &a, cudaStream_t s);
+
+// Id of the CUDA context current on this thread (unique for the life of the process,
+// unlike a context handle or a device ordinal); false if there is none or the driver
+// cannot say.
+bool current_context_id(unsigned long long *id);
+
+// Device address of a file-scope __device__ symbol in the current context, looked up with
+// `lookup` (a cudaGetSymbolAddress call) the first time on each device and again whenever
+// the current context differs from the one the cached address came from.
+struct CachedSymbol {
+    void *ptr = nullptr;
+    bool have_ctx = false;
+    unsigned long long ctx_id = 0;
+};
+void *cached_symbol_address(CachedSymbol *cache, int n, std::mutex &mu,
+                            cudaError_t (*lookup)(void **));
+
+// SM count and opt-in maximum of dynamic shared memory per block of device `dev`, read
+// once per device (148 and 232448 on a B200 if the query fails).
+int device_sm_count(int dev);
+int max_optin_smem(int dev);
+// The same for the current device.
+int current_sm_count();
 
 // Number of persistent decode CTAs the library launches on a device with `num_sms` SMs.
 int decode_grid_ctas(int num_sms);

@@ -140,9 +140,7 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(RopeArgs a) {
 }
 
 int grid_for(long long items, int threads) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = current_sm_count();
     long long blocks = (items + threads - 1) / threads;
     long long cap = (long long)sms * 8;  // 8 x 256 threads resident per SM
     if (blocks > cap) blocks = cap;

@@ -43,16 +43,22 @@ constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 
 
 template <int D, bool FP8>
 struct PGeo {
-    static constexpr int kSlabs = D / 64;                    // 128-byte column slabs
+    // E4M3 caches at head dim 128: the cache bytes are the operands of kind::f8f6f4 MMAs
+    // (one 128-byte swizzled row per key); at head dim 64 they are widened to f16 first.
+    static constexpr bool kF8 = FP8 && D == 128;
+    static constexpr bool kConv = FP8 && D != 128;
+    static constexpr int kSlabs = D / 64;                    // 128-byte column slabs of bf16 Q
     static constexpr int kSlabBytes = kRows * 128;           // 16 KB (128 rows x 128 B)
     static constexpr int kQBytes = kSlabs * kSlabBytes;      // one Q tile
-    static constexpr int kKVBytes = kSlabs * kSlabBytes;     // one K (or V) tile of 128 keys
+    static constexpr int kKVSlabs = kF8 ? 1 : kSlabs;        // 128-byte slabs of a K/V row
+    static constexpr int kKVBytes = kKVSlabs * kSlabBytes;   // one K (or V) tile of 128 keys
     // Separate K and V rings: K(j) is released as soon as S1(j) completes, V(j) after PV1(j),
     // so the K load that gates S(j+2) gets five MMAs of slack instead of two.  (A third K
-    // stage fits at D 128 in bf16 but measured 1-2 % slower than two.)
-    static constexpr int kKStages = D == 128 ? 2 : 4;
-    static constexpr int kVStages = D == 128 ? 2 : 4;
-    static constexpr int kStgBytes = FP8 ? kKeys * D : 0;    // raw E4M3 tile (K or V)
+    // stage fits at D 128 in bf16 but measured 1-2 % slower than two.)  E4M3 tiles are half
+    // the size, so their rings are twice as deep.
+    static constexpr int kKStages = kF8 ? 4 : (D == 128 ? 2 : 4);
+    static constexpr int kVStages = kF8 ? 4 : (D == 128 ? 2 : 4);
+    static constexpr int kStgBytes = kConv ? kKeys * D : 0;  // raw E4M3 tile (K or V)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = 2 * kQBytes;
     static constexpr int kOffV = kOffK + kKStages * kKVBytes;
@@ -67,6 +73,8 @@ struct PrefillParams {
     __nv_bfloat16 *out;
     const int32_t *cu_seqlens, *block_tables, *context_lens;
     int max_blocks, B, Hq, Hkv, n_qt;
+    int bs;          // tokens per physical block (8, 16 or 32)
+    int max_tokens;  // max_blocks * bs
     int n_items;  // work items (see decode_item); CTAs take them round robin
     long long num_blocks;
     float scale_log2;
@@ -113,6 +121,25 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "r"(0));
 }
 
+// The same two forms for E4M3 operands (kind::f8f6f4; the instruction descriptor's A/B type
+// fields are 0 = E4M3, so mma_idesc(M, N, b_mn_major, true) describes them too).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                          uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum), "r"(0), "r"(0), "r"(0),
+        "r"(0));
+}
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(bar) : "memory");
@@ -155,6 +182,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
@@ -182,6 +217,38 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
     uint32_t r;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"((uint16_t)two));
     return r;
+}
+
+// f16x2 <-> two E4M3 codes (round to nearest even, saturating); low half <-> low byte.
+__device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t h2) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h2));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Four fp32 values with |x| <= 448 -> a high and a low word of four E4M3 codes each, hi + lo
+// holding the value to about 8 significant bits: hi = E4M3(f16(x)), lo = E4M3 of the (exact)
+// f16 remainder.  Low value in the low byte.
+__device__ __forceinline__ void split_e4m3x4(float x0, float x1, float x2, float x3, uint32_t &hi,
+                                             uint32_t &lo) {
+    const uint32_t f01 = pack_f16x2(x0, x1), f23 = pack_f16x2(x2, x3);
+    const uint32_t h01 = f16x2_to_e4m3x2(f01), h23 = f16x2_to_e4m3x2(f23);
+    const uint32_t l01 = f16x2_to_e4m3x2(hsub2(f01, e4m3x2_to_f16x2(h01)));
+    const uint32_t l23 = f16x2_to_e4m3x2(hsub2(f23, e4m3x2_to_f16x2(h23)));
+    hi = h01 | (h23 << 16);
+    lo = l01 | (l23 << 16);
 }
 
 // bf16 -> f16, exact for |x| in [2^-17, 65504] (8 significant bits fit in f16's 11).
@@ -295,13 +362,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(b_pfull + 8 * i, 128);
             mbar_init(b_ofree + 8 * i, 128);
         }
-        // bf16: one arrival with the TMA byte count; FP8: the 64 converter threads
+        // one arrival with the TMA byte count; widened E4M3: the 64 converter threads
         for (int s = 0; s < KS; ++s) {
-            mbar_init(b_kfull + 8 * s, FP8 ? 64 : 1);
+            mbar_init(b_kfull + 8 * s, Geo::kConv ? 64 : 1);
             mbar_init(b_kempty + 8 * s, 1);
         }
         for (int s = 0; s < VS; ++s) {
-            mbar_init(b_vfull + 8 * s, FP8 ? 64 : 1);
+            mbar_init(b_vfull + 8 * s, Geo::kConv ? 64 : 1);
             mbar_init(b_vempty + 8 * s, 1);
         }
         mbar_init(b_stgfull, 1);
@@ -340,13 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
         }
-        const int oob = (int)min(p.num_blocks, (long long)(0x7fffffff / kBlockSize));
+        // first row past the cache: TMA reads it as zeros
+        const int oob = (int)min(p.num_blocks * p.bs, (long long)0x7fffffff);
         for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
             const Item it = decode_item(p, idx);
             if (!active(it)) continue;
             const int n_kv = it.n_kv;
-            const int Lc = min(it.L, p.max_blocks * kBlockSize);
-            const int nblk = (Lc + kBlockSize - 1) / kBlockSize;  // valid blocks of the sequence
+            const int Lc = min(it.L, p.max_tokens);
+            const int npiece = (Lc + kPiece - 1) / kPiece;  // 16-token pieces holding the sequence
             // Q tiles: the previous item's S MMAs must have finished reading the buffer
             if (lane == 0) {
                 if (*abort_flag || (li > 0 && !mbar_wait_bounded(b_qfree, (li - 1) & 1, p.err))) {
@@ -368,18 +436,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int gg = g + j;
                 const int ks = gg % KS, vs = gg % VS;
                 const uint32_t kpar = ((gg / KS) & 1) ^ 1, vpar = ((gg / VS) & 1) ^ 1;
-                int phys = oob;
+                // lane i < 8: cache rows of piece i of the tile (16 keys): one run of 16 from
+                // `phys` (16- and 32-token blocks) or two runs of 8 from `phys` and `phys1`
+                int phys = oob, phys1 = oob;
                 if (lane < 8) {
                     const int lb = j * 8 + lane;
-                    if (lb < nblk) {
-                        phys = __ldg(p.block_tables + (size_t)it.b * p.max_blocks + lb);
-                        if (phys < 0 || (long long)phys >= p.num_blocks) {
-                            atomicOr(p.err, kErrBounds);
-                            phys = oob;
+                    if (lb < npiece) {
+                        const int32_t *tab = p.block_tables + (size_t)it.b * p.max_blocks;
+                        auto row = [&](int entry, int off) {
+                            const int e = __ldg(tab + entry);
+                            if (e < 0 || (long long)e >= p.num_blocks) {
+                                atomicOr(p.err, kErrBounds);
+                                return oob;
+                            }
+                            return e * p.bs + off;
+                        };
+                        if (p.bs == 16) {
+                            phys = row(lb, 0);
+                        } else if (p.bs == 32) {
+                            phys = row(lb >> 1, (lb & 1) * 16);
+                        } else {
+                            phys = row(2 * lb, 0);
+                            if ((2 * lb + 1) * 8 < Lc) phys1 = row(2 * lb + 1, 0);
                         }
                     }
                 }
-                if constexpr (FP8) {
+                if constexpr (Geo::kConv) {
                     // raw E4M3 tiles go to the single staging buffer; the converter warps
                     // widen them into the MMA operand stage
                     if (lane == 0) {
@@ -390,23 +472,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                     if (!ok) break;
-                    int ph[8];
+                    int ph[8], ph1[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) ph[i] = __shfl_sync(0xffffffffu, phys, i);
+                    for (int i = 0; i < 8; ++i) {
+                        ph[i] = __shfl_sync(0xffffffffu, phys, i);
+                        ph1[i] = __shfl_sync(0xffffffffu, phys1, i);
+                    }
                     if (lane == 0) {
                         mbar_arrive_expect_tx(b_stgfull, 2 * Geo::kStgBytes);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            tma_load_3d(sStg + i * kBlockSize * D, &tm_k, b_stgfull, 0, it.kvh, ph[i] * kBlockSize);
-                            tma_load_3d(sStg + Geo::kStgBytes + i * kBlockSize * D, &tm_v, b_stgfull, 0, it.kvh,
-                                        ph[i] * kBlockSize);
+                            tma_load_3d(sStg + i * kPiece * D, &tm_k, b_stgfull, 0, it.kvh, ph[i]);
+                            tma_load_3d(sStg + Geo::kStgBytes + i * kPiece * D, &tm_v, b_stgfull, 0, it.kvh, ph[i]);
+                            if (p.bs == 8) {
+                                tma_load_3d(sStg + (i * kPiece + 8) * D, &tm_k, b_stgfull, 0, it.kvh, ph1[i]);
+                                tma_load_3d(sStg + Geo::kStgBytes + (i * kPiece + 8) * D, &tm_v, b_stgfull, 0,
+                                            it.kvh, ph1[i]);
+                            }
                         }
                         issued |= 1u << 16;
                         phase_bits = (phase_bits & ~(1u << 16)) | ((uint32_t)(gg & 1) << 16);
                     }
                     continue;
                 }
-                const bool fix = (Lc % kBlockSize) != 0 && j == (Lc - 1) / kKeys;
+                // the tile holding the sequence's partial last block: its rows past Lc hold
+                // whatever the block held before and are zeroed before use
+                const bool fix = (Lc % p.bs) != 0 && j == (Lc - 1) / kKeys;
                 if (lane == 0) {
                     if (*abort_flag || !mbar_wait_bounded(b_kempty + 8 * ks, kpar, p.err)) {
                         ok = false;
@@ -415,17 +506,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                int ph[8];
+                int ph[8], ph1[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) ph[i] = __shfl_sync(0xffffffffu, phys, i);
+                for (int i = 0; i < 8; ++i) {
+                    ph[i] = __shfl_sync(0xffffffffu, phys, i);
+                    ph1[i] = __shfl_sync(0xffffffffu, phys1, i);
+                }
+                // piece i of a tile = 16 rows x 128 bytes of each slab (8-token blocks: two boxes of 8)
+                auto load_tile = [&](uint32_t dst, const CUtensorMap *map, uint32_t bar) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        for (int s = 0; s < Geo::kKVSlabs; ++s) {
+                            tma_load_3d(dst + s * Geo::kSlabBytes + i * 2048, map, bar, 64 * s, it.kvh, ph[i]);
+                            if (p.bs == 8)
+                                tma_load_3d(dst + s * Geo::kSlabBytes + i * 2048 + 1024, map, bar, 64 * s, it.kvh,
+                                            ph1[i]);
+                        }
+                };
                 if (lane == 0) {
                     const uint32_t kb = b_kfull + 8 * ks;
                     mbar_arrive_expect_tx(kb, Geo::kKVBytes);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        for (int s = 0; s < Geo::kSlabs; ++s)
-                            tma_load_3d(sK + ks * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_k, kb,
-                                        64 * s, it.kvh, ph[i] * kBlockSize);
+                    load_tile(sK + ks * Geo::kKVBytes, &tm_k, kb);
                     issued |= 1u << ks;
                     phase_bits = (phase_bits & ~(1u << ks)) | ((uint32_t)((gg / KS) & 1) << ks);
                     // V of the same tile: its stage frees later (after PV1 of tile gg - VS)
@@ -435,11 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         const uint32_t vb = fix ? b_vraw : b_vfull + 8 * vs;
                         mbar_arrive_expect_tx(vb, Geo::kKVBytes);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            for (int s = 0; s < Geo::kSlabs; ++s)
-                                tma_load_3d(sV + vs * Geo::kKVBytes + s * Geo::kSlabBytes + i * 2048, &tm_v, vb,
-                                            64 * s, it.kvh, ph[i] * kBlockSize);
+                        load_tile(sV + vs * Geo::kKVBytes, &tm_v, vb);
                         if (!fix) {
                             issued |= 1u << (8 + vs);
                             phase_bits = (phase_bits & ~(1u << (8 + vs))) | ((uint32_t)((gg / VS) & 1) << (8 + vs));
@@ -461,12 +558,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++nfix;
                     if (landed) {
                         if (lane == 0) issued &= ~(1u << 17);
-                        const int blk_in_tile = ((Lc - 1) / kBlockSize) % 8;
-                        const int first = Lc % kBlockSize;
-                        const int rows = kBlockSize - first;
-                        for (int s = 0; s < Geo::kSlabs; ++s) {
-                            const uint32_t row0 = sV + vs * Geo::kKVBytes + s * Geo::kSlabBytes +
-                                                  blk_in_tile * 2048 + first * 128;
+                        // tile rows [Lc, end of that block) (the block lies inside the tile)
+                        const int first = Lc % kKeys;
+                        const int rows = ((Lc + p.bs - 1) / p.bs) * p.bs - Lc;
+                        for (int s = 0; s < Geo::kKVSlabs; ++s) {
+                            const uint32_t row0 = sV + vs * Geo::kKVBytes + s * Geo::kSlabBytes + first * 128;
                             for (int e = lane; e < rows * 8; e += 32)
                                 asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(row0 + e * 16),
                                              "r"(0)
@@ -499,26 +595,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idS = mma_idesc(kRows, kKeys, false, FP8);
+            constexpr uint32_t idS = mma_idesc(kRows, kKeys, false, FP8);  // (E4M3: type code 0, as f16)
             constexpr uint32_t idO = mma_idesc(kRows, D, true, FP8);
             const uint32_t tS[2] = {tmem + 0, tmem + 128};
             const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
             auto issue_s = [&](int i, int kst) {
+                if constexpr (Geo::kF8) {
+                    // S_i = (Q_hi + Q_lo) K^T: the Q tile holds its rows as E4M3 codes, the high
+                    // parts in slab 0 and the low parts in slab 1; 32 codes per k step
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk / 4) * Geo::kSlabBytes + (kk % 4) * 32;
-                    mma_ss(tS[i], sw128_desc(sQ + i * Geo::kQBytes + off, 16, 1024),
-                           sw128_desc(sK + kst * Geo::kKVBytes + off, 16, 1024), idS, kk > 0);
+                    for (int kk = 0; kk < D / 32; ++kk) {
+                        const uint64_t kd = sw128_desc(sK + kst * Geo::kKVBytes + kk * 32, 16, 1024);
+                        mma_ss_f8(tS[i], sw128_desc(sQ + i * Geo::kQBytes + kk * 32, 16, 1024), kd, idS, kk > 0);
+                        mma_ss_f8(tS[i], sw128_desc(sQ + i * Geo::kQBytes + Geo::kSlabBytes + kk * 32, 16, 1024),
+                                  kd, idS, 1u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk / 4) * Geo::kSlabBytes + (kk % 4) * 32;
+                        mma_ss(tS[i], sw128_desc(sQ + i * Geo::kQBytes + off, 16, 1024),
+                               sw128_desc(sK + kst * Geo::kKVBytes + off, 16, 1024), idS, kk > 0);
+                    }
                 }
                 mma_commit(b_sfull + 8 * i);
                 if (i == 1) mma_commit(b_kempty + 8 * kst);  // both S MMAs of this K tile issued
             };
             auto issue_pv = [&](int i, int vst, int j) {
+                if constexpr (Geo::kF8) {
+                    // O_i += (P_hi + P_lo) V: P as E4M3 codes in TMEM (4 keys per column; the high
+                    // parts in columns 0-31, the low in 32-63), V MN-major straight from the cache
 #pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk)
-                    mma_ts(tO[i], tS[i] + 8 * kk,
-                           sw128_desc(sV + vst * Geo::kKVBytes + kk * 2048, Geo::kSlabBytes, 1024), idO,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kKeys / 32; ++kk) {
+                        const uint64_t vd = sw128_desc(sV + vst * Geo::kKVBytes + kk * 4096, Geo::kSlabBytes, 1024);
+                        mma_ts_f8(tO[i], tS[i] + 8 * kk, vd, idO, (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_ts_f8(tO[i], tS[i] + 32 + 8 * kk, vd, idO, 1u);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk)
+                        mma_ts(tO[i], tS[i] + 8 * kk,
+                               sw128_desc(sV + vst * Geo::kKVBytes + kk * 2048, Geo::kSlabBytes, 1024), idO,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
             };
             bool ok = true;
             int li = 0, g = 0;
@@ -575,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(b_drain);
             mbar_wait_bounded(b_drain, 0, p.err);
         }
-    } else if (FP8 && warp >= 2) {
+    } else if (Geo::kConv && warp >= 2) {
         // ---------------------------------------------------------------- E4M3 -> f16
         // Warps 2-3 widen each raw tile into the swizzled operand layout (the same
         // 128-byte-swizzled K-major layout TMA produces for 16-bit caches).  V rows of keys
@@ -587,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int idx = blockIdx.x; idx < p.n_items && run; idx += gridDim.x) {
             const Item it = decode_item(p, idx);
             if (!active(it)) continue;
-            const int Lc = min(it.L, p.max_blocks * kBlockSize);
+            const int Lc = min(it.L, p.max_tokens);
             for (int j = 0; j < it.n_kv; ++j) {
                 const int gg = g + j;
                 const int ks = gg % KS, vs = gg % VS;
@@ -671,7 +790,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return false;
         };
-        auto prologue = [&](const Item &it, int li) {
+        // returns the reciprocal of the power-of-two scale applied to this thread's Q row
+        // before its E4M3 split (1 on the other paths)
+        auto prologue = [&](const Item &it, int li) -> float {
             const int row = it.row0[wg] + r;  // row within the sequence's new tokens
             const bool row_valid = row < it.n;
             const int pos = it.L - it.n + row;
@@ -781,9 +902,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if constexpr (FP8) {
-                // the FP8 path multiplies in f16: convert this row of Q (swizzle untouched), after
-                // both warpgroups finished rotating (they may share rows)
+            float qinv = 1.f;
+            if constexpr (Geo::kConv) {
+                // the widened-E4M3 path multiplies in f16: convert this row of Q (swizzle
+                // untouched), after both warpgroups finished rotating (they may share rows)
                 named_bar(2, 256);
                 if (ok) {
                     const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
@@ -799,26 +921,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            if constexpr (Geo::kF8) {
+                // E4M3 operands: after both warpgroups finished rotating, this thread turns its
+                // row of tile wg into 128 high and 128 low E4M3 codes, in place -- the high
+                // ones as slab 0's row, the low ones as slab 1's (each a 128-byte K-major
+                // swizzled row, the layout of an E4M3 A tile).  The row is first scaled by the
+                // power of two that puts its largest |q| in [224, 448]; the score scale takes
+                // the reciprocal.
+                named_bar(2, 256);
+                if (ok) {
+                    const uint32_t qrow = sQ + wg * Geo::kQBytes + r * 128;
+                    const uint32_t sw = (uint32_t)(r & 7);
+                    uint32_t w[64];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const uint4 x = lds128(qrow + (c >> 3) * Geo::kSlabBytes + (((c & 7) ^ sw) << 4));
+                        w[4 * c] = x.x;
+                        w[4 * c + 1] = x.y;
+                        w[4 * c + 2] = x.z;
+                        w[4 * c + 3] = x.w;
+                    }
+                    float amax = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16lo(w[i])), fabsf(bf16hi(w[i]))));
+                    const float sq = amax > 0.f
+                                         ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
+                                         : 1.f;
+                    qinv = 1.f / sq;  // exact: sq is a power of two
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {  // codes 16k .. 16k+15 = bf16 words 8k .. 8k+7
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t w0 = w[8 * k + 2 * j], w1 = w[8 * k + 2 * j + 1];
+                            split_e4m3x4(bf16lo(w0) * sq, bf16hi(w0) * sq, bf16lo(w1) * sq, bf16hi(w1) * sq, hw[j],
+                                         lw[j]);
+                        }
+                        const uint32_t off = (uint32_t)((k ^ sw) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(qrow + off), "r"(hw[0]),
+                                     "r"(hw[1]), "r"(hw[2]), "r"(hw[3]) : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(qrow + Geo::kSlabBytes + off),
+                                     "r"(lw[0]), "r"(lw[1]), "r"(lw[2]), "r"(lw[3]) : "memory");
+                    }
+                }
+            }
             fence_proxy_async_smem();
             mbar_arrive(b_qready);
+            return qinv;
         };
 
         // Q of item li+1 is rotated before the epilogue of item li, so the tensor pipe can
         // start the next item's S MMAs while this item's O is written out.
         Item it;
         bool have = next_item(it);
-        if (have) prologue(it, 0);
+        float qinv = 1.f;
+        if (have) qinv = prologue(it, 0);
         int li = 0, g = 0;
         while (have) {
             if (*abort_flag) alive = false;
             const int n_kv = it.n_kv;
-            const int Lc = min(it.L, p.max_blocks * kBlockSize);
+            const int Lc = min(it.L, p.max_tokens);
             if (Lc < it.L && r == 0 && wg == 0) atomicOr(p.err, kErrBounds);
             const int row = it.row0[wg] + r;              // row within the sequence's new tokens
             const bool row_valid = row < it.n;
             const int pos = it.L - it.n + row;
             const int limit = min(pos, Lc - 1);           // last visible key
-            const float c = p.scale_log2 * (p.k_scale ? __ldg(p.k_scale + it.kvh) : 1.f);
+            const float c = p.scale_log2 * (p.k_scale ? __ldg(p.k_scale + it.kvh) : 1.f) * qinv;
             // Every tcgen05.ld/st below is executed by all 32 lanes of the warp together (the
             // instructions are warp-aligned); per-row differences are data, not control flow.
             float m_used = -INFINITY, l_sum = 0.f;
@@ -867,16 +1035,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                  make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int h = 0; h < kKeys / 32; ++h) {  // 32 keys -> 16 packed columns
-                    uint32_t rr[16];
+                for (int h = 0; h < kKeys / 32; ++h) {  // 32 keys
+                    if constexpr (Geo::kF8) {
+                        // -> 8 columns of high E4M3 parts (4 keys each) at 8h, 8 of low parts at 32 + 8h
+                        uint32_t hw[8], lw[8];
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 x = __ffma2_rn(make_float2(s[h * 32 + e], s[h * 32 + e + 1]), c2, nm2);
-                        const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-                        acc[(e / 2) & 3] = __fadd2_rn(acc[(e / 2) & 3], pp);
-                        rr[e / 2] = FP8 ? pack_f16x2(pp.x, pp.y) : pack_bf16x2(pp.x, pp.y);
+                        for (int e = 0; e < 32; e += 4) {
+                            const float2 x0 = __ffma2_rn(make_float2(s[h * 32 + e], s[h * 32 + e + 1]), c2, nm2);
+                            const float2 x1 = __ffma2_rn(make_float2(s[h * 32 + e + 2], s[h * 32 + e + 3]), c2, nm2);
+                            const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y)), p1 = make_float2(ex2(x1.x), ex2(x1.y));
+                            acc[(e / 2) & 3] = __fadd2_rn(acc[(e / 2) & 3], p0);
+                            acc[(e / 2 + 1) & 3] = __fadd2_rn(acc[(e / 2 + 1) & 3], p1);
+                            split_e4m3x4(p0.x, p0.y, p1.x, p1.y, hw[e / 4], lw[e / 4]);
+                        }
+                        tmem_st8(tS + h * 8, hw);
+                        tmem_st8(tS + 32 + h * 8, lw);
+                    } else {
+                        // -> 16 packed columns
+                        uint32_t rr[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 x = __ffma2_rn(make_float2(s[h * 32 + e], s[h * 32 + e + 1]), c2, nm2);
+                            const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+                            acc[(e / 2) & 3] = __fadd2_rn(acc[(e / 2) & 3], pp);
+                            rr[e / 2] = FP8 ? pack_f16x2(pp.x, pp.y) : pack_bf16x2(pp.x, pp.y);
+                        }
+                        tmem_st16(tS + h * 16, rr);
                     }
-                    tmem_st16(tS + h * 16, rr);
                 }
                 l_sum += ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
                          ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
@@ -901,7 +1086,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             Item nxt;
             const bool have_next = next_item(nxt);
-            if (have_next) prologue(nxt, li + 1);
+            float qinv_next = 1.f;
+            if (have_next) qinv_next = prologue(nxt, li + 1);
             // ---- epilogue: O / l -> bf16 -> global (valid rows only)
             bool fin = alive && mbar_wait_bounded(b_ofinal, li & 1, p.err);
             if (!fin) alive = false;
@@ -940,6 +1126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++li;
             it = nxt;
             have = have_next;
+            qinv = qinv_next;
         }
     }
 
@@ -956,20 +1143,23 @@ cudaError_t run(const PrefillArgs &a, const PrefillParams &p, long long items, c
     // Q: 128-byte swizzled boxes of 64 bf16 x 128 rows (one operand slab each).  K/V: for
     // bf16 the same 128-byte swizzled 64-column boxes of one block (16 rows); for E4M3 one
     // plain box of a whole block row range (widened in shared memory by the kernel).
+    // E4M3 at head dim 128: one 128-byte-swizzled box per block (a whole 128-byte row per key).
+    using Geo = PGeo<D, FP8>;
     constexpr int esize = FP8 ? 1 : 2;
     CUtensorMap tq, tk, tv;
-    const uint64_t slots = (uint64_t)a.num_blocks * kBlockSize;
+    const uint64_t slots = (uint64_t)a.num_blocks * a.block_size;
+    const uint32_t box_rows = a.block_size == 8 ? 8u : (uint32_t)kPiece;
     const uint32_t inner = FP8 ? (uint32_t)D : 64u;
+    constexpr bool swz = !Geo::kConv;
     if (!encode_tensor_map_3d(&tq, a.q, 2, D, a.n_q_heads, a.num_tokens, 64, 1, kRows, true) ||
-        !encode_tensor_map_3d(&tk, a.k_cache, esize, D, a.n_kv_heads, slots, inner, 1, kBlockSize, !FP8) ||
-        !encode_tensor_map_3d(&tv, a.v_cache, esize, D, a.n_kv_heads, slots, inner, 1, kBlockSize, !FP8))
+        !encode_tensor_map_3d(&tk, a.k_cache, esize, D, a.n_kv_heads, slots, inner, 1, box_rows, swz) ||
+        !encode_tensor_map_3d(&tv, a.v_cache, esize, D, a.n_kv_heads, slots, inner, 1, box_rows, swz))
         return cudaErrorInvalidValue;
     auto k = prefill_kernel<D, FP8>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, PGeo<D, FP8>::kSmem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (shared memory allows one), items taken round robin
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = current_sm_count();
     const long long grid = items < sms ? items : sms;
     return launch_pdl(k, dim3((unsigned)grid), dim3(kThreads), PGeo<D, FP8>::kSmem, s, tq, tk, tv, p);
 }
@@ -983,6 +1173,8 @@ cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s) {
     p.block_tables = a.block_tables;
     p.context_lens = a.context_lens;
     p.max_blocks = a.max_blocks_per_seq;
+    p.bs = a.block_size;
+    p.max_tokens = (int)min((long long)a.max_blocks_per_seq * a.block_size, 0x7fffffffLL);
     p.B = a.num_seqs;
     p.Hq = a.n_q_heads;
     p.Hkv = a.n_kv_heads;

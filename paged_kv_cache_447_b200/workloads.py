@@ -100,8 +100,8 @@ def _randn_bf16(g: torch.Generator, *shape) -> torch.Tensor:
 
 
 def _fill_cache(g: torch.Generator, nb: int, hkv: int, d: int, fp8: bool,
-                k_scale=None, v_scale=None, nan_fill: bool = False):
-    shape = (nb, BLOCK_SIZE, hkv, d)
+                k_scale=None, v_scale=None, nan_fill: bool = False, block_size: int = BLOCK_SIZE):
+    shape = (nb, block_size, hkv, d)
     if nan_fill:
         if fp8:
             return (torch.full(shape, 0x7F, dtype=torch.uint8),
@@ -148,17 +148,18 @@ def _assign_blocks(perm: torch.Tensor, counts, max_blocks: int, shared=None) -> 
     return bt
 
 
-def _slots(bt: torch.Tensor, b: int, positions) -> list:
-    return [int(bt[b, p // BLOCK_SIZE]) * BLOCK_SIZE + p % BLOCK_SIZE for p in positions]
+def _slots(bt: torch.Tensor, b: int, positions, block_size: int = BLOCK_SIZE) -> list:
+    return [int(bt[b, p // block_size]) * block_size + p % block_size for p in positions]
 
 
-def _step(name, g, hq, hkv, d, new_counts, ctx_lens, bt, decode_seqs=0) -> Step:
+def _step(name, g, hq, hkv, d, new_counts, ctx_lens, bt, decode_seqs=0,
+          block_size: int = BLOCK_SIZE) -> Step:
     T = int(sum(new_counts))
     cu = torch.zeros(len(new_counts) + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(torch.tensor(new_counts, dtype=torch.int64), 0).to(torch.int32)
     slots = []
     for b, (n, L) in enumerate(zip(new_counts, ctx_lens)):
-        slots += _slots(bt, b, range(L - n, L))
+        slots += _slots(bt, b, range(L - n, L), block_size)
     return Step(name=name, q=_randn_bf16(g, T, hq, d), k=_randn_bf16(g, T, hkv, d),
                 v=_randn_bf16(g, T, hkv, d), slot_mapping=torch.tensor(slots, dtype=torch.int32),
                 cu_seqlens=cu, context_lens=torch.tensor(ctx_lens, dtype=torch.int32),
@@ -236,6 +237,27 @@ def shared_prefix(seed: int = 4, requests: int = 32, prefix: int = 2048, new: in
                [prefix + new] * requests, bt)
     return Workload("shared_prefix", seed, hq, hkv, d, nb, "bf16", kc, vc, [st],
                     max_pos=prefix + new, notes={"shared_prefix_blocks": shared})
+
+
+def paged_batch(seed: int, hq: int, hkv: int, d: int, news, ctxs, block_size: int = BLOCK_SIZE,
+                fp8: bool = False, decode_seqs: int = 0, spare_blocks: int = 3,
+                nan_fill: bool = False) -> Workload:
+    """One step over a freshly filled paged cache of any block size / head dim: sequence b
+    has ctxs[b] cached tokens, the last news[b] of them new in this step; its blocks come
+    from a seeded permutation of the pool.  (Block-size and head-dim variants.)"""
+    g = torch.Generator().manual_seed(seed)
+    counts = [-(-L // block_size) for L in ctxs]
+    nb = sum(counts) + spare_blocks
+    perm = torch.randperm(nb, generator=g)
+    bt = _assign_blocks(perm, counts, max_blocks=max(counts) + 1)
+    st = _step("batch", g, hq, hkv, d, list(news), list(ctxs), bt, decode_seqs=decode_seqs,
+               block_size=block_size)
+    ks = vs = None
+    if fp8:
+        ks, vs = _fp8_scales(st.k, st.v)
+    kc, vc = _fill_cache(g, nb, hkv, d, fp8, ks, vs, nan_fill=nan_fill, block_size=block_size)
+    return Workload("batch", seed, hq, hkv, d, nb, "fp8" if fp8 else "bf16", kc, vc, [st],
+                    max_pos=max(ctxs) + 1, k_scale=ks, v_scale=vs, block_size=block_size)
 
 
 def lognormal_lengths(g: torch.Generator, n: int, median: float = 1024.0, sigma: float = 1.0,

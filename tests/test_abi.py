@@ -60,8 +60,8 @@ def test_host_argument_checks_need_no_device():
     n = None
     # head_dim 96 is not compiled
     assert lib.pkv_kv_store(n, n, n, n, n, 4, 2, 96, 16, 32, 0, n, n, n, 0, n, n, 0, n) == -2
-    # block size 8 is not compiled
-    assert lib.pkv_kv_store(n, n, n, n, n, 4, 2, 64, 8, 32, 0, n, n, n, 0, n, n, 0, n) == -2
+    # block sizes other than 8, 16, 32 are not compiled
+    assert lib.pkv_kv_store(n, n, n, n, n, 4, 2, 64, 12, 32, 0, n, n, n, 0, n, n, 0, n) == -2
     # null pointers
     assert lib.pkv_kv_store(n, n, n, n, n, 4, 2, 64, 16, 32, 0, n, n, n, 0, n, n, 0, n) == -1
     # Hq not a multiple of Hkv
@@ -88,8 +88,8 @@ def test_block_helpers_host_checks_need_no_device():
     n = None
     buf = ctypes.create_string_buffer(64)
     p = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
-    # slot mapping: block size 8 not compiled; negative sizes; null pointers; empty is a no-op
-    assert lib.pkv_slot_mapping(p, p, 4, p, p, 2, 5, 8, 32, n) == -2
+    # slot mapping: block size 12 not compiled; negative sizes; null pointers; empty is a no-op
+    assert lib.pkv_slot_mapping(p, p, 4, p, p, 2, 5, 12, 32, n) == -2
     assert lib.pkv_slot_mapping(p, p, 4, p, p, -1, 5, 16, 32, n) == -1
     assert lib.pkv_slot_mapping(n, p, 4, p, p, 2, 5, 16, 32, n) == -1
     assert lib.pkv_slot_mapping(p, p, 0, p, p, 2, 5, 16, 32, n) == -1
@@ -121,3 +121,129 @@ def test_missing_library_fails_loudly():
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.startswith("raised") and "missing" in r.stdout
+
+
+# ---- the header's prototypes, the binding's ctypes signatures and a C caller agree
+
+_CTYPE = {"int": ctypes.c_int, "long long": ctypes.c_longlong, "size_t": ctypes.c_size_t,
+          "float": ctypes.c_float, "double": ctypes.c_double, "void": None}
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) for every function pkv.h declares."""
+    src = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"#[^\n]*", "", src)
+    protos = {}
+    for ret, name, params in re.findall(
+            r"((?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?\s*\**)\s*\b(pkv_[a-z0-9_]+)\s*\(([^)]*)\)\s*;",
+            src, flags=re.S):
+        ps = [p.strip() for p in params.split(",")]
+        types = []
+        for p in ps:
+            if p in ("void", ""):
+                continue
+            p = re.sub(r"\s+", " ", p)
+            t = re.sub(r"\s*\b[A-Za-z_][A-Za-z0-9_]*$", "", p)  # drop the parameter name
+            types.append(t.strip())
+        protos[name] = (re.sub(r"\s+", " ", ret.strip()), types)
+    return protos
+
+
+def _as_ctype(t: str):
+    t = t.replace("const ", "").strip()
+    if t.endswith("*") or t == "pkv_stream_t":
+        return "char*" if t == "char *" else ctypes.c_void_p
+    return _CTYPE[t]
+
+
+def test_binding_signatures_match_the_header():
+    """Every argtypes / restype the ctypes binding sets equals what pkv.h declares, in
+    order -- an int passed where the header has long long (or a swapped pair) fails."""
+    protos = _prototypes()
+    lib = binding.load_library()
+    assert set(protos) == set(_declared_symbols())
+    for name, (ret, params) in protos.items():
+        fn = getattr(lib, name)
+        want = [_as_ctype(p) for p in params]
+        got = list(fn.argtypes or [])
+        assert len(got) == len(want), (name, params)
+        for i, (g, w) in enumerate(zip(got, want)):
+            if w == "char*":
+                w = ctypes.c_char_p
+            assert g is w, f"{name} argument {i}: binding {g}, header {params[i]}"
+        wr = _as_ctype(ret)
+        if ret.replace(" ", "") == "constchar*":
+            wr = ctypes.c_char_p
+        assert fn.restype is wr, f"{name} returns {ret}, binding {fn.restype}"
+
+
+def _build_c_driver(tmp_path):
+    """Compile tests/abi_check.c against include/pkv.h only (-Wall -Werror) and link it to
+    the library."""
+    import subprocess
+    src = os.path.join(ROOT, "tests", "abi_check.c")
+    exe = str(tmp_path / "abi_check")
+    libdir = os.path.dirname(binding.library_path())
+    cuda = "/usr/local/cuda"
+    cmd = ["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-O1", "-I", os.path.join(ROOT, "include"),
+           "-I", f"{cuda}/include", src, "-o", exe, "-L", libdir, "-lpagedkv",
+           f"-Wl,-rpath,{libdir}", "-L", f"{cuda}/lib64", "-lcudart", f"-Wl,-rpath,{cuda}/lib64", "-lm"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    return exe
+
+
+def test_c_caller_host_entry_points(tmp_path):
+    """A C program that includes pkv.h calls every host-side entry point and the argument
+    checks that return before touching a device."""
+    import subprocess
+    exe = _build_c_driver(tmp_path)
+    r = subprocess.run([exe, "host"], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "host checks passed" in r.stdout
+
+
+@pytest.mark.gpu
+def test_c_caller_runs_the_hot_path(tmp_path):
+    """The same C program stores a tiny batch (K rotated), runs prefill and decode through
+    the header's prototypes with device buffers it allocates itself, and writes the outputs;
+    they must match the oracle."""
+    import subprocess
+    from paged_kv_cache_447_b200 import workloads as W
+    from helpers import oracle_attention, oracle_caches, oracle_store
+    exe = _build_c_driver(tmp_path)
+    wl = W.tiny(seed=1)
+    pre, dec = wl.steps
+    kc, vc = oracle_caches(wl)
+    files = {}
+
+    def put(name, arr):
+        path = str(tmp_path / name)
+        np.ascontiguousarray(arr).tofile(path)
+        files[name] = path
+
+    put("k_cache", kc)
+    put("v_cache", vc)
+    for tag, st in (("pre", pre), ("dec", dec)):
+        for f in ("q", "k", "v"):
+            put(f"{tag}_{f}", W.bits(getattr(st, f)))
+        for f in ("slot_mapping", "cu_seqlens", "context_lens", "block_tables"):
+            put(f"{tag}_{f}", getattr(st, f).numpy().astype(np.int32))
+    dims = [wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.num_blocks, wl.max_pos,
+            pre.num_seqs, pre.num_tokens, pre.block_tables.shape[1], pre.max_new_tokens,
+            dec.num_seqs, dec.num_tokens, dec.block_tables.shape[1]]
+    r = subprocess.run([exe, "device", str(tmp_path)] + [str(x) for x in dims],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    # oracle side: the same two steps
+    outs = {}
+    for tag, st in (("pre", pre), ("dec", dec)):
+        oracle_store(wl, st, kc, vc)
+        outs[tag] = oracle_attention(wl, st, kc, vc)
+    for tag, st in (("pre", pre), ("dec", dec)):
+        got = np.fromfile(str(tmp_path / f"out_{tag}"), dtype=np.uint16)
+        got = oracle.bf16_to_f64(got).reshape(outs[tag].shape)
+        err = np.abs(got - outs[tag])
+        assert err.max() <= 1e-2 and err.mean() <= 1e-3, (tag, err.max())
+    assert np.array_equal(np.fromfile(str(tmp_path / "k_cache_out"), dtype=np.uint16).reshape(kc.shape), kc)

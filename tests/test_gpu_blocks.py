@@ -129,3 +129,137 @@ def test_copy_on_write_divergence_decode(fp8):
     assert np.array_equal(cache_bits(dw.k_cache)[:2], before)
     ref = oracle_attention(wl, st, okc, ovc, rope=True)
     compare(out, ref, fp8=fp8, what=f"copy-on-write decode fp8={fp8}")
+
+
+# ---------------------------------------------------------------- block pool on the device
+
+def _pool_state(pool: torch.Tensor):
+    p = pool.cpu().numpy()
+    nb = (p.shape[0] - 4) // 2
+    return int(p[0]), p[4:4 + nb], p[4 + nb:]
+
+
+def _same_pool(gpu_pool, orc_pool):
+    n, stack, flags = _pool_state(gpu_pool)
+    nb = stack.shape[0]
+    assert n == int(orc_pool[0])
+    assert np.array_equal(stack[:n], orc_pool[1:1 + n])
+    assert np.array_equal(flags, orc_pool[1 + nb:])
+
+
+def test_block_pool_random_traffic_bit_exact():
+    """Batches of admissions and growth (some larger than the pool can cover) and frees of
+    finished sequences, on the device and in the oracle: after every call the free count,
+    the stack of free ids, the free flags and every table written are identical."""
+    rng = np.random.default_rng(3)
+    nb, mb = 96, 24
+    pool = pkv.block_pool(nb)
+    orc = oracle.pool_init(nb)
+    _same_pool(pool, orc)
+    live = {}
+    next_id = 0
+    refused = 0
+    for _ in range(120):
+        if live and rng.random() < 0.35:
+            ids = []
+            for s in rng.choice(list(live), size=min(len(live), int(rng.integers(1, 3))), replace=False):
+                ids += live.pop(int(s))[1]
+            pkv.block_pool_free(pool, torch.tensor(ids, dtype=torch.int32, device="cuda"))
+            assert oracle.pool_free(orc, ids) == 0
+            assert pkv.get_error() == 0
+        else:
+            batch = [(s, int(rng.integers(1, 30))) for s in list(live)[:4]]
+            for _ in range(int(rng.integers(0, 3))):
+                batch.append((next_id, int(rng.integers(1, 200))))
+                next_id += 1
+            if not batch:
+                continue
+            bt = np.full((len(batch), mb), -1, np.int32)
+            ctx, new = [], []
+            for i, (s, n) in enumerate(batch):
+                L0, table = live.get(s, (0, []))
+                bt[i, :len(table)] = table
+                ctx.append(L0 + n)
+                new.append(n)
+            cu = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+            ctx = np.array(ctx, np.int32)
+            bt_dev = torch.from_numpy(bt.copy()).cuda()
+            pkv.block_pool_alloc(pool, bt_dev, torch.from_numpy(cu).cuda(), torch.from_numpy(ctx).cuda())
+            rc = oracle.pool_alloc(orc, bt, cu, ctx)
+            code = pkv.get_error()
+            if rc != 0:
+                refused += 1
+                assert code in (-9, -6)
+            else:
+                assert code == 0
+                for i, (s, n) in enumerate(batch):
+                    live[s] = (int(ctx[i]), [int(x) for x in bt[i] if x >= 0])
+            assert np.array_equal(bt_dev.cpu().numpy(), bt)
+        _same_pool(pool, orc)
+    assert refused > 0  # the run did exercise the all-or-nothing refusal
+
+
+def test_block_pool_rejects_double_and_foreign_frees():
+    nb = 8
+    pool = pkv.block_pool(nb)
+    orc = oracle.pool_init(nb)
+    bt = torch.full((1, 4), -1, dtype=torch.int32, device="cuda")
+    cu = torch.tensor([0, 40], dtype=torch.int32, device="cuda")
+    ctx = torch.tensor([40], dtype=torch.int32, device="cuda")
+    pkv.block_pool_alloc(pool, bt, cu, ctx)
+    btn = np.full((1, 4), -1, np.int32)
+    oracle.pool_alloc(orc, btn, cu.cpu().numpy(), ctx.cpu().numpy())
+    assert pkv.get_error() == 0
+    ids = [2, 0, 2, 9, -1, 5, 1]   # 2 twice, 9 and -1 outside, 5 not allocated
+    pkv.block_pool_free(pool, torch.tensor(ids, dtype=torch.int32, device="cuda"))
+    assert pkv.get_error() == -6
+    assert oracle.pool_free(orc, ids) == 4
+    _same_pool(pool, orc)
+    assert _pool_state(pool)[0] == 8
+
+
+def test_block_pool_end_to_end_alloc_store_decode_free():
+    """Blocks from the pool, slots from the tables, the store and decode attention over
+    them, then the blocks back: the cache is what the oracle stores at the same slots and
+    the output matches the oracle."""
+    g = torch.Generator().manual_seed(12)
+    hq, hkv, d, nb, mb = 8, 2, 128, 64, 16
+    pool = pkv.block_pool(nb)
+    kc = torch.zeros((nb, 16, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    okc = np.zeros((nb, 16, hkv, d), np.uint16)
+    ovc = np.zeros_like(okc)
+    table = pkv.rope_build_table(512, d).cuda()
+    otab = oracle.rope_table(512, d)
+    bt = torch.full((3, mb), -1, dtype=torch.int32, device="cuda")
+    lens = [0, 0, 0]
+    for step, new in enumerate(([37, 5, 140], [1, 1, 1], [1, 20, 1])):
+        ctx = [L + n for L, n in zip(lens, new)]
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(new)]), dtype=torch.int32, device="cuda")
+        ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+        pkv.block_pool_alloc(pool, bt, cu, ctx_t)
+        T = sum(new)
+        slots = pkv.slot_mapping(bt, cu, ctx_t, T, nb)
+        k = W._randn_bf16(g, T, hkv, d).cuda()
+        v = W._randn_bf16(g, T, hkv, d).cuda()
+        q = W._randn_bf16(g, T, hq, d).cuda()
+        pkv.kv_store(k, v, kc, vc, slots, rope_cos_sin=table, cu_seqlens=cu, context_lens=ctx_t)
+        pos = oracle.positions(cu.cpu().numpy(), np.array(ctx, np.int32))
+        oracle.kv_store(W.bits(k.cpu()), W.bits(v.cpu()), okc, ovc, slots.cpu().numpy(), 16,
+                        table=otab, pos=pos)
+        out = pkv.paged_prefill_attention(q, kc, vc, cu, bt, ctx_t, max(new), rope_cos_sin=table)
+        torch.cuda.synchronize()
+        assert pkv.get_error() == 0
+        assert np.array_equal(W.bits(kc.cpu()), okc) and np.array_equal(W.bits(vc.cpu()), ovc)
+        ref = oracle.attention(W.bits(q.cpu()), okc, ovc, cu.cpu().numpy(), bt.cpu().numpy(),
+                               np.array(ctx, np.int32), 1.0 / np.sqrt(d), 16, hkv, table=otab)
+        err = np.abs(out.float().cpu().numpy() - ref)
+        assert err.max() <= 1e-2 and err.mean() <= 1e-3
+        lens = ctx
+    used = int(sum(-(-L // 16) for L in lens))
+    assert _pool_state(pool)[0] == nb - used
+    held = bt.cpu().numpy()
+    ids = torch.from_numpy(held[held >= 0].astype(np.int32)).cuda()
+    assert ids.numel() == used and len(set(ids.tolist())) == used
+    pkv.block_pool_free(pool, ids)
+    assert pkv.get_error() == 0 and _pool_state(pool)[0] == nb

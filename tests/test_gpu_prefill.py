@@ -62,17 +62,23 @@ def test_prefill_lengths(prefix, new):
 def test_prefill_shared_prefix_full_size_sampled():
     """The 32-request shared-prefix workload at full size (2048-token aliased prefix + 2048
     new tokens each, 32 q / 8 kv heads): the whole output is produced in the launch
-    configuration the benchmark times, and sampled rows are checked against the oracle."""
+    configuration the benchmark times (persistent CTAs, many items each), and three rows of
+    every 128-row tile of every request -- the tile's first and last rows and one drawn at
+    random -- are checked against the oracle for every q head (all 8 kv heads)."""
     wl = W.shared_prefix(seed=4)
     st = wl.steps[0]
     rng = np.random.default_rng(0)
     rows = []
-    for b in (0, 13, 31):
+    for b in range(st.num_seqs):
         base = int(st.cu_seqlens[b])
-        for r in (0, 1, 127, 128, 1000, 2046, 2047) + tuple(rng.integers(0, 2048, 6)):
-            for h in (0, 3, 17, 31):
-                rows.append((base + int(r), h))
+        n = int(st.cu_seqlens[b + 1]) - base
+        for t0 in range(0, n, 128):
+            last = min(t0 + 127, n - 1)
+            for r in (t0, last, int(rng.integers(t0, last + 1))):
+                for h in range(wl.n_q_heads):
+                    rows.append((base + r, h))
     rows = np.array(rows, dtype=np.int32)
+    assert len(rows) == 32 * 16 * 3 * 32
     out, ref = _prefill_case(wl, rows=rows)
     got = out[torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()]
     compare(got, ref, what="shared prefix sampled")

@@ -743,3 +743,98 @@ def test_copy_on_write_divergence_equals_private_copy():
     ref = oracle.attention(W.bits(q), kp, vp, cu, private, ctx, d ** -0.5, bs, hkv)
     assert np.array_equal(got, ref)
     assert np.array_equal(kc[0], before)
+
+
+# ----------------------------------------------------------------------------- block pool
+
+def test_block_pool_hand_worked_sequence():
+    """tests/golden/block_pool.txt: allocations in sequence order from the top of the free
+    stack, nothing taken for tokens that fit the blocks held, LIFO reuse of freed blocks, a
+    request the pool cannot cover refused whole, double and out-of-range frees rejected."""
+    pool = oracle.pool_init(8)
+    tables = {}
+    steps = {}
+    for r in _golden_rows("block_pool.txt"):
+        steps.setdefault(r[0], []).append(r)
+    for step in sorted(steps, key=int):
+        rows = steps[step]
+        if rows[0][1] == "free":
+            r = rows[0]
+            arrow = r.index("->")
+            ids = [int(x) for x in r[2:arrow]]
+            rej = oracle.pool_free(pool, ids)
+            tail = r[arrow + 1:]
+            assert int(pool[0]) == int(tail[tail.index(";") + 1])
+            assert rej == int(tail[-1])
+            continue
+        names = [r[2] for r in rows]
+        bt = np.full((len(rows), 8), -1, np.int32)
+        for i, name in enumerate(names):
+            held = tables.get(name, [])
+            bt[i, :len(held)] = held
+        ctx = np.array([int(r[3]) for r in rows], np.int32)
+        cu = np.concatenate([[0], np.cumsum([int(r[4]) for r in rows])]).astype(np.int32)
+        rc = oracle.pool_alloc(pool, bt, cu, ctx)
+        for i, r in enumerate(rows):
+            arrow = r.index("->")
+            semi = r.index(";")
+            want = r[arrow + 1:semi]
+            if want == ["refused"]:
+                assert rc == -1
+            else:
+                assert rc == 0
+                got = [int(x) for x in bt[i] if x >= 0]
+                assert got == [int(x) for x in want], (r, got)
+                tables[names[i]] = got
+            assert int(pool[0]) == int(r[semi + 1])
+
+
+def test_block_pool_invariants_under_random_traffic():
+    """Random admissions, growth and completions against a model kept with Python sets:
+    no block is ever held by two sequences or held and free at once, every held-or-free id
+    is accounted for, every sequence's table covers exactly ceil(L / 16) blocks, and a
+    refused request changes nothing."""
+    rng = np.random.default_rng(7)
+    nb = 64
+    pool = oracle.pool_init(nb)
+    live = {}          # seq -> (L, table list)
+    next_id = 0
+    for _ in range(400):
+        if live and rng.random() < 0.3:
+            s = int(rng.choice(list(live)))
+            _, table = live.pop(s)
+            assert oracle.pool_free(pool, table) == 0
+        else:
+            batch = []
+            for s in list(live)[:3]:
+                batch.append((s, int(rng.integers(1, 40))))
+            if rng.random() < 0.6:
+                batch.append((next_id, int(rng.integers(1, 90))))
+                next_id += 1
+            if not batch:
+                continue
+            bt = np.full((len(batch), 32), -1, np.int32)
+            ctx, new = [], []
+            for i, (s, n) in enumerate(batch):
+                L0, table = live.get(s, (0, []))
+                bt[i, :len(table)] = table
+                ctx.append(L0 + n)
+                new.append(n)
+            before = pool.copy()
+            cu = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+            rc = oracle.pool_alloc(pool, bt, cu, np.array(ctx, np.int32))
+            need = sum(-(-c // 16) - (-(-(c - n) // 16)) for c, n in zip(ctx, new))
+            if rc != 0:
+                assert need > int(before[0]) or max(-(-c // 16) for c in ctx) > 32
+                assert np.array_equal(pool, before)
+                continue
+            for i, (s, n) in enumerate(batch):
+                table = [int(x) for x in bt[i] if x >= 0]
+                assert len(table) == -(-ctx[i] // 16)
+                live[s] = (ctx[i], table)
+        held = [x for _, t in live.values() for x in t]
+        free = [int(x) for x in pool[1:1 + int(pool[0])]]
+        assert len(set(held)) == len(held) and len(set(free)) == len(free)
+        assert not set(held) & set(free) and len(held) + len(free) == nb
+        flags = pool[1 + nb:]
+        assert all(flags[x] == 1 for x in free) and all(flags[x] == 0 for x in held)

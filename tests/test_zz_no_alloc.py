@@ -7,16 +7,17 @@ synchronise the device.  For them the library offers a decode entry point withou
 workspace argument; it uses a fixed 8 MiB array inside the library's device image.
 
 These tests call it through the C ABI and check that two calls in a row give what the
-ordinary (workspace-taking) entry point gives, within the attention tolerance used by
-every other decode test.  The file is named so that pytest collects it last."""
-import numpy as np
+ordinary (workspace-taking) entry point gives.  Both run the same kernels with the same
+launch geometry on the same inputs, so the outputs must be identical bit for bit (which is
+within any tolerance): a stale or clobbered scratch array would show up as a difference.
+The file is named so that pytest collects it last."""
 import pytest
 import torch
 
 import paged_kv_cache_447_b200 as pkv
 from paged_kv_cache_447_b200 import workloads as W
 
-from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, FP8_MAX_ABS, DeviceWorkload
+from helpers import DeviceWorkload
 
 pytestmark = pytest.mark.gpu
 
@@ -39,13 +40,9 @@ def _both(d: DeviceWorkload, st: W.Step):
     return ref, out, free_before, free_after
 
 
-def _close(a: torch.Tensor, b: torch.Tensor, fp8: bool):
-    err = (a.float() - b.float()).abs()
+def _same(a: torch.Tensor, b: torch.Tensor):
     assert torch.isfinite(a.float()).all()
-    if fp8:
-        assert float(err.max()) <= FP8_MAX_ABS
-    else:
-        assert float(err.max()) <= BF16_MAX_ABS and float(err.mean()) <= BF16_MEAN_ABS
+    assert torch.equal(a, b), float((a.float() - b.float()).abs().max())
 
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
@@ -63,13 +60,14 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
                                           d.wl.head_dim) <= pkv.NOALLOC_SCRATCH_BYTES
     ref1, out1, _, _ = _both(d1, st1)
     ref2, out2, free_b, free_a = _both(d2, st2)
-    _close(out1, ref1, fp8=False)
-    _close(out2, ref2, fp8=True)
+    _same(out1, ref1)
+    _same(out2, ref2)
     # the second call allocated nothing on the device
     assert free_a == free_b
     # and repeating call 1 after call 2 (scratch left holding call 2's data) still matches
     ref1b, out1b, _, _ = _both(d1, st1)
-    _close(out1b, ref1, fp8=False)
+    _same(ref1b, ref1)
+    _same(out1b, ref1)
 
 
 def test_noalloc_rejects_calls_beyond_the_scratch_limit():
@@ -90,7 +88,5 @@ def test_noalloc_rejects_calls_beyond_the_scratch_limit():
     assert e.value.code == -8
     # nothing was enqueued and the device is fine
     assert pkv.get_error() == 0
-    out = pkv.paged_decode_attention_noalloc(st.q.cuda(), d.k_cache, d.v_cache,
-                                             st.block_tables.cuda(), st.context_lens.cuda())
-    torch.cuda.synchronize()
-    assert torch.isfinite(out.float()).all()
+    ref, out, _, _ = _both(d, st)
+    _same(out, ref)
