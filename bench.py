@@ -602,6 +602,8 @@ def main():
                 del rr
                 torch.cuda.empty_cache()
                 keep = {k: v for k, v in r.items() if k not in ("clocks",)}
+                if r.get("clocks"):
+                    keep["clocks"] = {k: r["clocks"][k] for k in ("sm_mhz", "reasons")}
                 if "attn_gbs" in r:
                     keep["attn_hbm_frac"] = r["attn_gbs"] / pk["hbm_gbs"]
                 if "prefill_tflops" in r:

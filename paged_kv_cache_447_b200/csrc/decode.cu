@@ -17,6 +17,7 @@ size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int h
 }
 
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t s) {
+    if (decode_tc_supported(a)) return launch_paged_decode_tc(a, s);
     return dispatch_decode<false>(a, s);
 }
 

@@ -870,11 +870,24 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
             __syncwarp();
             // p.v: lane owns dims [lane*DPL, (lane+1)*DPL)
             constexpr int DPL = Geo::kDimsPerLane;
+            static_assert(DPL == 2 || DPL == 4 || DPL == 8, "head dim 64, 128 or 256");
             auto pv_row = [&](int jj, const float *pw) {
                 float vf[DPL];
                 const uint32_t va = vs_a + jj * Geo::kRowBytes + lane * DPL * Geo::kElem;
                 if constexpr (FP8) {
-                    if constexpr (DPL == 4) {
+                    if constexpr (DPL == 8) {
+                        const uint2 w2 = lds64(va);
+                        const uint32_t ww[2] = {w2.x, w2.y};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t h2;
+                            const uint16_t pair = (uint16_t)(ww[q >> 1] >> (16 * (q & 1)));
+                            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+                            float2 f = __half22float2(*reinterpret_cast<__half2 *>(&h2));
+                            vf[2 * q] = f.x;
+                            vf[2 * q + 1] = f.y;
+                        }
+                    } else if constexpr (DPL == 4) {
                         const uint32_t w = lds32(va);
 #pragma unroll
                         for (int hb = 0; hb < 2; ++hb) {
@@ -895,7 +908,15 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                         vf[1] = f.y;
                     }
                 } else {
-                    if constexpr (DPL == 4) {
+                    if constexpr (DPL == 8) {
+                        const uint4 w = lds128(va);
+                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            vf[2 * q] = bf16lo(ww[q]);
+                            vf[2 * q + 1] = bf16hi(ww[q]);
+                        }
+                    } else if constexpr (DPL == 4) {
                         const uint2 w = lds64(va);
                         vf[0] = bf16lo(w.x);
                         vf[1] = bf16hi(w.x);

@@ -20,6 +20,7 @@ size_t decode_step_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, 
 }
 
 cudaError_t launch_paged_decode_step(const DecodeArgs &a, cudaStream_t s) {
+    if (decode_tc_supported(a)) return launch_paged_decode_step_tc(a, s);
     return dispatch_decode<true>(a, s);
 }
 

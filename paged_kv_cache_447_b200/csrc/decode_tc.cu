@@ -1,0 +1,820 @@
+// decode_tc.cu -- paged decode attention of grouped query heads over an E4M3 cache on the
+// 5th-generation tensor cores (tcgen05.mma kind::f8f6f4).
+//
+// "Inside the Nano-vLLM engine: KV cache, attention and tensor parallelism", §3 (one query
+// token per sequence against the cached K/V), §3.1 (tiles, softmax kept on chip), §3.2
+// (subtract the maximum); "LLM primer", §17.1 (decode is bound by memory bandwidth) and
+// §17.6 (an FP8 cache halves the bytes per token).  The result is that of decode_kernel;
+// what differs is how the arithmetic reaches the hardware.
+//
+// Work: persistent CTAs (one per SM) split the units -- 128-token tiles of one (sequence,
+// kv head), numbered sequence-major -- into equal contiguous ranges (stream-K); a range's
+// run of tiles of one (sequence, kv head) is a piece with one softmax state, merged with the
+// other pieces of its sequence by the combine kernel exactly as decode_kernel's partials.
+//   warp 0      TMA producer: the tile's K and V rows (8 boxes of 16 rows each, 128-byte
+//               swizzled, straight from the cache) into a 5-stage ring
+//   warp 1      TMEM owner and the one MMA-issuing thread
+//   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
+// Per tile:
+//   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
+//                 cache stores it (K-major), B = q as E4M3 rows -- the G heads' high parts in
+//                 rows 0..G-1, their low parts (the E4M3 remainder) in rows G..2G-1, zeros
+//                 after -- so one MMA yields both partial scores of every head in TMEM.
+//   softmax       thread t adds its two parts, masks past the context, takes the per-head
+//                 tile maxima across the four warps, updates the lazy running max (O is
+//                 rescaled only when a max grows by more than 2^8) and writes p as high and
+//                 low E4M3 parts into a shared-memory P tile: row h / G+h, byte t.
+//   O += P V      M = 64 (rows 0..2G-1 used), N = 128 dims, K = 128 tokens: A = the P tile,
+//                 B = the V tile MN-major as the cache stores it; O = rows h + rows G+h.
+// The MMA thread never blocks on one event: it polls for the next PV (P written) and the next
+// S^T (tile landed, S buffer free, the piece's q staged) and issues whichever is ready, PV
+// first, so a stage goes back to the producer as soon as its PV is issued.  S, P and q are
+// double-buffered, and so is O (by piece), so the epilogue of one piece overlaps the next
+// piece's MMAs; the next piece's q is staged before the epilogue.
+#include "decode_kernel.cuh"
+#include "tcgen05.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kTcThreads = 192;
+constexpr int kTcTile = 128;    // tokens per unit
+constexpr int kTcStages = 5;
+constexpr int kTcSoftmax0 = 2;  // first softmax warp
+constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
+constexpr uint32_t kTcO = 128;  // TMEM column of O buffer 0 (buffer 1 follows at +128)
+
+template <int G>
+struct TcGeo {
+    static constexpr int D = 128;
+    static constexpr int kKV = kTcTile * D;         // one E4M3 K (or V) tile: 16 KB
+    static constexpr int kStage = 2 * kKV;
+    static constexpr int kQ = 16 * 128;             // B operand of S^T: 16 rows x 128 codes
+    static constexpr int kP = 64 * 128;             // A operand of PV: 64 rows x 128 tokens
+    static constexpr int kOffQ = kTcStages * kStage;
+    static constexpr int kOffP = kOffQ + 2 * kQ;
+    static constexpr int kOffRed = kOffP + 2 * kP;  // [4 warps][8] floats x 2 (max, sum)
+    static constexpr int kOffQtmp = kOffRed + 2 * 4 * 8 * 4;  // rotated bf16 q [G][128]
+    static constexpr int kOffBar = kOffQtmp + 8 * 128 * 2;
+    static constexpr int kBars = 2 * kTcStages + 12;
+    static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
+    static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
+    static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
+};
+
+// Barrier indices (8 bytes each after kOffBar)
+constexpr int kBFull = 0;                 // [kTcStages]  K/V landed (TMA bytes)
+constexpr int kBEmpty = kTcStages;        // [kTcStages]  K/V consumed (PV commit)
+constexpr int kBSFull = 2 * kTcStages;    // [2] S^T in TMEM (commit)
+constexpr int kBSFree = kBSFull + 2;      // [2] softmax has read S^T (128 arrivals)
+constexpr int kBPFull = kBSFree + 2;      // [2] P tile written (128 arrivals)
+constexpr int kBPvDone = kBPFull + 2;     // [2] PV done reading P buffer (commit)
+constexpr int kBQFull = kBPvDone + 2;     // q staged for the piece (128 arrivals)
+constexpr int kBOFree = kBQFull + 1;      // [2] O buffer read by its piece's epilogue (32 arrivals)
+constexpr int kBDrain = kBOFree + 2;      // every MMA of the CTA has completed (commit)
+static_assert(kBDrain < 2 * kTcStages + 12, "barrier count");
+
+__device__ __forceinline__ uint32_t bar_at(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
+
+// Non-blocking test of an mbarrier phase (the MMA thread polls several).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Row r, byte c of a 128-byte-row swizzled tile (16-byte chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+    return (uint32_t)(r * 128 + ((((c >> 4) ^ (r & 7)) << 4) | (c & 15)));
+}
+
+// Decode step: store the step's new token of sequence b, kv head kvh (the newest of its L
+// tokens, row (L-1) % 128 of its last tile, cache slot `slot`) into the cache and into the
+// tile's K and V rows, which TMA filled with the slot's previous codes -- K rotated at L - 1,
+// both quantised from the fp64 quotient by the head's scale, as pkv_kv_store does.  One warp.
+__device__ __forceinline__ void tc_put_new_token(const DecodeParams &p, int b, int kvh, int L, int slot,
+                                                 uint32_t kt, uint32_t vt, int lane) {
+    constexpr int D = 128;
+    const int r = (L - 1) % kTcTile, pos = L - 1;
+    const float *rope = nullptr;
+    if (p.rope) {
+        if (pos >= p.max_pos) {
+            if (lane == 0) atomicOr(p.err, kErrBounds);
+            return;
+        }
+        rope = p.rope + (size_t)pos * D;
+    }
+    const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
+    const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
+    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;
+    const double ks = (double)__ldg(p.k_scale + kvh), vs = (double)__ldg(p.v_scale + kvh);
+    for (int i = lane; i < D / 2; i += 32) {
+        uint16_t kb[2] = {__ldg(kin + i), __ldg(kin + i + D / 2)};
+        const uint16_t vb[2] = {__ldg(vin + i), __ldg(vin + i + D / 2)};
+        if (rope) rope_pair_fast(kb[0], kb[1], __ldg(rope + i), __ldg(rope + D / 2 + i), kb[0], kb[1]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = i + h * (D / 2);
+            const uint32_t kc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[h]), ks));
+            const uint32_t vc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(vb[h]), vs));
+            static_cast<uint8_t *>(p.k_cache_w)[dst + e] = (uint8_t)kc;
+            static_cast<uint8_t *>(p.v_cache_w)[dst + e] = (uint8_t)vc;
+            asm volatile("st.shared.u8 [%0], %1;" ::"r"(kt + sw_off(r, e)), "r"(kc) : "memory");
+            asm volatile("st.shared.u8 [%0], %1;" ::"r"(vt + sw_off(r, e)), "r"(vc) : "memory");
+        }
+    }
+}
+
+template <int G, bool STEP>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const DecodeParams p) {
+    using Geo = TcGeo<G>;
+    constexpr int D = Geo::D;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (sbase - smem_u32(smem_raw));
+    const uint32_t sStages = sbase, sQ = sbase + Geo::kOffQ, sP = sbase + Geo::kOffP;
+    float *red = reinterpret_cast<float *>(smem + Geo::kOffRed);
+    uint16_t *qtmp = reinterpret_cast<uint16_t *>(smem + Geo::kOffQtmp);
+    const uint32_t bars = sbase + Geo::kOffBar;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Geo::kOffBar + 8 * Geo::kBars);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kOffBar + 8 * Geo::kBars + 4);
+    int *pfx = reinterpret_cast<int *>(smem + Geo::kOffPfx);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    pdl_wait();
+    pdl_trigger();
+    // prefix of the sequences' tile counts (units per sequence and kv head)
+    {
+        __shared__ int wsum[kTcThreads / 32];
+        __shared__ int carry_s;
+        if (threadIdx.x == 0) carry_s = 0;
+        __syncthreads();
+        for (int base = 0; base < p.B; base += kTcThreads) {
+            const int b = base + threadIdx.x;
+            int v = 0;
+            if (b < p.B) {
+                int L = __ldg(p.context_lens + b);
+                if (L < 0) L = 0;
+                if (L > p.max_tokens) {
+                    atomicOr(p.err, kErrBounds);
+                    L = p.max_tokens;
+                }
+                v = (L + kTcTile - 1) / kTcTile;
+            }
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) wsum[warp] = incl;
+            __syncthreads();
+            int before = carry_s;
+            for (int w = 0; w < warp; ++w) before += wsum[w];
+            if (b < p.B) pfx[b] = before + incl - v;
+            __syncthreads();
+            if (threadIdx.x == kTcThreads - 1) carry_s = before + incl;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) pfx[p.B] = carry_s;
+        __syncthreads();
+    }
+    const int Hu = p.Hkv;
+    const long long total = (long long)Hu * pfx[p.B];
+    if (!STEP && blockIdx.x == 0)
+        for (int i = threadIdx.x; i <= p.B; i += kTcThreads) p.prefix[i] = pfx[i];
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x)
+        if (pfx[b + 1] == pfx[b])
+            for (int e = threadIdx.x; e < p.Hq * D; e += kTcThreads)
+                p.out[(size_t)b * p.Hq * D + e] = __float2bfloat16_rn(0.f);
+    const long long U = total > 0 ? (total + p.nctas - 1) / p.nctas : 1;
+    const long long u0 = (long long)blockIdx.x * U;
+    const long long u1 = (u0 + U < total) ? u0 + U : total;
+    if (u0 >= u1) return;  // uniform across the CTA
+    const int nunits = (int)(u1 - u0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(bar_at(bars, kBFull + s), 1);
+            mbar_init(bar_at(bars, kBEmpty + s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_at(bars, kBSFull + i), 1);
+            mbar_init(bar_at(bars, kBSFree + i), 128);
+            mbar_init(bar_at(bars, kBPFull + i), 128);
+            mbar_init(bar_at(bars, kBPvDone + i), 1);
+        }
+        mbar_init(bar_at(bars, kBQFull), 128);
+        mbar_init(bar_at(bars, kBOFree), 32);
+        mbar_init(bar_at(bars, kBOFree + 1), 32);
+        mbar_init(bar_at(bars, kBDrain), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // zero the rows of the q and P operands that no head uses (rows 2G.. stay zero)
+    for (int i = threadIdx.x; i < (2 * Geo::kQ + 2 * Geo::kP) / 16; i += kTcThreads)
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(sQ + 16 * i), "r"(0u) : "memory");
+    fence_proxy_async_smem();
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
+                     ::"r"(smem_u32((const void *)tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // TMEM: S^T buffers at columns 0 and 16 (128 lanes x 16), O buffers at columns 128 and 256
+    // (rows 0..2G-1 of 64 x 128 each)
+
+    // unit k of this CTA -> (sequence, kv head, tile); `first` = a piece starts here
+    auto unit = [&](int k, int &b, int &kvh, int &tile, int &ntiles) {
+        UnitPos up = locate(pfx, p.B, Hu, u0 + k);
+        b = up.b;
+        kvh = up.kvh;
+        tile = up.blk;
+        ntiles = up.nb;
+    };
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+        }
+        const int oob = (int)(p.num_blocks * p.bs < 0x7fffffffLL ? p.num_blocks * p.bs : 0x7fffffff);
+        uint32_t issued = 0, phases = 0;
+        bool ok = true;
+        for (int k = 0; k < nunits && ok; ++k) {
+            int b, kvh, tile, ntiles;
+            unit(k, b, kvh, tile, ntiles);
+            const int L = min(__ldg(p.context_lens + b), p.max_tokens);
+            // lane i < 8: cache rows of the tile's piece i (16 tokens); two runs for 8-token blocks
+            int r0 = oob, r1 = oob;
+            if (lane < 8) {
+                const int pc = tile * 8 + lane;  // 16-token piece of the sequence
+                if (pc * 16 < L) {
+                    const int32_t *tab = p.block_tables + (size_t)b * p.max_blocks;
+                    if (p.bs == 16) {
+                        r0 = cache_row(p, __ldg(tab + pc), 0);
+                    } else if (p.bs == 32) {
+                        r0 = cache_row(p, __ldg(tab + (pc >> 1)), (pc & 1) * 16);
+                    } else {
+                        r0 = cache_row(p, __ldg(tab + 2 * pc), 0);
+                        if ((2 * pc + 1) * 8 < L) r1 = cache_row(p, __ldg(tab + 2 * pc + 1), 0);
+                    }
+                }
+            }
+            int rr0[8], rr1[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                rr0[i] = __shfl_sync(0xffffffffu, r0, i);
+                rr1[i] = __shfl_sync(0xffffffffu, r1, i);
+            }
+            if (lane == 0) {
+                const int s = k % kTcStages;
+                if (*abort_flag || !mbar_wait_bounded(bar_at(bars, kBEmpty + s), ((k / kTcStages) & 1) ^ 1, p.err)) {
+                    ok = false;
+                    *abort_flag = 1;
+                } else {
+                    const uint32_t fb = bar_at(bars, kBFull + s);
+                    const uint32_t dk = sStages + s * Geo::kStage, dv = dk + Geo::kKV;
+                    mbar_arrive_expect_tx(fb, Geo::kStage);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        tma_load_3d(dk + i * 2048, &tm_k, fb, 0, kvh, rr0[i]);
+                        tma_load_3d(dv + i * 2048, &tm_v, fb, 0, kvh, rr0[i]);
+                        if (p.bs == 8) {
+                            tma_load_3d(dk + i * 2048 + 1024, &tm_k, fb, 0, kvh, rr1[i]);
+                            tma_load_3d(dv + i * 2048 + 1024, &tm_v, fb, 0, kvh, rr1[i]);
+                        }
+                    }
+                    issued |= 1u << s;
+                    phases = (phases & ~(1u << s)) | ((uint32_t)((k / kTcStages) & 1) << s);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        }
+        if (lane == 0)  // never leave with a TMA copy landing in shared memory
+            for (int s = 0; s < kTcStages; ++s)
+                if ((issued >> s) & 1) mbar_wait_bounded(bar_at(bars, kBFull + s), (phases >> s) & 1, p.err);
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        // Lane 0 tests the barriers and issues; the whole warp walks the units (with STEP it
+        // stores the step's new token into the tile before that tile's S^T is issued).
+        constexpr uint32_t idS = tc::mma_idesc(128, 16, false, true);  // E4M3 x E4M3 -> f32
+        constexpr uint32_t idO = tc::mma_idesc(64, D, true, true);     // B (V) MN-major
+        int ks = 0, kp = 0;       // next S^T, next PV
+        int spc = -1, ppc = -1;   // piece of the last S^T / PV issued
+        bool s_known = false, p_known = false, s_first = false, p_first = false;
+        int sb_ = 0, skvh = 0, stile = 0, snt = 0;
+        bool ok = true;
+        int idle = 0;
+        unsigned long long t_idle = 0;
+        while (kp < nunits) {
+            bool did = false;
+            // ---- PV of tile kp, into the O buffer of its piece
+            if (kp < ks) {
+                if (!p_known) {
+                    int b, kvh, tile, nt;
+                    unit(kp, b, kvh, tile, nt);
+                    p_first = kp == 0 || tile == 0;
+                    p_known = true;
+                }
+                const int pc = ppc + (p_first ? 1 : 0);
+                int go = 0;
+                if (lane == 0)  // a piece's first PV overwrites its O buffer: piece pc-2's epilogue must have read it
+                    go = mbar_test(bar_at(bars, kBPFull + (kp & 1)), (kp >> 1) & 1) &&
+                         (!p_first || pc < 2 || mbar_test(bar_at(bars, kBOFree + (pc & 1)), ((pc >> 1) - 1) & 1));
+                if (__shfl_sync(0xffffffffu, go, 0)) {
+                    if (lane == 0) {
+                        tc::tc_fence_after();
+                        const uint32_t vd = sStages + (kp % kTcStages) * Geo::kStage + Geo::kKV;
+                        const uint32_t pd = sP + (kp & 1) * Geo::kP;
+                        const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(pc & 1);
+#pragma unroll
+                        for (int kk = 0; kk < kTcTile / 32; ++kk)
+                            tc::mma_ss_f8(tO, tc::sw128_desc(pd + 32 * kk, 16, 1024),
+                                          tc::sw128_desc(vd + 4096 * kk, 16384, 1024), idO,
+                                          (p_first && kk == 0) ? 0u : 1u);
+                        tc::mma_commit(bar_at(bars, kBEmpty + kp % kTcStages));
+                        tc::mma_commit(bar_at(bars, kBPvDone + (kp & 1)));
+                    }
+                    __syncwarp();
+                    ppc = pc;
+                    ++kp;
+                    p_known = false;
+                    did = true;
+                }
+            }
+            // ---- S^T of tile ks
+            if (ks < nunits) {
+                if (!s_known) {
+                    unit(ks, sb_, skvh, stile, snt);
+                    s_first = ks == 0 || stile == 0;
+                    s_known = true;
+                }
+                const int pc = spc + (s_first ? 1 : 0);
+                int go = 0;
+                if (lane == 0)
+                    go = mbar_test(bar_at(bars, kBFull + ks % kTcStages), (ks / kTcStages) & 1) &&
+                         (ks < 2 || mbar_test(bar_at(bars, kBSFree + (ks & 1)), ((ks - 2) >> 1) & 1)) &&
+                         (!s_first || mbar_test(bar_at(bars, kBQFull), pc & 1));
+                if (__shfl_sync(0xffffffffu, go, 0)) {
+                    const uint32_t kd = sStages + (ks % kTcStages) * Geo::kStage;
+                    if constexpr (STEP) {
+                        const int Lraw = __ldg(p.context_lens + sb_), L = min(Lraw, p.max_tokens);
+                        if (stile == snt - 1 && L == Lraw) {  // the sequence's last tile holds its new token
+                            const int e = __ldg(p.block_tables + (size_t)sb_ * p.max_blocks + (L - 1) / p.bs);
+                            if (e >= 0 && (long long)e < p.num_blocks)
+                                tc_put_new_token(p, sb_, skvh, L, e * p.bs + (L - 1) % p.bs, kd, kd + Geo::kKV, lane);
+                            fence_proxy_async_smem();  // the tensor cores read these rows next
+                            __syncwarp();
+                        }
+                    }
+                    if (lane == 0) {
+                        tc::tc_fence_after();
+                        const uint32_t qd = sQ + (pc & 1) * Geo::kQ;
+#pragma unroll
+                        for (int kk = 0; kk < D / 32; ++kk)
+                            tc::mma_ss_f8(tmem + 16 * (ks & 1), tc::sw128_desc(kd + 32 * kk, 16, 1024),
+                                          tc::sw128_desc(qd + 32 * kk, 16, 1024), idS, kk > 0);
+                        tc::mma_commit(bar_at(bars, kBSFull + (ks & 1)));
+                    }
+                    __syncwarp();
+                    spc = pc;
+                    ++ks;
+                    s_known = false;
+                    did = true;
+                }
+            }
+            if (did) {
+                idle = 0;
+                continue;
+            }
+            // nothing ready: yield the issue slots to the softmax warp on this SM sub-partition,
+            // and give up (error flag) after the wait limit without progress
+            int stop = 0;
+            if (lane == 0) {
+                if (*abort_flag) {
+                    stop = 1;
+                } else if (idle == 0) {
+                    t_idle = globaltimer();
+                } else if ((idle & 63) == 0 && globaltimer() - t_idle > kWaitLimitNs) {
+                    atomicOr(p.err, kErrTimeout);
+                    stop = 1;
+                }
+            }
+            if (__shfl_sync(0xffffffffu, stop, 0)) {
+                ok = false;
+                break;
+            }
+            ++idle;
+            __nanosleep(32);
+        }
+        if (!ok && lane == 0) *abort_flag = 1;
+        // drain: no MMA may still write TMEM when it is released
+        if (lane == 0) {
+            tc::mma_commit(bar_at(bars, kBDrain));
+            mbar_wait_bounded(bar_at(bars, kBDrain), 0, p.err);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- softmax / epilogue
+        const int sw = warp - kTcSoftmax0;               // 0..3
+        const int quad = warp & 3;                        // TMEM lanes 32*quad .. +31
+        const int t = quad * 32 + lane;                   // token of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int ct = threadIdx.x - 32 * kTcSoftmax0;    // 0..127
+        bool alive = true;
+        // Stage q of the piece starting at unit kk (piece index pc) into q buffer pc & 1: the
+        // G heads rotated at L-1, one power-of-two scale for the group (returned), high parts
+        // to rows 0..G-1 and low parts to rows G..2G-1.
+        auto stage_q = [&](int kk, int pc) -> float {
+            int b, kvh, tile, ntiles;
+            unit(kk, b, kvh, tile, ntiles);
+            const int L = min(__ldg(p.context_lens + b), p.max_tokens);
+            float amax = 0.f;
+            for (int e = ct; e < G * (D / 2); e += 128) {
+                const int h = e / (D / 2), i = e % (D / 2);
+                const uint16_t *qr = p.q + ((size_t)b * p.Hq + kvh * G + h) * D;
+                uint16_t x1 = __ldg(qr + i), x2 = __ldg(qr + i + D / 2);
+                if (p.rope) {
+                    const int pos = L - 1;
+                    if (pos >= 0 && pos < p.max_pos) {
+                        const float *row = p.rope + (size_t)pos * D;
+                        rope_pair_fast(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
+                    } else {
+                        atomicOr(p.err, kErrBounds);
+                    }
+                }
+                qtmp[h * D + i] = x1;
+                qtmp[h * D + i + D / 2] = x2;
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float((uint32_t)x1 << 16)),
+                                         fabsf(__uint_as_float((uint32_t)x2 << 16))));
+            }
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if (lane == 0) red[sw] = amax;
+            named_bar(kTcBar, 128);
+            amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+            named_bar(kTcBar, 128);  // red and qtmp are rewritten later
+            const float sq = amax > 0.f
+                                 ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
+                                 : 1.f;
+            const uint32_t qd = sQ + (pc & 1) * Geo::kQ;
+            for (int e = ct; e < G * (D / 4); e += 128) {  // four dims per thread
+                const int h = e / (D / 4), c = 4 * (e % (D / 4));
+                const uint2 w = *reinterpret_cast<const uint2 *>(qtmp + h * D + c);
+                uint32_t hi, lo;
+                tc::split_e4m3x4(bf16lo(w.x) * sq, bf16hi(w.x) * sq, bf16lo(w.y) * sq, bf16hi(w.y) * sq, hi, lo);
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(h, c)), "r"(hi) : "memory");
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(G + h, c)), "r"(lo) : "memory");
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_at(bars, kBQFull));
+            return sq;
+        };
+        int k = 0, piece = 0;
+        float sq = stage_q(0, 0);
+        while (k < nunits) {
+            int b, kvh, tile, ntiles;
+            unit(k, b, kvh, tile, ntiles);
+            const int piece_len = min(ntiles - tile, nunits - k);
+            const int L = min(__ldg(p.context_lens + b), p.max_tokens);
+            const bool whole = tile == 0 && piece_len == ntiles;
+            const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
+            const float sc = p.scale_log2 * __ldg(p.k_scale + kvh) / sq;
+            float mref[G], lsum[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                mref[h] = -INFINITY;
+                lsum[h] = 0.f;
+            }
+            for (int j = 0; j < piece_len; ++j, ++k) {
+                const int sb = k & 1, s = k % kTcStages;
+                bool got = alive && !*abort_flag && mbar_wait_bounded(bar_at(bars, kBSFull + sb), (k >> 1) & 1, p.err);
+                if (!__all_sync(0xffffffffu, got)) {
+                    alive = false;
+                    *abort_flag = 1;
+                }
+                float sv[G];
+                if (alive) {
+                    tc::tc_fence_after();
+                    uint32_t c[16];
+                    tc::tmem_ld16(tmem + lane_off + 16 * sb, c);
+                    tc::tc_wait_ld();
+                    const int valid = min(kTcTile, L - (tile + j) * kTcTile);
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        sv[h] = t < valid ? (__uint_as_float(c[h]) + __uint_as_float(c[G + h])) * sc : -INFINITY;
+                    if (t >= valid) {
+                        // V rows past the context would multiply P = 0 by whatever they hold
+                        const uint32_t vrow = sStages + s * Geo::kStage + Geo::kKV + t * 128;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + 16 * q), "r"(0u)
+                                         : "memory");
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) sv[h] = -INFINITY;
+                }
+                tc::tc_fence_before();
+                mbar_arrive(bar_at(bars, kBSFree + sb));
+                // per-head maxima of the tile over the 128 tokens
+                float mt[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float m = sv[h];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                    mt[h] = m;
+                }
+                if (lane == 0)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) red[8 * sw + h] = mt[h];
+                named_bar(kTcBar, 128);
+                float alpha[G];
+                bool rescale = false;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float m = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
+                    alpha[h] = 1.f;
+                    if (m > mref[h] + 8.0f) {  // (token 0 of a tile is always valid: m is finite)
+                        alpha[h] = ex2(mref[h] - m);
+                        mref[h] = m;
+                        rescale = rescale || j > 0;
+                    }
+                }
+                named_bar(kTcBar, 128);  // red is rewritten by the next tile
+                float pr[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    pr[h] = ex2(sv[h] - mref[h]);
+                    lsum[h] = lsum[h] * alpha[h] + pr[h];
+                }
+                // P buffer (k & 1) was last read by the PV of tile k - 2
+                const int pb = k & 1;
+                if (alive && k >= 2 && !mbar_wait_bounded(bar_at(bars, kBPvDone + pb), ((k - 2) >> 1) & 1, p.err)) {
+                    alive = false;
+                    *abort_flag = 1;
+                }
+                const uint32_t pd = sP + pb * Geo::kP;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    uint32_t hi, lo;  // (only the first of the four codes is used)
+                    tc::split_e4m3x4(pr[h], 0.f, 0.f, 0.f, hi, lo);
+                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(h, t)), "r"(hi & 0xFFu) : "memory");
+                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(G + h, t)), "r"(lo & 0xFFu) : "memory");
+                }
+                if (rescale && alive) {
+                    // O rows h and G+h (TMEM lanes 0..2G-1, warp quad 0) times alpha_h, once the
+                    // PV of the previous tile has finished
+                    const int pj = (k - 1) & 1;
+                    if (!mbar_wait_bounded(bar_at(bars, kBPvDone + pj), ((k - 1) >> 1) & 1, p.err)) {
+                        alive = false;
+                        *abort_flag = 1;
+                    }
+                    if (quad == 0 && __all_sync(0xffffffffu, alive)) {
+                        tc::tc_fence_after();
+                        float a = 1.f;
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+                            if (lane == h || lane == G + h) a = alpha[h];
+#pragma unroll 1
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t rr[32];
+                            tc::tmem_ld32(tO + c0, rr);
+                            tc::tc_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * a);
+                            tc::tmem_st32(tO + c0, rr);
+                        }
+                        tc::tc_wait_st();
+                    }
+                }
+                fence_proxy_async_smem();
+                tc::tc_fence_before();
+                mbar_arrive(bar_at(bars, kBPFull + pb));
+            }
+            // ---- end of the piece: the sums over the 128 tokens, the next piece's q, then the
+            // epilogue (O from TMEM), which overlaps the next piece's MMAs
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float l = lsum[h];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+                if (lane == 0) red[32 + 8 * sw + h] = l;
+            }
+            named_bar(kTcBar, 128);
+            const float sq_next = k < nunits ? stage_q(k, piece + 1) : 1.f;
+            if (quad == 0) {
+                const int jl = k - 1;  // the piece's last tile
+                bool fin = alive && mbar_wait_bounded(bar_at(bars, kBPvDone + (jl & 1)), (jl >> 1) & 1, p.err);
+                fin = __all_sync(0xffffffffu, fin);
+                if (!fin) {
+                    alive = false;
+                    *abort_flag = 1;
+                }
+                tc::tc_fence_after();
+                // lanes 0..G-1 hold O rows h (high parts of p), lanes G..2G-1 rows G+h (low parts)
+                const int h = lane < G ? lane : (lane < 2 * G ? lane - G : 0);
+                float m = -INFINITY;
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh)
+                    if (hh == h) m = mref[hh];
+                const float l = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
+                const int segu = b * Hu + kvh;
+                float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
+                const float vs = __ldg(p.v_scale + kvh);
+                const float inv = (l > 0.f && fin) ? vs / l : 0.f;
+                __nv_bfloat16 *orow = p.out + ((size_t)b * p.Hq + kvh * G + h) * D;
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t rr[32];
+                    if (fin) {
+                        tc::tmem_ld32(tO + c0, rr);
+                        tc::tc_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) rr[e] = 0u;
+                    }
+                    float o[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __uint_as_float(rr[e]) + __shfl_down_sync(0xffffffffu, __uint_as_float(rr[e]), G);
+                    if (lane < G) {
+                        if (whole) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                uint4 w;
+                                w.x = tc::pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+                                w.y = tc::pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+                                w.z = tc::pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+                                w.w = tc::pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+                                dst[v] = w;
+                            }
+                        } else {
+                            float4 *dst = reinterpret_cast<float4 *>(slot + h * D + c0);
+#pragma unroll
+                            for (int v = 0; v < 8; ++v)
+                                dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+                        }
+                    }
+                }
+                if (!whole && lane < G) {
+                    slot[G * D + lane] = m;
+                    slot[G * D + G + lane] = l;
+                }
+                tc::tc_fence_before();
+                mbar_arrive(bar_at(bars, kBOFree + (piece & 1)));
+                if constexpr (STEP) {
+                    if (!whole) {
+                        // the last of the CTAs c0..c1 that cut this segment merges it (as the
+                        // combine kernel does) and clears the counter for the next call
+                        __threadfence();
+                        __syncwarp();
+                        const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
+                        const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
+                        int last = 0;
+                        if (lane == 0) last = atomicAdd(p.counters + segu, 1) == c1 - c0;
+                        last = __shfl_sync(0xffffffffu, last, 0);
+                        if (last) {
+                            __threadfence();
+                            // four dims per lane: M = max m_c, o = sum e^(m_c - M) acc_c / sum e^(m_c - M) l_c
+#pragma unroll
+                            for (int i = 0; i < G * D / 128; ++i) {
+                                const int e = (i * 32 + lane) * 4, g = e / D, d = e % D;
+                                float M = -INFINITY;
+                                for (int cc = c0; cc <= c1; ++cc)
+                                    M = fmaxf(M, __ldcg(p.partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D + g));
+                                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                                float ls = 0.f;
+                                for (int cc = c0; cc <= c1; ++cc) {
+                                    const float *sl = p.partials + (size_t)(segu + cc) * (G * (D + 2));
+                                    const float mk = __ldcg(sl + G * D + g);
+                                    const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
+                                    const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));
+                                    acc.x += f * x.x;
+                                    acc.y += f * x.y;
+                                    acc.z += f * x.z;
+                                    acc.w += f * x.w;
+                                    ls += f * __ldcg(sl + G * D + G + g);
+                                }
+                                const float r = ls > 0.f ? vs / ls : 0.f;
+                                uint2 w;
+                                w.x = tc::pack_bf16x2(acc.x * r, acc.y * r);
+                                w.y = tc::pack_bf16x2(acc.z * r, acc.w * r);
+                                *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
+                            }
+                            if (lane == 0) p.counters[segu] = 0;
+                        }
+                    }
+                }
+            }
+            ++piece;
+            sq = sq_next;
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+    }
+}
+
+template <int G, bool STEP>
+cudaError_t launch_tc_g(DecodeParams prm, const DecodeArgs &a, int dev, cudaStream_t s) {
+    using Geo = TcGeo<G>;
+    auto kern = decode_tc_kernel<G, STEP>;
+    const size_t smem = (size_t)Geo::kOffPfx + (size_t)(a.num_seqs + 1) * 4 + 1024;
+    if (smem > (size_t)max_optin_smem(dev) - 2048) return cudaErrorNotSupported;
+    static std::atomic<int> attr_smem[kMaxDev];
+    static std::mutex attr_mu;
+    if ((size_t)attr_smem[dev].load(std::memory_order_acquire) < smem) {
+        std::lock_guard<std::mutex> lock(attr_mu);
+        if ((size_t)attr_smem[dev].load(std::memory_order_relaxed) < smem) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            attr_smem[dev].store((int)smem, std::memory_order_release);
+        }
+    }
+    prm.nctas = device_sm_count(dev);  // one CTA per SM
+    CUtensorMap tk, tv;
+    const uint64_t slots = (uint64_t)a.num_blocks * a.block_size;
+    const uint32_t box_rows = a.block_size == 8 ? 8u : 16u;
+    if (!encode_tensor_map_3d(&tk, a.k_cache, 1, 128, a.n_kv_heads, slots, 128, 1, box_rows, true) ||
+        !encode_tensor_map_3d(&tv, a.v_cache, 1, 128, a.n_kv_heads, slots, 128, 1, box_rows, true))
+        return cudaErrorUnknown;
+    cudaError_t e = launch_pdl(kern, dim3(prm.nctas), dim3(kTcThreads), smem, s, tk, tv, prm);
+    if (e != cudaSuccess || STEP) return e;
+    DecodeParams cp = prm;
+    return launch_pdl(combine_kernel<128, G, 1>, dim3(prm.nctas), dim3(128), 0, s, cp);
+}
+
+template <bool STEP>
+cudaError_t dispatch_tc(const DecodeArgs &a, cudaStream_t s) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    if (a.num_seqs == 0) return cudaSuccess;
+    DecodeParams prm;
+    prm.out = static_cast<__nv_bfloat16 *>(a.out);
+    prm.q = static_cast<const uint16_t *>(a.q);
+    prm.block_tables = a.block_tables;
+    prm.max_blocks = a.max_blocks_per_seq;
+    prm.context_lens = a.context_lens;
+    prm.B = a.num_seqs;
+    prm.Hq = a.n_q_heads;
+    prm.Hkv = a.n_kv_heads;
+    prm.num_blocks = a.num_blocks;
+    prm.bs = a.block_size;
+    prm.max_tokens = (int)std::min<long long>((long long)a.max_blocks_per_seq * a.block_size, 0x7fffffffLL);
+    prm.scale_log2 = a.scale * kLog2e;
+    prm.k_scale = a.k_scale;
+    prm.v_scale = a.v_scale;
+    prm.rope = a.rope;
+    prm.max_pos = a.max_pos;
+    prm.prefix = static_cast<int *>(a.workspace);
+    prm.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(a.workspace) +
+                                             align16((size_t)(a.num_seqs + 1) * sizeof(int)));
+    prm.err = a.err;
+    prm.k_new = static_cast<const uint16_t *>(a.k_new);
+    prm.v_new = static_cast<const uint16_t *>(a.v_new);
+    prm.k_cache_w = a.k_cache_w;
+    prm.v_cache_w = a.v_cache_w;
+    prm.counters = nullptr;
+    if (STEP)  // counters follow the attention workspace (see decode_step_workspace_bytes)
+        prm.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(a.workspace) +
+                                               decode_workspace_bytes(a.num_seqs, a.n_q_heads, a.n_kv_heads,
+                                                                      a.head_dim, device_sm_count(dev)));
+    switch (a.n_q_heads / a.n_kv_heads) {
+        case 2: return launch_tc_g<2, STEP>(prm, a, dev, s);
+        case 4: return launch_tc_g<4, STEP>(prm, a, dev, s);
+        case 8: return launch_tc_g<8, STEP>(prm, a, dev, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool decode_tc_supported(const DecodeArgs &a) {
+    const int G = a.n_q_heads / a.n_kv_heads;
+    return a.fp8 && a.head_dim == 128 && (G == 2 || G == 4 || G == 8);
+}
+
+cudaError_t launch_paged_decode_tc(const DecodeArgs &a, cudaStream_t s) { return dispatch_tc<false>(a, s); }
+cudaError_t launch_paged_decode_step_tc(const DecodeArgs &a, cudaStream_t s) { return dispatch_tc<true>(a, s); }
+
+}  // namespace pkv

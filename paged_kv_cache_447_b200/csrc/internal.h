@@ -137,6 +137,10 @@ size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int h
 // Its workspace is decode_workspace_bytes(...) followed by num_seqs * n_kv_heads int
 // counters that must be zero before the first call (every call leaves them zero).
 cudaError_t launch_paged_decode_step(const DecodeArgs &a, cudaStream_t s);
+// Grouped heads over an E4M3 cache at head dim 128 run on the tcgen05 decode kernel.
+bool decode_tc_supported(const DecodeArgs &a);
+cudaError_t launch_paged_decode_tc(const DecodeArgs &a, cudaStream_t s);
+cudaError_t launch_paged_decode_step_tc(const DecodeArgs &a, cudaStream_t s);
 size_t decode_step_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int head_dim,
                                    int num_sms);
 cudaError_t launch_paged_prefill(const PrefillArgs &a, cudaStream_t s);
