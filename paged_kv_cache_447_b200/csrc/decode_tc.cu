@@ -12,9 +12,10 @@
 // run of tiles of one (sequence, kv head) is a piece with one softmax state, merged with the
 // other pieces of its sequence by the combine kernel exactly as decode_kernel's partials.
 //   warp 0      TMA producer: the tile's K and V rows (8 boxes of 16 rows each, 128-byte
-//               swizzled, straight from the cache) into a 5-stage ring
-//   warp 1      TMEM owner and the one MMA-issuing thread
+//               swizzled, straight from the cache; one lane per box) into a 5-stage ring
+//   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
+//   warp 6      lane 0 issues the PV MMAs
 // Per tile:
 //   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
 //                 cache stores it (K-major), B = q as E4M3 rows -- the G heads' high parts in
@@ -26,18 +27,20 @@
 //                 low E4M3 parts into a shared-memory P tile: row h / G+h, byte t.
 //   O += P V      M = 64 (rows 0..2G-1 used), N = 128 dims, K = 128 tokens: A = the P tile,
 //                 B = the V tile MN-major as the cache stores it; O = rows h + rows G+h.
-// The MMA thread never blocks on one event: it polls for the next PV (P written) and the next
-// S^T (tile landed, S buffer free, the piece's q staged) and issues whichever is ready, PV
-// first, so a stage goes back to the producer as soon as its PV is issued.  S, P and q are
-// double-buffered, and so is O (by piece), so the epilogue of one piece overlaps the next
-// piece's MMAs; the next piece's q is staged before the epilogue.
+// S^T and PV are issued by two threads, each waiting only for its own inputs (S^T: tile
+// landed, S buffer free, the piece's q staged; PV: P written, O buffer free), so a stage goes
+// back to the producer as soon as its PV completes, and S^T of later tiles runs ahead.  They
+// touch disjoint TMEM columns and shared memory.  S, P and q are double-buffered, and so is
+// O (by piece), so the epilogue of one piece overlaps the next piece's MMAs; the next
+// piece's q is staged before the epilogue.
 #include "decode_kernel.cuh"
 #include "tcgen05.cuh"
 
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 224;
+constexpr int kTcPvWarp = 6;    // the PV issuer
 constexpr int kTcTile = 128;    // tokens per unit
 constexpr int kTcStages = 5;
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
@@ -71,23 +74,10 @@ constexpr int kBPFull = kBSFree + 2;      // [2] P tile written (128 arrivals)
 constexpr int kBPvDone = kBPFull + 2;     // [2] PV done reading P buffer (commit)
 constexpr int kBQFull = kBPvDone + 2;     // q staged for the piece (128 arrivals)
 constexpr int kBOFree = kBQFull + 1;      // [2] O buffer read by its piece's epilogue (32 arrivals)
-constexpr int kBDrain = kBOFree + 2;      // every MMA of the CTA has completed (commit)
+constexpr int kBDrain = kBOFree + 2;      // every MMA of the CTA has completed (2 commits)
 static_assert(kBDrain < 2 * kTcStages + 12, "barrier count");
 
 __device__ __forceinline__ uint32_t bar_at(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
-
-// Non-blocking test of an mbarrier phase (the MMA thread polls several).
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
 
 // Row r, byte c of a 128-byte-row swizzled tile (16-byte chunk index XOR row % 8).
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
@@ -215,7 +205,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(bar_at(bars, kBQFull), 128);
         mbar_init(bar_at(bars, kBOFree), 32);
         mbar_init(bar_at(bars, kBOFree + 1), 32);
-        mbar_init(bar_at(bars, kBDrain), 1);
+        mbar_init(bar_at(bars, kBDrain), 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -251,178 +241,129 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             prefetch_tmap(&tm_v);
         }
         const int oob = (int)(p.num_blocks * p.bs < 0x7fffffffLL ? p.num_blocks * p.bs : 0x7fffffff);
+        // this lane's box of every tile: 16-token piece `piece` (8-token blocks: half `half`,
+        // two boxes of 8 rows per piece); the boxes of a tile go out from their lanes at once
+        const bool two = p.bs == 8;
+        const int n_box = two ? 16 : 8;
+        const int half = two ? (lane & 1) : 0, bpiece = two ? (lane >> 1) : lane;
+        const uint32_t box_off = (uint32_t)(bpiece * 2048 + half * 1024);
         uint32_t issued = 0, phases = 0;
         bool ok = true;
         for (int k = 0; k < nunits && ok; ++k) {
             int b, kvh, tile, ntiles;
             unit(k, b, kvh, tile, ntiles);
             const int L = min(__ldg(p.context_lens + b), p.max_tokens);
-            // lane i < 8: cache rows of the tile's piece i (16 tokens); two runs for 8-token blocks
-            int r0 = oob, r1 = oob;
-            if (lane < 8) {
-                const int pc = tile * 8 + lane;  // 16-token piece of the sequence
-                if (pc * 16 < L) {
-                    const int32_t *tab = p.block_tables + (size_t)b * p.max_blocks;
-                    if (p.bs == 16) {
-                        r0 = cache_row(p, __ldg(tab + pc), 0);
-                    } else if (p.bs == 32) {
-                        r0 = cache_row(p, __ldg(tab + (pc >> 1)), (pc & 1) * 16);
-                    } else {
-                        r0 = cache_row(p, __ldg(tab + 2 * pc), 0);
-                        if ((2 * pc + 1) * 8 < L) r1 = cache_row(p, __ldg(tab + 2 * pc + 1), 0);
-                    }
+            int row = oob;
+            if (lane < n_box) {
+                const int pc = tile * 8 + bpiece;  // 16-token piece of the sequence
+                const int32_t *tab = p.block_tables + (size_t)b * p.max_blocks;
+                if (p.bs == 16) {
+                    if (pc * 16 < L) row = cache_row(p, __ldg(tab + pc), 0);
+                } else if (p.bs == 32) {
+                    if (pc * 16 < L) row = cache_row(p, __ldg(tab + (pc >> 1)), (pc & 1) * 16);
+                } else {
+                    const int e = 2 * pc + half;
+                    if (e * 8 < L) row = cache_row(p, __ldg(tab + e), 0);
                 }
             }
-            int rr0[8], rr1[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                rr0[i] = __shfl_sync(0xffffffffu, r0, i);
-                rr1[i] = __shfl_sync(0xffffffffu, r1, i);
-            }
+            const int s = k % kTcStages;
+            const uint32_t fb = bar_at(bars, kBFull + s);
             if (lane == 0) {
-                const int s = k % kTcStages;
                 if (*abort_flag || !mbar_wait_bounded(bar_at(bars, kBEmpty + s), ((k / kTcStages) & 1) ^ 1, p.err)) {
                     ok = false;
                     *abort_flag = 1;
                 } else {
-                    const uint32_t fb = bar_at(bars, kBFull + s);
-                    const uint32_t dk = sStages + s * Geo::kStage, dv = dk + Geo::kKV;
                     mbar_arrive_expect_tx(fb, Geo::kStage);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        tma_load_3d(dk + i * 2048, &tm_k, fb, 0, kvh, rr0[i]);
-                        tma_load_3d(dv + i * 2048, &tm_v, fb, 0, kvh, rr0[i]);
-                        if (p.bs == 8) {
-                            tma_load_3d(dk + i * 2048 + 1024, &tm_k, fb, 0, kvh, rr1[i]);
-                            tma_load_3d(dv + i * 2048 + 1024, &tm_v, fb, 0, kvh, rr1[i]);
-                        }
-                    }
                     issued |= 1u << s;
                     phases = (phases & ~(1u << s)) | ((uint32_t)((k / kTcStages) & 1) << s);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (ok && lane < n_box) {
+                const uint32_t dk = sStages + s * Geo::kStage;
+                tma_load_3d(dk + box_off, &tm_k, fb, 0, kvh, row);
+                tma_load_3d(dk + Geo::kKV + box_off, &tm_v, fb, 0, kvh, row);
+            }
         }
         if (lane == 0)  // never leave with a TMA copy landing in shared memory
             for (int s = 0; s < kTcStages; ++s)
                 if ((issued >> s) & 1) mbar_wait_bounded(bar_at(bars, kBFull + s), (phases >> s) & 1, p.err);
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        // Lane 0 tests the barriers and issues; the whole warp walks the units (with STEP it
-        // stores the step's new token into the tile before that tile's S^T is issued).
+        // ---------------------------------------------------------------- S^T issuer
+        // Lane 0 issues; the whole warp walks the units (with STEP it stores the step's new
+        // token into the tile before that tile's S^T is issued).
         constexpr uint32_t idS = tc::mma_idesc(128, 16, false, true);  // E4M3 x E4M3 -> f32
-        constexpr uint32_t idO = tc::mma_idesc(64, D, true, true);     // B (V) MN-major
-        int ks = 0, kp = 0;       // next S^T, next PV
-        int spc = -1, ppc = -1;   // piece of the last S^T / PV issued
-        bool s_known = false, p_known = false, s_first = false, p_first = false;
-        int sb_ = 0, skvh = 0, stile = 0, snt = 0;
+        auto wait0 = [&](int bi, uint32_t parity) -> bool {
+            bool r = true;
+            if (lane == 0) r = !*abort_flag && mbar_wait_bounded(bar_at(bars, bi), parity, p.err);
+            return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+        };
         bool ok = true;
-        int idle = 0;
-        unsigned long long t_idle = 0;
-        while (kp < nunits) {
-            bool did = false;
-            // ---- PV of tile kp, into the O buffer of its piece
-            if (kp < ks) {
-                if (!p_known) {
-                    int b, kvh, tile, nt;
-                    unit(kp, b, kvh, tile, nt);
-                    p_first = kp == 0 || tile == 0;
-                    p_known = true;
-                }
-                const int pc = ppc + (p_first ? 1 : 0);
-                int go = 0;
-                if (lane == 0)  // a piece's first PV overwrites its O buffer: piece pc-2's epilogue must have read it
-                    go = mbar_test(bar_at(bars, kBPFull + (kp & 1)), (kp >> 1) & 1) &&
-                         (!p_first || pc < 2 || mbar_test(bar_at(bars, kBOFree + (pc & 1)), ((pc >> 1) - 1) & 1));
-                if (__shfl_sync(0xffffffffu, go, 0)) {
-                    if (lane == 0) {
-                        tc::tc_fence_after();
-                        const uint32_t vd = sStages + (kp % kTcStages) * Geo::kStage + Geo::kKV;
-                        const uint32_t pd = sP + (kp & 1) * Geo::kP;
-                        const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(pc & 1);
-#pragma unroll
-                        for (int kk = 0; kk < kTcTile / 32; ++kk)
-                            tc::mma_ss_f8(tO, tc::sw128_desc(pd + 32 * kk, 16, 1024),
-                                          tc::sw128_desc(vd + 4096 * kk, 16384, 1024), idO,
-                                          (p_first && kk == 0) ? 0u : 1u);
-                        tc::mma_commit(bar_at(bars, kBEmpty + kp % kTcStages));
-                        tc::mma_commit(bar_at(bars, kBPvDone + (kp & 1)));
-                    }
+        int piece = -1;
+        for (int k = 0; k < nunits && ok; ++k) {
+            int b, kvh, tile, ntiles;
+            unit(k, b, kvh, tile, ntiles);
+            if (k == 0 || tile == 0) {
+                ++piece;
+                ok = wait0(kBQFull, piece & 1);
+            }
+            ok = ok && wait0(kBFull + k % kTcStages, (k / kTcStages) & 1) &&
+                 (k < 2 || wait0(kBSFree + (k & 1), ((k - 2) >> 1) & 1));
+            if (!ok) break;
+            const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
+            if constexpr (STEP) {
+                const int Lraw = __ldg(p.context_lens + b), L = min(Lraw, p.max_tokens);
+                if (tile == ntiles - 1 && L == Lraw) {  // the sequence's last tile holds its new token
+                    const int e = __ldg(p.block_tables + (size_t)b * p.max_blocks + (L - 1) / p.bs);
+                    if (e >= 0 && (long long)e < p.num_blocks)
+                        tc_put_new_token(p, b, kvh, L, e * p.bs + (L - 1) % p.bs, kd, kd + Geo::kKV, lane);
+                    fence_proxy_async_smem();  // the tensor cores read these rows next
                     __syncwarp();
-                    ppc = pc;
-                    ++kp;
-                    p_known = false;
-                    did = true;
                 }
             }
-            // ---- S^T of tile ks
-            if (ks < nunits) {
-                if (!s_known) {
-                    unit(ks, sb_, skvh, stile, snt);
-                    s_first = ks == 0 || stile == 0;
-                    s_known = true;
-                }
-                const int pc = spc + (s_first ? 1 : 0);
-                int go = 0;
-                if (lane == 0)
-                    go = mbar_test(bar_at(bars, kBFull + ks % kTcStages), (ks / kTcStages) & 1) &&
-                         (ks < 2 || mbar_test(bar_at(bars, kBSFree + (ks & 1)), ((ks - 2) >> 1) & 1)) &&
-                         (!s_first || mbar_test(bar_at(bars, kBQFull), pc & 1));
-                if (__shfl_sync(0xffffffffu, go, 0)) {
-                    const uint32_t kd = sStages + (ks % kTcStages) * Geo::kStage;
-                    if constexpr (STEP) {
-                        const int Lraw = __ldg(p.context_lens + sb_), L = min(Lraw, p.max_tokens);
-                        if (stile == snt - 1 && L == Lraw) {  // the sequence's last tile holds its new token
-                            const int e = __ldg(p.block_tables + (size_t)sb_ * p.max_blocks + (L - 1) / p.bs);
-                            if (e >= 0 && (long long)e < p.num_blocks)
-                                tc_put_new_token(p, sb_, skvh, L, e * p.bs + (L - 1) % p.bs, kd, kd + Geo::kKV, lane);
-                            fence_proxy_async_smem();  // the tensor cores read these rows next
-                            __syncwarp();
-                        }
-                    }
-                    if (lane == 0) {
-                        tc::tc_fence_after();
-                        const uint32_t qd = sQ + (pc & 1) * Geo::kQ;
-#pragma unroll
-                        for (int kk = 0; kk < D / 32; ++kk)
-                            tc::mma_ss_f8(tmem + 16 * (ks & 1), tc::sw128_desc(kd + 32 * kk, 16, 1024),
-                                          tc::sw128_desc(qd + 32 * kk, 16, 1024), idS, kk > 0);
-                        tc::mma_commit(bar_at(bars, kBSFull + (ks & 1)));
-                    }
-                    __syncwarp();
-                    spc = pc;
-                    ++ks;
-                    s_known = false;
-                    did = true;
-                }
-            }
-            if (did) {
-                idle = 0;
-                continue;
-            }
-            // nothing ready: yield the issue slots to the softmax warp on this SM sub-partition,
-            // and give up (error flag) after the wait limit without progress
-            int stop = 0;
             if (lane == 0) {
-                if (*abort_flag) {
-                    stop = 1;
-                } else if (idle == 0) {
-                    t_idle = globaltimer();
-                } else if ((idle & 63) == 0 && globaltimer() - t_idle > kWaitLimitNs) {
-                    atomicOr(p.err, kErrTimeout);
-                    stop = 1;
-                }
+                tc::tc_fence_after();
+                const uint32_t qd = sQ + (piece & 1) * Geo::kQ;
+#pragma unroll
+                for (int kk = 0; kk < D / 32; ++kk)
+                    tc::mma_ss_f8(tmem + 16 * (k & 1), tc::sw128_desc(kd + 32 * kk, 16, 1024),
+                                  tc::sw128_desc(qd + 32 * kk, 16, 1024), idS, kk > 0);
+                tc::mma_commit(bar_at(bars, kBSFull + (k & 1)));
             }
-            if (__shfl_sync(0xffffffffu, stop, 0)) {
-                ok = false;
-                break;
-            }
-            ++idle;
-            __nanosleep(32);
+            __syncwarp();
         }
         if (!ok && lane == 0) *abort_flag = 1;
-        // drain: no MMA may still write TMEM when it is released
+        if (lane == 0) tc::mma_commit(bar_at(bars, kBDrain));  // (with the PV issuer's commit)
+    } else if (warp == kTcPvWarp) {
+        // ---------------------------------------------------------------- PV issuer
+        constexpr uint32_t idO = tc::mma_idesc(64, D, true, true);  // B (V) MN-major
         if (lane == 0) {
+            bool ok = true;
+            int piece = -1;
+            for (int k = 0; k < nunits && ok; ++k) {
+                int b, kvh, tile, ntiles;
+                unit(k, b, kvh, tile, ntiles);
+                const bool first = k == 0 || tile == 0;
+                if (first) ++piece;
+                // a piece's first PV overwrites its O buffer: the epilogue of piece - 2 must
+                // have read it
+                ok = !*abort_flag && mbar_wait_bounded(bar_at(bars, kBPFull + (k & 1)), (k >> 1) & 1, p.err) &&
+                     (!first || piece < 2 ||
+                      mbar_wait_bounded(bar_at(bars, kBOFree + (piece & 1)), ((piece >> 1) - 1) & 1, p.err));
+                if (!ok) break;
+                tc::tc_fence_after();
+                const uint32_t vd = sStages + (k % kTcStages) * Geo::kStage + Geo::kKV;
+                const uint32_t pd = sP + (k & 1) * Geo::kP;
+                const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
+#pragma unroll
+                for (int kk = 0; kk < kTcTile / 32; ++kk)
+                    tc::mma_ss_f8(tO, tc::sw128_desc(pd + 32 * kk, 16, 1024),
+                                  tc::sw128_desc(vd + 4096 * kk, 16384, 1024), idO, (first && kk == 0) ? 0u : 1u);
+                tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
+                tc::mma_commit(bar_at(bars, kBPvDone + (k & 1)));
+            }
+            if (!ok) *abort_flag = 1;
+            // drain: no MMA of either issuer may still write TMEM when it is released
             tc::mma_commit(bar_at(bars, kBDrain));
             mbar_wait_bounded(bar_at(bars, kBDrain), 0, p.err);
         }

@@ -239,6 +239,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // first row past the cache: TMA reads it as zeros
         const int oob = (int)min(p.num_blocks * p.bs, (long long)0x7fffffff);
+        // The box of every K/V tile this lane loads: 16-key piece box_piece, half box_half
+        // (8-token blocks: two boxes of 8 rows per piece) and 64-column slab box_slab.  The
+        // boxes of a tile are issued by their lanes at once, so a freed stage refills with
+        // one warp instruction instead of a serial run of copies.
+        const bool two = p.bs == 8;
+        const int n_box = (two ? 16 : 8) * (Geo::kConv ? 1 : Geo::kKVSlabs);
+        const int box_half = two ? (lane & 1) : 0;
+        const int box_piece = two ? ((lane >> 1) & 7) : (lane & 7);
+        const int box_slab = two ? (lane >> 4) : (lane >> 3);
+        const uint32_t box_off = (uint32_t)(box_slab * Geo::kSlabBytes + box_piece * 2048 + box_half * 1024);
         for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
             const Item it = decode_item(p, idx);
             if (!active(it)) continue;
@@ -266,29 +276,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int gg = g + j;
                 const int ks = gg % KS, vs = gg % VS;
                 const uint32_t kpar = ((gg / KS) & 1) ^ 1, vpar = ((gg / VS) & 1) ^ 1;
-                // lane i < 8: cache rows of piece i of the tile (16 keys): one run of 16 from
-                // `phys` (16- and 32-token blocks) or two runs of 8 from `phys` and `phys1`
-                int phys = oob, phys1 = oob;
-                if (lane < 8) {
-                    const int lb = j * 8 + lane;
-                    if (lb < npiece) {
-                        const int32_t *tab = p.block_tables + (size_t)it.b * p.max_blocks;
-                        auto row = [&](int entry, int off) {
-                            const int e = __ldg(tab + entry);
-                            if (e < 0 || (long long)e >= p.num_blocks) {
-                                atomicOr(p.err, kErrBounds);
-                                return oob;
-                            }
-                            return e * p.bs + off;
-                        };
-                        if (p.bs == 16) {
-                            phys = row(lb, 0);
-                        } else if (p.bs == 32) {
-                            phys = row(lb >> 1, (lb & 1) * 16);
-                        } else {
-                            phys = row(2 * lb, 0);
-                            if ((2 * lb + 1) * 8 < Lc) phys1 = row(2 * lb + 1, 0);
-                        }
+                // This lane's box of the tile (see box_* above): its cache row, from its own
+                // block-table entry, or the first row past the cache (read as zeros).
+                int row = oob;
+                if (lane < n_box) {
+                    const int lb = j * 8 + box_piece;  // 16-token piece of the sequence
+                    int entry = lb, off = 0;
+                    bool valid = lb < npiece;
+                    if (p.bs == 32) {
+                        entry = lb >> 1;
+                        off = (lb & 1) * 16;
+                    } else if (p.bs == 8) {
+                        entry = 2 * lb + box_half;
+                        valid = entry * 8 < Lc;
+                    }
+                    if (valid) {
+                        const int e = __ldg(p.block_tables + (size_t)it.b * p.max_blocks + entry);
+                        if (e < 0 || (long long)e >= p.num_blocks) atomicOr(p.err, kErrBounds);
+                        else row = e * p.bs + off;
                     }
                 }
                 if constexpr (Geo::kConv) {
@@ -298,30 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (*abort_flag || !mbar_wait_bounded(b_stgempty, (gg & 1) ^ 1, p.err)) {
                             ok = false;
                             *abort_flag = 1;
+                        } else {
+                            mbar_arrive_expect_tx(b_stgfull, 2 * Geo::kStgBytes);
+                            issued |= 1u << 16;
+                            phase_bits = (phase_bits & ~(1u << 16)) | ((uint32_t)(gg & 1) << 16);
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                     if (!ok) break;
-                    int ph[8], ph1[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        ph[i] = __shfl_sync(0xffffffffu, phys, i);
-                        ph1[i] = __shfl_sync(0xffffffffu, phys1, i);
-                    }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(b_stgfull, 2 * Geo::kStgBytes);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            tma_load_3d(sStg + i * kPiece * D, &tm_k, b_stgfull, 0, it.kvh, ph[i]);
-                            tma_load_3d(sStg + Geo::kStgBytes + i * kPiece * D, &tm_v, b_stgfull, 0, it.kvh, ph[i]);
-                            if (p.bs == 8) {
-                                tma_load_3d(sStg + (i * kPiece + 8) * D, &tm_k, b_stgfull, 0, it.kvh, ph1[i]);
-                                tma_load_3d(sStg + Geo::kStgBytes + (i * kPiece + 8) * D, &tm_v, b_stgfull, 0,
-                                            it.kvh, ph1[i]);
-                            }
-                        }
-                        issued |= 1u << 16;
-                        phase_bits = (phase_bits & ~(1u << 16)) | ((uint32_t)(gg & 1) << 16);
+                    if (lane < n_box) {  // (one slab: the boxes are whole D-byte rows)
+                        const uint32_t off = (uint32_t)((box_piece * kPiece + box_half * 8) * D);
+                        tma_load_3d(sStg + off, &tm_k, b_stgfull, 0, it.kvh, row);
+                        tma_load_3d(sStg + Geo::kStgBytes + off, &tm_v, b_stgfull, 0, it.kvh, row);
                     }
                     continue;
                 }
@@ -336,37 +329,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                int ph[8], ph1[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    ph[i] = __shfl_sync(0xffffffffu, phys, i);
-                    ph1[i] = __shfl_sync(0xffffffffu, phys1, i);
-                }
-                // piece i of a tile = 16 rows x 128 bytes of each slab (8-token blocks: two boxes of 8)
-                auto load_tile = [&](uint32_t dst, const CUtensorMap *map, uint32_t bar) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        for (int s = 0; s < Geo::kKVSlabs; ++s) {
-                            tma_load_3d(dst + s * Geo::kSlabBytes + i * 2048, map, bar, 64 * s, it.kvh, ph[i]);
-                            if (p.bs == 8)
-                                tma_load_3d(dst + s * Geo::kSlabBytes + i * 2048 + 1024, map, bar, 64 * s, it.kvh,
-                                            ph1[i]);
-                        }
-                };
+                // lane 0 arms the barrier, then every box lane issues its own load
                 if (lane == 0) {
                     const uint32_t kb = b_kfull + 8 * ks;
                     mbar_arrive_expect_tx(kb, Geo::kKVBytes);
-                    load_tile(sK + ks * Geo::kKVBytes, &tm_k, kb);
                     issued |= 1u << ks;
                     phase_bits = (phase_bits & ~(1u << ks)) | ((uint32_t)((gg / KS) & 1) << ks);
-                    // V of the same tile: its stage frees later (after PV1 of tile gg - VS)
+                }
+                __syncwarp();
+                if (lane < n_box)
+                    tma_load_3d(sK + ks * Geo::kKVBytes + box_off, &tm_k, b_kfull + 8 * ks, 64 * box_slab, it.kvh, row);
+                // V of the same tile: its stage frees later (after PV1 of tile gg - VS)
+                const uint32_t vb = fix ? b_vraw : b_vfull + 8 * vs;
+                if (lane == 0) {
                     if (*abort_flag || !mbar_wait_bounded(b_vempty + 8 * vs, vpar, p.err)) {
                         ok = false;
                         *abort_flag = 1;
                     } else {
-                        const uint32_t vb = fix ? b_vraw : b_vfull + 8 * vs;
                         mbar_arrive_expect_tx(vb, Geo::kKVBytes);
-                        load_tile(sV + vs * Geo::kKVBytes, &tm_v, vb);
                         if (!fix) {
                             issued |= 1u << (8 + vs);
                             phase_bits = (phase_bits & ~(1u << (8 + vs))) | ((uint32_t)((gg / VS) & 1) << (8 + vs));
@@ -378,6 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                if (lane < n_box) tma_load_3d(sV + vs * Geo::kKVBytes + box_off, &tm_v, vb, 64 * box_slab, it.kvh, row);
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
                 if (fix) {
