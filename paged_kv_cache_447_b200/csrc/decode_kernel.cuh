@@ -131,6 +131,7 @@ struct Geometry {
     static constexpr int kStages = kStagesQ < kGroups ? kGroups : (kStagesQ > 64 ? 64 : kStagesQ);
     static_assert(kStages % kGroups == 0, "stage count must be a multiple of the consumer groups");
     static_assert(kConsumers % HPU == 0, "one consumer warp per head of a unit");
+    static_assert(HPU * 2 * D * kElem <= kConsumers * G * (D + 2) * 4, "new-token rows fit the merge scratch");
     static constexpr int kChunkElems = 16 / kElem;                     // elements per 16 B
     static constexpr int kChunks = kRowBytes / 16;                     // 16-B chunks per row
     static constexpr int kQuads = kChunkElems / 4;                     // float4 per chunk
@@ -322,58 +323,6 @@ __device__ __forceinline__ float merge_partials(const DecodeParams &p, int segu,
     }
     return lsum > 0.f ? o / lsum * vsc : 0.f;
 }
-
-// Decode step: store the step's new token of sequence b, kv head kvh -- the newest of its L
-// cached tokens, row (L-1) % 16 of its last 16-token tile, cache slot `slot` -- into the cache,
-// and into the stage's K and V tiles (which TMA filled with that slot's previous contents),
-// exactly as pkv_kv_store stores it: K rotated at position L - 1, E4M3 codes from the
-// fp64 quotient by the head's scale.  A position outside the RoPE table stores nothing
-// (bounds flag), as in pkv_kv_store.  One warp; `swizzled`: the 128-byte-swizzled tile
-// layout of the tensor-core consumers.
-template <int D, bool FP8, int kSlabStride, bool kSwizzled>
-__device__ __forceinline__ void put_new_token(const DecodeParams &p, int b, int kvh, int L, int slot,
-                                              uint32_t ks_a, uint32_t vs_a, int lane) {
-    constexpr int kElem = FP8 ? 1 : 2;
-    const int r = (L - 1) % kPiece, pos = L - 1;
-    const float *rope = nullptr;
-    if (p.rope) {
-        if (pos >= p.max_pos) {
-            if (lane == 0) atomicOr(p.err, kErrBounds);
-            return;
-        }
-        rope = p.rope + (size_t)pos * D;
-    }
-    const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
-    const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
-    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;  // element index
-    const double ks = FP8 ? (double)__ldg(p.k_scale + kvh) : 1.0;
-    const double vs = FP8 ? (double)__ldg(p.v_scale + kvh) : 1.0;
-    for (int i = lane; i < D / 2; i += 32) {
-        uint16_t kb[2] = {__ldg(kin + i), __ldg(kin + i + D / 2)};
-        const uint16_t vb[2] = {__ldg(vin + i), __ldg(vin + i + D / 2)};
-        if (rope) rope_pair_fast(kb[0], kb[1], __ldg(rope + i), __ldg(rope + D / 2 + i), kb[0], kb[1]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int e = i + h * (D / 2), byte = e * kElem;
-            const uint32_t off = kSwizzled ? swz<kSlabStride>(r, byte / 16) + (byte % 16)
-                                           : (uint32_t)(r * D * kElem + byte);
-            if constexpr (FP8) {
-                const uint32_t kc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[h]), ks));
-                const uint32_t vc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(vb[h]), vs));
-                static_cast<uint8_t *>(p.k_cache_w)[dst + e] = (uint8_t)kc;
-                static_cast<uint8_t *>(p.v_cache_w)[dst + e] = (uint8_t)vc;
-                asm volatile("st.shared.u8 [%0], %1;" ::"r"(ks_a + off), "r"(kc) : "memory");
-                asm volatile("st.shared.u8 [%0], %1;" ::"r"(vs_a + off), "r"(vc) : "memory");
-            } else {
-                static_cast<uint16_t *>(p.k_cache_w)[dst + e] = kb[h];
-                static_cast<uint16_t *>(p.v_cache_w)[dst + e] = vb[h];
-                asm volatile("st.shared.u16 [%0], %1;" ::"r"(ks_a + off), "h"(kb[h]) : "memory");
-                asm volatile("st.shared.u16 [%0], %1;" ::"r"(vs_a + off), "h"(vb[h]) : "memory");
-            }
-        }
-    }
-}
-
 
 template <int D, bool FP8, int G, int HPU, bool STEP>
 __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
@@ -578,6 +527,37 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
         const int L = min(__ldg(p.context_lens + b), p.max_tokens);
         const bool whole = (cur.blk == 0) && (piece_len == cur.nb);
 
+        // decode step: issue the loads of the new token (if this piece stores it) ahead of q's
+        constexpr int kNt = STEP ? (HPU * D / 2 + kConsumers * 32 - 1) / (kConsumers * 32) : 1;
+        uint16_t nt_k[kNt][2], nt_v[kNt][2];
+        float nt_c[kNt], nt_s[kNt];
+        bool nt_has = false;
+        int nt_e = -1, nt_lraw = -1;
+        if constexpr (STEP) {
+            nt_has = cur.blk + piece_len == cur.nb;
+            if (nt_has) {
+                const int pos = L - 1;
+                nt_lraw = __ldg(p.context_lens + b);
+                nt_e = __ldg(p.block_tables + (size_t)b * p.max_blocks + pos / p.bs);
+                const bool rope_ok = p.rope && pos < p.max_pos;
+#pragma unroll
+                for (int j = 0; j < kNt; ++j) {
+                    const int e2 = ct + j * kConsumers * 32;
+                    if (e2 >= HPU * D / 2) break;
+                    const int hh = e2 / (D / 2), i = e2 % (D / 2), kvo = kvg * HPU + hh;
+                    const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvo) * D;
+                    const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvo) * D;
+                    nt_k[j][0] = __ldg(kin + i);
+                    nt_k[j][1] = __ldg(kin + i + D / 2);
+                    nt_v[j][0] = __ldg(vin + i);
+                    nt_v[j][1] = __ldg(vin + i + D / 2);
+                    if (rope_ok) {
+                        nt_c[j] = __ldg(p.rope + (size_t)pos * D + i);
+                        nt_s[j] = __ldg(p.rope + (size_t)pos * D + D / 2 + i);
+                    }
+                }
+            }
+        }
         // ---- stage q for this (b, kv-head group): rotate (optional), scale, split layout
         for (int e = ct; e < HPU * G * D / 2; e += kConsumers * 32) {
             const int hh = e / (G * D / 2), g = (e / (D / 2)) % G, i = e % (D / 2);
@@ -610,6 +590,55 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                 const int c = dim / Geo::kChunkElems, w = dim % Geo::kChunkElems;
                 const int quad = w / 4, comp = w % 4;
                 qs[hh * G * D + ((g * Geo::kQuads + quad) * Geo::kChunks + c) * 4 + comp] = val[r];
+            }
+        }
+        bool nt_ok = false;
+        if constexpr (STEP) {
+            // The step's new token of this group's heads, when this piece holds its sequence's
+            // last block (and the context was not clipped to the block table): K rotated at
+            // L - 1 and V, converted as the cache stores them (E4M3 codes from the fp64
+            // quotient by the head's scale, as pkv_kv_store does), go into the cache and into
+            // mrg, which is free until the piece's merge.  The warp that takes the last block
+            // copies its head's rows from there into its tile, so no global load sits on that
+            // warp's path.  (The loads were issued before q's, in nt_*.)
+            if (nt_has) {
+                const int pos = L - 1;
+                const bool rope_ok = !p.rope || pos < p.max_pos;
+                if (!rope_ok && ct == 0) atomicOr(p.err, kErrBounds);
+                nt_ok = L == nt_lraw && rope_ok && nt_e >= 0 && (long long)nt_e < p.num_blocks;
+                if (nt_ok) {
+                    const int slot = nt_e * p.bs + pos % p.bs;
+                    uint8_t *nt = reinterpret_cast<uint8_t *>(mrg);
+#pragma unroll
+                    for (int j = 0; j < kNt; ++j) {
+                        const int e2 = ct + j * kConsumers * 32;
+                        if (e2 >= HPU * D / 2) break;
+                        const int hh = e2 / (D / 2), i = e2 % (D / 2), kvo = kvg * HPU + hh;
+                        uint16_t kb[2] = {nt_k[j][0], nt_k[j][1]};
+                        if (p.rope) rope_pair_fast(kb[0], kb[1], nt_c[j], nt_s[j], kb[0], kb[1]);
+                        const size_t dst = ((size_t)slot * p.Hkv + kvo) * D;  // element index
+                        uint8_t *krow = nt + 2 * hh * Geo::kRowBytes, *vrow = krow + Geo::kRowBytes;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int el = i + h * (D / 2);
+                            if constexpr (FP8) {
+                                const uint32_t kc =
+                                    f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[h]), (double)__ldg(p.k_scale + kvo)));
+                                const uint32_t vc =
+                                    f64_to_e4m3(__ddiv_rn(bf16_to_f64(nt_v[j][h]), (double)__ldg(p.v_scale + kvo)));
+                                static_cast<uint8_t *>(p.k_cache_w)[dst + el] = (uint8_t)kc;
+                                static_cast<uint8_t *>(p.v_cache_w)[dst + el] = (uint8_t)vc;
+                                krow[el] = (uint8_t)kc;
+                                vrow[el] = (uint8_t)vc;
+                            } else {
+                                static_cast<uint16_t *>(p.k_cache_w)[dst + el] = kb[h];
+                                static_cast<uint16_t *>(p.v_cache_w)[dst + el] = nt_v[j][h];
+                                reinterpret_cast<uint16_t *>(krow)[el] = kb[h];
+                                reinterpret_cast<uint16_t *>(vrow)[el] = nt_v[j][h];
+                            }
+                        }
+                    }
+                }
             }
         }
         named_bar(kMergeBar, kConsumers * 32);
@@ -650,13 +679,20 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
             const uint32_t ks_a = smem_u32(stages + s * Geo::kStageBytes) + hsel * kHeadStride;
             const uint32_t vs_a = ks_a + HPU * Geo::kTileBytes;
             if constexpr (STEP) {
-                // the sequence's last block holds the step's new token (not when the context
-                // was clipped to the block table)
-                if (blk == cur.nb - 1 && L == __ldg(p.context_lens + b)) {
-                    const int e = __ldg(p.block_tables + (size_t)b * p.max_blocks + (L - 1) / p.bs);
-                    if (e >= 0 && (long long)e < p.num_blocks)
-                        put_new_token<D, FP8, kSlabStride, kMma>(p, b, kvh, L, e * p.bs + (L - 1) % p.bs, ks_a,
-                                                                 vs_a, lane);
+                // the sequence's last block holds the step's new token: its rows, staged in
+                // mrg with the piece's q, replace the slot's previous contents in the tile
+                if (blk == cur.nb - 1 && nt_ok) {
+                    const int r = (L - 1) % kPiece;
+                    const uint8_t *krow = reinterpret_cast<const uint8_t *>(mrg) + 2 * hsel * Geo::kRowBytes;
+                    for (int c = lane; c < Geo::kChunks; c += 32) {  // 16-byte chunks of the row
+                        const uint4 kx = *reinterpret_cast<const uint4 *>(krow + 16 * c);
+                        const uint4 vx = *reinterpret_cast<const uint4 *>(krow + Geo::kRowBytes + 16 * c);
+                        const uint32_t off = kMma ? swz<kSlabStride>(r, c) : (uint32_t)(r * Geo::kRowBytes + 16 * c);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(ks_a + off), "r"(kx.x),
+                                     "r"(kx.y), "r"(kx.z), "r"(kx.w) : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vs_a + off), "r"(vx.x),
+                                     "r"(vx.y), "r"(vx.z), "r"(vx.w) : "memory");
+                    }
                     fence_proxy_async_smem();  // before the stage is refilled by TMA
                     __syncwarp();
                 }
@@ -968,6 +1004,10 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
         }
 
         // ---- merge the four consumer warps' states for this piece
+        if constexpr (STEP) {
+            // mrg still holds the staged new-token rows until every warp is past its blocks
+            if (nt_ok) named_bar(kMergeBar, kConsumers * 32);
+        }
         if constexpr (kMma) {
             float lw = lr;
             lw += __shfl_xor_sync(0xffffffffu, lw, 1);

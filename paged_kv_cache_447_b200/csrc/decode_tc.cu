@@ -39,10 +39,13 @@
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 224;
+constexpr int kTcThreads = 288;
 constexpr int kTcPvWarp = 6;    // the PV issuer
+constexpr int kTcQWarp = 7;     // the q stager
+constexpr int kTcEpiWarp = 8;   // the epilogue (warp 8: TMEM lanes 0-31, where O's rows live)
 constexpr int kTcTile = 128;    // tokens per unit
 constexpr int kTcStages = 5;
+constexpr int kTcQBufs = 4;     // q buffers: the stager runs up to this many pieces ahead
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
 constexpr uint32_t kTcO = 128;  // TMEM column of O buffer 0 (buffer 1 follows at +128)
@@ -55,27 +58,32 @@ struct TcGeo {
     static constexpr int kQ = 16 * 128;             // B operand of S^T: 16 rows x 128 codes
     static constexpr int kP = 64 * 128;             // A operand of PV: 64 rows x 128 tokens
     static constexpr int kOffQ = kTcStages * kStage;
-    static constexpr int kOffP = kOffQ + 2 * kQ;
-    static constexpr int kOffRed = kOffP + 2 * kP;  // [4 warps][8] floats x 2 (max, sum)
-    static constexpr int kOffQtmp = kOffRed + 2 * 4 * 8 * 4;  // rotated bf16 q [G][128]
+    static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
+    static constexpr int kOffRed = kOffP + 2 * kP;          // [4 warps][8] floats x 2 (max, sum)
+    static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;  // [2 O buffers][m | l][8] floats
+    static constexpr int kOffSq = kOffStats + 2 * 2 * 8 * 4;   // [kTcQBufs] q scales
+    static constexpr int kOffQtmp = kOffSq + 16 * 4;           // rotated bf16 q [G][128] (stager)
     static constexpr int kOffBar = kOffQtmp + 8 * 128 * 2;
-    static constexpr int kBars = 2 * kTcStages + 12;
+    static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 15;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
     static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
 };
 
 // Barrier indices (8 bytes each after kOffBar)
-constexpr int kBFull = 0;                 // [kTcStages]  K/V landed (TMA bytes)
-constexpr int kBEmpty = kTcStages;        // [kTcStages]  K/V consumed (PV commit)
-constexpr int kBSFull = 2 * kTcStages;    // [2] S^T in TMEM (commit)
-constexpr int kBSFree = kBSFull + 2;      // [2] softmax has read S^T (128 arrivals)
-constexpr int kBPFull = kBSFree + 2;      // [2] P tile written (128 arrivals)
-constexpr int kBPvDone = kBPFull + 2;     // [2] PV done reading P buffer (commit)
-constexpr int kBQFull = kBPvDone + 2;     // q staged for the piece (128 arrivals)
-constexpr int kBOFree = kBQFull + 1;      // [2] O buffer read by its piece's epilogue (32 arrivals)
-constexpr int kBDrain = kBOFree + 2;      // every MMA of the CTA has completed (2 commits)
-static_assert(kBDrain < 2 * kTcStages + 12, "barrier count");
+constexpr int kBFull = 0;                   // [kTcStages]  K/V landed (TMA bytes)
+constexpr int kBEmpty = kTcStages;          // [kTcStages]  K/V consumed (PV commit)
+constexpr int kBSFull = 2 * kTcStages;      // [2] S^T in TMEM (commit)
+constexpr int kBSFree = kBSFull + 2;        // [2] softmax has read S^T (128 arrivals)
+constexpr int kBPFull = kBSFree + 2;        // [2] P tile written (128 arrivals)
+constexpr int kBPvDone = kBPFull + 2;       // [2] PV done reading P buffer (commit)
+constexpr int kBQFull = kBPvDone + 2;       // [kTcQBufs] q staged (stager)
+constexpr int kBQEmpty = kBQFull + kTcQBufs;  // [kTcQBufs] q buffer read by its S^T MMAs (softmax)
+constexpr int kBOReady = kBQEmpty + kTcQBufs;  // [2] the piece's last PV has completed (commit)
+constexpr int kBStats = kBOReady + 2;       // [2] the piece's (m, l) written (softmax)
+constexpr int kBOFree = kBStats + 2;        // [2] O buffer and stats read by the epilogue (32 arrivals)
+constexpr int kBDrain = kBOFree + 2;        // every MMA of the CTA has completed (2 commits)
+static_assert(kBDrain < 2 * kTcStages + 2 * kTcQBufs + 15, "barrier count");
 
 __device__ __forceinline__ uint32_t bar_at(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
 
@@ -84,40 +92,93 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
     return (uint32_t)(r * 128 + ((((c >> 4) ^ (r & 7)) << 4) | (c & 15)));
 }
 
-// Decode step: store the step's new token of sequence b, kv head kvh (the newest of its L
-// tokens, row (L-1) % 128 of its last tile, cache slot `slot`) into the cache and into the
-// tile's K and V rows, which TMA filled with the slot's previous codes -- K rotated at L - 1,
-// both quantised from the fp64 quotient by the head's scale, as pkv_kv_store does.  One warp.
-__device__ __forceinline__ void tc_put_new_token(const DecodeParams &p, int b, int kvh, int L, int slot,
-                                                 uint32_t kt, uint32_t vt, int lane) {
+// Position of a unit in the walk over (sequence, kv head, tile): the issuers and the
+// producer's lanes step through their units one by one instead of searching each time.
+struct TcCursor {
+    int b, kvh, tile, nt;
+};
+
+__device__ __forceinline__ TcCursor tc_cursor(const int *pfx, int B, int Hkv, long long u) {
+    const UnitPos up = locate(pfx, B, Hkv, u);
+    return TcCursor{up.b, up.kvh, up.blk, up.nb};
+}
+
+__device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int Hkv) {
+    if (++c.tile < c.nt) return;
+    c.tile = 0;
+    if (++c.kvh < Hkv) return;
+    c.kvh = 0;
+    do {
+        ++c.b;
+        c.nt = c.b < B ? pfx[c.b + 1] - pfx[c.b] : 1;
+    } while (c.b < B && c.nt == 0);
+}
+
+// Decode step: the step's new token of sequence b, kv head kvh -- the newest of its L tokens,
+// row (L-1) % 128 of its last tile, cache slot `slot`.  fetch() loads what it needs (K and V
+// as bf16, the RoPE row, the slot) when the piece starts, so the loads overlap the piece's
+// waits; put() then rotates K at L - 1, quantises both from the fp64 quotient by the head's
+// scale (as pkv_kv_store does) and stores the codes into the cache and into the tile's K
+// and V rows, which TMA filled with the slot's previous codes.  One warp; lane i holds
+// dims i, i + 32, i + 64, i + 96.
+struct TcNewToken {
+    uint16_t k[4], v[4];
+    float c[2], sn[2];
+    int slot;   // -1: nothing to store
+    bool rope;
+};
+
+__device__ __forceinline__ void tc_fetch_new_token(const DecodeParams &p, int b, int kvh, TcNewToken &t, int lane) {
     constexpr int D = 128;
-    const int r = (L - 1) % kTcTile, pos = L - 1;
-    const float *rope = nullptr;
-    if (p.rope) {
-        if (pos >= p.max_pos) {
-            if (lane == 0) atomicOr(p.err, kErrBounds);
-            return;
-        }
-        rope = p.rope + (size_t)pos * D;
+    const int Lraw = __ldg(p.context_lens + b), L = min(Lraw, p.max_tokens);
+    t.slot = -1;
+    t.rope = p.rope != nullptr;
+    if (L != Lraw || L < 1) return;  // clipped to the block table: the kernel stores nothing
+    const int pos = L - 1;
+    if (p.rope && pos >= p.max_pos) {
+        if (lane == 0) atomicOr(p.err, kErrBounds);
+        return;
     }
+    const int e = __ldg(p.block_tables + (size_t)b * p.max_blocks + pos / p.bs);
+    if (e < 0 || (long long)e >= p.num_blocks) return;  // (the producer flags a bad entry)
+    t.slot = e * p.bs + pos % p.bs;
     const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
     const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
-    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;
-    const double ks = (double)__ldg(p.k_scale + kvh), vs = (double)__ldg(p.v_scale + kvh);
-    for (int i = lane; i < D / 2; i += 32) {
-        uint16_t kb[2] = {__ldg(kin + i), __ldg(kin + i + D / 2)};
-        const uint16_t vb[2] = {__ldg(vin + i), __ldg(vin + i + D / 2)};
-        if (rope) rope_pair_fast(kb[0], kb[1], __ldg(rope + i), __ldg(rope + D / 2 + i), kb[0], kb[1]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int e = i + h * (D / 2);
-            const uint32_t kc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[h]), ks));
-            const uint32_t vc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(vb[h]), vs));
-            static_cast<uint8_t *>(p.k_cache_w)[dst + e] = (uint8_t)kc;
-            static_cast<uint8_t *>(p.v_cache_w)[dst + e] = (uint8_t)vc;
-            asm volatile("st.shared.u8 [%0], %1;" ::"r"(kt + sw_off(r, e)), "r"(kc) : "memory");
-            asm volatile("st.shared.u8 [%0], %1;" ::"r"(vt + sw_off(r, e)), "r"(vc) : "memory");
+    for (int j = 0; j < 4; ++j) {
+        t.k[j] = __ldg(kin + lane + 32 * j);
+        t.v[j] = __ldg(vin + lane + 32 * j);
+    }
+    if (p.rope) {
+        const float *row = p.rope + (size_t)pos * D;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {  // the pairs (i, i + 64) for i = lane, lane + 32
+            t.c[j] = __ldg(row + lane + 32 * j);
+            t.sn[j] = __ldg(row + D / 2 + lane + 32 * j);
         }
+    }
+}
+
+__device__ __forceinline__ void tc_put_new_token(const DecodeParams &p, int kvh, int L, const TcNewToken &t,
+                                                 uint32_t kt, uint32_t vt, int lane) {
+    constexpr int D = 128;
+    if (t.slot < 0) return;
+    const int r = (L - 1) % kTcTile;
+    uint16_t kb[4] = {t.k[0], t.k[1], t.k[2], t.k[3]};
+    if (t.rope)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) rope_pair_fast(kb[j], kb[j + 2], t.c[j], t.sn[j], kb[j], kb[j + 2]);
+    const size_t dst = ((size_t)t.slot * p.Hkv + kvh) * D;
+    const double ks = (double)__ldg(p.k_scale + kvh), vs = (double)__ldg(p.v_scale + kvh);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int e = lane + 32 * j;
+        const uint32_t kc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[j]), ks));
+        const uint32_t vc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(t.v[j]), vs));
+        static_cast<uint8_t *>(p.k_cache_w)[dst + e] = (uint8_t)kc;
+        static_cast<uint8_t *>(p.v_cache_w)[dst + e] = (uint8_t)vc;
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(kt + sw_off(r, e)), "r"(kc) : "memory");
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(vt + sw_off(r, e)), "r"(vc) : "memory");
     }
 }
 
@@ -132,6 +193,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t *smem = smem_raw + (sbase - smem_u32(smem_raw));
     const uint32_t sStages = sbase, sQ = sbase + Geo::kOffQ, sP = sbase + Geo::kOffP;
     float *red = reinterpret_cast<float *>(smem + Geo::kOffRed);
+    float *stats = reinterpret_cast<float *>(smem + Geo::kOffStats);  // [O buffer][m | l][8]
+    float *sqbuf = reinterpret_cast<float *>(smem + Geo::kOffSq);     // [q buffer]
     uint16_t *qtmp = reinterpret_cast<uint16_t *>(smem + Geo::kOffQtmp);
     const uint32_t bars = sbase + Geo::kOffBar;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Geo::kOffBar + 8 * Geo::kBars);
@@ -201,16 +264,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar_at(bars, kBSFree + i), 128);
             mbar_init(bar_at(bars, kBPFull + i), 128);
             mbar_init(bar_at(bars, kBPvDone + i), 1);
+            mbar_init(bar_at(bars, kBOReady + i), 1);
+            mbar_init(bar_at(bars, kBStats + i), 1);
+            mbar_init(bar_at(bars, kBOFree + i), 32);
         }
-        mbar_init(bar_at(bars, kBQFull), 128);
-        mbar_init(bar_at(bars, kBOFree), 32);
-        mbar_init(bar_at(bars, kBOFree + 1), 32);
+        for (int i = 0; i < kTcQBufs; ++i) {
+            mbar_init(bar_at(bars, kBQFull + i), 1);
+            mbar_init(bar_at(bars, kBQEmpty + i), 1);
+        }
         mbar_init(bar_at(bars, kBDrain), 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // zero the rows of the q and P operands that no head uses (rows 2G.. stay zero)
-    for (int i = threadIdx.x; i < (2 * Geo::kQ + 2 * Geo::kP) / 16; i += kTcThreads)
+    // zero the q and P operands: the rows no head uses (2G.. of q, 2G.. of P) stay zero
+    for (int i = threadIdx.x; i < (kTcQBufs * Geo::kQ + 2 * Geo::kP) / 16; i += kTcThreads)
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(sQ + 16 * i), "r"(0u) : "memory");
     fence_proxy_async_smem();
     if (warp == 1) {
@@ -225,13 +292,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // TMEM: S^T buffers at columns 0 and 16 (128 lanes x 16), O buffers at columns 128 and 256
     // (rows 0..2G-1 of 64 x 128 each)
 
-    // unit k of this CTA -> (sequence, kv head, tile); `first` = a piece starts here
+    // unit k of this CTA -> (sequence, kv head, tile of the sequence, its tile count)
     auto unit = [&](int k, int &b, int &kvh, int &tile, int &ntiles) {
         UnitPos up = locate(pfx, p.B, Hu, u0 + k);
         b = up.b;
         kvh = up.kvh;
         tile = up.blk;
         ntiles = up.nb;
+    };
+    // a bounded wait by lane 0 of the calling warp, its outcome broadcast to the warp (the
+    // __syncwarp orders the other lanes' accesses after lane 0's acquire)
+    auto wait0 = [&](int bi, uint32_t parity) -> bool {
+        bool r = true;
+        if (lane == 0) r = !*abort_flag && mbar_wait_bounded(bar_at(bars, bi), parity, p.err);
+        __syncwarp();
+        return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
     };
 
     if (warp == 0) {
@@ -241,22 +316,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             prefetch_tmap(&tm_v);
         }
         const int oob = (int)(p.num_blocks * p.bs < 0x7fffffffLL ? p.num_blocks * p.bs : 0x7fffffff);
-        // this lane's box of every tile: 16-token piece `piece` (8-token blocks: half `half`,
-        // two boxes of 8 rows per piece); the boxes of a tile go out from their lanes at once
+        // Lanes cover a batch of tiles: lane = tile of the batch * boxes + box, a box being
+        // 16-token piece `bpiece` of the tile (8-token blocks: half `half`, two boxes of 8
+        // rows per piece).  One pass of block-table loads serves the whole batch, and each
+        // box is issued by its own lane.
         const bool two = p.bs == 8;
-        const int n_box = two ? 16 : 8;
-        const int half = two ? (lane & 1) : 0, bpiece = two ? (lane >> 1) : lane;
+        const int n_box = two ? 16 : 8, tpb = 32 / n_box;
+        const int bt = lane / n_box, bx = lane % n_box;
+        const int half = two ? (bx & 1) : 0, bpiece = two ? (bx >> 1) : bx;
         const uint32_t box_off = (uint32_t)(bpiece * 2048 + half * 1024);
+        TcCursor cur = tc_cursor(pfx, p.B, Hu, u0 + min(bt, nunits - 1));  // this lane's tile
         uint32_t issued = 0, phases = 0;
         bool ok = true;
-        for (int k = 0; k < nunits && ok; ++k) {
-            int b, kvh, tile, ntiles;
-            unit(k, b, kvh, tile, ntiles);
-            const int L = min(__ldg(p.context_lens + b), p.max_tokens);
+        for (int k0 = 0; k0 < nunits && ok; k0 += tpb) {
             int row = oob;
-            if (lane < n_box) {
-                const int pc = tile * 8 + bpiece;  // 16-token piece of the sequence
-                const int32_t *tab = p.block_tables + (size_t)b * p.max_blocks;
+            if (k0 + bt < nunits) {
+                const int L = min(__ldg(p.context_lens + cur.b), p.max_tokens);
+                const int pc = cur.tile * 8 + bpiece;  // 16-token piece of the sequence
+                const int32_t *tab = p.block_tables + (size_t)cur.b * p.max_blocks;
                 if (p.bs == 16) {
                     if (pc * 16 < L) row = cache_row(p, __ldg(tab + pc), 0);
                 } else if (p.bs == 32) {
@@ -266,24 +343,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (e * 8 < L) row = cache_row(p, __ldg(tab + e), 0);
                 }
             }
-            const int s = k % kTcStages;
-            const uint32_t fb = bar_at(bars, kBFull + s);
-            if (lane == 0) {
-                if (*abort_flag || !mbar_wait_bounded(bar_at(bars, kBEmpty + s), ((k / kTcStages) & 1) ^ 1, p.err)) {
-                    ok = false;
-                    *abort_flag = 1;
-                } else {
-                    mbar_arrive_expect_tx(fb, Geo::kStage);
-                    issued |= 1u << s;
-                    phases = (phases & ~(1u << s)) | ((uint32_t)((k / kTcStages) & 1) << s);
+            const int kvh = cur.kvh;
+            for (int t = 0; t < tpb && k0 + t < nunits; ++t) {
+                const int k = k0 + t, s = k % kTcStages;
+                const uint32_t fb = bar_at(bars, kBFull + s);
+                if (lane == 0) {
+                    if (*abort_flag ||
+                        !mbar_wait_bounded(bar_at(bars, kBEmpty + s), ((k / kTcStages) & 1) ^ 1, p.err)) {
+                        ok = false;
+                        *abort_flag = 1;
+                    } else {
+                        mbar_arrive_expect_tx(fb, Geo::kStage);
+                        issued |= 1u << s;
+                        phases = (phases & ~(1u << s)) | ((uint32_t)((k / kTcStages) & 1) << s);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                if (bt == t) {
+                    const uint32_t dk = sStages + s * Geo::kStage;
+                    tma_load_3d(dk + box_off, &tm_k, fb, 0, kvh, row);
+                    tma_load_3d(dk + Geo::kKV + box_off, &tm_v, fb, 0, kvh, row);
                 }
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (ok && lane < n_box) {
-                const uint32_t dk = sStages + s * Geo::kStage;
-                tma_load_3d(dk + box_off, &tm_k, fb, 0, kvh, row);
-                tma_load_3d(dk + Geo::kKV + box_off, &tm_v, fb, 0, kvh, row);
-            }
+            // this lane's tile of the next batch
+            for (int t = 0; t < tpb; ++t) tc_next(cur, pfx, p.B, Hu);
         }
         if (lane == 0)  // never leave with a TMA copy landing in shared memory
             for (int s = 0; s < kTcStages; ++s)
@@ -293,37 +377,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // Lane 0 issues; the whole warp walks the units (with STEP it stores the step's new
         // token into the tile before that tile's S^T is issued).
         constexpr uint32_t idS = tc::mma_idesc(128, 16, false, true);  // E4M3 x E4M3 -> f32
-        auto wait0 = [&](int bi, uint32_t parity) -> bool {
-            bool r = true;
-            if (lane == 0) r = !*abort_flag && mbar_wait_bounded(bar_at(bars, bi), parity, p.err);
-            return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
-        };
         bool ok = true;
         int piece = -1;
-        for (int k = 0; k < nunits && ok; ++k) {
-            int b, kvh, tile, ntiles;
-            unit(k, b, kvh, tile, ntiles);
+        TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
+        TcNewToken nt;
+        for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
+            const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
             if (k == 0 || tile == 0) {
                 ++piece;
-                ok = wait0(kBQFull, piece & 1);
+                // a piece that ends its sequence stores the step's new token: fetch it now
+                if (STEP && k + (ntiles - 1 - tile) < nunits) tc_fetch_new_token(p, b, kvh, nt, lane);
+                ok = wait0(kBQFull + piece % kTcQBufs, (piece / kTcQBufs) & 1);
             }
             ok = ok && wait0(kBFull + k % kTcStages, (k / kTcStages) & 1) &&
                  (k < 2 || wait0(kBSFree + (k & 1), ((k - 2) >> 1) & 1));
             if (!ok) break;
             const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
             if constexpr (STEP) {
-                const int Lraw = __ldg(p.context_lens + b), L = min(Lraw, p.max_tokens);
-                if (tile == ntiles - 1 && L == Lraw) {  // the sequence's last tile holds its new token
-                    const int e = __ldg(p.block_tables + (size_t)b * p.max_blocks + (L - 1) / p.bs);
-                    if (e >= 0 && (long long)e < p.num_blocks)
-                        tc_put_new_token(p, b, kvh, L, e * p.bs + (L - 1) % p.bs, kd, kd + Geo::kKV, lane);
+                if (tile == ntiles - 1) {  // the sequence's last tile holds its new token
+                    tc_put_new_token(p, kvh, min(__ldg(p.context_lens + b), p.max_tokens), nt, kd, kd + Geo::kKV,
+                                     lane);
                     fence_proxy_async_smem();  // the tensor cores read these rows next
                     __syncwarp();
                 }
             }
             if (lane == 0) {
                 tc::tc_fence_after();
-                const uint32_t qd = sQ + (piece & 1) * Geo::kQ;
+                const uint32_t qd = sQ + (piece % kTcQBufs) * Geo::kQ;
 #pragma unroll
                 for (int kk = 0; kk < D / 32; ++kk)
                     tc::mma_ss_f8(tmem + 16 * (k & 1), tc::sw128_desc(kd + 32 * kk, 16, 1024),
@@ -340,10 +420,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             bool ok = true;
             int piece = -1;
-            for (int k = 0; k < nunits && ok; ++k) {
-                int b, kvh, tile, ntiles;
-                unit(k, b, kvh, tile, ntiles);
-                const bool first = k == 0 || tile == 0;
+            TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
+            for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
+                const bool first = k == 0 || cur.tile == 0;
+                const bool last = k == nunits - 1 || cur.tile == cur.nt - 1;
                 if (first) ++piece;
                 // a piece's first PV overwrites its O buffer: the epilogue of piece - 2 must
                 // have read it
@@ -361,6 +441,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                   tc::sw128_desc(vd + 4096 * kk, 16384, 1024), idO, (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
                 tc::mma_commit(bar_at(bars, kBPvDone + (k & 1)));
+                if (last) tc::mma_commit(bar_at(bars, kBOReady + (piece & 1)));
             }
             if (!ok) *abort_flag = 1;
             // drain: no MMA of either issuer may still write TMEM when it is released
@@ -368,34 +449,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait_bounded(bar_at(bars, kBDrain), 0, p.err);
         }
         __syncwarp();
-    } else {
-        // ---------------------------------------------------------------- softmax / epilogue
-        const int sw = warp - kTcSoftmax0;               // 0..3
-        const int quad = warp & 3;                        // TMEM lanes 32*quad .. +31
-        const int t = quad * 32 + lane;                   // token of the tile = TMEM lane
-        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int ct = threadIdx.x - 32 * kTcSoftmax0;    // 0..127
-        bool alive = true;
-        // Stage q of the piece starting at unit kk (piece index pc) into q buffer pc & 1: the
-        // G heads rotated at L-1, one power-of-two scale for the group (returned), high parts
-        // to rows 0..G-1 and low parts to rows G..2G-1.
-        auto stage_q = [&](int kk, int pc) -> float {
-            int b, kvh, tile, ntiles;
-            unit(kk, b, kvh, tile, ntiles);
+    } else if (warp == kTcQWarp) {
+        // ---------------------------------------------------------------- q stager
+        // For each piece in turn, into q buffer piece % kTcQBufs: the G heads' q rotated at
+        // L - 1, scaled by one power of two for the group (kept in sqbuf) and split into high
+        // parts (rows 0..G-1) and low parts (rows G..2G-1) as E4M3 codes.  Runs up to
+        // kTcQBufs pieces ahead of the softmax.
+        TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
+        int k = 0;
+        for (int pc = 0; k < nunits; ++pc) {
+            const int b = cur.b, kvh = cur.kvh;
+            const int piece_len = min(cur.nt - cur.tile, nunits - k);
+            const int slot = pc % kTcQBufs;
+            if (!wait0(kBQEmpty + slot, ((pc / kTcQBufs) & 1) ^ 1)) {
+                if (lane == 0) *abort_flag = 1;
+                break;
+            }
             const int L = min(__ldg(p.context_lens + b), p.max_tokens);
+            const int pos = L - 1;
+            const bool rope_ok = p.rope && pos >= 0 && pos < p.max_pos;
+            if (p.rope && !rope_ok && lane == 0) atomicOr(p.err, kErrBounds);
             float amax = 0.f;
-            for (int e = ct; e < G * (D / 2); e += 128) {
+#pragma unroll 4
+            for (int e = lane; e < G * (D / 2); e += 32) {
                 const int h = e / (D / 2), i = e % (D / 2);
                 const uint16_t *qr = p.q + ((size_t)b * p.Hq + kvh * G + h) * D;
                 uint16_t x1 = __ldg(qr + i), x2 = __ldg(qr + i + D / 2);
-                if (p.rope) {
-                    const int pos = L - 1;
-                    if (pos >= 0 && pos < p.max_pos) {
-                        const float *row = p.rope + (size_t)pos * D;
-                        rope_pair_fast(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
-                    } else {
-                        atomicOr(p.err, kErrBounds);
-                    }
+                if (rope_ok) {
+                    const float *row = p.rope + (size_t)pos * D;
+                    rope_pair_fast(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
                 }
                 qtmp[h * D + i] = x1;
                 qtmp[h * D + i + D / 2] = x2;
@@ -404,15 +486,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            if (lane == 0) red[sw] = amax;
-            named_bar(kTcBar, 128);
-            amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-            named_bar(kTcBar, 128);  // red and qtmp are rewritten later
             const float sq = amax > 0.f
                                  ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
                                  : 1.f;
-            const uint32_t qd = sQ + (pc & 1) * Geo::kQ;
-            for (int e = ct; e < G * (D / 4); e += 128) {  // four dims per thread
+            __syncwarp();  // qtmp complete
+            const uint32_t qd = sQ + slot * Geo::kQ;
+            for (int e = lane; e < G * (D / 4); e += 32) {  // four dims per lane and step
                 const int h = e / (D / 4), c = 4 * (e % (D / 4));
                 const uint2 w = *reinterpret_cast<const uint2 *>(qtmp + h * D + c);
                 uint32_t hi, lo;
@@ -420,19 +499,146 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(h, c)), "r"(hi) : "memory");
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(G + h, c)), "r"(lo) : "memory");
             }
+            if (lane == 0) sqbuf[slot] = sq;
             fence_proxy_async_smem();
-            mbar_arrive(bar_at(bars, kBQFull));
-            return sq;
-        };
-        int k = 0, piece = 0;
-        float sq = stage_q(0, 0);
-        while (k < nunits) {
+            __syncwarp();  // (qtmp is rewritten by the next piece)
+            if (lane == 0) mbar_arrive(bar_at(bars, kBQFull + slot));
+            k += piece_len;
+            for (int t = 0; t < piece_len; ++t) tc_next(cur, pfx, p.B, Hu);
+        }
+    } else if (warp == kTcEpiWarp) {
+        // ---------------------------------------------------------------- epilogue
+        // For each piece in turn, once its last PV has completed and the softmax has left its
+        // (m, l): O (TMEM lanes 0..2G-1 of O buffer piece & 1) -> the output rows (a whole
+        // segment) or the piece's partial slot, then O buffer free.
+        int k = 0;
+        for (int piece = 0; k < nunits; ++piece) {
+            int b, kvh, tile, ntiles;
+            unit(k, b, kvh, tile, ntiles);
+            const int piece_len = min(ntiles - tile, nunits - k);
+            const bool whole = tile == 0 && piece_len == ntiles;
+            const int ob = piece & 1;
+            const bool fin = wait0(kBStats + ob, (piece >> 1) & 1) && wait0(kBOReady + ob, (piece >> 1) & 1);
+            if (!fin && lane == 0) *abort_flag = 1;
+            tc::tc_fence_after();
+            // lanes 0..G-1 hold O rows h (high parts of p), lanes G..2G-1 rows G+h (low parts)
+            const int h = lane < G ? lane : (lane < 2 * G ? lane - G : 0);
+            const float m = stats[ob * 16 + h], l = stats[ob * 16 + 8 + h];
+            const int segu = b * Hu + kvh;
+            float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
+            const float vs = __ldg(p.v_scale + kvh);
+            const float inv = (l > 0.f && fin) ? vs / l : 0.f;
+            const uint32_t tO = tmem + kTcO + 128u * (uint32_t)ob;
+            __nv_bfloat16 *orow = p.out + ((size_t)b * p.Hq + kvh * G + h) * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t rr[32];
+                if (fin) {
+                    tc::tmem_ld32(tO + c0, rr);
+                    tc::tc_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) rr[e] = 0u;
+                }
+                float o[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    o[e] = __uint_as_float(rr[e]) + __shfl_down_sync(0xffffffffu, __uint_as_float(rr[e]), G);
+                if (lane < G) {
+                    if (whole) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 w;
+                            w.x = tc::pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
+                            w.y = tc::pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
+                            w.z = tc::pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
+                            w.w = tc::pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
+                            dst[v] = w;
+                        }
+                    } else {
+                        float4 *dst = reinterpret_cast<float4 *>(slot + h * D + c0);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+                    }
+                }
+            }
+            if (!whole && lane < G) {
+                slot[G * D + lane] = m;
+                slot[G * D + G + lane] = l;
+            }
+            tc::tc_fence_before();
+            mbar_arrive(bar_at(bars, kBOFree + ob));
+            if constexpr (STEP) {
+                if (!whole) {
+                    // the last of the CTAs c0..c1 that cut this segment merges it (as the
+                    // combine kernel does) and clears the counter for the next call
+                    __threadfence();
+                    __syncwarp();
+                    const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
+                    const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
+                    int last = 0;
+                    if (lane == 0) last = atomicAdd(p.counters + segu, 1) == c1 - c0;
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    if (last) {
+                        __threadfence();
+                        // four dims per lane: M = max m_c, o = sum e^(m_c - M) acc_c / sum e^(m_c - M) l_c
+#pragma unroll
+                        for (int i = 0; i < G * D / 128; ++i) {
+                            const int e = (i * 32 + lane) * 4, g = e / D, d = e % D;
+                            float M = -INFINITY;
+                            for (int cc = c0; cc <= c1; ++cc)
+                                M = fmaxf(M, __ldcg(p.partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D + g));
+                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                            float ls = 0.f;
+                            for (int cc = c0; cc <= c1; ++cc) {
+                                const float *sl = p.partials + (size_t)(segu + cc) * (G * (D + 2));
+                                const float mk = __ldcg(sl + G * D + g);
+                                const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
+                                const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));
+                                acc.x += f * x.x;
+                                acc.y += f * x.y;
+                                acc.z += f * x.z;
+                                acc.w += f * x.w;
+                                ls += f * __ldcg(sl + G * D + G + g);
+                            }
+                            const float r = ls > 0.f ? vs / ls : 0.f;
+                            uint2 w;
+                            w.x = tc::pack_bf16x2(acc.x * r, acc.y * r);
+                            w.y = tc::pack_bf16x2(acc.z * r, acc.w * r);
+                            *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
+                        }
+                        if (lane == 0) p.counters[segu] = 0;
+                    }
+                }
+            }
+            k += piece_len;
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax (warps 2-5)
+        const int sw = warp - kTcSoftmax0;               // 0..3
+        const int quad = warp & 3;                        // TMEM lanes 32*quad .. +31
+        const int t = quad * 32 + lane;                   // token of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int ct = threadIdx.x - 32 * kTcSoftmax0;    // 0..127
+        bool alive = true;
+        int k = 0;
+        for (int piece = 0; k < nunits; ++piece) {
             int b, kvh, tile, ntiles;
             unit(k, b, kvh, tile, ntiles);
             const int piece_len = min(ntiles - tile, nunits - k);
             const int L = min(__ldg(p.context_lens + b), p.max_tokens);
-            const bool whole = tile == 0 && piece_len == ntiles;
+            const int qslot = piece % kTcQBufs;
             const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
+            // the piece's q scale (and q) from the stager
+            const bool qok = alive && !*abort_flag &&
+                             mbar_wait_bounded(bar_at(bars, kBQFull + qslot), (piece / kTcQBufs) & 1, p.err);
+            if (!__all_sync(0xffffffffu, qok)) {
+                alive = false;
+                *abort_flag = 1;
+            }
+            const float sq = alive ? sqbuf[qslot] : 1.f;
             const float sc = p.scale_log2 * __ldg(p.k_scale + kvh) / sq;
             float mref[G], lsum[G];
 #pragma unroll
@@ -547,8 +753,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::tc_fence_before();
                 mbar_arrive(bar_at(bars, kBPFull + pb));
             }
-            // ---- end of the piece: the sums over the 128 tokens, the next piece's q, then the
-            // epilogue (O from TMEM), which overlaps the next piece's MMAs
+            // q buffer qslot is free: every S^T of the piece has completed (each SFull was waited)
+            if (ct == 0) mbar_arrive(bar_at(bars, kBQEmpty + qslot));
+            // ---- end of the piece: its (m, l) per head for the epilogue warp
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float l = lsum[h];
@@ -557,114 +764,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (lane == 0) red[32 + 8 * sw + h] = l;
             }
             named_bar(kTcBar, 128);
-            const float sq_next = k < nunits ? stage_q(k, piece + 1) : 1.f;
             if (quad == 0) {
-                const int jl = k - 1;  // the piece's last tile
-                bool fin = alive && mbar_wait_bounded(bar_at(bars, kBPvDone + (jl & 1)), (jl >> 1) & 1, p.err);
-                fin = __all_sync(0xffffffffu, fin);
-                if (!fin) {
+                // stats buffer piece & 1 was last read by the epilogue of piece - 2
+                bool ok = alive && (piece < 2 || wait0(kBOFree + (piece & 1), ((piece >> 1) - 1) & 1));
+                if (!__all_sync(0xffffffffu, ok)) {
                     alive = false;
                     *abort_flag = 1;
                 }
-                tc::tc_fence_after();
-                // lanes 0..G-1 hold O rows h (high parts of p), lanes G..2G-1 rows G+h (low parts)
-                const int h = lane < G ? lane : (lane < 2 * G ? lane - G : 0);
-                float m = -INFINITY;
+                if (lane < G) {
+                    float m = -INFINITY;
 #pragma unroll
-                for (int hh = 0; hh < G; ++hh)
-                    if (hh == h) m = mref[hh];
-                const float l = red[32 + h] + red[40 + h] + red[48 + h] + red[56 + h];
-                const int segu = b * Hu + kvh;
-                float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
-                const float vs = __ldg(p.v_scale + kvh);
-                const float inv = (l > 0.f && fin) ? vs / l : 0.f;
-                __nv_bfloat16 *orow = p.out + ((size_t)b * p.Hq + kvh * G + h) * D;
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t rr[32];
-                    if (fin) {
-                        tc::tmem_ld32(tO + c0, rr);
-                        tc::tc_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) rr[e] = 0u;
-                    }
-                    float o[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        o[e] = __uint_as_float(rr[e]) + __shfl_down_sync(0xffffffffu, __uint_as_float(rr[e]), G);
-                    if (lane < G) {
-                        if (whole) {
-                            uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                uint4 w;
-                                w.x = tc::pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
-                                w.y = tc::pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
-                                w.z = tc::pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
-                                w.w = tc::pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
-                                dst[v] = w;
-                            }
-                        } else {
-                            float4 *dst = reinterpret_cast<float4 *>(slot + h * D + c0);
-#pragma unroll
-                            for (int v = 0; v < 8; ++v)
-                                dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
-                        }
-                    }
+                    for (int hh = 0; hh < G; ++hh)
+                        if (hh == lane) m = mref[hh];
+                    stats[(piece & 1) * 16 + lane] = m;
+                    stats[(piece & 1) * 16 + 8 + lane] = red[32 + lane] + red[40 + lane] + red[48 + lane] + red[56 + lane];
                 }
-                if (!whole && lane < G) {
-                    slot[G * D + lane] = m;
-                    slot[G * D + G + lane] = l;
-                }
-                tc::tc_fence_before();
-                mbar_arrive(bar_at(bars, kBOFree + (piece & 1)));
-                if constexpr (STEP) {
-                    if (!whole) {
-                        // the last of the CTAs c0..c1 that cut this segment merges it (as the
-                        // combine kernel does) and clears the counter for the next call
-                        __threadfence();
-                        __syncwarp();
-                        const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
-                        const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
-                        int last = 0;
-                        if (lane == 0) last = atomicAdd(p.counters + segu, 1) == c1 - c0;
-                        last = __shfl_sync(0xffffffffu, last, 0);
-                        if (last) {
-                            __threadfence();
-                            // four dims per lane: M = max m_c, o = sum e^(m_c - M) acc_c / sum e^(m_c - M) l_c
-#pragma unroll
-                            for (int i = 0; i < G * D / 128; ++i) {
-                                const int e = (i * 32 + lane) * 4, g = e / D, d = e % D;
-                                float M = -INFINITY;
-                                for (int cc = c0; cc <= c1; ++cc)
-                                    M = fmaxf(M, __ldcg(p.partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D + g));
-                                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                                float ls = 0.f;
-                                for (int cc = c0; cc <= c1; ++cc) {
-                                    const float *sl = p.partials + (size_t)(segu + cc) * (G * (D + 2));
-                                    const float mk = __ldcg(sl + G * D + g);
-                                    const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
-                                    const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));
-                                    acc.x += f * x.x;
-                                    acc.y += f * x.y;
-                                    acc.z += f * x.z;
-                                    acc.w += f * x.w;
-                                    ls += f * __ldcg(sl + G * D + G + g);
-                                }
-                                const float r = ls > 0.f ? vs / ls : 0.f;
-                                uint2 w;
-                                w.x = tc::pack_bf16x2(acc.x * r, acc.y * r);
-                                w.y = tc::pack_bf16x2(acc.z * r, acc.w * r);
-                                *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
-                            }
-                            if (lane == 0) p.counters[segu] = 0;
-                        }
-                    }
-                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_at(bars, kBStats + (piece & 1)));
             }
-            ++piece;
-            sq = sq_next;
         }
     }
 
