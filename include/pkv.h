@@ -108,8 +108,8 @@ size_t pkv_cache_bytes(int num_layers, long long num_blocks, int block_size, int
  *   slot_mapping  [num_tokens] int32; -1 = skip the token
  *   k_scale,
  *   v_scale       [n_kv_heads] fp32, required for PKV_FP8_E4M3 (ignored for bf16):
- *                 code = E4M3(value / scale), quotient in fp64, round to nearest even,
- *                 saturated to +-448
+ *                 code = E4M3(value / scale): the exact quotient rounded to nearest even
+ *                 (the same code as rounding its fp64 value), saturated to +-448
  *   rope_cos_sin  RoPE table or NULL; when given, K is rotated at its position before it
  *                 is stored (V never is), and cu_seqlens/context_lens/num_seqs/max_pos
  *                 must describe the batch; otherwise they are ignored and may be NULL/0
@@ -266,8 +266,8 @@ size_t pkv_decode_step_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_hea
  *                 p % block_size of block block_tables[b][p / block_size] (ENG §2.2), so
  *                 no slot mapping is taken; a sequence with L_b = 0 has no new token.
  *   k_cache,
- *   v_cache       written at those slots (E4M3 codes for PKV_FP8_E4M3, from the fp64 quotient
- *                 by the head's scale, as in pkv_kv_store)
+ *   v_cache       written at those slots (E4M3 codes for PKV_FP8_E4M3, of the quotient by
+ *                 the head's scale, as in pkv_kv_store)
  *   other arguments as pkv_paged_decode_attention (rope_cos_sin rotates both the new K and q
  *   at L_b - 1)
  *   workspace     at least pkv_decode_step_workspace_bytes(...) bytes, 16-byte aligned,

@@ -85,6 +85,39 @@ __device__ __forceinline__ uint32_t f64_to_e4m3(double x) {
     return sign | (E << 3) | M;
 }
 
+// E4M3 code (round to nearest even, saturating at 448) of the exact quotient x / s for s > 0:
+// the code f64_to_e4m3 gives for the fp64 quotient, computed in fp32.  Every rounding
+// midpoint between two E4M3 values is an fp32 value and the fp32 quotient is correctly
+// rounded, so it lies on the exact quotient's side of every midpoint unless it is one; then
+// the sign of the residual x - q s (one fused multiply-add: the sign of a nonzero result is
+// exact) tells where the exact quotient lies, and q moves one fp32 ulp that way, crossing no
+// other midpoint.  (The fp64 quotient of a bf16 by an fp32 value is never rounded onto a
+// midpoint either: that would need a quotient within 2^-53 of one, while a bf16 x differs
+// from m * s, when not equal, by at least 2^-29 of it.)
+__device__ __forceinline__ uint32_t e4m3_of_quotient(float x, float s) {
+    if (!(s > 0.f) || isnan(x)) return f64_to_e4m3((double)x / (double)s);  // (a NaN keeps its sign)
+    float q = __fdiv_rn(x, s);
+    const float a = fabsf(q);
+    bool mid;
+    if (a < 0.015625f) {  // E4M3 subnormal grid 2^-9: midpoints at odd multiples of 2^-10
+        const float t = a * 1024.f;  // exact
+        const int ti = (int)t;
+        mid = (float)ti == t && (ti & 1) != 0;
+    } else {  // 4 significant bits: a midpoint has bit 19 alone set below them
+        mid = a < 448.f && (__float_as_uint(a) & 0xFFFFFu) == 0x80000u;
+    }
+    if (mid) {
+        const float r = __fmaf_rn(-q, s, x);
+        if (r != 0.f) {
+            const bool away = (r > 0.f) == (q > 0.f);  // the exact quotient has the larger magnitude
+            q = __uint_as_float(__float_as_uint(q) + (away ? 1u : 0xFFFFFFFFu));
+        }
+    }
+    uint16_t c;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "f"(0.f), "f"(q));
+    return c & 0xFFu;
+}
+
 // ------------------------------------------------------------------------------ PTX
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

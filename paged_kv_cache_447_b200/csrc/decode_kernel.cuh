@@ -596,8 +596,8 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
         if constexpr (STEP) {
             // The step's new token of this group's heads, when this piece holds its sequence's
             // last block (and the context was not clipped to the block table): K rotated at
-            // L - 1 and V, converted as the cache stores them (E4M3 codes from the fp64
-            // quotient by the head's scale, as pkv_kv_store does), go into the cache and into
+            // L - 1 and V, converted as the cache stores them (E4M3 codes of the exact quotient
+            // by the head's scale, as pkv_kv_store does), go into the cache and into
             // mrg, which is free until the piece's merge.  The warp that takes the last block
             // copies its head's rows from there into its tile, so no global load sits on that
             // warp's path.  (The loads were issued before q's, in nt_*.)
@@ -623,9 +623,9 @@ __global__ void __launch_bounds__(Geometry<D, FP8, G, HPU>::kThreads,
                             const int el = i + h * (D / 2);
                             if constexpr (FP8) {
                                 const uint32_t kc =
-                                    f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[h]), (double)__ldg(p.k_scale + kvo)));
+                                    e4m3_of_quotient(__uint_as_float((uint32_t)kb[h] << 16), __ldg(p.k_scale + kvo));
                                 const uint32_t vc =
-                                    f64_to_e4m3(__ddiv_rn(bf16_to_f64(nt_v[j][h]), (double)__ldg(p.v_scale + kvo)));
+                                    e4m3_of_quotient(__uint_as_float((uint32_t)nt_v[j][h] << 16), __ldg(p.v_scale + kvo));
                                 static_cast<uint8_t *>(p.k_cache_w)[dst + el] = (uint8_t)kc;
                                 static_cast<uint8_t *>(p.v_cache_w)[dst + el] = (uint8_t)vc;
                                 krow[el] = (uint8_t)kc;

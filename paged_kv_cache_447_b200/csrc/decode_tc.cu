@@ -16,6 +16,9 @@
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
 //   warp 6      lane 0 issues the PV MMAs
+//   warp 7      q stager: each piece's q (rotated, scaled, split), its context length and
+//               scales, up to 4 pieces ahead
+//   warp 8      epilogue: O of a finished piece -> output rows or a partial slot
 // Per tile:
 //   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
 //                 cache stores it (K-major), B = q as E4M3 rows -- the G heads' high parts in
@@ -24,15 +27,16 @@
 //   softmax       thread t adds its two parts, masks past the context, takes the per-head
 //                 tile maxima across the four warps, updates the lazy running max (O is
 //                 rescaled only when a max grows by more than 2^8) and writes p as high and
-//                 low E4M3 parts into a shared-memory P tile: row h / G+h, byte t.
-//   O += P V      M = 64 (rows 0..2G-1 used), N = 128 dims, K = 128 tokens: A = the P tile,
-//                 B = the V tile MN-major as the cache stores it; O = rows h + rows G+h.
+//                 low E4M3 parts into a shared-memory P tile: row h / 8+h, byte t.
+//   O += P V      M = 64, N = 128 dims, K = 128 tokens, twice: A = the P tile from row 0 (high
+//                 parts in rows 0..G-1) and from row 8 (low parts in rows 8..8+G-1), B = the V
+//                 tile MN-major as the cache stores it; O rows 0..G-1 = the G heads.
 // S^T and PV are issued by two threads, each waiting only for its own inputs (S^T: tile
 // landed, S buffer free, the piece's q staged; PV: P written, O buffer free), so a stage goes
 // back to the producer as soon as its PV completes, and S^T of later tiles runs ahead.  They
-// touch disjoint TMEM columns and shared memory.  S, P and q are double-buffered, and so is
-// O (by piece), so the epilogue of one piece overlaps the next piece's MMAs; the next
-// piece's q is staged before the epilogue.
+// touch disjoint TMEM columns and shared memory.  S and P are double-buffered, q has 4
+// buffers and O two (by piece), so neither the next piece's q nor the last piece's epilogue
+// holds up the tiles.
 #include "decode_kernel.cuh"
 #include "tcgen05.cuh"
 
@@ -50,19 +54,39 @@ constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
 constexpr uint32_t kTcO = 128;  // TMEM column of O buffer 0 (buffer 1 follows at +128)
 
+// What the q stager knows of a piece, for the softmax warps.
+struct TcMeta {
+    int b, kvh, tile, ntiles, piece_len, L;
+    float sc;  // score scale in exp2 units, over the q scale: scale * log2(e) * k_scale / sq
+    float vs;  // the head's V scale
+    int nt_row;  // decode step: tile row of the new token staged in the slot's codes, or -1
+};
+
+// What the softmax hands the epilogue warp per piece: the piece and its per-head (m, l).
+struct TcStats {
+    float m[8], l[8];
+    int b, kvh, ntiles, whole, piece_len;
+    float vs;
+    int pad[2];
+};
+
 template <int G>
 struct TcGeo {
     static constexpr int D = 128;
     static constexpr int kKV = kTcTile * D;         // one E4M3 K (or V) tile: 16 KB
     static constexpr int kStage = 2 * kKV;
     static constexpr int kQ = 16 * 128;             // B operand of S^T: 16 rows x 128 codes
-    static constexpr int kP = 64 * 128;             // A operand of PV: 64 rows x 128 tokens
+    // A operands of PV: p's high parts in rows 0..G-1 (read as rows 0..63) and its low parts
+    // in rows 8..8+G-1 (read as rows 8..71, i.e. again rows 0..G-1 of that operand), so two
+    // MMAs add both into O rows 0..G-1; 80 rows x 128 tokens
+    static constexpr int kP = 80 * 128;
     static constexpr int kOffQ = kTcStages * kStage;
     static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
     static constexpr int kOffRed = kOffP + 2 * kP;          // [4 warps][8] floats x 2 (max, sum)
-    static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;  // [2 O buffers][m | l][8] floats
-    static constexpr int kOffSq = kOffStats + 2 * 2 * 8 * 4;   // [kTcQBufs] q scales
-    static constexpr int kOffQtmp = kOffSq + 16 * 4;           // rotated bf16 q [G][128] (stager)
+    static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [2] TcStats
+    static constexpr int kOffMeta = kOffStats + 2 * (int)sizeof(TcStats);   // [kTcQBufs] TcMeta
+    static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
+    static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // rotated bf16 q [G][128]
     static constexpr int kOffBar = kOffQtmp + 8 * 128 * 2;
     static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 15;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
@@ -115,71 +139,54 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
 }
 
 // Decode step: the step's new token of sequence b, kv head kvh -- the newest of its L tokens,
-// row (L-1) % 128 of its last tile, cache slot `slot`.  fetch() loads what it needs (K and V
-// as bf16, the RoPE row, the slot) when the piece starts, so the loads overlap the piece's
-// waits; put() then rotates K at L - 1, quantises both from the fp64 quotient by the head's
-// scale (as pkv_kv_store does) and stores the codes into the cache and into the tile's K
-// and V rows, which TMA filled with the slot's previous codes.  One warp; lane i holds
-// dims i, i + 32, i + 64, i + 96.
-struct TcNewToken {
-    uint16_t k[4], v[4];
-    float c[2], sn[2];
-    int slot;   // -1: nothing to store
-    bool rope;
-};
-
-__device__ __forceinline__ void tc_fetch_new_token(const DecodeParams &p, int b, int kvh, TcNewToken &t, int lane) {
+// cache slot `slot`.  Run by the q stager when it stages a piece that ends the sequence: K
+// rotated at L - 1, both K and V quantised to the E4M3 code of the exact quotient by the
+// head's scale (as pkv_kv_store does), stored into the cache and into `codes` (128 K codes, then 128 V codes),
+// from where the S^T issuer patches the tile that TMA filled with the slot's previous codes.
+// Returns false (nothing stored) when the context was clipped to the block table, the
+// position is outside the RoPE table (bounds flag) or the block entry is outside the pool
+// (the producer flags that one).  One warp; lane i takes dims i, i + 32, i + 64, i + 96.
+__device__ __forceinline__ bool tc_stage_new_token(const DecodeParams &p, int b, int kvh, uint8_t *codes,
+                                                   int lane) {
     constexpr int D = 128;
     const int Lraw = __ldg(p.context_lens + b), L = min(Lraw, p.max_tokens);
-    t.slot = -1;
-    t.rope = p.rope != nullptr;
-    if (L != Lraw || L < 1) return;  // clipped to the block table: the kernel stores nothing
+    if (L != Lraw || L < 1) return false;
     const int pos = L - 1;
     if (p.rope && pos >= p.max_pos) {
         if (lane == 0) atomicOr(p.err, kErrBounds);
-        return;
+        return false;
     }
     const int e = __ldg(p.block_tables + (size_t)b * p.max_blocks + pos / p.bs);
-    if (e < 0 || (long long)e >= p.num_blocks) return;  // (the producer flags a bad entry)
-    t.slot = e * p.bs + pos % p.bs;
+    if (e < 0 || (long long)e >= p.num_blocks) return false;
+    const int slot = e * p.bs + pos % p.bs;
     const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
     const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
+    uint16_t kb[4], vb[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        t.k[j] = __ldg(kin + lane + 32 * j);
-        t.v[j] = __ldg(vin + lane + 32 * j);
+        kb[j] = __ldg(kin + lane + 32 * j);
+        vb[j] = __ldg(vin + lane + 32 * j);
     }
     if (p.rope) {
         const float *row = p.rope + (size_t)pos * D;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {  // the pairs (i, i + 64) for i = lane, lane + 32
-            t.c[j] = __ldg(row + lane + 32 * j);
-            t.sn[j] = __ldg(row + D / 2 + lane + 32 * j);
-        }
+        for (int j = 0; j < 2; ++j)  // the pairs (i, i + 64) for i = lane, lane + 32
+            rope_pair_fast(kb[j], kb[j + 2], __ldg(row + lane + 32 * j), __ldg(row + D / 2 + lane + 32 * j), kb[j],
+                           kb[j + 2]);
     }
-}
-
-__device__ __forceinline__ void tc_put_new_token(const DecodeParams &p, int kvh, int L, const TcNewToken &t,
-                                                 uint32_t kt, uint32_t vt, int lane) {
-    constexpr int D = 128;
-    if (t.slot < 0) return;
-    const int r = (L - 1) % kTcTile;
-    uint16_t kb[4] = {t.k[0], t.k[1], t.k[2], t.k[3]};
-    if (t.rope)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) rope_pair_fast(kb[j], kb[j + 2], t.c[j], t.sn[j], kb[j], kb[j + 2]);
-    const size_t dst = ((size_t)t.slot * p.Hkv + kvh) * D;
-    const double ks = (double)__ldg(p.k_scale + kvh), vs = (double)__ldg(p.v_scale + kvh);
+    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;
+    const float ks = __ldg(p.k_scale + kvh), vs = __ldg(p.v_scale + kvh);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int e = lane + 32 * j;
-        const uint32_t kc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(kb[j]), ks));
-        const uint32_t vc = f64_to_e4m3(__ddiv_rn(bf16_to_f64(t.v[j]), vs));
-        static_cast<uint8_t *>(p.k_cache_w)[dst + e] = (uint8_t)kc;
-        static_cast<uint8_t *>(p.v_cache_w)[dst + e] = (uint8_t)vc;
-        asm volatile("st.shared.u8 [%0], %1;" ::"r"(kt + sw_off(r, e)), "r"(kc) : "memory");
-        asm volatile("st.shared.u8 [%0], %1;" ::"r"(vt + sw_off(r, e)), "r"(vc) : "memory");
+        const int d = lane + 32 * j;
+        const uint8_t kc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)kb[j] << 16), ks);
+        const uint8_t vc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)vb[j] << 16), vs);
+        static_cast<uint8_t *>(p.k_cache_w)[dst + d] = kc;
+        static_cast<uint8_t *>(p.v_cache_w)[dst + d] = vc;
+        codes[d] = kc;
+        codes[D + d] = vc;
     }
+    return true;
 }
 
 template <int G, bool STEP>
@@ -193,8 +200,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t *smem = smem_raw + (sbase - smem_u32(smem_raw));
     const uint32_t sStages = sbase, sQ = sbase + Geo::kOffQ, sP = sbase + Geo::kOffP;
     float *red = reinterpret_cast<float *>(smem + Geo::kOffRed);
-    float *stats = reinterpret_cast<float *>(smem + Geo::kOffStats);  // [O buffer][m | l][8]
-    float *sqbuf = reinterpret_cast<float *>(smem + Geo::kOffSq);     // [q buffer]
+    TcStats *stats = reinterpret_cast<TcStats *>(smem + Geo::kOffStats);  // [O buffer]
+    TcMeta *meta = reinterpret_cast<TcMeta *>(smem + Geo::kOffMeta);      // [q buffer]
+    uint8_t *newcodes = smem + Geo::kOffNew;                               // [q buffer][256]
     uint16_t *qtmp = reinterpret_cast<uint16_t *>(smem + Geo::kOffQtmp);
     const uint32_t bars = sbase + Geo::kOffBar;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Geo::kOffBar + 8 * Geo::kBars);
@@ -292,14 +300,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // TMEM: S^T buffers at columns 0 and 16 (128 lanes x 16), O buffers at columns 128 and 256
     // (rows 0..2G-1 of 64 x 128 each)
 
-    // unit k of this CTA -> (sequence, kv head, tile of the sequence, its tile count)
-    auto unit = [&](int k, int &b, int &kvh, int &tile, int &ntiles) {
-        UnitPos up = locate(pfx, p.B, Hu, u0 + k);
-        b = up.b;
-        kvh = up.kvh;
-        tile = up.blk;
-        ntiles = up.nb;
-    };
     // a bounded wait by lane 0 of the calling warp, its outcome broadcast to the warp (the
     // __syncwarp orders the other lanes' accesses after lane 0's acquire)
     auto wait0 = [&](int bi, uint32_t parity) -> bool {
@@ -380,13 +380,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool ok = true;
         int piece = -1;
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
-        TcNewToken nt;
         for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
             const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
             if (k == 0 || tile == 0) {
                 ++piece;
-                // a piece that ends its sequence stores the step's new token: fetch it now
-                if (STEP && k + (ntiles - 1 - tile) < nunits) tc_fetch_new_token(p, b, kvh, nt, lane);
                 ok = wait0(kBQFull + piece % kTcQBufs, (piece / kTcQBufs) & 1);
             }
             ok = ok && wait0(kBFull + k % kTcStages, (k / kTcStages) & 1) &&
@@ -394,9 +391,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok) break;
             const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
             if constexpr (STEP) {
-                if (tile == ntiles - 1) {  // the sequence's last tile holds its new token
-                    tc_put_new_token(p, kvh, min(__ldg(p.context_lens + b), p.max_tokens), nt, kd, kd + Geo::kKV,
-                                     lane);
+                const int qs = piece % kTcQBufs, r = meta[qs].nt_row;
+                if (tile == ntiles - 1 && r >= 0) {
+                    // the sequence's last tile holds its new token: the stager's codes replace
+                    // the slot's previous contents in the K and V rows
+                    if (lane < 16) {
+                        const int c = 16 * (lane & 7);
+                        const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + qs * 256 + (lane >> 3) * D + c);
+                        const uint32_t dst = kd + (lane >> 3) * Geo::kKV + sw_off(r, c);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(x.x), "r"(x.y),
+                                     "r"(x.z), "r"(x.w) : "memory");
+                    }
                     fence_proxy_async_smem();  // the tensor cores read these rows next
                     __syncwarp();
                 }
@@ -436,9 +441,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint32_t pd = sP + (k & 1) * Geo::kP;
                 const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
 #pragma unroll
-                for (int kk = 0; kk < kTcTile / 32; ++kk)
-                    tc::mma_ss_f8(tO, tc::sw128_desc(pd + 32 * kk, 16, 1024),
-                                  tc::sw128_desc(vd + 4096 * kk, 16384, 1024), idO, (first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < kTcTile / 32; ++kk) {
+                    const uint64_t vdesc = tc::sw128_desc(vd + 4096 * kk, 16384, 1024);
+                    tc::mma_ss_f8(tO, tc::sw128_desc(pd + 32 * kk, 16, 1024), vdesc, idO, (first && kk == 0) ? 0u : 1u);
+                    tc::mma_ss_f8(tO, tc::sw128_desc(pd + 1024 + 32 * kk, 16, 1024), vdesc, idO, 1u);  // low parts
+                }
                 tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
                 tc::mma_commit(bar_at(bars, kBPvDone + (k & 1)));
                 if (last) tc::mma_commit(bar_at(bars, kBOReady + (piece & 1)));
@@ -452,7 +459,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == kTcQWarp) {
         // ---------------------------------------------------------------- q stager
         // For each piece in turn, into q buffer piece % kTcQBufs: the G heads' q rotated at
-        // L - 1, scaled by one power of two for the group (kept in sqbuf) and split into high
+        // L - 1, scaled by one power of two for the group and split into high
         // parts (rows 0..G-1) and low parts (rows G..2G-1) as E4M3 codes.  Runs up to
         // kTcQBufs pieces ahead of the softmax.
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
@@ -499,7 +506,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(h, c)), "r"(hi) : "memory");
                 asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(G + h, c)), "r"(lo) : "memory");
             }
-            if (lane == 0) sqbuf[slot] = sq;
+            int nt_row = -1;
+            if constexpr (STEP) {
+                if (piece_len == cur.nt - cur.tile &&  // the piece ends its sequence
+                    tc_stage_new_token(p, b, kvh, newcodes + slot * 256, lane))
+                    nt_row = (L - 1) % kTcTile;
+            }
+            if (lane == 0) {
+                TcMeta &mt = meta[slot];
+                mt.nt_row = nt_row;
+                mt.b = b;
+                mt.kvh = kvh;
+                mt.tile = cur.tile;
+                mt.ntiles = cur.nt;
+                mt.piece_len = piece_len;
+                mt.L = L;
+                mt.sc = p.scale_log2 * __ldg(p.k_scale + kvh) / sq;
+                mt.vs = __ldg(p.v_scale + kvh);
+            }
             fence_proxy_async_smem();
             __syncwarp();  // (qtmp is rewritten by the next piece)
             if (lane == 0) mbar_arrive(bar_at(bars, kBQFull + slot));
@@ -508,42 +532,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     } else if (warp == kTcEpiWarp) {
         // ---------------------------------------------------------------- epilogue
-        // For each piece in turn, once its last PV has completed and the softmax has left its
-        // (m, l): O (TMEM lanes 0..2G-1 of O buffer piece & 1) -> the output rows (a whole
-        // segment) or the piece's partial slot, then O buffer free.
+        // For each piece in turn, once its last PV has completed and the softmax has left the
+        // piece's description and (m, l): O (TMEM lanes 0..G-1 of O buffer piece & 1) -> the
+        // output rows (a whole segment) or the piece's partial slot, then O buffer free.
         int k = 0;
         for (int piece = 0; k < nunits; ++piece) {
-            int b, kvh, tile, ntiles;
-            unit(k, b, kvh, tile, ntiles);
-            const int piece_len = min(ntiles - tile, nunits - k);
-            const bool whole = tile == 0 && piece_len == ntiles;
             const int ob = piece & 1;
             const bool fin = wait0(kBStats + ob, (piece >> 1) & 1) && wait0(kBOReady + ob, (piece >> 1) & 1);
-            if (!fin && lane == 0) *abort_flag = 1;
+            if (!fin) {
+                if (lane == 0) *abort_flag = 1;
+                break;
+            }
             tc::tc_fence_after();
-            // lanes 0..G-1 hold O rows h (high parts of p), lanes G..2G-1 rows G+h (low parts)
-            const int h = lane < G ? lane : (lane < 2 * G ? lane - G : 0);
-            const float m = stats[ob * 16 + h], l = stats[ob * 16 + 8 + h];
+            const TcStats &st = stats[ob];
+            const int b = st.b, kvh = st.kvh, ntiles = st.ntiles, piece_len = st.piece_len;
+            const bool whole = st.whole != 0;
+            const float vs = st.vs;
+            const int h = lane < G ? lane : 0;  // lanes 0..G-1 hold O rows h
+            const float m = st.m[h], l = st.l[h];
             const int segu = b * Hu + kvh;
             float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
-            const float vs = __ldg(p.v_scale + kvh);
-            const float inv = (l > 0.f && fin) ? vs / l : 0.f;
+            const float inv = l > 0.f ? vs / l : 0.f;
             const uint32_t tO = tmem + kTcO + 128u * (uint32_t)ob;
             __nv_bfloat16 *orow = p.out + ((size_t)b * p.Hq + kvh * G + h) * D;
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t rr[32];
-                if (fin) {
-                    tc::tmem_ld32(tO + c0, rr);
-                    tc::tc_wait_ld();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) rr[e] = 0u;
-                }
+                tc::tmem_ld32(tO + c0, rr);
+                tc::tc_wait_ld();
                 float o[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    o[e] = __uint_as_float(rr[e]) + __shfl_down_sync(0xffffffffu, __uint_as_float(rr[e]), G);
+                for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(rr[e]);
                 if (lane < G) {
                     if (whole) {
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
@@ -603,10 +622,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                 acc.w += f * x.w;
                                 ls += f * __ldcg(sl + G * D + G + g);
                             }
-                            const float r = ls > 0.f ? vs / ls : 0.f;
+                            // (rounded as the combine kernel rounds: o / l * v_scale)
+                            const bool any = ls > 0.f;
                             uint2 w;
-                            w.x = tc::pack_bf16x2(acc.x * r, acc.y * r);
-                            w.y = tc::pack_bf16x2(acc.z * r, acc.w * r);
+                            w.x = tc::pack_bf16x2(any ? acc.x / ls * vs : 0.f, any ? acc.y / ls * vs : 0.f);
+                            w.y = tc::pack_bf16x2(any ? acc.z / ls * vs : 0.f, any ? acc.w / ls * vs : 0.f);
                             *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
                         }
                         if (lane == 0) p.counters[segu] = 0;
@@ -624,22 +644,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int ct = threadIdx.x - 32 * kTcSoftmax0;    // 0..127
         bool alive = true;
         int k = 0;
+        TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
         for (int piece = 0; k < nunits; ++piece) {
-            int b, kvh, tile, ntiles;
-            unit(k, b, kvh, tile, ntiles);
+            const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
             const int piece_len = min(ntiles - tile, nunits - k);
-            const int L = min(__ldg(p.context_lens + b), p.max_tokens);
             const int qslot = piece % kTcQBufs;
             const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
-            // the piece's q scale (and q) from the stager
+            // the piece's context length and scales (and q) from the stager
             const bool qok = alive && !*abort_flag &&
                              mbar_wait_bounded(bar_at(bars, kBQFull + qslot), (piece / kTcQBufs) & 1, p.err);
             if (!__all_sync(0xffffffffu, qok)) {
                 alive = false;
                 *abort_flag = 1;
             }
-            const float sq = alive ? sqbuf[qslot] : 1.f;
-            const float sc = p.scale_log2 * __ldg(p.k_scale + kvh) / sq;
+            const int L = alive ? meta[qslot].L : 1;
+            const float sc = alive ? meta[qslot].sc : 0.f;
+            const float vsc = alive ? meta[qslot].vs : 0.f;
             float mref[G], lsum[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -721,10 +741,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     uint32_t hi, lo;  // (only the first of the four codes is used)
                     tc::split_e4m3x4(pr[h], 0.f, 0.f, 0.f, hi, lo);
                     asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(h, t)), "r"(hi & 0xFFu) : "memory");
-                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(G + h, t)), "r"(lo & 0xFFu) : "memory");
+                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(8 + h, t)), "r"(lo & 0xFFu) : "memory");
                 }
                 if (rescale && alive) {
-                    // O rows h and G+h (TMEM lanes 0..2G-1, warp quad 0) times alpha_h, once the
+                    // O rows h (TMEM lanes 0..G-1, warp quad 0) times alpha_h, once the
                     // PV of the previous tile has finished
                     const int pj = (k - 1) & 1;
                     if (!mbar_wait_bounded(bar_at(bars, kBPvDone + pj), ((k - 1) >> 1) & 1, p.err)) {
@@ -736,7 +756,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         float a = 1.f;
 #pragma unroll
                         for (int h = 0; h < G; ++h)
-                            if (lane == h || lane == G + h) a = alpha[h];
+                            if (lane == h) a = alpha[h];
 #pragma unroll 1
                         for (int c0 = 0; c0 < D; c0 += 32) {
                             uint32_t rr[32];
@@ -771,17 +791,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     alive = false;
                     *abort_flag = 1;
                 }
+                TcStats &st = stats[piece & 1];
                 if (lane < G) {
                     float m = -INFINITY;
 #pragma unroll
                     for (int hh = 0; hh < G; ++hh)
                         if (hh == lane) m = mref[hh];
-                    stats[(piece & 1) * 16 + lane] = m;
-                    stats[(piece & 1) * 16 + 8 + lane] = red[32 + lane] + red[40 + lane] + red[48 + lane] + red[56 + lane];
+                    st.m[lane] = m;
+                    st.l[lane] = red[32 + lane] + red[40 + lane] + red[48 + lane] + red[56 + lane];
+                }
+                if (lane == 0) {
+                    st.b = b;
+                    st.kvh = kvh;
+                    st.ntiles = ntiles;
+                    st.whole = tile == 0 && piece_len == ntiles;
+                    st.piece_len = piece_len;
+                    st.vs = vsc;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_at(bars, kBStats + (piece & 1)));
             }
+            for (int j = 0; j < piece_len; ++j) tc_next(cur, pfx, p.B, Hu);
         }
     }
 

@@ -37,14 +37,15 @@ __device__ __forceinline__ void rotate_chunk(Chunk &x, const float *cos_row, con
     x.hi = *reinterpret_cast<uint4 *>(rb);
 }
 
-// Quantise 8 bf16 values (one 16-byte chunk) to 8 E4M3 codes with scale s.
-__device__ __forceinline__ uint2 quantize_chunk(uint4 v, double s) {
+// Quantise 8 bf16 values (one 16-byte chunk) to 8 E4M3 codes with scale s: each the code of
+// the exact quotient (e4m3_of_quotient).
+__device__ __forceinline__ uint2 quantize_chunk(uint4 v, float s) {
     const uint16_t *e = reinterpret_cast<const uint16_t *>(&v);
     uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) lo |= f64_to_e4m3(__ddiv_rn(bf16_to_f64(e[i]), s)) << (8 * i);
+    for (int i = 0; i < 4; ++i) lo |= e4m3_of_quotient(__uint_as_float((uint32_t)e[i] << 16), s) << (8 * i);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) hi |= f64_to_e4m3(__ddiv_rn(bf16_to_f64(e[4 + i]), s)) << (8 * i);
+    for (int i = 0; i < 4; ++i) hi |= e4m3_of_quotient(__uint_as_float((uint32_t)e[4 + i] << 16), s) << (8 * i);
     return make_uint2(lo, hi);
 }
 
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(256) kv_store_kernel(StoreArgs a) {
         }
         const size_t dst = ((size_t)slot * H + h) * D;
         if (FP8) {
-            const double ksc = (double)__ldg(a.k_scale + h), vsc = (double)__ldg(a.v_scale + h);
+            const float ksc = __ldg(a.k_scale + h), vsc = __ldg(a.v_scale + h);
             uint2 *kd = reinterpret_cast<uint2 *>(static_cast<uint8_t *>(a.k_cache) + dst);
             uint2 *vd = reinterpret_cast<uint2 *>(static_cast<uint8_t *>(a.v_cache) + dst);
             kd[c] = quantize_chunk(kx.lo, ksc);

@@ -311,3 +311,34 @@ def test_bounded_wait_times_out_and_context_survives():
     assert pkv.get_error() == 0                       # cleared
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum()) == 8.0
+
+
+@pytest.mark.parametrize("scales", [(1.0, 0.0625), (0.3, 3.0), (1e-3, 7.0), (448.0, 2.0 ** -9)])
+def test_kv_store_e4m3_every_bf16_value(scales):
+    """The E4M3 quantiser of kv_store on every bf16 bit pattern (NaN included), for two heads
+    with their own scales: code for code as the oracle's (fp64 quotient, round to nearest
+    even, saturate).  Scales that are powers of two put many quotients exactly on rounding
+    midpoints, where the product's fp32 shortcut has to take the exact decision."""
+    H, D = 2, 128
+    vals = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    T = 65536 // (H * D) * 2                   # every pattern once per head
+    k = np.concatenate([vals, vals]).reshape(T, H, D)
+    v = k[::-1].copy()
+    bs = 16
+    NB = T // bs
+    slots = np.arange(T, dtype=np.int32)
+    ks = np.array(scales, dtype=np.float32)
+    vs = ks[::-1].copy()
+    kc = np.zeros((NB, bs, H, D), dtype=np.uint8)
+    vc = np.zeros_like(kc)
+    oracle.kv_store(k, v, kc, vc, slots, bs, fp8=True, k_scale=ks, v_scale=vs)
+    dk = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).cuda()
+    dv = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda()
+    gk = torch.zeros((NB, bs, H, D), dtype=torch.uint8, device="cuda")
+    gv = torch.zeros_like(gk)
+    pkv.kv_store(dk, dv, gk, gv, torch.from_numpy(slots).cuda(), k_scale=torch.from_numpy(ks).cuda(),
+                 v_scale=torch.from_numpy(vs).cuda())
+    torch.cuda.synchronize()
+    _assert_no_device_error()
+    assert np.array_equal(gk.cpu().numpy(), kc)
+    assert np.array_equal(gv.cpu().numpy(), vc)
