@@ -16,8 +16,9 @@
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
 //   warp 6      lane 0 issues the PV MMAs
-//   warp 7      q stager: each piece's q (rotated, scaled, split), its context length and
-//               scales, up to 4 pieces ahead
+//   warps 7, 9  q stagers (even / odd pieces): each piece's q (rotated, scaled, split), its
+//               context length and scales, and (decode step) its new token, up to 4 pieces
+//               ahead
 //   warp 8      epilogue: O of a finished piece -> output rows or a partial slot
 // Per tile:
 //   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
@@ -43,9 +44,10 @@
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 288;
+constexpr int kTcThreads = 320;
 constexpr int kTcPvWarp = 6;    // the PV issuer
-constexpr int kTcQWarp = 7;     // the q stager
+constexpr int kTcQWarp = 7;     // q stager of the even pieces
+constexpr int kTcQWarp2 = 9;    // q stager of the odd pieces
 constexpr int kTcEpiWarp = 8;   // the epilogue (warp 8: TMEM lanes 0-31, where O's rows live)
 constexpr int kTcTile = 128;    // tokens per unit
 constexpr int kTcStages = 5;
@@ -86,8 +88,8 @@ struct TcGeo {
     static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [2] TcStats
     static constexpr int kOffMeta = kOffStats + 2 * (int)sizeof(TcStats);   // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
-    static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // rotated bf16 q [G][128]
-    static constexpr int kOffBar = kOffQtmp + 8 * 128 * 2;
+    static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [2 stagers] rotated bf16 q [8][128]
+    static constexpr int kOffBar = kOffQtmp + 2 * 8 * 128 * 2;
     static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 15;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
@@ -136,57 +138,6 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
         ++c.b;
         c.nt = c.b < B ? pfx[c.b + 1] - pfx[c.b] : 1;
     } while (c.b < B && c.nt == 0);
-}
-
-// Decode step: the step's new token of sequence b, kv head kvh -- the newest of its L tokens,
-// cache slot `slot`.  Run by the q stager when it stages a piece that ends the sequence: K
-// rotated at L - 1, both K and V quantised to the E4M3 code of the exact quotient by the
-// head's scale (as pkv_kv_store does), stored into the cache and into `codes` (128 K codes, then 128 V codes),
-// from where the S^T issuer patches the tile that TMA filled with the slot's previous codes.
-// Returns false (nothing stored) when the context was clipped to the block table, the
-// position is outside the RoPE table (bounds flag) or the block entry is outside the pool
-// (the producer flags that one).  One warp; lane i takes dims i, i + 32, i + 64, i + 96.
-__device__ __forceinline__ bool tc_stage_new_token(const DecodeParams &p, int b, int kvh, uint8_t *codes,
-                                                   int lane) {
-    constexpr int D = 128;
-    const int Lraw = __ldg(p.context_lens + b), L = min(Lraw, p.max_tokens);
-    if (L != Lraw || L < 1) return false;
-    const int pos = L - 1;
-    if (p.rope && pos >= p.max_pos) {
-        if (lane == 0) atomicOr(p.err, kErrBounds);
-        return false;
-    }
-    const int e = __ldg(p.block_tables + (size_t)b * p.max_blocks + pos / p.bs);
-    if (e < 0 || (long long)e >= p.num_blocks) return false;
-    const int slot = e * p.bs + pos % p.bs;
-    const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
-    const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
-    uint16_t kb[4], vb[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        kb[j] = __ldg(kin + lane + 32 * j);
-        vb[j] = __ldg(vin + lane + 32 * j);
-    }
-    if (p.rope) {
-        const float *row = p.rope + (size_t)pos * D;
-#pragma unroll
-        for (int j = 0; j < 2; ++j)  // the pairs (i, i + 64) for i = lane, lane + 32
-            rope_pair_fast(kb[j], kb[j + 2], __ldg(row + lane + 32 * j), __ldg(row + D / 2 + lane + 32 * j), kb[j],
-                           kb[j + 2]);
-    }
-    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;
-    const float ks = __ldg(p.k_scale + kvh), vs = __ldg(p.v_scale + kvh);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int d = lane + 32 * j;
-        const uint8_t kc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)kb[j] << 16), ks);
-        const uint8_t vc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)vb[j] << 16), vs);
-        static_cast<uint8_t *>(p.k_cache_w)[dst + d] = kc;
-        static_cast<uint8_t *>(p.v_cache_w)[dst + d] = vc;
-        codes[d] = kc;
-        codes[D + d] = vc;
-    }
-    return true;
 }
 
 template <int G, bool STEP>
@@ -381,7 +332,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int piece = -1;
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
         for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
-            const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
+            const int tile = cur.tile, ntiles = cur.nt;
             if (k == 0 || tile == 0) {
                 ++piece;
                 ok = wait0(kBQFull + piece % kTcQBufs, (piece / kTcQBufs) & 1);
@@ -456,77 +407,161 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait_bounded(bar_at(bars, kBDrain), 0, p.err);
         }
         __syncwarp();
-    } else if (warp == kTcQWarp) {
-        // ---------------------------------------------------------------- q stager
-        // For each piece in turn, into q buffer piece % kTcQBufs: the G heads' q rotated at
-        // L - 1, scaled by one power of two for the group and split into high
-        // parts (rows 0..G-1) and low parts (rows G..2G-1) as E4M3 codes.  Runs up to
-        // kTcQBufs pieces ahead of the softmax.
+    } else if (warp == kTcQWarp || warp == kTcQWarp2) {
+        // ---------------------------------------------------------------- q stagers
+        // Two warps take the pieces in turn (even / odd), each into q buffer piece % kTcQBufs:
+        // the G heads' q rotated at L - 1, scaled by one power of two for the group and split
+        // into high parts (rows 0..G-1) and low parts (rows G..2G-1) as E4M3 codes, plus the
+        // piece's description, and (decode step) the new token of a piece that ends its
+        // sequence.  All loads of a piece go out in one round (the RoPE row serves q and the
+        // new K alike: both rotate at L - 1); the next piece's context length is fetched
+        // while this one is staged.  Run up to kTcQBufs pieces ahead of the softmax.
+        constexpr int D2 = D / 2;
+        const int par = warp == kTcQWarp ? 0 : 1;
+        uint16_t *qt = qtmp + par * (8 * D);
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
         int k = 0;
+        // context length of the next piece this warp stages
+        auto next_own = [&](TcCursor c, int kk, int pc) -> int {  // (by value: a look-ahead)
+            while (kk < nunits && (pc & 1) != par) {
+                const int pl = min(c.nt - c.tile, nunits - kk);
+                kk += pl;
+                for (int t = 0; t < pl; ++t) tc_next(c, pfx, p.B, Hu);
+                ++pc;
+            }
+            return kk < nunits ? __ldg(p.context_lens + c.b) : 0;
+        };
+        int Lraw = next_own(cur, 0, 0);
         for (int pc = 0; k < nunits; ++pc) {
             const int b = cur.b, kvh = cur.kvh;
             const int piece_len = min(cur.nt - cur.tile, nunits - k);
-            const int slot = pc % kTcQBufs;
-            if (!wait0(kBQEmpty + slot, ((pc / kTcQBufs) & 1) ^ 1)) {
-                if (lane == 0) *abort_flag = 1;
-                break;
-            }
-            const int L = min(__ldg(p.context_lens + b), p.max_tokens);
-            const int pos = L - 1;
-            const bool rope_ok = p.rope && pos >= 0 && pos < p.max_pos;
-            if (p.rope && !rope_ok && lane == 0) atomicOr(p.err, kErrBounds);
-            float amax = 0.f;
-#pragma unroll 4
-            for (int e = lane; e < G * (D / 2); e += 32) {
-                const int h = e / (D / 2), i = e % (D / 2);
-                const uint16_t *qr = p.q + ((size_t)b * p.Hq + kvh * G + h) * D;
-                uint16_t x1 = __ldg(qr + i), x2 = __ldg(qr + i + D / 2);
-                if (rope_ok) {
-                    const float *row = p.rope + (size_t)pos * D;
-                    rope_pair_fast(x1, x2, __ldg(row + i), __ldg(row + D / 2 + i), x1, x2);
-                }
-                qtmp[h * D + i] = x1;
-                qtmp[h * D + i + D / 2] = x2;
-                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float((uint32_t)x1 << 16)),
-                                         fabsf(__uint_as_float((uint32_t)x2 << 16))));
-            }
+            const bool ends = piece_len == cur.nt - cur.tile;  // the piece ends its sequence
+            if ((pc & 1) == par) {
+                const int slot = pc % kTcQBufs;
+                const int L = min(Lraw, p.max_tokens), pos = L - 1;
+                const bool rope_ok = p.rope && pos >= 0 && pos < p.max_pos;
+                if (p.rope && !rope_ok && lane == 0) atomicOr(p.err, kErrBounds);
+                // ---- one round of loads: q pairs (i, i + 64) for i = lane, lane + 32 of every
+                // head, their RoPE factors, the new token's K and V and its block entry
+                uint16_t qx[G][2][2];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const float sq = amax > 0.f
-                                 ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
-                                 : 1.f;
-            __syncwarp();  // qtmp complete
-            const uint32_t qd = sQ + slot * Geo::kQ;
-            for (int e = lane; e < G * (D / 4); e += 32) {  // four dims per lane and step
-                const int h = e / (D / 4), c = 4 * (e % (D / 4));
-                const uint2 w = *reinterpret_cast<const uint2 *>(qtmp + h * D + c);
-                uint32_t hi, lo;
-                tc::split_e4m3x4(bf16lo(w.x) * sq, bf16hi(w.x) * sq, bf16lo(w.y) * sq, bf16hi(w.y) * sq, hi, lo);
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(h, c)), "r"(hi) : "memory");
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(G + h, c)), "r"(lo) : "memory");
+                for (int h = 0; h < G; ++h)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const uint16_t *qr = p.q + ((size_t)b * p.Hq + kvh * G + h) * D + lane + 32 * j;
+                        qx[h][j][0] = __ldg(qr);
+                        qx[h][j][1] = __ldg(qr + D2);
+                    }
+                float rc[2] = {1.f, 1.f}, rs[2] = {0.f, 0.f};
+                if (rope_ok)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        rc[j] = __ldg(p.rope + (size_t)pos * D + lane + 32 * j);
+                        rs[j] = __ldg(p.rope + (size_t)pos * D + D2 + lane + 32 * j);
+                    }
+                bool nt_go = false;
+                int nt_e = -1;
+                uint16_t nk[2][2], nv[2][2];
+                if constexpr (STEP) {
+                    // (nothing is stored when the context was clipped to the block table or the
+                    // position is outside the RoPE table; a bad block entry is the producer's to flag)
+                    nt_go = ends && L == Lraw && L >= 1 && (!p.rope || rope_ok);
+                    if (nt_go) {
+                        nt_e = __ldg(p.block_tables + (size_t)b * p.max_blocks + pos / p.bs);
+                        const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
+                        const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            nk[j][0] = __ldg(kin + lane + 32 * j);
+                            nk[j][1] = __ldg(kin + lane + 32 * j + D2);
+                            nv[j][0] = __ldg(vin + lane + 32 * j);
+                            nv[j][1] = __ldg(vin + lane + 32 * j + D2);
+                        }
+                    }
+                }
+                const float ksc = __ldg(p.k_scale + kvh), vsc = __ldg(p.v_scale + kvh);
+                // the following piece's context length, while this one is computed
+                TcCursor nc = cur;
+                for (int t = 0; t < piece_len; ++t) tc_next(nc, pfx, p.B, Hu);
+                const int Lnext = next_own(nc, k + piece_len, pc + 1);
+                // ---- the slot must be free before it is written
+                if (!wait0(kBQEmpty + slot, ((pc / kTcQBufs) & 1) ^ 1)) {
+                    if (lane == 0) *abort_flag = 1;
+                    break;
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        uint16_t x1 = qx[h][j][0], x2 = qx[h][j][1];
+                        if (rope_ok) rope_pair_fast(x1, x2, rc[j], rs[j], x1, x2);
+                        qt[h * D + lane + 32 * j] = x1;
+                        qt[h * D + lane + 32 * j + D2] = x2;
+                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float((uint32_t)x1 << 16)),
+                                                 fabsf(__uint_as_float((uint32_t)x2 << 16))));
+                    }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                const float sq = amax > 0.f
+                                     ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
+                                     : 1.f;
+                __syncwarp();  // qt complete
+                const uint32_t qd = sQ + slot * Geo::kQ;
+                for (int e = lane; e < G * (D / 4); e += 32) {  // four dims per lane and step
+                    const int h = e / (D / 4), c = 4 * (e % (D / 4));
+                    const uint2 w = *reinterpret_cast<const uint2 *>(qt + h * D + c);
+                    uint32_t hi, lo;
+                    tc::split_e4m3x4(bf16lo(w.x) * sq, bf16hi(w.x) * sq, bf16lo(w.y) * sq, bf16hi(w.y) * sq, hi,
+                                     lo);
+                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(h, c)), "r"(hi) : "memory");
+                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(G + h, c)), "r"(lo) : "memory");
+                }
+                int nt_row = -1;
+                if constexpr (STEP) {
+                    if (nt_go && nt_e >= 0 && (long long)nt_e < p.num_blocks) {
+                        // K rotated at L - 1, both quantised to the E4M3 code of the exact
+                        // quotient by the head's scale (as pkv_kv_store does), into the cache
+                        // and into the slot's codes (128 K, then 128 V)
+                        const size_t dst = ((size_t)(nt_e * p.bs + pos % p.bs) * p.Hkv + kvh) * D;
+                        uint8_t *codes = newcodes + slot * 256;
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            uint16_t k1 = nk[j][0], k2 = nk[j][1];
+                            if (p.rope) rope_pair_fast(k1, k2, rc[j], rs[j], k1, k2);
+                            const uint16_t kb[2] = {k1, k2};
+#pragma unroll
+                            for (int hf = 0; hf < 2; ++hf) {
+                                const int d = lane + 32 * j + hf * D2;
+                                const uint8_t kc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)kb[hf] << 16), ksc);
+                                const uint8_t vc =
+                                    (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)nv[j][hf] << 16), vsc);
+                                static_cast<uint8_t *>(p.k_cache_w)[dst + d] = kc;
+                                static_cast<uint8_t *>(p.v_cache_w)[dst + d] = vc;
+                                codes[d] = kc;
+                                codes[D + d] = vc;
+                            }
+                        }
+                        nt_row = pos % kTcTile;
+                    }
+                }
+                if (lane == 0) {
+                    TcMeta &mt = meta[slot];
+                    mt.nt_row = nt_row;
+                    mt.b = b;
+                    mt.kvh = kvh;
+                    mt.tile = cur.tile;
+                    mt.ntiles = cur.nt;
+                    mt.piece_len = piece_len;
+                    mt.L = L;
+                    mt.sc = p.scale_log2 * ksc / sq;
+                    mt.vs = vsc;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();  // (qt is rewritten by this warp's next piece)
+                if (lane == 0) mbar_arrive(bar_at(bars, kBQFull + slot));
+                Lraw = Lnext;
             }
-            int nt_row = -1;
-            if constexpr (STEP) {
-                if (piece_len == cur.nt - cur.tile &&  // the piece ends its sequence
-                    tc_stage_new_token(p, b, kvh, newcodes + slot * 256, lane))
-                    nt_row = (L - 1) % kTcTile;
-            }
-            if (lane == 0) {
-                TcMeta &mt = meta[slot];
-                mt.nt_row = nt_row;
-                mt.b = b;
-                mt.kvh = kvh;
-                mt.tile = cur.tile;
-                mt.ntiles = cur.nt;
-                mt.piece_len = piece_len;
-                mt.L = L;
-                mt.sc = p.scale_log2 * __ldg(p.k_scale + kvh) / sq;
-                mt.vs = __ldg(p.v_scale + kvh);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();  // (qtmp is rewritten by the next piece)
-            if (lane == 0) mbar_arrive(bar_at(bars, kBQFull + slot));
             k += piece_len;
             for (int t = 0; t < piece_len; ++t) tc_next(cur, pfx, p.B, Hu);
         }
