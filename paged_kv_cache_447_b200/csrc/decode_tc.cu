@@ -36,7 +36,7 @@
 // landed, S buffer free, the piece's q staged; PV: P written, O buffer free), so a stage goes
 // back to the producer as soon as its PV completes, and S^T of later tiles runs ahead.  They
 // touch disjoint TMEM columns and shared memory.  S and P are double-buffered, q has 4
-// buffers and O two (by piece), so neither the next piece's q nor the last piece's epilogue
+// buffers and O three (by piece), so neither the next piece's q nor the last pieces' epilogues
 // holds up the tiles.
 #include "decode_kernel.cuh"
 #include "tcgen05.cuh"
@@ -54,7 +54,8 @@ constexpr int kTcStages = 5;
 constexpr int kTcQBufs = 4;     // q buffers: the stager runs up to this many pieces ahead
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
-constexpr uint32_t kTcO = 128;  // TMEM column of O buffer 0 (buffer 1 follows at +128)
+constexpr uint32_t kTcO = 128;  // TMEM column of O buffer 0 (buffers 1, 2 follow at +128, +256)
+constexpr int kTcOBufs = 3;     // O buffers (and stats slots): the epilogue may lag two pieces
 
 // What the q stager knows of a piece, for the softmax warps.
 struct TcMeta {
@@ -86,11 +87,11 @@ struct TcGeo {
     static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
     static constexpr int kOffRed = kOffP + 2 * kP;          // [4 warps][8] floats x 2 (max, sum)
     static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [2] TcStats
-    static constexpr int kOffMeta = kOffStats + 2 * (int)sizeof(TcStats);   // [kTcQBufs] TcMeta
+    static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
     static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [2 stagers] rotated bf16 q [8][128]
     static constexpr int kOffBar = kOffQtmp + 2 * 8 * 128 * 2;
-    static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 15;
+    static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 18;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
     static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
@@ -105,11 +106,11 @@ constexpr int kBPFull = kBSFree + 2;        // [2] P tile written (128 arrivals)
 constexpr int kBPvDone = kBPFull + 2;       // [2] PV done reading P buffer (commit)
 constexpr int kBQFull = kBPvDone + 2;       // [kTcQBufs] q staged (stager)
 constexpr int kBQEmpty = kBQFull + kTcQBufs;  // [kTcQBufs] q buffer read by its S^T MMAs (softmax)
-constexpr int kBOReady = kBQEmpty + kTcQBufs;  // [2] the piece's last PV has completed (commit)
-constexpr int kBStats = kBOReady + 2;       // [2] the piece's (m, l) written (softmax)
-constexpr int kBOFree = kBStats + 2;        // [2] O buffer and stats read by the epilogue (32 arrivals)
-constexpr int kBDrain = kBOFree + 2;        // every MMA of the CTA has completed (2 commits)
-static_assert(kBDrain < 2 * kTcStages + 2 * kTcQBufs + 15, "barrier count");
+constexpr int kBOReady = kBQEmpty + kTcQBufs;  // [kTcOBufs] the piece's last PV has completed (commit)
+constexpr int kBStats = kBOReady + kTcOBufs;   // [kTcOBufs] the piece's (m, l) written (softmax)
+constexpr int kBOFree = kBStats + kTcOBufs;    // [kTcOBufs] O buffer and stats read by the epilogue (32 arrivals)
+constexpr int kBDrain = kBOFree + kTcOBufs;    // every MMA of the CTA has completed (2 commits)
+static_assert(kBDrain < 2 * kTcStages + 2 * kTcQBufs + 18, "barrier count");
 
 __device__ __forceinline__ uint32_t bar_at(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
 
@@ -223,6 +224,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar_at(bars, kBSFree + i), 128);
             mbar_init(bar_at(bars, kBPFull + i), 128);
             mbar_init(bar_at(bars, kBPvDone + i), 1);
+        }
+        for (int i = 0; i < kTcOBufs; ++i) {
             mbar_init(bar_at(bars, kBOReady + i), 1);
             mbar_init(bar_at(bars, kBStats + i), 1);
             mbar_init(bar_at(bars, kBOFree + i), 32);
@@ -248,8 +251,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM: S^T buffers at columns 0 and 16 (128 lanes x 16), O buffers at columns 128 and 256
-    // (rows 0..2G-1 of 64 x 128 each)
+    // TMEM: S^T buffers at columns 0 and 16 (128 lanes x 16), O buffers at columns 128, 256
+    // and 384 (rows 0..G-1 of 64 x 128 each)
 
     // a bounded wait by lane 0 of the calling warp, its outcome broadcast to the warp (the
     // __syncwarp orders the other lanes' accesses after lane 0's acquire)
@@ -277,24 +280,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int half = two ? (bx & 1) : 0, bpiece = two ? (bx >> 1) : bx;
         const uint32_t box_off = (uint32_t)(bpiece * 2048 + half * 1024);
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0 + min(bt, nunits - 1));  // this lane's tile
+        // Loads of this lane's block-table entry and context length for the tile k0 + bt;
+        // they are issued one batch ahead, so their latency hides behind the waits and
+        // copies of the batch before.  (The entry is read only where it lies inside the
+        // table row; whether the box holds tokens is decided once L is known.)
+        auto fetch = [&](int k0, int &e, int &L) {
+            e = -1;
+            L = 0;
+            if (k0 + bt < nunits) {
+                const int pc = cur.tile * 8 + bpiece;  // 16-token piece of the sequence
+                const int idx = p.bs == 16 ? pc : (p.bs == 32 ? (pc >> 1) : 2 * pc + half);
+                if (idx < p.max_blocks) e = __ldg(p.block_tables + (size_t)cur.b * p.max_blocks + idx);
+                L = __ldg(p.context_lens + cur.b);
+            }
+        };
+        auto row_of = [&](int e, int L) -> int {
+            L = min(L, p.max_tokens);
+            const int pc = cur.tile * 8 + bpiece;
+            const bool inside = p.bs == 8 ? (2 * pc + half) * 8 < L : pc * 16 < L;
+            return inside ? cache_row(p, e, p.bs == 32 ? (pc & 1) * 16 : 0) : oob;
+        };
+        int e_cur, L_cur;
+        fetch(0, e_cur, L_cur);
         uint32_t issued = 0, phases = 0;
         bool ok = true;
         for (int k0 = 0; k0 < nunits && ok; k0 += tpb) {
-            int row = oob;
-            if (k0 + bt < nunits) {
-                const int L = min(__ldg(p.context_lens + cur.b), p.max_tokens);
-                const int pc = cur.tile * 8 + bpiece;  // 16-token piece of the sequence
-                const int32_t *tab = p.block_tables + (size_t)cur.b * p.max_blocks;
-                if (p.bs == 16) {
-                    if (pc * 16 < L) row = cache_row(p, __ldg(tab + pc), 0);
-                } else if (p.bs == 32) {
-                    if (pc * 16 < L) row = cache_row(p, __ldg(tab + (pc >> 1)), (pc & 1) * 16);
-                } else {
-                    const int e = 2 * pc + half;
-                    if (e * 8 < L) row = cache_row(p, __ldg(tab + e), 0);
-                }
-            }
+            const int row = k0 + bt < nunits ? row_of(e_cur, L_cur) : oob;
             const int kvh = cur.kvh;
+            // this lane's tile of the next batch, and its loads
+            for (int t = 0; t < tpb; ++t) tc_next(cur, pfx, p.B, Hu);
+            fetch(k0 + tpb, e_cur, L_cur);
             for (int t = 0; t < tpb && k0 + t < nunits; ++t) {
                 const int k = k0 + t, s = k % kTcStages;
                 const uint32_t fb = bar_at(bars, kBFull + s);
@@ -317,8 +332,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tma_load_3d(dk + Geo::kKV + box_off, &tm_v, fb, 0, kvh, row);
                 }
             }
-            // this lane's tile of the next batch
-            for (int t = 0; t < tpb; ++t) tc_next(cur, pfx, p.B, Hu);
         }
         if (lane == 0)  // never leave with a TMA copy landing in shared memory
             for (int s = 0; s < kTcStages; ++s)
@@ -381,16 +394,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const bool first = k == 0 || cur.tile == 0;
                 const bool last = k == nunits - 1 || cur.tile == cur.nt - 1;
                 if (first) ++piece;
-                // a piece's first PV overwrites its O buffer: the epilogue of piece - 2 must
-                // have read it
+                // a piece's first PV overwrites its O buffer: the epilogue of piece - kTcOBufs
+                // must have read it
                 ok = !*abort_flag && mbar_wait_bounded(bar_at(bars, kBPFull + (k & 1)), (k >> 1) & 1, p.err) &&
-                     (!first || piece < 2 ||
-                      mbar_wait_bounded(bar_at(bars, kBOFree + (piece & 1)), ((piece >> 1) - 1) & 1, p.err));
+                     (!first || piece < kTcOBufs ||
+                      mbar_wait_bounded(bar_at(bars, kBOFree + piece % kTcOBufs), (piece / kTcOBufs - 1) & 1, p.err));
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint32_t vd = sStages + (k % kTcStages) * Geo::kStage + Geo::kKV;
                 const uint32_t pd = sP + (k & 1) * Geo::kP;
-                const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
+                const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece % kTcOBufs);
 #pragma unroll
                 for (int kk = 0; kk < kTcTile / 32; ++kk) {
                     const uint64_t vdesc = tc::sw128_desc(vd + 4096 * kk, 16384, 1024);
@@ -399,7 +412,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
                 tc::mma_commit(bar_at(bars, kBPvDone + (k & 1)));
-                if (last) tc::mma_commit(bar_at(bars, kBOReady + (piece & 1)));
+                if (last) tc::mma_commit(bar_at(bars, kBOReady + piece % kTcOBufs));
             }
             if (!ok) *abort_flag = 1;
             // drain: no MMA of either issuer may still write TMEM when it is released
@@ -568,12 +581,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == kTcEpiWarp) {
         // ---------------------------------------------------------------- epilogue
         // For each piece in turn, once its last PV has completed and the softmax has left the
-        // piece's description and (m, l): O (TMEM lanes 0..G-1 of O buffer piece & 1) -> the
+        // piece's description and (m, l): O (TMEM lanes 0..G-1 of its O buffer) -> the
         // output rows (a whole segment) or the piece's partial slot, then O buffer free.
         int k = 0;
         for (int piece = 0; k < nunits; ++piece) {
-            const int ob = piece & 1;
-            const bool fin = wait0(kBStats + ob, (piece >> 1) & 1) && wait0(kBOReady + ob, (piece >> 1) & 1);
+            const int ob = piece % kTcOBufs, ph = (piece / kTcOBufs) & 1;
+            const bool fin = wait0(kBStats + ob, ph) && wait0(kBOReady + ob, ph);
             if (!fin) {
                 if (lane == 0) *abort_flag = 1;
                 break;
@@ -590,33 +603,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float inv = l > 0.f ? vs / l : 0.f;
             const uint32_t tO = tmem + kTcO + 128u * (uint32_t)ob;
             __nv_bfloat16 *orow = p.out + ((size_t)b * p.Hq + kvh * G + h) * D;
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t rr[32];
-                tc::tmem_ld32(tO + c0, rr);
-                tc::tc_wait_ld();
-                float o[32];
+            // 32 columns of the row, scaled and stored (lanes 0..G-1)
+            auto put = [&](int c0, const uint32_t (&rr)[32]) {
+                if (lane >= G) return;
+                if (whole) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(rr[e]);
-                if (lane < G) {
-                    if (whole) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint4 w;
-                            w.x = tc::pack_bf16x2(o[8 * v + 0] * inv, o[8 * v + 1] * inv);
-                            w.y = tc::pack_bf16x2(o[8 * v + 2] * inv, o[8 * v + 3] * inv);
-                            w.z = tc::pack_bf16x2(o[8 * v + 4] * inv, o[8 * v + 5] * inv);
-                            w.w = tc::pack_bf16x2(o[8 * v + 6] * inv, o[8 * v + 7] * inv);
-                            dst[v] = w;
-                        }
-                    } else {
-                        float4 *dst = reinterpret_cast<float4 *>(slot + h * D + c0);
-#pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+                    for (int v = 0; v < 4; ++v) {
+                        uint4 w;
+                        w.x = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv, __uint_as_float(rr[8 * v + 1]) * inv);
+                        w.y = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv, __uint_as_float(rr[8 * v + 3]) * inv);
+                        w.z = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv, __uint_as_float(rr[8 * v + 5]) * inv);
+                        w.w = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv, __uint_as_float(rr[8 * v + 7]) * inv);
+                        dst[v] = w;
                     }
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(slot + h * D + c0);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
+                                             __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
                 }
+            };
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 64) {  // two loads per wait
+                uint32_t ra[32], rb[32];
+                tc::tmem_ld32(tO + c0, ra);
+                tc::tmem_ld32(tO + c0 + 32, rb);
+                tc::tc_wait_ld();
+                put(c0, ra);
+                put(c0 + 32, rb);
             }
             if (!whole && lane < G) {
                 slot[G * D + lane] = m;
@@ -684,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
             const int piece_len = min(ntiles - tile, nunits - k);
             const int qslot = piece % kTcQBufs;
-            const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece & 1);
+            const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece % kTcOBufs);
             // the piece's context length and scales (and q) from the stager
             const bool qok = alive && !*abort_flag &&
                              mbar_wait_bounded(bar_at(bars, kBQFull + qslot), (piece / kTcQBufs) & 1, p.err);
@@ -820,13 +836,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             named_bar(kTcBar, 128);
             if (quad == 0) {
-                // stats buffer piece & 1 was last read by the epilogue of piece - 2
-                bool ok = alive && (piece < 2 || wait0(kBOFree + (piece & 1), ((piece >> 1) - 1) & 1));
+                // the stats slot was last read by the epilogue of piece - kTcOBufs
+                bool ok = alive && (piece < kTcOBufs ||
+                                    wait0(kBOFree + piece % kTcOBufs, (piece / kTcOBufs - 1) & 1));
                 if (!__all_sync(0xffffffffu, ok)) {
                     alive = false;
                     *abort_flag = 1;
                 }
-                TcStats &st = stats[piece & 1];
+                TcStats &st = stats[piece % kTcOBufs];
                 if (lane < G) {
                     float m = -INFINITY;
 #pragma unroll
@@ -844,7 +861,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     st.vs = vsc;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_at(bars, kBStats + (piece & 1)));
+                if (lane == 0) mbar_arrive(bar_at(bars, kBStats + piece % kTcOBufs));
             }
             for (int j = 0; j < piece_len; ++j) tc_next(cur, pfx, p.B, Hu);
         }
