@@ -94,8 +94,13 @@ __device__ __forceinline__ uint32_t f64_to_e4m3(double x) {
 // other midpoint.  (The fp64 quotient of a bf16 by an fp32 value is never rounded onto a
 // midpoint either: that would need a quotient within 2^-53 of one, while a bf16 x differs
 // from m * s, when not equal, by at least 2^-29 of it.)
+// (out of line: a rare path whose fp64 code would crowd the callers' instruction cache)
+static __device__ __noinline__ uint32_t e4m3_of_quotient_f64(float x, float s) {
+    return f64_to_e4m3((double)x / (double)s);
+}
+
 __device__ __forceinline__ uint32_t e4m3_of_quotient(float x, float s) {
-    if (!(s > 0.f) || isnan(x)) return f64_to_e4m3((double)x / (double)s);  // (a NaN keeps its sign)
+    if (!(s > 0.f) || isnan(x)) return e4m3_of_quotient_f64(x, s);  // (a NaN keeps its sign)
     float q = __fdiv_rn(x, s);
     const float a = fabsf(q);
     bool mid;

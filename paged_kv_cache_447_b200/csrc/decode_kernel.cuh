@@ -1123,6 +1123,8 @@ __device__ __forceinline__ int find_seq_global(const int *pfx, int B, int Hkv, l
 
 template <int D, int G, int HPU>
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
+    constexpr int kSmemPfx = 4096;  // sequences whose prefix is searched in shared memory
+    __shared__ int spfx[kSmemPfx];
     pdl_wait();
     pdl_trigger();
     const int c = blockIdx.x;
@@ -1132,7 +1134,16 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     const long long U = (total + p.nctas - 1) / p.nctas;
     const long long x = (long long)c * U;
     if (x >= total) return;
-    const int b = find_seq_global(p.prefix, p.B, Hu, x);
+    // the segment holding boundary x: one coalesced copy of the prefix, then a search in
+    // shared memory (the search in global memory would chain a load per step)
+    int b;
+    if (p.B + 1 <= kSmemPfx) {
+        for (int i = threadIdx.x; i <= p.B; i += blockDim.x) spfx[i] = __ldg(p.prefix + i);
+        __syncthreads();
+        b = find_seq(spfx, p.B, Hu, x);
+    } else {
+        b = find_seq_global(p.prefix, p.B, Hu, x);
+    }
     const int pb = __ldg(p.prefix + b), nb = __ldg(p.prefix + b + 1) - pb;
     const int kvg = (int)((x - (long long)Hu * pb) / nb);
     const long long start = (long long)Hu * pb + (long long)kvg * nb;
@@ -1140,12 +1151,41 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeParams p) {
     const int c0 = (int)(start / U), c1 = (int)((start + nb - 1) / U);
     if (c0 != c - 1) return;                         // an earlier boundary's CTA merges it
     const int segu = b * Hu + kvg;
-    for (int e = threadIdx.x; e < HPU * G * D; e += blockDim.x) {
+    // four dims per thread, every load of a thread issued before it is used; the arithmetic
+    // is merge_partials' for each dim (the same order, so the same rounding).  A slot holds
+    // G * (D + 2) floats, so slots start on 16 bytes only when that is a multiple of 4.
+    for (int e4 = threadIdx.x; e4 < HPU * G * D / 4; e4 += blockDim.x) {
+        const int e = 4 * e4;
         const int hd = e / (G * D), g = (e / D) % G, d = e % D;
         const int kvo = kvg * HPU + hd;
+        float M = -INFINITY;
+        for (int cc = c0; cc <= c1; ++cc)
+            M = fmaxf(M, __ldcg(p.partials + (size_t)(HPU * (segu + cc) + hd) * (G * (D + 2)) + G * D + g));
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lsum = 0.f;
+        for (int cc = c0; cc <= c1; ++cc) {
+            const float *slot = p.partials + (size_t)(HPU * (segu + cc) + hd) * (G * (D + 2));
+            const float mk = __ldcg(slot + G * D + g);
+            const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
+            float4 a;
+            if constexpr ((G * (D + 2)) % 4 == 0) {  // slots 16-byte aligned: one vector load
+                a = __ldcg(reinterpret_cast<const float4 *>(slot + g * D + d));
+            } else {
+                a = make_float4(__ldcg(slot + g * D + d), __ldcg(slot + g * D + d + 1), __ldcg(slot + g * D + d + 2),
+                                __ldcg(slot + g * D + d + 3));
+            }
+            o.x += f * a.x;
+            o.y += f * a.y;
+            o.z += f * a.z;
+            o.w += f * a.w;
+            lsum += f * __ldcg(slot + G * D + G + g);
+        }
         const float vsc = p.v_scale ? __ldg(p.v_scale + kvo) : 1.f;
-        p.out[((size_t)b * p.Hq + kvo * G + g) * D + d] =
-            __float2bfloat16_rn(merge_partials<D, G, HPU>(p, segu, hd, g, d, c0, c1, vsc));
+        const bool any = lsum > 0.f;
+        uint2 w;
+        w.x = pack_bf16x2(any ? o.x / lsum * vsc : 0.f, any ? o.y / lsum * vsc : 0.f);
+        w.y = pack_bf16x2(any ? o.z / lsum * vsc : 0.f, any ? o.w / lsum * vsc : 0.f);
+        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvo * G + g) * D + d) = w;
     }
 }
 

@@ -141,6 +141,82 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
     } while (c.b < B && c.nt == 0);
 }
 
+// Decode step, run by a q stager when a piece ends its sequence: the new token's K (rotated
+// at L - 1 by the RoPE factors rc/rs, when a table is given) and V, quantised to the E4M3
+// code of the exact quotient by the head's scale (as pkv_kv_store does), into cache slot
+// `slot` and into `codes` (128 K codes, then 128 V codes), from where the S^T issuer patches
+// the tile.  Lane i holds the pairs (i, i + 64) and (i + 32, i + 96).  Out of line: it runs
+// once per sequence, and inlined it would crowd the stager's loop in the instruction cache.
+__device__ __noinline__ void tc_store_new_token(const DecodeParams &p, int kvh, int slot, const uint16_t (&nk)[2][2],
+                                                const uint16_t (&nv)[2][2], const float (&rc)[2],
+                                                const float (&rs)[2], uint8_t *codes, int lane) {
+    constexpr int D = 128, D2 = 64;
+    const float ksc = __ldg(p.k_scale + kvh), vsc = __ldg(p.v_scale + kvh);
+    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        uint16_t k1 = nk[j][0], k2 = nk[j][1];
+        if (p.rope) rope_pair_fast(k1, k2, rc[j], rs[j], k1, k2);
+        const uint16_t kb[2] = {k1, k2};
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int d = lane + 32 * j + hf * D2;
+            const uint8_t kc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)kb[hf] << 16), ksc);
+            const uint8_t vc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)nv[j][hf] << 16), vsc);
+            static_cast<uint8_t *>(p.k_cache_w)[dst + d] = kc;
+            static_cast<uint8_t *>(p.v_cache_w)[dst + d] = vc;
+            codes[d] = kc;
+            codes[D + d] = vc;
+        }
+    }
+}
+
+// Decode step, run by the epilogue warp after it wrote the partial slot of a piece that is
+// not a whole segment: the CTAs c0..c1 that cut the segment each add one arrival; the last to
+// arrive merges their partials (as the combine kernel does, rounded alike: o / l * v_scale)
+// and clears the counter for the next call.  Out of line: it runs at most twice per CTA.
+template <int G>
+__device__ __noinline__ void tc_merge_if_last(const DecodeParams &p, const int *pfx, int Hu, long long U, int b,
+                                              int kvh, int ntiles, int segu, float vs, int lane) {
+    constexpr int D = 128;
+    __threadfence();
+    __syncwarp();
+    const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
+    const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
+    int last = 0;
+    if (lane == 0) last = atomicAdd(p.counters + segu, 1) == c1 - c0;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __threadfence();
+    // four dims per lane: M = max m_c, o = sum e^(m_c - M) acc_c / sum e^(m_c - M) l_c
+#pragma unroll
+    for (int i = 0; i < G * D / 128; ++i) {
+        const int e = (i * 32 + lane) * 4, g = e / D, d = e % D;
+        float M = -INFINITY;
+        for (int cc = c0; cc <= c1; ++cc)
+            M = fmaxf(M, __ldcg(p.partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D + g));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float ls = 0.f;
+        for (int cc = c0; cc <= c1; ++cc) {
+            const float *sl = p.partials + (size_t)(segu + cc) * (G * (D + 2));
+            const float mk = __ldcg(sl + G * D + g);
+            const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
+            const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
+            acc.x += f * x.x;
+            acc.y += f * x.y;
+            acc.z += f * x.z;
+            acc.w += f * x.w;
+            ls += f * __ldcg(sl + G * D + G + g);
+        }
+        const bool any = ls > 0.f;
+        uint2 w;
+        w.x = tc::pack_bf16x2(any ? acc.x / ls * vs : 0.f, any ? acc.y / ls * vs : 0.f);
+        w.y = tc::pack_bf16x2(any ? acc.z / ls * vs : 0.f, any ? acc.w / ls * vs : 0.f);
+        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
+    }
+    if (lane == 0) p.counters[segu] = 0;
+}
+
 template <int G, bool STEP>
 __global__ void __launch_bounds__(kTcThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -533,28 +609,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 int nt_row = -1;
                 if constexpr (STEP) {
                     if (nt_go && nt_e >= 0 && (long long)nt_e < p.num_blocks) {
-                        // K rotated at L - 1, both quantised to the E4M3 code of the exact
-                        // quotient by the head's scale (as pkv_kv_store does), into the cache
-                        // and into the slot's codes (128 K, then 128 V)
-                        const size_t dst = ((size_t)(nt_e * p.bs + pos % p.bs) * p.Hkv + kvh) * D;
-                        uint8_t *codes = newcodes + slot * 256;
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            uint16_t k1 = nk[j][0], k2 = nk[j][1];
-                            if (p.rope) rope_pair_fast(k1, k2, rc[j], rs[j], k1, k2);
-                            const uint16_t kb[2] = {k1, k2};
-#pragma unroll
-                            for (int hf = 0; hf < 2; ++hf) {
-                                const int d = lane + 32 * j + hf * D2;
-                                const uint8_t kc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)kb[hf] << 16), ksc);
-                                const uint8_t vc =
-                                    (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)nv[j][hf] << 16), vsc);
-                                static_cast<uint8_t *>(p.k_cache_w)[dst + d] = kc;
-                                static_cast<uint8_t *>(p.v_cache_w)[dst + d] = vc;
-                                codes[d] = kc;
-                                codes[D + d] = vc;
-                            }
-                        }
+                        tc_store_new_token(p, kvh, nt_e * p.bs + pos % p.bs, nk, nv, rc, rs, newcodes + slot * 256,
+                                           lane);
                         nt_row = pos % kTcTile;
                     }
                 }
@@ -641,48 +697,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc::tc_fence_before();
             mbar_arrive(bar_at(bars, kBOFree + ob));
             if constexpr (STEP) {
-                if (!whole) {
-                    // the last of the CTAs c0..c1 that cut this segment merges it (as the
-                    // combine kernel does) and clears the counter for the next call
-                    __threadfence();
-                    __syncwarp();
-                    const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
-                    const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
-                    int last = 0;
-                    if (lane == 0) last = atomicAdd(p.counters + segu, 1) == c1 - c0;
-                    last = __shfl_sync(0xffffffffu, last, 0);
-                    if (last) {
-                        __threadfence();
-                        // four dims per lane: M = max m_c, o = sum e^(m_c - M) acc_c / sum e^(m_c - M) l_c
-#pragma unroll
-                        for (int i = 0; i < G * D / 128; ++i) {
-                            const int e = (i * 32 + lane) * 4, g = e / D, d = e % D;
-                            float M = -INFINITY;
-                            for (int cc = c0; cc <= c1; ++cc)
-                                M = fmaxf(M, __ldcg(p.partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D + g));
-                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                            float ls = 0.f;
-                            for (int cc = c0; cc <= c1; ++cc) {
-                                const float *sl = p.partials + (size_t)(segu + cc) * (G * (D + 2));
-                                const float mk = __ldcg(sl + G * D + g);
-                                const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
-                                const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));
-                                acc.x += f * x.x;
-                                acc.y += f * x.y;
-                                acc.z += f * x.z;
-                                acc.w += f * x.w;
-                                ls += f * __ldcg(sl + G * D + G + g);
-                            }
-                            // (rounded as the combine kernel rounds: o / l * v_scale)
-                            const bool any = ls > 0.f;
-                            uint2 w;
-                            w.x = tc::pack_bf16x2(any ? acc.x / ls * vs : 0.f, any ? acc.y / ls * vs : 0.f);
-                            w.y = tc::pack_bf16x2(any ? acc.z / ls * vs : 0.f, any ? acc.w / ls * vs : 0.f);
-                            *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
-                        }
-                        if (lane == 0) p.counters[segu] = 0;
-                    }
-                }
+                if (!whole) tc_merge_if_last<G>(p, pfx, Hu, U, b, kvh, ntiles, segu, vs, lane);
             }
             k += piece_len;
         }
