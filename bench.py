@@ -196,6 +196,12 @@ def code_sha256(path: str) -> str:
     return hashlib.sha256(src.encode()).hexdigest()
 
 
+def sources_sha256(paths) -> str:
+    """code_sha256 over several sources (a kernel and the headers it is built from)."""
+    import hashlib
+    return hashlib.sha256("".join(code_sha256(os.path.join(ROOT, q)) for q in paths).encode()).hexdigest()
+
+
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch (read + write) from the committed ncu record in profiles/, or
     None if there is none for this kernel and workload or the kernel's code has changed
@@ -206,11 +212,21 @@ def recorded_traffic(kernel: str, workload: str):
             rec = json.load(f).get(kernel)
         if not rec or rec.get("workload") != workload:
             return None
-        if not code_sha256(os.path.join(ROOT, rec["src"])).startswith(rec["code_sha256_prefix"]):
+        if not sources_sha256(rec["src"]).startswith(rec["code_sha256_prefix"]):
             return None
         return int(rec["dram_bytes_read"]) + int(rec["dram_bytes_write"])
-    except (OSError, ValueError, KeyError):
+    except (OSError, ValueError, KeyError, TypeError):
         return None
+
+
+def timed_kernel(wl, decode: bool) -> str:
+    """Name of the kernel the bench's attention events bracket for this workload."""
+    if not decode:
+        return "prefill_kernel"
+    g = wl.n_q_heads // wl.n_kv_heads
+    if wl.cache_dtype == "fp8" and wl.head_dim == 128 and g in (2, 4, 8):
+        return "decode_tc_kernel"
+    return "decode_kernel"
 
 
 # ----------------------------------------------------------------------------- runner
@@ -246,6 +262,11 @@ class Runner:
             self.ws_step = pkv.decode_step_workspace(B, wl.n_q_heads, wl.n_kv_heads, wl.head_dim)
             self.dec_bt = self.dev["block_tables"][:B].contiguous()
             self.dec_ctx = self.dev["context_lens"][:B].contiguous()
+            self.dec_slots = self.dev["slot_mapping"][:B].contiguous()
+            self.dec_cu = torch.arange(B + 1, dtype=torch.int32, device=self.dec_ctx.device)
+            # the library's automatic choice: one launch up to one segment per SM
+            sms = torch.cuda.get_device_properties(self.dec_ctx.device).multi_processor_count
+            self.step_fused = B * wl.n_kv_heads <= sms
             self.ws = torch.empty(pkv.decode_workspace_bytes(B, wl.n_q_heads, wl.n_kv_heads,
                                                              wl.head_dim),
                                   dtype=torch.uint8, device="cuda")
@@ -270,7 +291,9 @@ class Runner:
 
     def launches_per_step(self) -> int:
         if self.fused:
-            n = (1 if self.B else 0) + (2 if self.P else 0)  # decode step; store + prefill
+            # decode step (one launch, or store + attention + merge); store + prefill
+            dec = 1 if getattr(self, "step_fused", True) else 3
+            n = (dec if self.B else 0) + (2 if self.P else 0)
         else:
             n = 1 + (2 if self.B else 0) + (1 if self.P else 0)  # store, decode + merge, prefill
         return n * self.layers
@@ -290,9 +313,18 @@ class Runner:
                              cu_seqlens=self.pre_cu, context_lens=self.pre_ctx)
             if self.B:
                 q = d["q"][:self.B]
+                # The decode step runs as one launch for a latency-bound batch and as store +
+                # attention + merge otherwise (the library's automatic mode).  The recorded
+                # pass times the attention kernels alone: for a split step the store runs
+                # first, outside the events.
+                split_rec = record and dominant == "decode" and self.fused and not self.step_fused
+                if split_rec:
+                    pkv.kv_store(self.dec_k, self.dec_v, kc, vc, self.dec_slots, k_scale=self.k_scale,
+                                 v_scale=self.v_scale, rope_cos_sin=self.table,
+                                 cu_seqlens=self.dec_cu, context_lens=self.dec_ctx)
                 if record and dominant == "decode":
                     e0 = torch.cuda.Event(enable_timing=True); e0.record(s)
-                if self.fused:
+                if self.fused and not split_rec:
                     pkv.paged_decode_step(q, self.dec_k, self.dec_v, kc, vc, self.dec_bt,
                                           self.dec_ctx, self.ws_step, scale=wl.scale,
                                           k_scale=self.k_scale, v_scale=self.v_scale,
@@ -398,7 +430,9 @@ def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=Tr
     attn_ms = r.attn_ms()
     res = {"workload": name, "step_ms": step_ms, "step_us": step_ms * 1e3, "layers": layers,
            "clocks": clocks, "gpu_launches": r.launches_per_step() * steps,
-           "decode_path": "fused step" if fused else "store + attention + merge"}
+           "decode_path": ("decode step, " + ("one launch" if getattr(r, "step_fused", False)
+                                                  else "store + attention + merge")) if fused
+                          else "kv_store + paged_decode_attention"}
     hbm = (pk or FALLBACK_PEAKS)["hbm_gbs"]
     if r.B:
         kv_bytes = decode_kv_bytes(st, wl.n_kv_heads, wl.head_dim, esize) * layers
@@ -569,8 +603,7 @@ def main():
         "decode_tok_s_per_layer": res.get("decode_tok_s_per_layer"),
         "roofline": {"bound": bound, "achieved": ach, "peak": peak, "unit": runit,
                      "frac": ach / peak,
-                     "traffic": recorded_traffic("decode_kernel" if runner.B else "prefill_kernel",
-                                                 args.workload),
+                     "traffic": recorded_traffic(timed_kernel(wl, bool(runner.B)), args.workload),
                      "kernel": "paged_decode_attention" if runner.B else "paged_prefill_attention",
                      "peak_source": pk_kind, "kernel_ms": res.get("attn_kernel_ms")},
         "clocks": res["clocks"],

@@ -253,8 +253,10 @@ size_t pkv_decode_step_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_hea
                                        int head_dim);
 
 /*
- * pkv_paged_decode_step -- one whole decode step in one launch: store each sequence's new
- * token into the paged cache and run decode attention over the cache including it
+ * pkv_paged_decode_step -- one whole decode step: store each sequence's new token into the
+ * paged cache and run decode attention over the cache including it.  In one launch when
+ * the batch is latency-bound (see pkv_set_decode_step_mode); otherwise the store runs as
+ * its own launch before the attention and its merge, chained on the stream
  * (ENG §2.1: every decode step appends the new token's K/V to the cache and attends over
  * all of it; PRM §17.1: decode is one token per sequence per step and its latency is the
  * time per output token; ENG §6.3: fusing kernels).  The result is that of
@@ -285,6 +287,20 @@ int pkv_paged_decode_step(void *out, const void *q, const void *k, const void *v
                           float scale, int cache_dtype, const float *k_scale,
                           const float *v_scale, const float *rope_cos_sin, int max_pos,
                           void *workspace, size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * pkv_set_decode_step_mode -- how pkv_paged_decode_step runs, for the whole process:
+ *   PKV_STEP_AUTO   one launch when num_seqs * n_kv_heads <= the device's SM count (the
+ *                   latency-bound case), else store + attention + merge (measured faster
+ *                   for large batches); the default
+ *   PKV_STEP_FUSED  always one launch
+ *   PKV_STEP_SPLIT  always store, then attention and merge
+ * The outputs and cache bytes are the same in every mode.  Returns the previous mode, or
+ * PKV_E_INVALID for an unknown one (nothing changes).  Host-side only; not thread-safe
+ * against concurrent decode-step calls that should see a change.
+ */
+enum pkv_step_mode { PKV_STEP_AUTO = 0, PKV_STEP_FUSED = 1, PKV_STEP_SPLIT = 2 };
+int pkv_set_decode_step_mode(int mode);
 
 /*
  * pkv_paged_prefill_attention -- causal attention of a chunk of new tokens per sequence

@@ -21,6 +21,7 @@ _BINDING_NAMES = {
     "paged_decode_attention_noalloc", "NOALLOC_SCRATCH_BYTES", "slot_mapping", "copy_blocks",
     "paged_decode_step", "decode_step_workspace_bytes", "decode_step_workspace",
     "block_pool", "block_pool_alloc", "block_pool_free",
+    "set_decode_step_mode", "STEP_AUTO", "STEP_FUSED", "STEP_SPLIT",
     "rope_build_table", "decode_workspace_bytes", "cache_bytes", "get_error", "strerror",
     "debug_wait_timeout", "version", "library_path", "load_library", "PagedKVError",
     "BF16", "FP8_E4M3",

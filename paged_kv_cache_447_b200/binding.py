@@ -78,6 +78,7 @@ def load_library():
         "pkv_copy_blocks": ([P, P, P, I, I, I, I, LL, I, P], I),
         "pkv_get_error": ([P], I),
         "pkv_debug_wait_timeout": ([LL, P], I),
+        "pkv_set_decode_step_mode": ([I], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -215,6 +216,18 @@ def block_pool_free(pool, block_ids, *, stream=None) -> None:
     n = block_ids.numel()
     _check("pkv_block_pool_free", load_library().pkv_block_pool_free(
         _p(pool), _pool_blocks(pool), _p(block_ids) if n else None, n, _stream(stream)))
+
+
+STEP_AUTO, STEP_FUSED, STEP_SPLIT = 0, 1, 2
+
+
+def set_decode_step_mode(mode: int) -> int:
+    """How paged_decode_step runs (STEP_AUTO / STEP_FUSED / STEP_SPLIT); returns the previous
+    mode."""
+    r = load_library().pkv_set_decode_step_mode(int(mode))
+    if r < 0:
+        raise PagedKVError("pkv_set_decode_step_mode", r)
+    return r
 
 
 def copy_blocks(k_cache, v_cache, block_pairs, *, stream=None) -> None:

@@ -477,6 +477,11 @@ int pkv_paged_decode_step(void *out, const void *q, const void *k, const void *v
     return status_of(e);
 }
 
+int pkv_set_decode_step_mode(int mode) {
+    if (mode != PKV_STEP_AUTO && mode != PKV_STEP_FUSED && mode != PKV_STEP_SPLIT) return PKV_E_INVALID;
+    return set_decode_step_mode(mode);
+}
+
 int pkv_paged_prefill_attention(void *out, const void *q, const void *k_cache,
                                 const void *v_cache, const int32_t *cu_seqlens,
                                 const int32_t *block_tables, int max_blocks_per_seq,

@@ -16,9 +16,9 @@
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
 //   warp 6      lane 0 issues the PV MMAs
-//   warps 7, 9  q stagers (even / odd pieces): each piece's q (rotated, scaled, split), its
-//               context length and scales, and (decode step) its new token, up to 4 pieces
-//               ahead
+//   warps 7, 9-11  q stagers (piece i to stager i % 4): each piece's q (rotated, scaled,
+//               split), its context length and scales, and (decode step) its new token,
+//               up to 4 pieces ahead
 //   warp 8      epilogue: O of a finished piece -> output rows or a partial slot
 // Per tile:
 //   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
@@ -44,10 +44,10 @@
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 384;
 constexpr int kTcPvWarp = 6;    // the PV issuer
-constexpr int kTcQWarp = 7;     // q stager of the even pieces
-constexpr int kTcQWarp2 = 9;    // q stager of the odd pieces
+constexpr int kTcStagers = 4;   // q stagers (warps 7, 9, 10, 11): stager i takes pieces i, i+4, ...
+__device__ __forceinline__ int tc_stager_index(int warp) { return warp == 7 ? 0 : (warp >= 9 ? warp - 8 : -1); }
 constexpr int kTcEpiWarp = 8;   // the epilogue (warp 8: TMEM lanes 0-31, where O's rows live)
 constexpr int kTcTile = 128;    // tokens per unit
 constexpr int kTcStages = 5;
@@ -90,7 +90,7 @@ struct TcGeo {
     static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
     static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [2 stagers] rotated bf16 q [8][128]
-    static constexpr int kOffBar = kOffQtmp + 2 * 8 * 128 * 2;
+    static constexpr int kOffBar = kOffQtmp + kTcStagers * 8 * 128 * 2;
     static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 18;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
@@ -147,24 +147,26 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
 // `slot` and into `codes` (128 K codes, then 128 V codes), from where the S^T issuer patches
 // the tile.  Lane i holds the pairs (i, i + 64) and (i + 32, i + 96).  Out of line: it runs
 // once per sequence, and inlined it would crowd the stager's loop in the instruction cache.
-__device__ __noinline__ void tc_store_new_token(const DecodeParams &p, int kvh, int slot, const uint16_t (&nk)[2][2],
+// (It takes plain values, not the kernel's parameter block: a reference to that would move
+// the block into local memory for the whole kernel.)
+__device__ __noinline__ void tc_store_new_token(uint8_t *k_cache, uint8_t *v_cache, int Hkv, float ksc, float vsc,
+                                                bool rope, int kvh, int slot, const uint16_t (&nk)[2][2],
                                                 const uint16_t (&nv)[2][2], const float (&rc)[2],
                                                 const float (&rs)[2], uint8_t *codes, int lane) {
     constexpr int D = 128, D2 = 64;
-    const float ksc = __ldg(p.k_scale + kvh), vsc = __ldg(p.v_scale + kvh);
-    const size_t dst = ((size_t)slot * p.Hkv + kvh) * D;
+    const size_t dst = ((size_t)slot * Hkv + kvh) * D;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         uint16_t k1 = nk[j][0], k2 = nk[j][1];
-        if (p.rope) rope_pair_fast(k1, k2, rc[j], rs[j], k1, k2);
+        if (rope) rope_pair_fast(k1, k2, rc[j], rs[j], k1, k2);
         const uint16_t kb[2] = {k1, k2};
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int d = lane + 32 * j + hf * D2;
             const uint8_t kc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)kb[hf] << 16), ksc);
             const uint8_t vc = (uint8_t)e4m3_of_quotient(__uint_as_float((uint32_t)nv[j][hf] << 16), vsc);
-            static_cast<uint8_t *>(p.k_cache_w)[dst + d] = kc;
-            static_cast<uint8_t *>(p.v_cache_w)[dst + d] = vc;
+            k_cache[dst + d] = kc;
+            v_cache[dst + d] = vc;
             codes[d] = kc;
             codes[D + d] = vc;
         }
@@ -174,47 +176,73 @@ __device__ __noinline__ void tc_store_new_token(const DecodeParams &p, int kvh, 
 // Decode step, run by the epilogue warp after it wrote the partial slot of a piece that is
 // not a whole segment: the CTAs c0..c1 that cut the segment each add one arrival; the last to
 // arrive merges their partials (as the combine kernel does, rounded alike: o / l * v_scale)
-// and clears the counter for the next call.  Out of line: it runs at most twice per CTA.
+// and clears the counter for the next call.  Out of line: it runs at most twice per CTA (and
+// takes plain values, not the kernel's parameter block, for the reason given above).
 template <int G>
-__device__ __noinline__ void tc_merge_if_last(const DecodeParams &p, const int *pfx, int Hu, long long U, int b,
-                                              int kvh, int ntiles, int segu, float vs, int lane) {
+__device__ __noinline__ void tc_merge_if_last(int *counters, const float *partials, __nv_bfloat16 *out, int Hq,
+                                              const int *pfx, int Hu, long long U, int b, int kvh, int ntiles,
+                                              int segu, float vs, int lane) {
     constexpr int D = 128;
     __threadfence();
     __syncwarp();
     const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
     const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
     int last = 0;
-    if (lane == 0) last = atomicAdd(p.counters + segu, 1) == c1 - c0;
+    if (lane == 0) last = atomicAdd(counters + segu, 1) == c1 - c0;
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
     __threadfence();
-    // four dims per lane: M = max m_c, o = sum e^(m_c - M) acc_c / sum e^(m_c - M) l_c
+    // lane: dims 4*lane .. 4*lane+3 of every head g.  M_g = max m_c, o = sum e^(m_c - M) acc_c
+    // / sum e^(m_c - M) l_c, accumulated over c in order (as the combine kernel does); the
+    // heads' loads of one CTA slot go out together.
+    const int d = 4 * lane;
+    float M[G];
 #pragma unroll
-    for (int i = 0; i < G * D / 128; ++i) {
-        const int e = (i * 32 + lane) * 4, g = e / D, d = e % D;
-        float M = -INFINITY;
-        for (int cc = c0; cc <= c1; ++cc)
-            M = fmaxf(M, __ldcg(p.partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D + g));
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float ls = 0.f;
-        for (int cc = c0; cc <= c1; ++cc) {
-            const float *sl = p.partials + (size_t)(segu + cc) * (G * (D + 2));
-            const float mk = __ldcg(sl + G * D + g);
-            const float f = (mk == -INFINITY) ? 0.f : ex2(mk - M);
-            const float4 x = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
-            acc.x += f * x.x;
-            acc.y += f * x.y;
-            acc.z += f * x.z;
-            acc.w += f * x.w;
-            ls += f * __ldcg(sl + G * D + G + g);
-        }
-        const bool any = ls > 0.f;
-        uint2 w;
-        w.x = tc::pack_bf16x2(any ? acc.x / ls * vs : 0.f, any ? acc.y / ls * vs : 0.f);
-        w.y = tc::pack_bf16x2(any ? acc.z / ls * vs : 0.f, any ? acc.w / ls * vs : 0.f);
-        *reinterpret_cast<uint2 *>(p.out + ((size_t)b * p.Hq + kvh * G + g) * D + d) = w;
+    for (int g = 0; g < G; ++g) M[g] = -INFINITY;
+    for (int cc = c0; cc <= c1; ++cc) {
+        const float *sl = partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D;
+        float mk[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) mk[g] = __ldcg(sl + g);
+#pragma unroll
+        for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], mk[g]);
     }
-    if (lane == 0) p.counters[segu] = 0;
+    float4 acc[G];
+    float ls[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+        ls[g] = 0.f;
+    }
+    for (int cc = c0; cc <= c1; ++cc) {
+        const float *sl = partials + (size_t)(segu + cc) * (G * (D + 2));
+        float mk[G], lk[G];
+        float4 x[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            mk[g] = __ldcg(sl + G * D + g);
+            lk[g] = __ldcg(sl + G * D + G + g);
+            x[g] = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float f = (mk[g] == -INFINITY) ? 0.f : ex2(mk[g] - M[g]);
+            acc[g].x += f * x[g].x;
+            acc[g].y += f * x[g].y;
+            acc[g].z += f * x[g].z;
+            acc[g].w += f * x[g].w;
+            ls[g] += f * lk[g];
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const bool any = ls[g] > 0.f;
+        uint2 w;
+        w.x = tc::pack_bf16x2(any ? acc[g].x / ls[g] * vs : 0.f, any ? acc[g].y / ls[g] * vs : 0.f);
+        w.y = tc::pack_bf16x2(any ? acc[g].z / ls[g] * vs : 0.f, any ? acc[g].w / ls[g] * vs : 0.f);
+        *reinterpret_cast<uint2 *>(out + ((size_t)b * Hq + kvh * G + g) * D + d) = w;
+    }
+    if (lane == 0) counters[segu] = 0;
 }
 
 template <int G, bool STEP>
@@ -496,9 +524,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait_bounded(bar_at(bars, kBDrain), 0, p.err);
         }
         __syncwarp();
-    } else if (warp == kTcQWarp || warp == kTcQWarp2) {
+    } else if (tc_stager_index(warp) >= 0) {
         // ---------------------------------------------------------------- q stagers
-        // Two warps take the pieces in turn (even / odd), each into q buffer piece % kTcQBufs:
+        // Four warps take the pieces in turn (piece i to stager i % 4), each into q buffer
+        // piece % kTcQBufs (its own):
         // the G heads' q rotated at L - 1, scaled by one power of two for the group and split
         // into high parts (rows 0..G-1) and low parts (rows G..2G-1) as E4M3 codes, plus the
         // piece's description, and (decode step) the new token of a piece that ends its
@@ -506,13 +535,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // new K alike: both rotate at L - 1); the next piece's context length is fetched
         // while this one is staged.  Run up to kTcQBufs pieces ahead of the softmax.
         constexpr int D2 = D / 2;
-        const int par = warp == kTcQWarp ? 0 : 1;
+        const int par = tc_stager_index(warp);
         uint16_t *qt = qtmp + par * (8 * D);
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
         int k = 0;
         // context length of the next piece this warp stages
         auto next_own = [&](TcCursor c, int kk, int pc) -> int {  // (by value: a look-ahead)
-            while (kk < nunits && (pc & 1) != par) {
+            while (kk < nunits && pc % kTcStagers != par) {
                 const int pl = min(c.nt - c.tile, nunits - kk);
                 kk += pl;
                 for (int t = 0; t < pl; ++t) tc_next(c, pfx, p.B, Hu);
@@ -525,7 +554,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int b = cur.b, kvh = cur.kvh;
             const int piece_len = min(cur.nt - cur.tile, nunits - k);
             const bool ends = piece_len == cur.nt - cur.tile;  // the piece ends its sequence
-            if ((pc & 1) == par) {
+            if (pc % kTcStagers == par) {
                 const int slot = pc % kTcQBufs;
                 const int L = min(Lraw, p.max_tokens), pos = L - 1;
                 const bool rope_ok = p.rope && pos >= 0 && pos < p.max_pos;
@@ -609,8 +638,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 int nt_row = -1;
                 if constexpr (STEP) {
                     if (nt_go && nt_e >= 0 && (long long)nt_e < p.num_blocks) {
-                        tc_store_new_token(p, kvh, nt_e * p.bs + pos % p.bs, nk, nv, rc, rs, newcodes + slot * 256,
-                                           lane);
+                        tc_store_new_token(static_cast<uint8_t *>(p.k_cache_w), static_cast<uint8_t *>(p.v_cache_w), p.Hkv,
+                                           ksc, vsc, p.rope != nullptr, kvh, nt_e * p.bs + pos % p.bs, nk, nv, rc, rs,
+                                           newcodes + slot * 256, lane);
                         nt_row = pos % kTcTile;
                     }
                 }
@@ -697,7 +727,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc::tc_fence_before();
             mbar_arrive(bar_at(bars, kBOFree + ob));
             if constexpr (STEP) {
-                if (!whole) tc_merge_if_last<G>(p, pfx, Hu, U, b, kvh, ntiles, segu, vs, lane);
+                if (!whole)
+                    tc_merge_if_last<G>(p.counters, p.partials, p.out, p.Hq, pfx, Hu, U, b, kvh, ntiles, segu, vs, lane);
             }
             k += piece_len;
         }

@@ -23,6 +23,10 @@ struct StoreArgs {
     const int32_t *cu_seqlens, *context_lens;
     int num_seqs;
     int *err;
+    // decode step (slot_mapping NULL): token t is sequence t's new token, at position
+    // context_lens[t] - 1, its slot read from the block table
+    const int32_t *block_tables = nullptr;
+    int max_blocks = 0, block_size = 16;
 };
 
 struct RopeArgs {
@@ -137,6 +141,7 @@ size_t decode_workspace_bytes(int num_seqs, int n_q_heads, int n_kv_heads, int h
 // Its workspace is decode_workspace_bytes(...) followed by num_seqs * n_kv_heads int
 // counters that must be zero before the first call (every call leaves them zero).
 cudaError_t launch_paged_decode_step(const DecodeArgs &a, cudaStream_t s);
+int set_decode_step_mode(int mode);  // returns the previous mode (PKV_STEP_*)
 // Grouped heads over an E4M3 cache at head dim 128 run on the tcgen05 decode kernel.
 bool decode_tc_supported(const DecodeArgs &a);
 cudaError_t launch_paged_decode_tc(const DecodeArgs &a, cudaStream_t s);

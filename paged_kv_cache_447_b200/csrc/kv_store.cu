@@ -62,8 +62,24 @@ __global__ void __launch_bounds__(256) kv_store_kernel(StoreArgs a) {
         const long long th = it / cpr;
         const int h = (int)(th % H);
         const int t = (int)(th / H);
-        const int slot = __ldg(a.slot_mapping + t);
-        if (slot < 0) continue;                      // padding token
+        int slot;
+        long long step_pos = -1;
+        if (a.slot_mapping) {
+            slot = __ldg(a.slot_mapping + t);
+            if (slot < 0) continue;                  // padding token
+        } else {
+            // decode step: sequence t's new token at L - 1 (none for an empty sequence, and
+            // none when the context exceeds the block table: attention flags that one)
+            const int L = __ldg(a.context_lens + t);
+            if (L < 1 || (long long)L > (long long)a.max_blocks * a.block_size) continue;
+            step_pos = L - 1;
+            const int e = __ldg(a.block_tables + (size_t)t * a.max_blocks + (int)(step_pos / a.block_size));
+            if (e < 0 || (long long)e * a.block_size >= a.num_slots) {
+                atomicOr(a.err, kErrBounds);
+                continue;
+            }
+            slot = e * a.block_size + (int)(step_pos % a.block_size);
+        }
         if ((long long)slot >= a.num_slots) {        // never write outside the cache
             atomicOr(a.err, kErrBounds);
             continue;
@@ -74,9 +90,12 @@ __global__ void __launch_bounds__(256) kv_store_kernel(StoreArgs a) {
         Chunk kx{__ldg(ks + c), __ldg(ks + c + cpr)};
         Chunk vx{__ldg(vs + c), __ldg(vs + c + cpr)};
         if (ROPE) {
-            const int b = owner_seq(a.cu_seqlens, a.num_seqs, t);
-            const int n = __ldg(a.cu_seqlens + b + 1) - __ldg(a.cu_seqlens + b);
-            const long long pos = (long long)__ldg(a.context_lens + b) - n + (t - __ldg(a.cu_seqlens + b));
+            long long pos = step_pos;
+            if (a.slot_mapping) {
+                const int b = owner_seq(a.cu_seqlens, a.num_seqs, t);
+                const int n = __ldg(a.cu_seqlens + b + 1) - __ldg(a.cu_seqlens + b);
+                pos = (long long)__ldg(a.context_lens + b) - n + (t - __ldg(a.cu_seqlens + b));
+            }
             if (pos < 0 || pos >= a.max_pos) {
                 atomicOr(a.err, kErrBounds);
                 continue;

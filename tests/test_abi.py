@@ -104,6 +104,20 @@ def test_block_helpers_host_checks_need_no_device():
     assert lib.pkv_copy_blocks(n, n, n, 0, 2, 64, 16, 32, 0, n) == 0
 
 
+def test_decode_step_mode_control():
+    """The decode-step mode: unknown modes are refused and change nothing; a set returns the
+    previous mode."""
+    lib = binding.load_library()
+    assert lib.pkv_set_decode_step_mode(7) == -1
+    assert lib.pkv_set_decode_step_mode(-1) == -1
+    prev = pkv.set_decode_step_mode(pkv.STEP_SPLIT)
+    assert prev == pkv.STEP_AUTO
+    assert pkv.set_decode_step_mode(pkv.STEP_FUSED) == pkv.STEP_SPLIT
+    assert pkv.set_decode_step_mode(pkv.STEP_AUTO) == pkv.STEP_FUSED
+    with pytest.raises(pkv.PagedKVError):
+        pkv.set_decode_step_mode(3)
+
+
 def test_workspace_size_is_positive_and_monotone():
     a = pkv.decode_workspace_bytes(64, 32, 32, 128)
     b = pkv.decode_workspace_bytes(128, 32, 32, 128)

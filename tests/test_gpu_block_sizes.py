@@ -48,9 +48,10 @@ def test_slots_store_and_prefill(bs, d, hq, hkv, fp8):
     compare(out, oracle_attention(wl, st, kc, vc), fp8=fp8, what=f"prefill bs={bs}")
 
 
+@pytest.mark.parametrize("mode", ["fused", "split"])
 @pytest.mark.parametrize("bs", [8, 32])
 @pytest.mark.parametrize("d,hq,hkv,fp8", SHAPES)
-def test_decode_and_decode_step(bs, d, hq, hkv, fp8):
+def test_decode_and_decode_step(bs, d, hq, hkv, fp8, mode):
     ctxs = _lengths(bs) + [4096, 2 * bs + 3]
     wl = W.paged_batch(200 + bs + d + hq, hq, hkv, d, [1] * len(ctxs), ctxs, block_size=bs,
                        fp8=fp8, decode_seqs=len(ctxs))
@@ -60,16 +61,21 @@ def test_decode_and_decode_step(bs, d, hq, hkv, fp8):
     ref = a.decode(st)
     b = DeviceWorkload(wl)
     ws = pkv.decode_step_workspace(st.num_seqs, hq, hkv, d)
-    out = pkv.paged_decode_step(st.q.cuda(), st.k.cuda(), st.v.cuda(), b.k_cache, b.v_cache,
-                                st.block_tables.cuda(), st.context_lens.cuda(), ws, scale=wl.scale,
-                                k_scale=b.k_scale, v_scale=b.v_scale, rope_cos_sin=b.table)
-    torch.cuda.synchronize()
+    pkv.set_decode_step_mode(pkv.STEP_FUSED if mode == "fused" else pkv.STEP_SPLIT)
+    try:
+        out = pkv.paged_decode_step(st.q.cuda(), st.k.cuda(), st.v.cuda(), b.k_cache, b.v_cache,
+                                    st.block_tables.cuda(), st.context_lens.cuda(), ws, scale=wl.scale,
+                                    k_scale=b.k_scale, v_scale=b.v_scale, rope_cos_sin=b.table)
+        torch.cuda.synchronize()
+    finally:
+        pkv.set_decode_step_mode(pkv.STEP_AUTO)
     assert pkv.get_error() == 0
     assert torch.equal(b.k_cache, a.k_cache) and torch.equal(b.v_cache, a.v_cache)
     assert torch.equal(out, ref)
-    kc, vc = oracle_caches(wl)
-    oracle_store(wl, st, kc, vc)
-    compare(ref, oracle_attention(wl, st, kc, vc), fp8=fp8, what=f"decode bs={bs}")
+    if mode == "fused":
+        kc, vc = oracle_caches(wl)
+        oracle_store(wl, st, kc, vc)
+        compare(ref, oracle_attention(wl, st, kc, vc), fp8=fp8, what=f"decode bs={bs}")
 
 
 @pytest.mark.parametrize("bs", [8, 32])

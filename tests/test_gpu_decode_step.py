@@ -1,7 +1,8 @@
-"""GPU parity of the one-launch decode step (pkv_paged_decode_step): storing each sequence's
-new token and attending over the cache in one kernel gives the same cache bytes and the same
-output bits as pkv_kv_store followed by pkv_paged_decode_attention, matches the oracle, and
-leaves the workspace's counters at zero for the next call."""
+"""GPU parity of the decode step (pkv_paged_decode_step): storing each sequence's new token and
+attending over the cache -- in one kernel, or as store + attention + merge, or as the batch
+size picks -- gives the same cache bytes and the same output bits as pkv_kv_store followed
+by pkv_paged_decode_attention, matches the oracle, and leaves the workspace's counters at
+zero for the next call."""
 import numpy as np
 import pytest
 import torch
@@ -49,19 +50,25 @@ def _check(wl: W.Workload, oracle_rows=None):
     a = DeviceWorkload(wl)
     a.store(st)
     ref = a.decode(st)
-    b = DeviceWorkload(wl)
-    ws = pkv.decode_step_workspace(st.num_seqs, wl.n_q_heads, wl.n_kv_heads, wl.head_dim)
-    for _ in range(2):  # twice in a row: the first call must leave its counters at zero
-        out = pkv.paged_decode_step(st.q.cuda(), st.k.cuda(), st.v.cuda(), b.k_cache, b.v_cache,
-                                    st.block_tables.cuda(), st.context_lens.cuda(), ws,
-                                    scale=wl.scale, k_scale=b.k_scale, v_scale=b.v_scale,
-                                    rope_cos_sin=b.table)
-        torch.cuda.synchronize()
-        assert pkv.get_error() == 0
-        assert torch.equal(b.k_cache, a.k_cache) and torch.equal(b.v_cache, a.v_cache)
-        assert torch.equal(out, ref), float((out.float() - ref.float()).abs().max())
-    nctr = st.num_seqs * wl.n_kv_heads * 4
-    assert int(ws[-((nctr + 15) // 16 * 16):].count_nonzero()) == 0
+    # every mode: one launch, store + attention + merge, and whichever the batch size picks
+    for mode in (pkv.STEP_FUSED, pkv.STEP_SPLIT, pkv.STEP_AUTO):
+        pkv.set_decode_step_mode(mode)
+        try:
+            b = DeviceWorkload(wl)
+            ws = pkv.decode_step_workspace(st.num_seqs, wl.n_q_heads, wl.n_kv_heads, wl.head_dim)
+            for _ in range(2):  # twice in a row: the first call must leave its counters at zero
+                out = pkv.paged_decode_step(st.q.cuda(), st.k.cuda(), st.v.cuda(), b.k_cache,
+                                            b.v_cache, st.block_tables.cuda(), st.context_lens.cuda(),
+                                            ws, scale=wl.scale, k_scale=b.k_scale,
+                                            v_scale=b.v_scale, rope_cos_sin=b.table)
+                torch.cuda.synchronize()
+                assert pkv.get_error() == 0
+                assert torch.equal(b.k_cache, a.k_cache) and torch.equal(b.v_cache, a.v_cache), mode
+                assert torch.equal(out, ref), (mode, float((out.float() - ref.float()).abs().max()))
+            nctr = st.num_seqs * wl.n_kv_heads * 4
+            assert int(ws[-((nctr + 15) // 16 * 16):].count_nonzero()) == 0
+        finally:
+            pkv.set_decode_step_mode(pkv.STEP_AUTO)
     if oracle_rows is not False:
         kc, vc = oracle_caches(wl)
         oracle_store(wl, st, kc, vc)
@@ -124,9 +131,16 @@ def test_decode_step_groups_and_head_dims(hq, hkv, d, fp8):
     _check(_lognormal_batch(30 + hq + d, hq, hkv, d, fp8))
 
 
-def test_decode_step_empty_and_out_of_table():
+@pytest.fixture(params=["fused", "split"])
+def step_mode(request):
+    pkv.set_decode_step_mode(pkv.STEP_FUSED if request.param == "fused" else pkv.STEP_SPLIT)
+    yield request.param
+    pkv.set_decode_step_mode(pkv.STEP_AUTO)
+
+
+def test_decode_step_empty_and_out_of_table(step_mode):
     """A sequence with no context stores nothing and gets a zero row; a block-table entry
-    outside the pool stores nothing and raises the bounds flag."""
+    outside the pool stores nothing and raises the bounds flag (in both step modes)."""
     wl = W.qwen_decode(seed=2, batch=6)
     st = wl.steps[0]
     ctx = st.context_lens.clone()
