@@ -16,10 +16,10 @@
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
 //   warp 6      lane 0 issues the PV MMAs
-//   warps 7, 9-11  q stagers (piece i to stager i % 4): each piece's q (rotated, scaled,
+//   warps 7, 12-14  q stagers (piece i to stager i % 4): each piece's q (rotated, scaled,
 //               split), its context length and scales, and (decode step) its new token,
 //               up to 4 pieces ahead
-//   warp 8      epilogue: O of a finished piece -> output rows or a partial slot
+//   warps 8-11  epilogue, thread = dim: O of a finished piece -> output rows or a partial slot
 // Per tile:
 //   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
 //                 cache stores it (K-major), B = q as E4M3 rows -- the G heads' high parts in
@@ -29,32 +29,37 @@
 //                 tile maxima across the four warps, updates the lazy running max (O is
 //                 rescaled only when a max grows by more than 2^8) and writes p as high and
 //                 low E4M3 parts into a shared-memory P tile: row h / 8+h, byte t.
-//   O += P V      M = 64, N = 128 dims, K = 128 tokens, twice: A = the P tile from row 0 (high
-//                 parts in rows 0..G-1) and from row 8 (low parts in rows 8..8+G-1), B = the V
-//                 tile MN-major as the cache stores it; O rows 0..G-1 = the G heads.
+//   O^T += V^T P^T  M = 128 dims, N = 16, K = 128 tokens: A = the V tile read MN-major as the
+//                 cache stores it, B = the P tile's 16 rows (K-major), so column h of O^T
+//                 gathers the heads' high parts and column 8+h their low parts; the epilogue
+//                 adds the two.  (Taking O transposed keeps the MMA at the 16 columns the
+//                 heads need instead of 64 rows of which G are used.)
 // S^T and PV are issued by two threads, each waiting only for its own inputs (S^T: tile
 // landed, S buffer free, the piece's q staged; PV: P written, O buffer free), so a stage goes
 // back to the producer as soon as its PV completes, and S^T of later tiles runs ahead.  They
 // touch disjoint TMEM columns and shared memory.  S and P are double-buffered, q has 4
 // buffers and O three (by piece), so neither the next piece's q nor the last pieces' epilogues
-// holds up the tiles.
+// holds up the tiles.  TMEM: S^T at columns 0 and 16, O^T buffers at 32, 48 and 64 (128 lanes
+// x 16 columns each).
 #include "decode_kernel.cuh"
 #include "tcgen05.cuh"
 
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 384;
+constexpr int kTcThreads = 480;
 constexpr int kTcPvWarp = 6;    // the PV issuer
-constexpr int kTcStagers = 4;   // q stagers (warps 7, 9, 10, 11): stager i takes pieces i, i+4, ...
-__device__ __forceinline__ int tc_stager_index(int warp) { return warp == 7 ? 0 : (warp >= 9 ? warp - 8 : -1); }
-constexpr int kTcEpiWarp = 8;   // the epilogue (warp 8: TMEM lanes 0-31, where O's rows live)
+constexpr int kTcStagers = 4;   // q stagers (warps 7, 12, 13, 14): stager i takes pieces i, i+4, ...
+__device__ __forceinline__ int tc_stager_index(int warp) { return warp == 7 ? 0 : (warp >= 12 ? warp - 11 : -1); }
+constexpr int kTcEpiWarp = 8;   // the epilogue: warps 8-11, one per TMEM lane quarter (O^T rows = dims)
+constexpr int kTcEpiBar = 2;    // named barrier of the 128 epilogue threads
 constexpr int kTcTile = 128;    // tokens per unit
 constexpr int kTcStages = 5;
 constexpr int kTcQBufs = 4;     // q buffers: the stager runs up to this many pieces ahead
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
-constexpr uint32_t kTcO = 128;  // TMEM column of O buffer 0 (buffers 1, 2 follow at +128, +256)
+constexpr uint32_t kTcO = 32;   // TMEM column of O^T buffer 0 (buffers 1, 2 follow at +16, +32)
+constexpr uint32_t kTcCols = 128;  // TMEM columns allocated (a power of two >= 32 + 16 * kTcOBufs)
 constexpr int kTcOBufs = 3;     // O buffers (and stats slots): the epilogue may lag two pieces
 
 // What the q stager knows of a piece, for the softmax warps.
@@ -79,17 +84,16 @@ struct TcGeo {
     static constexpr int kKV = kTcTile * D;         // one E4M3 K (or V) tile: 16 KB
     static constexpr int kStage = 2 * kKV;
     static constexpr int kQ = 16 * 128;             // B operand of S^T: 16 rows x 128 codes
-    // A operands of PV: p's high parts in rows 0..G-1 (read as rows 0..63) and its low parts
-    // in rows 8..8+G-1 (read as rows 8..71, i.e. again rows 0..G-1 of that operand), so two
-    // MMAs add both into O rows 0..G-1; 80 rows x 128 tokens
-    static constexpr int kP = 80 * 128;
+    // B operand of PV: p's high parts in rows 0..G-1, its low parts in rows 8..8+G-1, zeros in
+    // the other rows; 16 rows x 128 tokens
+    static constexpr int kP = 16 * 128;
     static constexpr int kOffQ = kTcStages * kStage;
     static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
     static constexpr int kOffRed = kOffP + 2 * kP;          // [4 warps][8] floats x 2 (max, sum)
-    static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [2] TcStats
+    static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [kTcOBufs] TcStats
     static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
-    static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [2 stagers] rotated bf16 q [8][128]
+    static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [kTcStagers] rotated bf16 q [8][128]
     static constexpr int kOffBar = kOffQtmp + kTcStagers * 8 * 128 * 2;
     static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 18;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int i = 0; i < kTcOBufs; ++i) {
             mbar_init(bar_at(bars, kBOReady + i), 1);
             mbar_init(bar_at(bars, kBStats + i), 1);
-            mbar_init(bar_at(bars, kBOFree + i), 32);
+            mbar_init(bar_at(bars, kBOFree + i), 128);
         }
         for (int i = 0; i < kTcQBufs; ++i) {
             mbar_init(bar_at(bars, kBQFull + i), 1);
@@ -347,16 +351,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(sQ + 16 * i), "r"(0u) : "memory");
     fence_proxy_async_smem();
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
-                     ::"r"(smem_u32((const void *)tmem_slot)));
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32((const void *)tmem_slot)), "n"(kTcCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM: S^T buffers at columns 0 and 16 (128 lanes x 16), O buffers at columns 128, 256
-    // and 384 (rows 0..G-1 of 64 x 128 each)
+    // TMEM: S^T buffers at columns 0 and 16, O^T buffers at 32, 48, 64 (128 lanes x 16 each)
 
     // a bounded wait by lane 0 of the calling warp, its outcome broadcast to the warp (the
     // __syncwarp orders the other lanes' accesses after lane 0's acquire)
@@ -489,7 +492,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) tc::mma_commit(bar_at(bars, kBDrain));  // (with the PV issuer's commit)
     } else if (warp == kTcPvWarp) {
         // ---------------------------------------------------------------- PV issuer
-        constexpr uint32_t idO = tc::mma_idesc(64, D, true, true);  // B (V) MN-major
+        constexpr uint32_t idO = tc::mma_idesc(128, 16, false, true) | tc::kIdescAMnMajor;  // A (V^T) MN-major
         if (lane == 0) {
             bool ok = true;
             int piece = -1;
@@ -507,13 +510,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::tc_fence_after();
                 const uint32_t vd = sStages + (k % kTcStages) * Geo::kStage + Geo::kKV;
                 const uint32_t pd = sP + (k & 1) * Geo::kP;
-                const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece % kTcOBufs);
+                const uint32_t tO = tmem + kTcO + 16u * (uint32_t)(piece % kTcOBufs);
 #pragma unroll
-                for (int kk = 0; kk < kTcTile / 32; ++kk) {
-                    const uint64_t vdesc = tc::sw128_desc(vd + 4096 * kk, 16384, 1024);
-                    tc::mma_ss_f8(tO, tc::sw128_desc(pd + 32 * kk, 16, 1024), vdesc, idO, (first && kk == 0) ? 0u : 1u);
-                    tc::mma_ss_f8(tO, tc::sw128_desc(pd + 1024 + 32 * kk, 16, 1024), vdesc, idO, 1u);  // low parts
-                }
+                for (int kk = 0; kk < kTcTile / 32; ++kk)  // 32 tokens per MMA
+                    tc::mma_ss_f8(tO, tc::sw128_desc(vd + 4096 * kk, 16384, 1024), tc::sw128_desc(pd + 32 * kk, 16, 1024),
+                                  idO, (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
                 tc::mma_commit(bar_at(bars, kBPvDone + (k & 1)));
                 if (last) tc::mma_commit(bar_at(bars, kBOReady + piece % kTcOBufs));
@@ -664,16 +665,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             k += piece_len;
             for (int t = 0; t < piece_len; ++t) tc_next(cur, pfx, p.B, Hu);
         }
-    } else if (warp == kTcEpiWarp) {
+    } else if (warp >= kTcEpiWarp && warp < kTcEpiWarp + 4) {
         // ---------------------------------------------------------------- epilogue
         // For each piece in turn, once its last PV has completed and the softmax has left the
-        // piece's description and (m, l): O (TMEM lanes 0..G-1 of its O buffer) -> the
-        // output rows (a whole segment) or the piece's partial slot, then O buffer free.
+        // piece's description and (m, l): thread = dim d (TMEM lane d of O^T), the heads'
+        // columns h + 8+h -> the output rows (a whole segment) or the piece's partial slot,
+        // then O buffer free.
+        const int quad = warp & 3;
+        const int d = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         int k = 0;
         for (int piece = 0; k < nunits; ++piece) {
             const int ob = piece % kTcOBufs, ph = (piece / kTcOBufs) & 1;
             const bool fin = wait0(kBStats + ob, ph) && wait0(kBOReady + ob, ph);
-            if (!fin) {
+            // the four warps leave together (the decode step's merge has them meet again)
+            if (named_bar_any(kTcEpiBar, 128, !fin)) {
                 if (lane == 0) *abort_flag = 1;
                 break;
             }
@@ -682,53 +688,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int b = st.b, kvh = st.kvh, ntiles = st.ntiles, piece_len = st.piece_len;
             const bool whole = st.whole != 0;
             const float vs = st.vs;
-            const int h = lane < G ? lane : 0;  // lanes 0..G-1 hold O rows h
-            const float m = st.m[h], l = st.l[h];
-            const int segu = b * Hu + kvh;
-            float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
-            const float inv = l > 0.f ? vs / l : 0.f;
-            const uint32_t tO = tmem + kTcO + 128u * (uint32_t)ob;
-            __nv_bfloat16 *orow = p.out + ((size_t)b * p.Hq + kvh * G + h) * D;
-            // 32 columns of the row, scaled and stored (lanes 0..G-1)
-            auto put = [&](int c0, const uint32_t (&rr)[32]) {
-                if (lane >= G) return;
-                if (whole) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c0);
+            float m[G], l[G];
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        w.x = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv, __uint_as_float(rr[8 * v + 1]) * inv);
-                        w.y = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv, __uint_as_float(rr[8 * v + 3]) * inv);
-                        w.z = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv, __uint_as_float(rr[8 * v + 5]) * inv);
-                        w.w = tc::pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv, __uint_as_float(rr[8 * v + 7]) * inv);
-                        dst[v] = w;
-                    }
-                } else {
-                    float4 *dst = reinterpret_cast<float4 *>(slot + h * D + c0);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v)
-                        dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
-                                             __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
-                }
-            };
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 64) {  // two loads per wait
-                uint32_t ra[32], rb[32];
-                tc::tmem_ld32(tO + c0, ra);
-                tc::tmem_ld32(tO + c0 + 32, rb);
-                tc::tc_wait_ld();
-                put(c0, ra);
-                put(c0 + 32, rb);
+            for (int h = 0; h < G; ++h) {
+                m[h] = st.m[h];
+                l[h] = st.l[h];
             }
-            if (!whole && lane < G) {
-                slot[G * D + lane] = m;
-                slot[G * D + G + lane] = l;
-            }
+            uint32_t rr[16];
+            tc::tmem_ld16(tmem + lane_off + kTcO + 16u * (uint32_t)ob, rr);
+            tc::tc_wait_ld();
             tc::tc_fence_before();
-            mbar_arrive(bar_at(bars, kBOFree + ob));
-            if constexpr (STEP) {
-                if (!whole)
-                    tc_merge_if_last<G>(p.counters, p.partials, p.out, p.Hq, pfx, Hu, U, b, kvh, ntiles, segu, vs, lane);
+            mbar_arrive(bar_at(bars, kBOFree + ob));  // O buffer and stats slot read
+            float o[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) o[h] = __uint_as_float(rr[h]) + __uint_as_float(rr[8 + h]);
+            const int segu = b * Hu + kvh;
+            if (whole) {
+#pragma unroll
+                for (int h = 0; h < G; ++h)
+                    p.out[((size_t)b * p.Hq + kvh * G + h) * D + d] =
+                        __float2bfloat16_rn(l[h] > 0.f ? o[h] * (vs / l[h]) : 0.f);
+            } else {
+                float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
+#pragma unroll
+                for (int h = 0; h < G; ++h) slot[h * D + d] = o[h];
+                if (quad == 0 && lane < G) {
+                    float mh = 0.f, lh = 0.f;
+#pragma unroll
+                    for (int h = 0; h < G; ++h)
+                        if (lane == h) {
+                            mh = m[h];
+                            lh = l[h];
+                        }
+                    slot[G * D + lane] = mh;
+                    slot[G * D + G + lane] = lh;
+                }
+                if constexpr (STEP) {
+                    // every epilogue thread's part of the slot is written (and fenced) before
+                    // the first epilogue warp counts the CTA in
+                    __threadfence();
+                    named_bar(kTcEpiBar, 128);
+                    if (quad == 0)
+                        tc_merge_if_last<G>(p.counters, p.partials, p.out, p.Hq, pfx, Hu, U, b, kvh, ntiles, segu, vs,
+                                            lane);
+                }
             }
             k += piece_len;
         }
@@ -746,7 +749,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
             const int piece_len = min(ntiles - tile, nunits - k);
             const int qslot = piece % kTcQBufs;
-            const uint32_t tO = tmem + kTcO + 128u * (uint32_t)(piece % kTcOBufs);
+            const uint32_t tO = tmem + lane_off + kTcO + 16u * (uint32_t)(piece % kTcOBufs);  // this lane's dim
             // the piece's context length and scales (and q) from the stager
             const bool qok = alive && !*abort_flag &&
                              mbar_wait_bounded(bar_at(bars, kBQFull + qslot), (piece / kTcQBufs) & 1, p.err);
@@ -794,32 +797,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 tc::tc_fence_before();
                 mbar_arrive(bar_at(bars, kBSFree + sb));
-                // per-head maxima of the tile over the 128 tokens
-                float mt[G];
+                // The running max of a head moves only when the tile's maximum exceeds it by
+                // more than 2^8.  One barrier-vote asks whether any token's score does; only then
+                // are the tile maxima reduced (always on a piece's first tile, whose running max
+                // is -inf).  (No second barrier guards `red`: the next write to it follows the
+                // next tile's vote, which every thread reaches after its reads.)
+                bool grow = false;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    float m = sv[h];
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                    mt[h] = m;
-                }
-                if (lane == 0)
-#pragma unroll
-                    for (int h = 0; h < G; ++h) red[8 * sw + h] = mt[h];
-                named_bar(kTcBar, 128);
+                for (int h = 0; h < G; ++h) grow = grow || sv[h] > mref[h] + 8.0f;
                 float alpha[G];
-                bool rescale = false;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float m = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
-                    alpha[h] = 1.f;
-                    if (m > mref[h] + 8.0f) {  // (token 0 of a tile is always valid: m is finite)
-                        alpha[h] = ex2(mref[h] - m);
-                        mref[h] = m;
-                        rescale = rescale || j > 0;
+                for (int h = 0; h < G; ++h) alpha[h] = 1.f;
+                bool rescale = false;
+                if (named_bar_any(kTcBar, 128, grow)) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        float m = sv[h];
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                        if (lane == 0) red[8 * sw + h] = m;
+                    }
+                    named_bar(kTcBar, 128);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float m = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
+                        if (m > mref[h] + 8.0f) {  // (token 0 of a tile is always valid: m is finite)
+                            alpha[h] = ex2(mref[h] - m);
+                            mref[h] = m;
+                            rescale = rescale || j > 0;
+                        }
                     }
                 }
-                named_bar(kTcBar, 128);  // red is rewritten by the next tile
                 float pr[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
@@ -834,35 +842,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 const uint32_t pd = sP + pb * Geo::kP;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    uint32_t hi, lo;  // (only the first of the four codes is used)
-                    tc::split_e4m3x4(pr[h], 0.f, 0.f, 0.f, hi, lo);
-                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(h, t)), "r"(hi & 0xFFu) : "memory");
-                    asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(8 + h, t)), "r"(lo & 0xFFu) : "memory");
+                for (int h0 = 0; h0 < G; h0 += 4) {  // four heads per conversion (G = 2: two)
+                    uint32_t hi, lo;
+                    tc::split_e4m3x4(pr[h0], h0 + 1 < G ? pr[h0 + 1] : 0.f, h0 + 2 < G ? pr[h0 + 2] : 0.f,
+                                     h0 + 3 < G ? pr[h0 + 3] : 0.f, hi, lo);
+#pragma unroll
+                    for (int i = 0; i < 4 && h0 + i < G; ++i) {
+                        const int h = h0 + i;
+                        asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(h, t)), "r"((hi >> (8 * i)) & 0xFFu)
+                                     : "memory");
+                        asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(8 + h, t)),
+                                     "r"((lo >> (8 * i)) & 0xFFu) : "memory");
+                    }
                 }
                 if (rescale && alive) {
-                    // O rows h (TMEM lanes 0..G-1, warp quad 0) times alpha_h, once the
+                    // O^T columns h and 8+h times alpha_h (each thread its dim's lane), once the
                     // PV of the previous tile has finished
                     const int pj = (k - 1) & 1;
                     if (!mbar_wait_bounded(bar_at(bars, kBPvDone + pj), ((k - 1) >> 1) & 1, p.err)) {
                         alive = false;
                         *abort_flag = 1;
                     }
-                    if (quad == 0 && __all_sync(0xffffffffu, alive)) {
+                    if (__all_sync(0xffffffffu, alive)) {
                         tc::tc_fence_after();
-                        float a = 1.f;
+                        uint32_t rr[16];
+                        tc::tmem_ld16(tO, rr);
+                        tc::tc_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < G; ++h)
-                            if (lane == h) a = alpha[h];
-#pragma unroll 1
-                        for (int c0 = 0; c0 < D; c0 += 32) {
-                            uint32_t rr[32];
-                            tc::tmem_ld32(tO + c0, rr);
-                            tc::tc_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * a);
-                            tc::tmem_st32(tO + c0, rr);
+                        for (int h = 0; h < G; ++h) {
+                            rr[h] = __float_as_uint(__uint_as_float(rr[h]) * alpha[h]);
+                            rr[8 + h] = __float_as_uint(__uint_as_float(rr[8 + h]) * alpha[h]);
                         }
+                        tc::tmem_st16(tO, rr);
                         tc::tc_wait_st();
                     }
                 }
@@ -917,7 +928,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc::tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTcCols));
     }
 }
 

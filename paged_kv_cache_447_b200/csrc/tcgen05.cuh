@@ -27,6 +27,9 @@ __host__ __device__ constexpr uint32_t mma_idesc(int M, int N, bool b_mn_major, 
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction-descriptor bit that reads A MN-major (M contiguous) instead of K-major.
+constexpr uint32_t kIdescAMnMajor = 1u << 15;
+
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                        uint32_t accum) {
     asm volatile(
