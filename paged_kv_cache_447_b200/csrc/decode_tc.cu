@@ -37,10 +37,10 @@
 // S^T and PV are issued by two threads, each waiting only for its own inputs (S^T: tile
 // landed, S buffer free, the piece's q staged; PV: P written, O buffer free), so a stage goes
 // back to the producer as soon as its PV completes, and S^T of later tiles runs ahead.  They
-// touch disjoint TMEM columns and shared memory.  S and P are double-buffered, q has 4
-// buffers and O three (by piece), so neither the next piece's q nor the last pieces' epilogues
-// holds up the tiles.  TMEM: S^T at columns 0 and 16, O^T buffers at 32, 48 and 64 (128 lanes
-// x 16 columns each).
+// touch disjoint TMEM columns and shared memory.  S and P have four buffers each (so neither
+// MMA's round trip stalls the softmax), q eight and O three (by piece), so neither the next
+// pieces' q nor the last pieces' epilogues holds up the tiles.  TMEM: S^T at columns 0, 16, 32
+// and 48, O^T buffers at 64, 80 and 96 (128 lanes x 16 columns each).
 #include "decode_kernel.cuh"
 #include "tcgen05.cuh"
 
@@ -55,11 +55,13 @@ constexpr int kTcEpiWarp = 8;   // the epilogue: warps 8-11, one per TMEM lane q
 constexpr int kTcEpiBar = 2;    // named barrier of the 128 epilogue threads
 constexpr int kTcTile = 128;    // tokens per unit
 constexpr int kTcStages = 5;
-constexpr int kTcQBufs = 4;     // q buffers: the stager runs up to this many pieces ahead
+constexpr int kTcQBufs = 8;     // q buffers: the stagers run up to this many pieces ahead
+constexpr int kTcSBufs = 4;     // S^T buffers in TMEM (16 columns each)
+constexpr int kTcPBufs = 4;     // P tiles in shared memory (2 KB each)
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
-constexpr uint32_t kTcO = 32;   // TMEM column of O^T buffer 0 (buffers 1, 2 follow at +16, +32)
-constexpr uint32_t kTcCols = 128;  // TMEM columns allocated (a power of two >= 32 + 16 * kTcOBufs)
+constexpr uint32_t kTcO = 16 * kTcSBufs;  // TMEM column of O^T buffer 0 (the others follow, 16 apart)
+constexpr uint32_t kTcCols = 128;  // TMEM columns allocated (a power of two >= kTcO + 16 * kTcOBufs)
 constexpr int kTcOBufs = 3;     // O buffers (and stats slots): the epilogue may lag two pieces
 
 // What the q stager knows of a piece, for the softmax warps.
@@ -89,13 +91,13 @@ struct TcGeo {
     static constexpr int kP = 16 * 128;
     static constexpr int kOffQ = kTcStages * kStage;
     static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
-    static constexpr int kOffRed = kOffP + 2 * kP;          // [4 warps][8] floats x 2 (max, sum)
+    static constexpr int kOffRed = kOffP + kTcPBufs * kP;   // [4 warps][8] floats x 2 (max, sum)
     static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [kTcOBufs] TcStats
     static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
     static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [kTcStagers] rotated bf16 q [8][128]
     static constexpr int kOffBar = kOffQtmp + kTcStagers * 8 * 128 * 2;
-    static constexpr int kBars = 2 * kTcStages + 2 * kTcQBufs + 18;
+    static constexpr int kBars = 2 * kTcStages + 2 * kTcSBufs + 2 * kTcPBufs + 2 * kTcQBufs + 3 * kTcOBufs + 1;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
     static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
@@ -104,17 +106,17 @@ struct TcGeo {
 // Barrier indices (8 bytes each after kOffBar)
 constexpr int kBFull = 0;                   // [kTcStages]  K/V landed (TMA bytes)
 constexpr int kBEmpty = kTcStages;          // [kTcStages]  K/V consumed (PV commit)
-constexpr int kBSFull = 2 * kTcStages;      // [2] S^T in TMEM (commit)
-constexpr int kBSFree = kBSFull + 2;        // [2] softmax has read S^T (128 arrivals)
-constexpr int kBPFull = kBSFree + 2;        // [2] P tile written (128 arrivals)
-constexpr int kBPvDone = kBPFull + 2;       // [2] PV done reading P buffer (commit)
-constexpr int kBQFull = kBPvDone + 2;       // [kTcQBufs] q staged (stager)
+constexpr int kBSFull = 2 * kTcStages;           // [kTcSBufs] S^T in TMEM (commit)
+constexpr int kBSFree = kBSFull + kTcSBufs;      // [kTcSBufs] softmax has read S^T (128 arrivals)
+constexpr int kBPFull = kBSFree + kTcSBufs;      // [kTcPBufs] P tile written (128 arrivals)
+constexpr int kBPvDone = kBPFull + kTcPBufs;     // [kTcPBufs] PV done reading P buffer (commit)
+constexpr int kBQFull = kBPvDone + kTcPBufs;     // [kTcQBufs] q staged (stager)
 constexpr int kBQEmpty = kBQFull + kTcQBufs;  // [kTcQBufs] q buffer read by its S^T MMAs (softmax)
 constexpr int kBOReady = kBQEmpty + kTcQBufs;  // [kTcOBufs] the piece's last PV has completed (commit)
 constexpr int kBStats = kBOReady + kTcOBufs;   // [kTcOBufs] the piece's (m, l) written (softmax)
 constexpr int kBOFree = kBStats + kTcOBufs;    // [kTcOBufs] O buffer and stats read by the epilogue (32 arrivals)
 constexpr int kBDrain = kBOFree + kTcOBufs;    // every MMA of the CTA has completed (2 commits)
-static_assert(kBDrain < 2 * kTcStages + 2 * kTcQBufs + 18, "barrier count");
+static_assert(kBDrain + 1 == TcGeo<8>::kBars, "barrier count");
 
 __device__ __forceinline__ uint32_t bar_at(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
 
@@ -327,9 +329,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_init(bar_at(bars, kBFull + s), 1);
             mbar_init(bar_at(bars, kBEmpty + s), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kTcSBufs; ++i) {
             mbar_init(bar_at(bars, kBSFull + i), 1);
             mbar_init(bar_at(bars, kBSFree + i), 128);
+        }
+        for (int i = 0; i < kTcPBufs; ++i) {
             mbar_init(bar_at(bars, kBPFull + i), 128);
             mbar_init(bar_at(bars, kBPvDone + i), 1);
         }
@@ -347,7 +351,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fence_mbar_init();
     }
     // zero the q and P operands: the rows no head uses (2G.. of q, 2G.. of P) stay zero
-    for (int i = threadIdx.x; i < (kTcQBufs * Geo::kQ + 2 * Geo::kP) / 16; i += kTcThreads)
+    for (int i = threadIdx.x; i < (kTcQBufs * Geo::kQ + kTcPBufs * Geo::kP) / 16; i += kTcThreads)
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(sQ + 16 * i), "r"(0u) : "memory");
     fence_proxy_async_smem();
     if (warp == 1) {
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM: S^T buffers at columns 0 and 16, O^T buffers at 32, 48, 64 (128 lanes x 16 each)
+    // TMEM: S^T buffers at columns 0..63, O^T buffers at 64..111 (128 lanes x 16 each)
 
     // a bounded wait by lane 0 of the calling warp, its outcome broadcast to the warp (the
     // __syncwarp orders the other lanes' accesses after lane 0's acquire)
@@ -458,7 +462,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 ok = wait0(kBQFull + piece % kTcQBufs, (piece / kTcQBufs) & 1);
             }
             ok = ok && wait0(kBFull + k % kTcStages, (k / kTcStages) & 1) &&
-                 (k < 2 || wait0(kBSFree + (k & 1), ((k - 2) >> 1) & 1));
+                 (k < kTcSBufs || wait0(kBSFree + k % kTcSBufs, ((k - kTcSBufs) / kTcSBufs) & 1));
             if (!ok) break;
             const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
             if constexpr (STEP) {
@@ -482,9 +486,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const uint32_t qd = sQ + (piece % kTcQBufs) * Geo::kQ;
 #pragma unroll
                 for (int kk = 0; kk < D / 32; ++kk)
-                    tc::mma_ss_f8(tmem + 16 * (k & 1), tc::sw128_desc(kd + 32 * kk, 16, 1024),
+                    tc::mma_ss_f8(tmem + 16 * (k % kTcSBufs), tc::sw128_desc(kd + 32 * kk, 16, 1024),
                                   tc::sw128_desc(qd + 32 * kk, 16, 1024), idS, kk > 0);
-                tc::mma_commit(bar_at(bars, kBSFull + (k & 1)));
+                tc::mma_commit(bar_at(bars, kBSFull + k % kTcSBufs));
             }
             __syncwarp();
         }
@@ -503,20 +507,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (first) ++piece;
                 // a piece's first PV overwrites its O buffer: the epilogue of piece - kTcOBufs
                 // must have read it
-                ok = !*abort_flag && mbar_wait_bounded(bar_at(bars, kBPFull + (k & 1)), (k >> 1) & 1, p.err) &&
+                ok = !*abort_flag &&
+                     mbar_wait_bounded(bar_at(bars, kBPFull + k % kTcPBufs), (k / kTcPBufs) & 1, p.err) &&
                      (!first || piece < kTcOBufs ||
                       mbar_wait_bounded(bar_at(bars, kBOFree + piece % kTcOBufs), (piece / kTcOBufs - 1) & 1, p.err));
                 if (!ok) break;
                 tc::tc_fence_after();
                 const uint32_t vd = sStages + (k % kTcStages) * Geo::kStage + Geo::kKV;
-                const uint32_t pd = sP + (k & 1) * Geo::kP;
+                const uint32_t pd = sP + (k % kTcPBufs) * Geo::kP;
                 const uint32_t tO = tmem + kTcO + 16u * (uint32_t)(piece % kTcOBufs);
 #pragma unroll
                 for (int kk = 0; kk < kTcTile / 32; ++kk)  // 32 tokens per MMA
                     tc::mma_ss_f8(tO, tc::sw128_desc(vd + 4096 * kk, 16384, 1024), tc::sw128_desc(pd + 32 * kk, 16, 1024),
                                   idO, (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
-                tc::mma_commit(bar_at(bars, kBPvDone + (k & 1)));
+                tc::mma_commit(bar_at(bars, kBPvDone + k % kTcPBufs));
                 if (last) tc::mma_commit(bar_at(bars, kBOReady + piece % kTcOBufs));
             }
             if (!ok) *abort_flag = 1;
@@ -767,8 +772,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 lsum[h] = 0.f;
             }
             for (int j = 0; j < piece_len; ++j, ++k) {
-                const int sb = k & 1, s = k % kTcStages;
-                bool got = alive && !*abort_flag && mbar_wait_bounded(bar_at(bars, kBSFull + sb), (k >> 1) & 1, p.err);
+                const int sb = k % kTcSBufs, s = k % kTcStages;
+                bool got = alive && !*abort_flag &&
+                           mbar_wait_bounded(bar_at(bars, kBSFull + sb), (k / kTcSBufs) & 1, p.err);
                 if (!__all_sync(0xffffffffu, got)) {
                     alive = false;
                     *abort_flag = 1;
@@ -834,9 +840,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     pr[h] = ex2(sv[h] - mref[h]);
                     lsum[h] = lsum[h] * alpha[h] + pr[h];
                 }
-                // P buffer (k & 1) was last read by the PV of tile k - 2
-                const int pb = k & 1;
-                if (alive && k >= 2 && !mbar_wait_bounded(bar_at(bars, kBPvDone + pb), ((k - 2) >> 1) & 1, p.err)) {
+                // P buffer pb was last read by the PV of tile k - kTcPBufs
+                const int pb = k % kTcPBufs;
+                if (alive && k >= kTcPBufs &&
+                    !mbar_wait_bounded(bar_at(bars, kBPvDone + pb), ((k - kTcPBufs) / kTcPBufs) & 1, p.err)) {
                     alive = false;
                     *abort_flag = 1;
                 }
@@ -858,8 +865,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (rescale && alive) {
                     // O^T columns h and 8+h times alpha_h (each thread its dim's lane), once the
                     // PV of the previous tile has finished
-                    const int pj = (k - 1) & 1;
-                    if (!mbar_wait_bounded(bar_at(bars, kBPvDone + pj), ((k - 1) >> 1) & 1, p.err)) {
+                    const int pj = (k - 1) % kTcPBufs;
+                    if (!mbar_wait_bounded(bar_at(bars, kBPvDone + pj), ((k - 1) / kTcPBufs) & 1, p.err)) {
                         alive = false;
                         *abort_flag = 1;
                     }
