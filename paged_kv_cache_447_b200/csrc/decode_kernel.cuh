@@ -99,6 +99,11 @@ struct DecodeParams {
     const uint16_t *k_new, *v_new;
     void *k_cache_w, *v_cache_w;
     int *counters;
+    // tensor-core decode without the step: one arrival counter per CTA (the segment whose
+    // first piece is that CTA's last), its high 48 bits naming the call (`epoch`), so the
+    // workspace needs no zeroing
+    unsigned long long *ectr = nullptr;
+    unsigned long long epoch = 0;
 };
 
 template <int D, bool FP8, int G, int HPU>

@@ -8,9 +8,10 @@
 // what differs is how the arithmetic reaches the hardware.
 //
 // Work: persistent CTAs (one per SM) split the units -- 128-token tiles of one (sequence,
-// kv head), numbered sequence-major -- into equal contiguous ranges (stream-K); a range's
-// run of tiles of one (sequence, kv head) is a piece with one softmax state, merged with the
-// other pieces of its sequence by the combine kernel exactly as decode_kernel's partials.
+// kv head), numbered sequence-major -- into contiguous ranges of equal cost (stream-K, a
+// segment's first tile costing a little more); a range's run of tiles of one (sequence, kv
+// head) is a piece with one softmax state.  A segment cut by several CTAs is merged, in the
+// combine kernel's arithmetic, by whichever of them finishes its piece last.
 //   warp 0      TMA producer: the tile's K and V rows (8 boxes of 16 rows each, 128-byte
 //               swizzled, straight from the cache; one lane per box) into a 5-stage ring
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
@@ -41,6 +42,8 @@
 // MMA's round trip stalls the softmax), q eight and O three (by piece), so neither the next
 // pieces' q nor the last pieces' epilogues holds up the tiles.  TMEM: S^T at columns 0, 16, 32
 // and 48, O^T buffers at 64, 80 and 96 (128 lanes x 16 columns each).
+#include <random>
+
 #include "decode_kernel.cuh"
 #include "tcgen05.cuh"
 
@@ -103,6 +106,9 @@ struct TcGeo {
     static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
 };
 
+// Shared-memory bytes of the [B + 1] tile prefix (the CTAs' first units follow, 8-byte aligned).
+__host__ __device__ constexpr int tc_pfx_bytes(int B) { return ((B + 1) * 4 + 7) & ~7; }
+
 // Barrier indices (8 bytes each after kOffBar)
 constexpr int kBFull = 0;                   // [kTcStages]  K/V landed (TMA bytes)
 constexpr int kBEmpty = kTcStages;          // [kTcStages]  K/V consumed (PV commit)
@@ -147,6 +153,54 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
     } while (c.b < B && c.nt == 0);
 }
 
+// Cost-balanced split.  A tile costs kTcUnitCost and a (sequence, kv head) segment's first
+// tile kTcPieceCost more (the piece's q, its first tile's full maximum, its epilogue: measured
+// at about two thirds of a tile), so a CTA with many short sequences takes fewer tiles.
+// key(u) = kTcUnitCost * u + kTcPieceCost * (segments starting at or before u) rises by at
+// most kTcUnitCost + kTcPieceCost per unit; CTA c starts at the first unit with key(u) * n >=
+// c * Ctot (Ctot = key past the last unit), so with Ctot >= (kTcUnitCost + kTcPieceCost) * n
+// every CTA gets at least one unit.
+constexpr int kTcUnitCost = 3, kTcPieceCost = 2;
+
+// The first unit whose key reaches thr (0 < thr, thr + kTcUnitCost <= Ctot); ne[b] counts the
+// sequences before b that hold at least one tile.
+__device__ __forceinline__ long long tc_unit_at_key(const int *pfx, const int *ne, int B, int Hu, long long thr) {
+    auto base = [&](int b) {
+        return (long long)Hu * ((long long)kTcUnitCost * pfx[b] + (long long)kTcPieceCost * ne[b]);
+    };
+    int lo = 0, hi = B - 1;  // the first sequence whose last key reaches thr
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (base(mid + 1) >= thr + kTcUnitCost) hi = mid;
+        else lo = mid + 1;
+    }
+    const long long nt = pfx[lo + 1] - pfx[lo];
+    long long u = (long long)Hu * pfx[lo];
+    const long long r = thr - (base(lo) + kTcPieceCost);  // past the sequence's first key
+    if (r > 0) {
+        const long long seg = kTcUnitCost * nt + kTcPieceCost;  // key span of one kv head
+        long long kvh = r / seg, tile = 0;
+        const long long rem = r - kvh * seg;
+        if (rem > 0) {
+            if (rem <= kTcUnitCost * (nt - 1)) tile = (rem + kTcUnitCost - 1) / kTcUnitCost;
+            else ++kvh;  // past this head's last tile: the next head's first
+        }
+        u += kvh * nt + tile;
+    }
+    return u;
+}
+
+// The CTA whose range holds unit u: the last c < n with start[c] <= u.
+__device__ __forceinline__ int tc_owner(const long long *start, int n, long long u) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (start[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
 // Decode step, run by a q stager when a piece ends its sequence: the new token's K (rotated
 // at L - 1 by the RoPE factors rc/rs, when a table is given) and V, quantised to the E4M3
 // code of the exact quotient by the head's scale (as pkv_kv_store does), into cache slot
@@ -179,22 +233,45 @@ __device__ __noinline__ void tc_store_new_token(uint8_t *k_cache, uint8_t *v_cac
     }
 }
 
-// Decode step, run by the epilogue warp after it wrote the partial slot of a piece that is
-// not a whole segment: the CTAs c0..c1 that cut the segment each add one arrival; the last to
+// One arrival on a counter whose high 48 bits name the call and whose low 16 bits count: a
+// count another call left (or whatever the workspace held) gives way to this call's first
+// arrival.  Returns the arrivals so far, this one included (0, with the timeout flag, after
+// a bounded number of lost races).
+__device__ __forceinline__ unsigned tc_arrive_epoch(unsigned long long *ctr, unsigned long long epoch, int *err) {
+    unsigned long long cur = atomicAdd(ctr, 0ull);
+    for (int i = 0; i < (1 << 16); ++i) {
+        const unsigned long long nv = (cur >> 16) == epoch ? cur + 1 : (epoch << 16) | 1ull;
+        const unsigned long long prev = atomicCAS(ctr, cur, nv);
+        if (prev == cur) return (unsigned)(nv & 0xFFFFu);
+        cur = prev;
+    }
+    atomicOr(err, kErrTimeout);
+    return 0;
+}
+
+// Run by the first epilogue warp after the partial slot of a piece that is not a whole
+// segment is written: the CTAs c0..c1 that cut the segment each add one arrival; the last to
 // arrive merges their partials (as the combine kernel does, rounded alike: o / l * v_scale)
-// and clears the counter for the next call.  Out of line: it runs at most twice per CTA (and
-// takes plain values, not the kernel's parameter block, for the reason given above).
-template <int G>
-__device__ __noinline__ void tc_merge_if_last(int *counters, const float *partials, __nv_bfloat16 *out, int Hq,
-                                              const int *pfx, int Hu, long long U, int b, int kvh, int ntiles,
-                                              int segu, float vs, int lane) {
+// and clears the counter for the next call.  The decode step counts on a per-segment counter
+// the caller zeroed once; the plain decode on call-tagged counters, one per CTA (c0's: a
+// CTA's last piece is the first piece of at most one split segment).  Out of line: it runs at
+// most twice per CTA (and takes plain values, not the kernel's parameter block, for the
+// reason given above).
+template <int G, bool EPOCH>
+__device__ __noinline__ void tc_merge_if_last(int *counters, unsigned long long *ectr, unsigned long long epoch,
+                                              int *err, const float *partials, __nv_bfloat16 *out, int Hq,
+                                              const int *pfx, int Hu, const long long *start_of, int n, int b,
+                                              int kvh, int ntiles, int segu, float vs, int lane) {
     constexpr int D = 128;
     __threadfence();
     __syncwarp();
     const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
-    const int c0 = (int)(start / U), c1 = (int)((start + ntiles - 1) / U);
+    const int c0 = tc_owner(start_of, n, start), c1 = tc_owner(start_of, n, start + ntiles - 1);
     int last = 0;
-    if (lane == 0) last = atomicAdd(counters + segu, 1) == c1 - c0;
+    if (lane == 0) {
+        if constexpr (EPOCH) last = tc_arrive_epoch(ectr + c0, epoch, err) == (unsigned)(c1 - c0 + 1);
+        else last = atomicAdd(counters + segu, 1) == c1 - c0;
+    }
     last = __shfl_sync(0xffffffffu, last, 0);
     if (!last) return;
     __threadfence();
@@ -248,7 +325,10 @@ __device__ __noinline__ void tc_merge_if_last(int *counters, const float *partia
         w.y = tc::pack_bf16x2(any ? acc[g].z / ls[g] * vs : 0.f, any ? acc[g].w / ls[g] * vs : 0.f);
         *reinterpret_cast<uint2 *>(out + ((size_t)b * Hq + kvh * G + g) * D + d) = w;
     }
-    if (lane == 0) counters[segu] = 0;
+    if (lane == 0) {
+        if constexpr (EPOCH) atomicExch(ectr + c0, 0ull);
+        else counters[segu] = 0;
+    }
 }
 
 template <int G, bool STEP>
@@ -274,11 +354,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     pdl_wait();
     pdl_trigger();
-    // prefix of the sequences' tile counts (units per sequence and kv head)
+    // prefix of the sequences' tile counts (units per sequence and kv head), and of the
+    // sequences that hold any tile (in the stage ring, free until the producer starts)
+    int *ne = reinterpret_cast<int *>(smem);
     {
-        __shared__ int wsum[kTcThreads / 32];
-        __shared__ int carry_s;
-        if (threadIdx.x == 0) carry_s = 0;
+        __shared__ int wsum[kTcThreads / 32][2];
+        __shared__ int carry_s[2];
+        if (threadIdx.x == 0) carry_s[0] = carry_s[1] = 0;
         __syncthreads();
         for (int base = 0; base < p.B; base += kTcThreads) {
             const int b = base + threadIdx.x;
@@ -292,35 +374,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 v = (L + kTcTile - 1) / kTcTile;
             }
-            int incl = v;
+            const int e = v > 0 ? 1 : 0;
+            int incl = v, incl_e = e;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
+                const int ye = __shfl_up_sync(0xffffffffu, incl_e, o);
+                if (lane >= o) {
+                    incl += y;
+                    incl_e += ye;
+                }
             }
-            if (lane == 31) wsum[warp] = incl;
+            if (lane == 31) {
+                wsum[warp][0] = incl;
+                wsum[warp][1] = incl_e;
+            }
             __syncthreads();
-            int before = carry_s;
-            for (int w = 0; w < warp; ++w) before += wsum[w];
-            if (b < p.B) pfx[b] = before + incl - v;
+            int before = carry_s[0], before_e = carry_s[1];
+            for (int w = 0; w < warp; ++w) {
+                before += wsum[w][0];
+                before_e += wsum[w][1];
+            }
+            if (b < p.B) {
+                pfx[b] = before + incl - v;
+                ne[b] = before_e + incl_e - e;
+            }
             __syncthreads();
-            if (threadIdx.x == kTcThreads - 1) carry_s = before + incl;
+            if (threadIdx.x == kTcThreads - 1) {
+                carry_s[0] = before + incl;
+                carry_s[1] = before_e + incl_e;
+            }
             __syncthreads();
         }
-        if (threadIdx.x == 0) pfx[p.B] = carry_s;
+        if (threadIdx.x == 0) {
+            pfx[p.B] = carry_s[0];
+            ne[p.B] = carry_s[1];
+        }
         __syncthreads();
     }
     const int Hu = p.Hkv;
     const long long total = (long long)Hu * pfx[p.B];
-    if (!STEP && blockIdx.x == 0)
-        for (int i = threadIdx.x; i <= p.B; i += kTcThreads) p.prefix[i] = pfx[i];
+    // every CTA's first unit (start_of[n] = total): cost-balanced where every CTA then gets a
+    // unit, else equal counts (a problem of a few tiles: the last CTAs may get none)
+    long long *start_of = reinterpret_cast<long long *>(smem + Geo::kOffPfx + tc_pfx_bytes(p.B));
+    {
+        const int n = p.nctas;
+        const long long ctot = kTcUnitCost * total + (long long)kTcPieceCost * Hu * ne[p.B];
+        const bool by_cost = ctot >= (long long)(kTcUnitCost + kTcPieceCost) * n;
+        const long long U = total > 0 ? (total + n - 1) / n : 1;
+        for (int c = threadIdx.x; c <= n; c += kTcThreads) {
+            long long u;
+            if (c == 0) u = 0;
+            else if (c == n) u = total;
+            else if (by_cost) u = tc_unit_at_key(pfx, ne, p.B, Hu, ((long long)c * ctot + n - 1) / n);
+            else u = min((long long)c * U, total);
+            start_of[c] = u;
+        }
+        __syncthreads();  // (ne's space is the stage ring's from here on)
+    }
     for (int b = blockIdx.x; b < p.B; b += gridDim.x)
         if (pfx[b + 1] == pfx[b])
             for (int e = threadIdx.x; e < p.Hq * D; e += kTcThreads)
                 p.out[(size_t)b * p.Hq * D + e] = __float2bfloat16_rn(0.f);
-    const long long U = total > 0 ? (total + p.nctas - 1) / p.nctas : 1;
-    const long long u0 = (long long)blockIdx.x * U;
-    const long long u1 = (u0 + U < total) ? u0 + U : total;
+    const long long u0 = start_of[blockIdx.x];
+    const long long u1 = start_of[blockIdx.x + 1];
     if (u0 >= u1) return;  // uniform across the CTA
     const int nunits = (int)(u1 - u0);
 
@@ -728,15 +845,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     slot[G * D + lane] = mh;
                     slot[G * D + G + lane] = lh;
                 }
-                if constexpr (STEP) {
-                    // every epilogue thread's part of the slot is written (and fenced) before
-                    // the first epilogue warp counts the CTA in
-                    __threadfence();
-                    named_bar(kTcEpiBar, 128);
-                    if (quad == 0)
-                        tc_merge_if_last<G>(p.counters, p.partials, p.out, p.Hq, pfx, Hu, U, b, kvh, ntiles, segu, vs,
-                                            lane);
-                }
+                // every epilogue thread's part of the slot is written (and fenced) before the
+                // first epilogue warp counts the CTA in
+                __threadfence();
+                named_bar(kTcEpiBar, 128);
+                if (quad == 0)
+                    tc_merge_if_last<G, !STEP>(p.counters, p.ectr, p.epoch, p.err, p.partials, p.out, p.Hq, pfx, Hu,
+                                               start_of, p.nctas, b, kvh, ntiles, segu, vs, lane);
             }
             k += piece_len;
         }
@@ -939,11 +1054,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 }
 
+// A 48-bit tag per launch, never 0, starting from a per-process random point so that a
+// workspace's leftover contents (another call's or another process's) do not match it.
+unsigned long long next_call_tag() {
+    static std::atomic<unsigned long long> next{[] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 32 | rd()) & ((1ull << 47) - 1);
+    }()};
+    for (;;) {
+        const unsigned long long t = next.fetch_add(1, std::memory_order_relaxed) & ((1ull << 48) - 1);
+        if (t != 0) return t;
+    }
+}
+
 template <int G, bool STEP>
 cudaError_t launch_tc_g(DecodeParams prm, const DecodeArgs &a, int dev, cudaStream_t s) {
     using Geo = TcGeo<G>;
     auto kern = decode_tc_kernel<G, STEP>;
-    const size_t smem = (size_t)Geo::kOffPfx + (size_t)(a.num_seqs + 1) * 4 + 1024;
+    const int nctas = device_sm_count(dev);  // one CTA per SM
+    const size_t smem = (size_t)Geo::kOffPfx + (size_t)tc_pfx_bytes(a.num_seqs) + (size_t)(nctas + 1) * 8 + 1024;
+    // the prologue's second prefix borrows the stage ring
+    if ((size_t)(a.num_seqs + 1) * 4 > (size_t)kTcStages * Geo::kStage) return cudaErrorNotSupported;
     if (smem > (size_t)max_optin_smem(dev) - 2048) return cudaErrorNotSupported;
     static std::atomic<int> attr_smem[kMaxDev];
     static std::mutex attr_mu;
@@ -955,17 +1086,24 @@ cudaError_t launch_tc_g(DecodeParams prm, const DecodeArgs &a, int dev, cudaStre
             attr_smem[dev].store((int)smem, std::memory_order_release);
         }
     }
-    prm.nctas = device_sm_count(dev);  // one CTA per SM
+    prm.nctas = nctas;
+    if (!STEP) {
+        // the call-tagged merge counters, past the partial slots the split can use (one per
+        // (sequence, kv head) plus one per CTA; the workspace holds one more per CTA)
+        const size_t used = (size_t)a.num_seqs * a.n_kv_heads + nctas;
+        const size_t have = (size_t)a.num_seqs * a.n_kv_heads + 2 * (size_t)decode_grid_ctas(nctas);
+        if ((have - used) * (size_t)(G * (128 + 2)) * sizeof(float) < (size_t)nctas * sizeof(unsigned long long))
+            return cudaErrorNotSupported;
+        prm.ectr = reinterpret_cast<unsigned long long *>(prm.partials + used * (size_t)(G * (128 + 2)));
+        prm.epoch = next_call_tag();
+    }
     CUtensorMap tk, tv;
     const uint64_t slots = (uint64_t)a.num_blocks * a.block_size;
     const uint32_t box_rows = a.block_size == 8 ? 8u : 16u;
     if (!encode_tensor_map_3d(&tk, a.k_cache, 1, 128, a.n_kv_heads, slots, 128, 1, box_rows, true) ||
         !encode_tensor_map_3d(&tv, a.v_cache, 1, 128, a.n_kv_heads, slots, 128, 1, box_rows, true))
         return cudaErrorUnknown;
-    cudaError_t e = launch_pdl(kern, dim3(prm.nctas), dim3(kTcThreads), smem, s, tk, tv, prm);
-    if (e != cudaSuccess || STEP) return e;
-    DecodeParams cp = prm;
-    return launch_pdl(combine_kernel<128, G, 1>, dim3(prm.nctas), dim3(128), 0, s, cp);
+    return launch_pdl(kern, dim3(prm.nctas), dim3(kTcThreads), smem, s, tk, tv, prm);
 }
 
 template <bool STEP>
