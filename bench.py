@@ -224,7 +224,7 @@ def timed_kernel(wl, decode: bool) -> str:
     if not decode:
         return "prefill_kernel"
     g = wl.n_q_heads // wl.n_kv_heads
-    if wl.cache_dtype == "fp8" and wl.head_dim == 128 and g in (2, 4, 8):
+    if wl.cache_dtype == "fp8" and wl.head_dim == 128 and g in (2, 4, 8) and wl.n_kv_heads % 2 == 0:
         return "decode_tc_kernel"
     return "decode_kernel"
 

@@ -208,6 +208,56 @@ bool encode_tensor_map_3d_strided(CUtensorMap *map, const void *base, int esize,
     return true;
 }
 
+// 4-D tiled map with explicit byte strides for dims 1..3 (in any order), cached like the
+// 3-D one.
+bool encode_tensor_map_4d_strided(CUtensorMap *map, const void *base, int esize, const uint64_t (&dim)[4],
+                                  const uint64_t (&stride)[3], const uint32_t (&boxdim)[4], bool swizzle128,
+                                  int promo_bytes) {
+    struct Key {
+        const void *base;
+        int esize, promo;
+        uint64_t d[4], s[3];
+        uint32_t b[4];
+        bool swz;
+        bool operator==(const Key &o) const {
+            return base == o.base && esize == o.esize && promo == o.promo && swz == o.swz &&
+                   memcmp(d, o.d, sizeof d) == 0 && memcmp(s, o.s, sizeof s) == 0 &&
+                   memcmp(b, o.b, sizeof b) == 0;
+        }
+    };
+    struct Entry {
+        Key key;
+        CUtensorMap map;
+        bool used;
+    };
+    constexpr int kEntries = 64;
+    thread_local Entry cache[kEntries] = {};
+    thread_local int next = 0;
+    Key key{base, esize, promo_bytes, {dim[0], dim[1], dim[2], dim[3]}, {stride[0], stride[1], stride[2]},
+            {boxdim[0], boxdim[1], boxdim[2], boxdim[3]}, swizzle128};
+    for (int i = 0; i < kEntries; ++i)
+        if (cache[i].used && cache[i].key == key) {
+            *map = cache[i].map;
+            return true;
+        }
+    if (!encoder()) return false;
+    const cuuint64_t dims[4] = {dim[0], dim[1], dim[2], dim[3]};
+    const cuuint64_t strides[3] = {stride[0], stride[1], stride[2]};
+    const cuuint32_t box[4] = {boxdim[0], boxdim[1], boxdim[2], boxdim[3]};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapL2promotion promo = promo_bytes >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                         : promo_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                              : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+    CUresult r = g_encode(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                          4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, promo,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    cache[next] = Entry{key, *map, true};
+    next = (next + 1) % kEntries;
+    return true;
+}
+
 // 3-D tiled map over a row-major [d2, d1, d0] tensor of `esize`-byte elements.  L2 fetches
 // are promoted to one contiguous row at most: a wider promotion would drag in the next
 // head's row of the same slot, which the paged layout does not read next.

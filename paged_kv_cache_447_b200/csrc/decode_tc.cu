@@ -8,40 +8,40 @@
 // what differs is how the arithmetic reaches the hardware.
 //
 // Work: persistent CTAs (one per SM) split the units -- 128-token tiles of one (sequence,
-// kv head), numbered sequence-major -- into contiguous ranges of equal cost (stream-K, a
-// segment's first tile costing a little more); a range's run of tiles of one (sequence, kv
-// head) is a piece with one softmax state.  A segment cut by several CTAs is merged, in the
-// combine kernel's arithmetic, by whichever of them finishes its piece last.
-//   warp 0      TMA producer: the tile's K and V rows (8 boxes of 16 rows each, 128-byte
-//               swizzled, straight from the cache; one lane per box) into a 5-stage ring
+// pair of adjacent kv heads), numbered sequence-major -- into contiguous ranges of equal cost
+// (stream-K, a segment's first tile costing a little more); a range's run of tiles of one
+// segment is a piece with one softmax state per head.  A segment cut by several CTAs is
+// merged, in the combine kernel's arithmetic, by whichever of them finishes its piece last.
+//
+// Why pairs of heads: a TMA box costs the copy engine about the same up to several KB, and
+// one box of 16 tokens of two adjacent heads (their rows sit side by side in the cache) is
+// 4 KB where one head's is 2 KB, so the producer issues half as many boxes per byte.  The
+// cache is read through a 4-D map (dim, slot % 8, head, slot / 8): a box lands as
+// [slot / 8][head][slot % 8][128 bytes], so each head's rows form 8-row, 1024-byte swizzle
+// atoms 2048 bytes apart -- a canonical K-major operand (K) and MN-major operand (V).
+//   warp 0      TMA producer: a tile's K and V boxes (one lane per box) into a 3-stage ring
+//               of 64 KB stages
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
 //   warp 6      lane 0 issues the PV MMAs
 //   warps 7, 12-14  q stagers (piece i to stager i % 4): each piece's q (rotated, scaled,
-//               split), its context length and scales, and (decode step) its new token,
-//               up to 4 pieces ahead
-//   warps 8-11  epilogue, thread = dim: O of a finished piece -> output rows or a partial slot
-// Per tile:
-//   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = the K tile as the
-//                 cache stores it (K-major), B = q as E4M3 rows -- the G heads' high parts in
-//                 rows 0..G-1, their low parts (the E4M3 remainder) in rows G..2G-1, zeros
-//                 after -- so one MMA yields both partial scores of every head in TMEM.
-//   softmax       thread t adds its two parts, masks past the context, takes the per-head
-//                 tile maxima across the four warps, updates the lazy running max (O is
-//                 rescaled only when a max grows by more than 2^8) and writes p as high and
-//                 low E4M3 parts into a shared-memory P tile: row h / 8+h, byte t.
-//   O^T += V^T P^T  M = 128 dims, N = 16, K = 128 tokens: A = the V tile read MN-major as the
-//                 cache stores it, B = the P tile's 16 rows (K-major), so column h of O^T
-//                 gathers the heads' high parts and column 8+h their low parts; the epilogue
-//                 adds the two.  (Taking O transposed keeps the MMA at the 16 columns the
-//                 heads need instead of 64 rows of which G are used.)
-// S^T and PV are issued by two threads, each waiting only for its own inputs (S^T: tile
-// landed, S buffer free, the piece's q staged; PV: P written, O buffer free), so a stage goes
-// back to the producer as soon as its PV completes, and S^T of later tiles runs ahead.  They
-// touch disjoint TMEM columns and shared memory.  S and P have four buffers each (so neither
-// MMA's round trip stalls the softmax), q eight and O three (by piece), so neither the next
-// pieces' q nor the last pieces' epilogues holds up the tiles.  TMEM: S^T at columns 0, 16, 32
-// and 48, O^T buffers at 64, 80 and 96 (128 lanes x 16 columns each).
+//               split), its context length and scales, and (decode step) its new token
+//   warps 8-11  epilogue, thread = dim: O of a finished piece -> output rows or partial slots
+// Per tile, for each head h of the pair:
+//   S^T = K Q^T   M = 128 tokens, N = 16, K = 128 dims (4 MMAs of 32): A = head h's K rows
+//                 as the cache stores them (K-major), B = q as E4M3 rows -- the G heads'
+//                 high parts in rows 0..G-1, their low parts (the E4M3 remainder) in rows
+//                 G..2G-1, zeros after -- so one MMA yields both partial scores of every head.
+//   softmax       thread t adds its two parts, masks past the context, updates the lazy
+//                 running max (O is rescaled only when a max grows by more than 2^8) and
+//                 writes p as high and low E4M3 parts into a shared-memory P tile: row g /
+//                 8+g, byte t.
+//   O^T += V^T P^T  M = 128 dims, N = 16, K = 128 tokens: A = head h's V rows read MN-major,
+//                 B = the P tile's 16 rows (K-major), so column g of O^T gathers the high
+//                 parts and column 8+g the low parts; the epilogue adds the two.
+// S^T and PV are issued by two threads, each waiting only for its own inputs, so a stage goes
+// back to the producer as soon as its PV completes and S^T of later tiles runs ahead.  TMEM:
+// S^T buffers of 32 columns (16 per head) at 0..127, O^T buffers of 32 columns at 128..223.
 #include <random>
 
 #include "decode_kernel.cuh"
@@ -56,53 +56,60 @@ constexpr int kTcStagers = 4;   // q stagers (warps 7, 12, 13, 14): stager i tak
 __device__ __forceinline__ int tc_stager_index(int warp) { return warp == 7 ? 0 : (warp >= 12 ? warp - 11 : -1); }
 constexpr int kTcEpiWarp = 8;   // the epilogue: warps 8-11, one per TMEM lane quarter (O^T rows = dims)
 constexpr int kTcEpiBar = 2;    // named barrier of the 128 epilogue threads
+constexpr int kTcHP = 2;        // kv heads per unit
 constexpr int kTcTile = 128;    // tokens per unit
-constexpr int kTcStages = 5;
-constexpr int kTcQBufs = 8;     // q buffers: the stagers run up to this many pieces ahead
-constexpr int kTcSBufs = 4;     // S^T buffers in TMEM (16 columns each)
-constexpr int kTcPBufs = 4;     // P tiles in shared memory (2 KB each)
+constexpr int kTcStages = 3;    // 64 KB stages
+constexpr int kTcQBufs = 4;     // q buffers: the stagers run up to this many pieces ahead
+constexpr int kTcSBufs = 4;     // S^T buffers in TMEM
+constexpr int kTcPBufs = 2;     // P tiles in shared memory
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
-constexpr uint32_t kTcO = 16 * kTcSBufs;  // TMEM column of O^T buffer 0 (the others follow, 16 apart)
-constexpr uint32_t kTcCols = 128;  // TMEM columns allocated (a power of two >= kTcO + 16 * kTcOBufs)
 constexpr int kTcOBufs = 3;     // O buffers (and stats slots): the epilogue may lag two pieces
+constexpr uint32_t kTcSCols = 16 * kTcHP;             // TMEM columns of one S^T (or O^T) buffer
+constexpr uint32_t kTcO = kTcSCols * kTcSBufs;        // TMEM column of O^T buffer 0
+constexpr uint32_t kTcCols = 256;                     // TMEM columns allocated (a power of two)
+static_assert(kTcO + kTcSCols * kTcOBufs <= kTcCols, "TMEM plan");
 
 // What the q stager knows of a piece, for the softmax warps.
 struct TcMeta {
-    int b, kvh, tile, ntiles, piece_len, L;
-    float sc;  // score scale in exp2 units, over the q scale: scale * log2(e) * k_scale / sq
-    float vs;  // the head's V scale
-    int nt_row;  // decode step: tile row of the new token staged in the slot's codes, or -1
+    int b, hp, tile, ntiles, piece_len, L;
+    float sc[kTcHP];  // score scale in exp2 units, over the q scale: scale * log2(e) * k_scale / sq
+    float vs[kTcHP];  // the heads' V scales
+    int nt_row;       // decode step: tile row of the new token staged in the slot's codes, or -1
+    int pad;
 };
 
-// What the softmax hands the epilogue warp per piece: the piece and its per-head (m, l).
+// What the softmax hands the epilogue per piece: the piece and its per-head (m, l).
 struct TcStats {
-    float m[8], l[8];
-    int b, kvh, ntiles, whole, piece_len;
-    float vs;
-    int pad[2];
+    float m[kTcHP][8], l[kTcHP][8];
+    int b, hp, ntiles, whole, piece_len;
+    float vs[kTcHP];
+    int pad;
 };
 
 template <int G>
 struct TcGeo {
     static constexpr int D = 128;
-    static constexpr int kKV = kTcTile * D;         // one E4M3 K (or V) tile: 16 KB
+    static constexpr int kHead = kTcTile * D;       // one head's E4M3 K (or V) tile: 16 KB
+    static constexpr int kKV = kTcHP * kHead;       // the pair's K (or V): 32 KB
     static constexpr int kStage = 2 * kKV;
-    static constexpr int kQ = 16 * 128;             // B operand of S^T: 16 rows x 128 codes
-    // B operand of PV: p's high parts in rows 0..G-1, its low parts in rows 8..8+G-1, zeros in
-    // the other rows; 16 rows x 128 tokens
-    static constexpr int kP = 16 * 128;
+    static constexpr int kQ1 = 16 * 128;            // B operand of one head's S^T: 16 rows x 128 codes
+    static constexpr int kQ = kTcHP * kQ1;
+    // B operand of one head's PV: p's high parts in rows 0..G-1, its low parts in rows
+    // 8..8+G-1, zeros in the other rows; 16 rows x 128 tokens
+    static constexpr int kP1 = 16 * 128;
+    static constexpr int kP = kTcHP * kP1;
     static constexpr int kOffQ = kTcStages * kStage;
     static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
-    static constexpr int kOffRed = kOffP + kTcPBufs * kP;   // [4 warps][8] floats x 2 (max, sum)
-    static constexpr int kOffStats = kOffRed + 2 * 4 * 8 * 4;              // [kTcOBufs] TcStats
+    static constexpr int kOffRed = kOffP + kTcPBufs * kP;          // [4 warps][16] maxima, then sums
+    static constexpr int kOffStats = kOffRed + 2 * 4 * 16 * 4;     // [kTcOBufs] TcStats
     static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
-    static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);   // [kTcQBufs][256] new-token codes
-    static constexpr int kOffQtmp = kOffNew + kTcQBufs * 256;                   // [kTcStagers] rotated bf16 q [8][128]
-    static constexpr int kOffBar = kOffQtmp + kTcStagers * 8 * 128 * 2;
+    static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);     // [q buffer][head][256] new-token codes
+    static constexpr int kOffBar = kOffNew + kTcQBufs * kTcHP * 256;
     static constexpr int kBars = 2 * kTcStages + 2 * kTcSBufs + 2 * kTcPBufs + 2 * kTcQBufs + 3 * kTcOBufs + 1;
-    static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
+    static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
+    static_assert(kOffBar % 8 == 0 && kOffNew % 16 == 0, "mbarriers and code rows aligned");
     static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
 };
 
@@ -110,18 +117,18 @@ struct TcGeo {
 __host__ __device__ constexpr int tc_pfx_bytes(int B) { return ((B + 1) * 4 + 7) & ~7; }
 
 // Barrier indices (8 bytes each after kOffBar)
-constexpr int kBFull = 0;                   // [kTcStages]  K/V landed (TMA bytes)
-constexpr int kBEmpty = kTcStages;          // [kTcStages]  K/V consumed (PV commit)
+constexpr int kBFull = 0;                        // [kTcStages]  K/V landed (TMA bytes)
+constexpr int kBEmpty = kTcStages;               // [kTcStages]  K/V consumed (PV commit)
 constexpr int kBSFull = 2 * kTcStages;           // [kTcSBufs] S^T in TMEM (commit)
 constexpr int kBSFree = kBSFull + kTcSBufs;      // [kTcSBufs] softmax has read S^T (128 arrivals)
 constexpr int kBPFull = kBSFree + kTcSBufs;      // [kTcPBufs] P tile written (128 arrivals)
 constexpr int kBPvDone = kBPFull + kTcPBufs;     // [kTcPBufs] PV done reading P buffer (commit)
 constexpr int kBQFull = kBPvDone + kTcPBufs;     // [kTcQBufs] q staged (stager)
-constexpr int kBQEmpty = kBQFull + kTcQBufs;  // [kTcQBufs] q buffer read by its S^T MMAs (softmax)
-constexpr int kBOReady = kBQEmpty + kTcQBufs;  // [kTcOBufs] the piece's last PV has completed (commit)
-constexpr int kBStats = kBOReady + kTcOBufs;   // [kTcOBufs] the piece's (m, l) written (softmax)
-constexpr int kBOFree = kBStats + kTcOBufs;    // [kTcOBufs] O buffer and stats read by the epilogue (32 arrivals)
-constexpr int kBDrain = kBOFree + kTcOBufs;    // every MMA of the CTA has completed (2 commits)
+constexpr int kBQEmpty = kBQFull + kTcQBufs;     // [kTcQBufs] q buffer read by its S^T MMAs (softmax)
+constexpr int kBOReady = kBQEmpty + kTcQBufs;    // [kTcOBufs] the piece's last PV has completed (commit)
+constexpr int kBStats = kBOReady + kTcOBufs;     // [kTcOBufs] the piece's (m, l) written (softmax)
+constexpr int kBOFree = kBStats + kTcOBufs;      // [kTcOBufs] O buffer and stats read by the epilogue (128 arrivals)
+constexpr int kBDrain = kBOFree + kTcOBufs;      // every MMA of the CTA has completed (2 commits)
 static_assert(kBDrain + 1 == TcGeo<8>::kBars, "barrier count");
 
 __device__ __forceinline__ uint32_t bar_at(uint32_t base, int i) { return base + 8u * (uint32_t)i; }
@@ -131,35 +138,40 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
     return (uint32_t)(r * 128 + ((((c >> 4) ^ (r & 7)) << 4) | (c & 15)));
 }
 
-// Position of a unit in the walk over (sequence, kv head, tile): the issuers and the
+// Byte c of token t of head h in a stage's K (or V) tile, as the 4-D boxes land it.
+__device__ __forceinline__ uint32_t kv_off(int t, int h, int c) {
+    return (uint32_t)((t >> 3) * 2048 + h * 1024) + sw_off(t & 7, c);
+}
+
+// Position of a unit in the walk over (sequence, head pair, tile): the issuers and the
 // producer's lanes step through their units one by one instead of searching each time.
 struct TcCursor {
-    int b, kvh, tile, nt;
+    int b, hp, tile, nt;
 };
 
-__device__ __forceinline__ TcCursor tc_cursor(const int *pfx, int B, int Hkv, long long u) {
-    const UnitPos up = locate(pfx, B, Hkv, u);
+__device__ __forceinline__ TcCursor tc_cursor(const int *pfx, int B, int Hu, long long u) {
+    const UnitPos up = locate(pfx, B, Hu, u);
     return TcCursor{up.b, up.kvh, up.blk, up.nb};
 }
 
-__device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int Hkv) {
+__device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int Hu) {
     if (++c.tile < c.nt) return;
     c.tile = 0;
-    if (++c.kvh < Hkv) return;
-    c.kvh = 0;
+    if (++c.hp < Hu) return;
+    c.hp = 0;
     do {
         ++c.b;
         c.nt = c.b < B ? pfx[c.b + 1] - pfx[c.b] : 1;
     } while (c.b < B && c.nt == 0);
 }
 
-// Cost-balanced split.  A tile costs kTcUnitCost and a (sequence, kv head) segment's first
-// tile kTcPieceCost more (the piece's q, its first tile's full maximum, its epilogue: measured
-// at about two thirds of a tile), so a CTA with many short sequences takes fewer tiles.
-// key(u) = kTcUnitCost * u + kTcPieceCost * (segments starting at or before u) rises by at
-// most kTcUnitCost + kTcPieceCost per unit; CTA c starts at the first unit with key(u) * n >=
-// c * Ctot (Ctot = key past the last unit), so with Ctot >= (kTcUnitCost + kTcPieceCost) * n
-// every CTA gets at least one unit.
+// Cost-balanced split.  A tile costs kTcUnitCost and a segment's first tile kTcPieceCost more
+// (the piece's q, its first tile's full maximum, its epilogue: measured at about two thirds
+// of a tile), so a CTA with many short sequences takes fewer tiles.  key(u) = kTcUnitCost * u
+// + kTcPieceCost * (segments starting at or before u) rises by at most kTcUnitCost +
+// kTcPieceCost per unit; CTA c starts at the first unit with key(u) * n >= c * Ctot (Ctot =
+// key past the last unit), so with Ctot >= (kTcUnitCost + kTcPieceCost) * n every CTA gets
+// at least one unit.
 constexpr int kTcUnitCost = 3, kTcPieceCost = 2;
 
 // The first unit whose key reaches thr (0 < thr, thr + kTcUnitCost <= Ctot); ne[b] counts the
@@ -178,14 +190,14 @@ __device__ __forceinline__ long long tc_unit_at_key(const int *pfx, const int *n
     long long u = (long long)Hu * pfx[lo];
     const long long r = thr - (base(lo) + kTcPieceCost);  // past the sequence's first key
     if (r > 0) {
-        const long long seg = kTcUnitCost * nt + kTcPieceCost;  // key span of one kv head
-        long long kvh = r / seg, tile = 0;
-        const long long rem = r - kvh * seg;
+        const long long seg = kTcUnitCost * nt + kTcPieceCost;  // key span of one segment
+        long long sg = r / seg, tile = 0;
+        const long long rem = r - sg * seg;
         if (rem > 0) {
             if (rem <= kTcUnitCost * (nt - 1)) tile = (rem + kTcUnitCost - 1) / kTcUnitCost;
-            else ++kvh;  // past this head's last tile: the next head's first
+            else ++sg;  // past this segment's last tile: the next segment's first
         }
-        u += kvh * nt + tile;
+        u += sg * nt + tile;
     }
     return u;
 }
@@ -249,23 +261,25 @@ __device__ __forceinline__ unsigned tc_arrive_epoch(unsigned long long *ctr, uns
     return 0;
 }
 
-// Run by the first epilogue warp after the partial slot of a piece that is not a whole
-// segment is written: the CTAs c0..c1 that cut the segment each add one arrival; the last to
-// arrive merges their partials (as the combine kernel does, rounded alike: o / l * v_scale)
-// and clears the counter for the next call.  The decode step counts on a per-segment counter
-// the caller zeroed once; the plain decode on call-tagged counters, one per CTA (c0's: a
-// CTA's last piece is the first piece of at most one split segment).  Out of line: it runs at
-// most twice per CTA (and takes plain values, not the kernel's parameter block, for the
-// reason given above).
+
+// Run by the first epilogue warp after the partial slots of a piece that is not a whole
+// segment are written: the CTAs c0..c1 that cut the segment each add one arrival; the last to
+// arrive merges their partials, head by head (as the combine kernel does, rounded alike:
+// o / l * v_scale), and clears the counter for the next call.  The decode step counts on a
+// per-segment counter the caller zeroed once; the plain decode on call-tagged counters, one
+// per CTA (c0's: a CTA's last piece is the first piece of at most one split segment).  A
+// segment's partials sit in slots kTcHP * (segment + c) + head.  Out of line: it runs at most
+// twice per CTA (and takes plain values, not the kernel's parameter block, for the reason
+// given above).
 template <int G, bool EPOCH>
 __device__ __noinline__ void tc_merge_if_last(int *counters, unsigned long long *ectr, unsigned long long epoch,
                                               int *err, const float *partials, __nv_bfloat16 *out, int Hq,
                                               const int *pfx, int Hu, const long long *start_of, int n, int b,
-                                              int kvh, int ntiles, int segu, float vs, int lane) {
+                                              int hp, int ntiles, int segu, float vs0, float vs1, int lane) {
     constexpr int D = 128;
     __threadfence();
     __syncwarp();
-    const long long start = (long long)Hu * pfx[b] + (long long)kvh * ntiles;
+    const long long start = (long long)Hu * pfx[b] + (long long)hp * ntiles;
     const int c0 = tc_owner(start_of, n, start), c1 = tc_owner(start_of, n, start + ntiles - 1);
     int last = 0;
     if (lane == 0) {
@@ -279,51 +293,55 @@ __device__ __noinline__ void tc_merge_if_last(int *counters, unsigned long long 
     // / sum e^(m_c - M) l_c, accumulated over c in order (as the combine kernel does); the
     // heads' loads of one CTA slot go out together.
     const int d = 4 * lane;
-    float M[G];
+#pragma unroll 1
+    for (int h = 0; h < kTcHP; ++h) {
+        const float vs = h == 0 ? vs0 : vs1;
+        float M[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) M[g] = -INFINITY;
-    for (int cc = c0; cc <= c1; ++cc) {
-        const float *sl = partials + (size_t)(segu + cc) * (G * (D + 2)) + G * D;
-        float mk[G];
+        for (int g = 0; g < G; ++g) M[g] = -INFINITY;
+        for (int cc = c0; cc <= c1; ++cc) {
+            const float *sl = partials + (size_t)(kTcHP * (segu + cc) + h) * (G * (D + 2)) + G * D;
+            float mk[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) mk[g] = __ldcg(sl + g);
+            for (int g = 0; g < G; ++g) mk[g] = __ldcg(sl + g);
 #pragma unroll
-        for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], mk[g]);
-    }
-    float4 acc[G];
-    float ls[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-        ls[g] = 0.f;
-    }
-    for (int cc = c0; cc <= c1; ++cc) {
-        const float *sl = partials + (size_t)(segu + cc) * (G * (D + 2));
-        float mk[G], lk[G];
-        float4 x[G];
+            for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], mk[g]);
+        }
+        float4 acc[G];
+        float ls[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            mk[g] = __ldcg(sl + G * D + g);
-            lk[g] = __ldcg(sl + G * D + G + g);
-            x[g] = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
+            acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+            ls[g] = 0.f;
+        }
+        for (int cc = c0; cc <= c1; ++cc) {
+            const float *sl = partials + (size_t)(kTcHP * (segu + cc) + h) * (G * (D + 2));
+            float mk[G], lk[G];
+            float4 x[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                mk[g] = __ldcg(sl + G * D + g);
+                lk[g] = __ldcg(sl + G * D + G + g);
+                x[g] = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float f = (mk[g] == -INFINITY) ? 0.f : ex2(mk[g] - M[g]);
+                acc[g].x += f * x[g].x;
+                acc[g].y += f * x[g].y;
+                acc[g].z += f * x[g].z;
+                acc[g].w += f * x[g].w;
+                ls[g] += f * lk[g];
+            }
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const float f = (mk[g] == -INFINITY) ? 0.f : ex2(mk[g] - M[g]);
-            acc[g].x += f * x[g].x;
-            acc[g].y += f * x[g].y;
-            acc[g].z += f * x[g].z;
-            acc[g].w += f * x[g].w;
-            ls[g] += f * lk[g];
+            const bool any = ls[g] > 0.f;
+            uint2 w;
+            w.x = tc::pack_bf16x2(any ? acc[g].x / ls[g] * vs : 0.f, any ? acc[g].y / ls[g] * vs : 0.f);
+            w.y = tc::pack_bf16x2(any ? acc[g].z / ls[g] * vs : 0.f, any ? acc[g].w / ls[g] * vs : 0.f);
+            *reinterpret_cast<uint2 *>(out + ((size_t)b * Hq + (hp * kTcHP + h) * G + g) * D + d) = w;
         }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const bool any = ls[g] > 0.f;
-        uint2 w;
-        w.x = tc::pack_bf16x2(any ? acc[g].x / ls[g] * vs : 0.f, any ? acc[g].y / ls[g] * vs : 0.f);
-        w.y = tc::pack_bf16x2(any ? acc[g].z / ls[g] * vs : 0.f, any ? acc[g].w / ls[g] * vs : 0.f);
-        *reinterpret_cast<uint2 *>(out + ((size_t)b * Hq + kvh * G + g) * D + d) = w;
     }
     if (lane == 0) {
         if constexpr (EPOCH) atomicExch(ectr + c0, 0ull);
@@ -344,8 +362,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float *red = reinterpret_cast<float *>(smem + Geo::kOffRed);
     TcStats *stats = reinterpret_cast<TcStats *>(smem + Geo::kOffStats);  // [O buffer]
     TcMeta *meta = reinterpret_cast<TcMeta *>(smem + Geo::kOffMeta);      // [q buffer]
-    uint8_t *newcodes = smem + Geo::kOffNew;                               // [q buffer][256]
-    uint16_t *qtmp = reinterpret_cast<uint16_t *>(smem + Geo::kOffQtmp);
+    uint8_t *newcodes = smem + Geo::kOffNew;                               // [q buffer][head][256]
     const uint32_t bars = sbase + Geo::kOffBar;
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + Geo::kOffBar + 8 * Geo::kBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Geo::kOffBar + 8 * Geo::kBars + 4);
@@ -412,7 +429,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         __syncthreads();
     }
-    const int Hu = p.Hkv;
+    const int Hu = p.Hkv / kTcHP;  // head pairs
     const long long total = (long long)Hu * pfx[p.B];
     // every CTA's first unit (start_of[n] = total): cost-balanced where every CTA then gets a
     // unit, else equal counts (a problem of a few tiles: the last CTAs may get none)
@@ -467,7 +484,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
     }
-    // zero the q and P operands: the rows no head uses (2G.. of q, 2G.. of P) stay zero
+    // zero the q and P operands: the rows no head uses (2G.. of q, G..7 and 8+G.. of P) stay zero
     for (int i = threadIdx.x; i < (kTcQBufs * Geo::kQ + kTcPBufs * Geo::kP) / 16; i += kTcThreads)
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(sQ + 16 * i), "r"(0u) : "memory");
     fence_proxy_async_smem();
@@ -480,7 +497,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM: S^T buffers at columns 0..63, O^T buffers at 64..111 (128 lanes x 16 each)
+    // TMEM: S^T buffers at columns 0..127, O^T buffers at 128..223 (128 lanes x 32 each: 16 per head)
 
     // a bounded wait by lane 0 of the calling warp, its outcome broadcast to the warp (the
     // __syncwarp orders the other lanes' accesses after lane 0's acquire)
@@ -497,16 +514,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
         }
-        const int oob = (int)(p.num_blocks * p.bs < 0x7fffffffLL ? p.num_blocks * p.bs : 0x7fffffff);
-        // Lanes cover a batch of tiles: lane = tile of the batch * boxes + box, a box being
-        // 16-token piece `bpiece` of the tile (8-token blocks: half `half`, two boxes of 8
-        // rows per piece).  One pass of block-table loads serves the whole batch, and each
-        // box is issued by its own lane.
-        const bool two = p.bs == 8;
-        const int n_box = two ? 16 : 8, tpb = 32 / n_box;
+        // A box is one block's bs tokens (8, 16 or 32) of the pair's two heads; lanes cover a
+        // batch of tiles: lane = tile of the batch * boxes + box.  One pass of block-table
+        // loads serves the whole batch, and each box is issued by its own lane.
+        const int n_box = kTcTile / p.bs, tpb = 32 / n_box;
         const int bt = lane / n_box, bx = lane % n_box;
-        const int half = two ? (bx & 1) : 0, bpiece = two ? (bx >> 1) : bx;
-        const uint32_t box_off = (uint32_t)(bpiece * 2048 + half * 1024);
+        const uint32_t box_off = (uint32_t)(bx * p.bs * 256);
+        // the slot / 8 coordinate just past the cache: the copy engine fills such a box with zeros
+        const int oob = (int)(p.num_blocks * p.bs / 8 < 0x7fffffffLL ? p.num_blocks * p.bs / 8 : 0x7fffffff);
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0 + min(bt, nunits - 1));  // this lane's tile
         // Loads of this lane's block-table entry and context length for the tile k0 + bt;
         // they are issued one batch ahead, so their latency hides behind the waits and
@@ -516,25 +531,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             e = -1;
             L = 0;
             if (k0 + bt < nunits) {
-                const int pc = cur.tile * 8 + bpiece;  // 16-token piece of the sequence
-                const int idx = p.bs == 16 ? pc : (p.bs == 32 ? (pc >> 1) : 2 * pc + half);
+                const int idx = cur.tile * n_box + bx;
                 if (idx < p.max_blocks) e = __ldg(p.block_tables + (size_t)cur.b * p.max_blocks + idx);
                 L = __ldg(p.context_lens + cur.b);
             }
         };
-        auto row_of = [&](int e, int L) -> int {
+        auto coord_of = [&](int e, int L) -> int {
             L = min(L, p.max_tokens);
-            const int pc = cur.tile * 8 + bpiece;
-            const bool inside = p.bs == 8 ? (2 * pc + half) * 8 < L : pc * 16 < L;
-            return inside ? cache_row(p, e, p.bs == 32 ? (pc & 1) * 16 : 0) : oob;
+            if ((cur.tile * n_box + bx) * p.bs >= L) return oob;  // no token of the context
+            if (e < 0 || (long long)e >= p.num_blocks) {
+                atomicOr(p.err, kErrBounds);
+                return oob;
+            }
+            return e * (p.bs / 8);
         };
         int e_cur, L_cur;
         fetch(0, e_cur, L_cur);
         uint32_t issued = 0, phases = 0;
         bool ok = true;
         for (int k0 = 0; k0 < nunits && ok; k0 += tpb) {
-            const int row = k0 + bt < nunits ? row_of(e_cur, L_cur) : oob;
-            const int kvh = cur.kvh;
+            const int co = k0 + bt < nunits ? coord_of(e_cur, L_cur) : oob;
+            const int hp = cur.hp;
             // this lane's tile of the next batch, and its loads
             for (int t = 0; t < tpb; ++t) tc_next(cur, pfx, p.B, Hu);
             fetch(k0 + tpb, e_cur, L_cur);
@@ -556,8 +573,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ok) break;
                 if (bt == t) {
                     const uint32_t dk = sStages + s * Geo::kStage;
-                    tma_load_3d(dk + box_off, &tm_k, fb, 0, kvh, row);
-                    tma_load_3d(dk + Geo::kKV + box_off, &tm_v, fb, 0, kvh, row);
+                    tma_load_4d(dk + box_off, &tm_k, fb, 0, 0, kTcHP * hp, co);
+                    tma_load_4d(dk + Geo::kKV + box_off, &tm_v, fb, 0, 0, kTcHP * hp, co);
                 }
             }
         }
@@ -566,51 +583,58 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if ((issued >> s) & 1) mbar_wait_bounded(bar_at(bars, kBFull + s), (phases >> s) & 1, p.err);
     } else if (warp == 1) {
         // ---------------------------------------------------------------- S^T issuer
-        // Lane 0 issues; the whole warp walks the units (with STEP it stores the step's new
-        // token into the tile before that tile's S^T is issued).
-        constexpr uint32_t idS = tc::mma_idesc(128, 16, false, true);  // E4M3 x E4M3 -> f32
-        bool ok = true;
-        int piece = -1;
-        TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
-        for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
-            const int tile = cur.tile, ntiles = cur.nt;
-            if (k == 0 || tile == 0) {
-                ++piece;
-                ok = wait0(kBQFull + piece % kTcQBufs, (piece / kTcQBufs) & 1);
-            }
-            ok = ok && wait0(kBFull + k % kTcStages, (k / kTcStages) & 1) &&
-                 (k < kTcSBufs || wait0(kBSFree + k % kTcSBufs, ((k - kTcSBufs) / kTcSBufs) & 1));
-            if (!ok) break;
-            const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
-            if constexpr (STEP) {
-                const int qs = piece % kTcQBufs, r = meta[qs].nt_row;
-                if (tile == ntiles - 1 && r >= 0) {
-                    // the sequence's last tile holds its new token: the stager's codes replace
-                    // the slot's previous contents in the K and V rows
-                    if (lane < 16) {
-                        const int c = 16 * (lane & 7);
-                        const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + qs * 256 + (lane >> 3) * D + c);
-                        const uint32_t dst = kd + (lane >> 3) * Geo::kKV + sw_off(r, c);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(x.x), "r"(x.y),
-                                     "r"(x.z), "r"(x.w) : "memory");
-                    }
-                    fence_proxy_async_smem();  // the tensor cores read these rows next
-                    __syncwarp();
+        // Lane 0 alone walks the units and issues (with STEP it first stores the step's new
+        // token into the tile that holds it); the other lanes wait for the TMEM release.
+        if (lane == 0) {
+            constexpr uint32_t idS = tc::mma_idesc(128, 16, false, true);  // E4M3 x E4M3 -> f32
+            bool ok = true;
+            int piece = -1;
+            TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
+            for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
+                const int tile = cur.tile, ntiles = cur.nt;
+                if (k == 0 || tile == 0) {
+                    ++piece;
+                    ok = !*abort_flag &&
+                         mbar_wait_bounded(bar_at(bars, kBQFull + piece % kTcQBufs), (piece / kTcQBufs) & 1, p.err);
                 }
-            }
-            if (lane == 0) {
+                ok = ok && !*abort_flag &&
+                     mbar_wait_bounded(bar_at(bars, kBFull + k % kTcStages), (k / kTcStages) & 1, p.err) &&
+                     (k < kTcSBufs ||
+                      mbar_wait_bounded(bar_at(bars, kBSFree + k % kTcSBufs), ((k - kTcSBufs) / kTcSBufs) & 1, p.err));
+                if (!ok) break;
+                const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
+                if constexpr (STEP) {
+                    const int qs = piece % kTcQBufs, r = meta[qs].nt_row;
+                    if (tile == ntiles - 1 && r >= 0) {
+                        // the sequence's last tile holds its new token: the stager's codes
+                        // replace the slot's previous contents in both heads' K and V rows
+#pragma unroll 1
+                        for (int i = 0; i < 2 * kTcHP * 8; ++i) {
+                            const int h = i >> 4, kv = (i >> 3) & 1, c = 16 * (i & 7);
+                            const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + (qs * kTcHP + h) * 256 +
+                                                                             kv * D + c);
+                            const uint32_t dst = kd + kv * Geo::kKV + kv_off(r, h, c);
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(x.x), "r"(x.y),
+                                         "r"(x.z), "r"(x.w) : "memory");
+                        }
+                        fence_proxy_async_smem();  // the tensor cores read these rows next
+                    }
+                }
                 tc::tc_fence_after();
                 const uint32_t qd = sQ + (piece % kTcQBufs) * Geo::kQ;
 #pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk)
-                    tc::mma_ss_f8(tmem + 16 * (k % kTcSBufs), tc::sw128_desc(kd + 32 * kk, 16, 1024),
-                                  tc::sw128_desc(qd + 32 * kk, 16, 1024), idS, kk > 0);
+                for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        tc::mma_ss_f8(tmem + kTcSCols * (k % kTcSBufs) + 16 * h,
+                                      tc::sw128_desc(kd + 1024 * h + 32 * kk, 16, 2048),
+                                      tc::sw128_desc(qd + Geo::kQ1 * h + 32 * kk, 16, 1024), idS, kk > 0);
                 tc::mma_commit(bar_at(bars, kBSFull + k % kTcSBufs));
             }
-            __syncwarp();
+            if (!ok) *abort_flag = 1;
+            tc::mma_commit(bar_at(bars, kBDrain));  // (with the PV issuer's commit)
         }
-        if (!ok && lane == 0) *abort_flag = 1;
-        if (lane == 0) tc::mma_commit(bar_at(bars, kBDrain));  // (with the PV issuer's commit)
+        __syncwarp();
     } else if (warp == kTcPvWarp) {
         // ---------------------------------------------------------------- PV issuer
         constexpr uint32_t idO = tc::mma_idesc(128, 16, false, true) | tc::kIdescAMnMajor;  // A (V^T) MN-major
@@ -632,11 +656,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::tc_fence_after();
                 const uint32_t vd = sStages + (k % kTcStages) * Geo::kStage + Geo::kKV;
                 const uint32_t pd = sP + (k % kTcPBufs) * Geo::kP;
-                const uint32_t tO = tmem + kTcO + 16u * (uint32_t)(piece % kTcOBufs);
+                const uint32_t tO = tmem + kTcO + kTcSCols * (uint32_t)(piece % kTcOBufs);
 #pragma unroll
-                for (int kk = 0; kk < kTcTile / 32; ++kk)  // 32 tokens per MMA
-                    tc::mma_ss_f8(tO, tc::sw128_desc(vd + 4096 * kk, 16384, 1024), tc::sw128_desc(pd + 32 * kk, 16, 1024),
-                                  idO, (first && kk == 0) ? 0u : 1u);
+                for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                    for (int kk = 0; kk < kTcTile / 32; ++kk)  // 32 tokens per MMA
+                        tc::mma_ss_f8(tO + 16 * h, tc::sw128_desc(vd + 1024 * h + 8192 * kk, 16384, 2048),
+                                      tc::sw128_desc(pd + Geo::kP1 * h + 32 * kk, 16, 1024), idO,
+                                      (first && kk == 0) ? 0u : 1u);
                 tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
                 tc::mma_commit(bar_at(bars, kBPvDone + k % kTcPBufs));
                 if (last) tc::mma_commit(bar_at(bars, kBOReady + piece % kTcOBufs));
@@ -650,16 +677,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (tc_stager_index(warp) >= 0) {
         // ---------------------------------------------------------------- q stagers
         // Four warps take the pieces in turn (piece i to stager i % 4), each into q buffer
-        // piece % kTcQBufs (its own):
-        // the G heads' q rotated at L - 1, scaled by one power of two for the group and split
-        // into high parts (rows 0..G-1) and low parts (rows G..2G-1) as E4M3 codes, plus the
-        // piece's description, and (decode step) the new token of a piece that ends its
-        // sequence.  All loads of a piece go out in one round (the RoPE row serves q and the
-        // new K alike: both rotate at L - 1); the next piece's context length is fetched
-        // while this one is staged.  Run up to kTcQBufs pieces ahead of the softmax.
+        // piece % kTcQBufs: per head of the pair its G q heads rotated at L - 1, scaled by one
+        // power of two and split into high parts (rows 0..G-1) and low parts (rows G..2G-1)
+        // as E4M3 codes, plus the piece's description, and (decode step) the new token of a
+        // piece that ends its sequence.  Lane i holds dims i, i + 32, i + 64, i + 96 of every
+        // q head (the RoPE pairs (i, i + 64) and (i + 32, i + 96)).  All loads of a piece go
+        // out in one round; the next piece's context length is fetched while this one is
+        // staged.
         constexpr int D2 = D / 2;
         const int par = tc_stager_index(warp);
-        uint16_t *qt = qtmp + par * (8 * D);
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
         int k = 0;
         // context length of the next piece this warp stages
@@ -674,7 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         };
         int Lraw = next_own(cur, 0, 0);
         for (int pc = 0; k < nunits; ++pc) {
-            const int b = cur.b, kvh = cur.kvh;
+            const int b = cur.b, hp = cur.hp;
             const int piece_len = min(cur.nt - cur.tile, nunits - k);
             const bool ends = piece_len == cur.nt - cur.tile;  // the piece ends its sequence
             if (pc % kTcStagers == par) {
@@ -682,16 +708,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int L = min(Lraw, p.max_tokens), pos = L - 1;
                 const bool rope_ok = p.rope && pos >= 0 && pos < p.max_pos;
                 if (p.rope && !rope_ok && lane == 0) atomicOr(p.err, kErrBounds);
-                // ---- one round of loads: q pairs (i, i + 64) for i = lane, lane + 32 of every
-                // head, their RoPE factors, the new token's K and V and its block entry
-                uint16_t qx[G][2][2];
+                // ---- one round of loads: every q head's four dims, their RoPE factors, the
+                // new token's K and V and its block entry
+                uint16_t qx[kTcHP][G][4];
 #pragma unroll
-                for (int h = 0; h < G; ++h)
+                for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const uint16_t *qr = p.q + ((size_t)b * p.Hq + kvh * G + h) * D + lane + 32 * j;
-                        qx[h][j][0] = __ldg(qr);
-                        qx[h][j][1] = __ldg(qr + D2);
+                    for (int g = 0; g < G; ++g) {
+                        const uint16_t *qr = p.q + ((size_t)b * p.Hq + (hp * kTcHP + h) * G + g) * D + lane;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) qx[h][g][j] = __ldg(qr + 32 * j);
                     }
                 float rc[2] = {1.f, 1.f}, rs[2] = {0.f, 0.f};
                 if (rope_ok)
@@ -702,25 +728,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                 bool nt_go = false;
                 int nt_e = -1;
-                uint16_t nk[2][2], nv[2][2];
+                uint16_t nk[kTcHP][2][2], nv[kTcHP][2][2];
                 if constexpr (STEP) {
                     // (nothing is stored when the context was clipped to the block table or the
                     // position is outside the RoPE table; a bad block entry is the producer's to flag)
                     nt_go = ends && L == Lraw && L >= 1 && (!p.rope || rope_ok);
                     if (nt_go) {
                         nt_e = __ldg(p.block_tables + (size_t)b * p.max_blocks + pos / p.bs);
-                        const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + kvh) * D;
-                        const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + kvh) * D;
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            nk[j][0] = __ldg(kin + lane + 32 * j);
-                            nk[j][1] = __ldg(kin + lane + 32 * j + D2);
-                            nv[j][0] = __ldg(vin + lane + 32 * j);
-                            nv[j][1] = __ldg(vin + lane + 32 * j + D2);
+                        for (int h = 0; h < kTcHP; ++h) {
+                            const uint16_t *kin = p.k_new + ((size_t)b * p.Hkv + hp * kTcHP + h) * D;
+                            const uint16_t *vin = p.v_new + ((size_t)b * p.Hkv + hp * kTcHP + h) * D;
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                nk[h][j][0] = __ldg(kin + lane + 32 * j);
+                                nk[h][j][1] = __ldg(kin + lane + 32 * j + D2);
+                                nv[h][j][0] = __ldg(vin + lane + 32 * j);
+                                nv[h][j][1] = __ldg(vin + lane + 32 * j + D2);
+                            }
                         }
                     }
                 }
-                const float ksc = __ldg(p.k_scale + kvh), vsc = __ldg(p.v_scale + kvh);
+                float ksc[kTcHP], vsc[kTcHP];
+#pragma unroll
+                for (int h = 0; h < kTcHP; ++h) {
+                    ksc[h] = __ldg(p.k_scale + hp * kTcHP + h);
+                    vsc[h] = __ldg(p.v_scale + hp * kTcHP + h);
+                }
                 // the following piece's context length, while this one is computed
                 TcCursor nc = cur;
                 for (int t = 0; t < piece_len; ++t) tc_next(nc, pfx, p.B, Hu);
@@ -730,40 +764,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (lane == 0) *abort_flag = 1;
                     break;
                 }
-                float amax = 0.f;
+                const uint32_t qd = sQ + slot * Geo::kQ;
+                float sqh[kTcHP];
 #pragma unroll
-                for (int h = 0; h < G; ++h)
+                for (int h = 0; h < kTcHP; ++h) {
+                    float x[G][4];
+                    float amax = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        uint16_t x1 = qx[h][j][0], x2 = qx[h][j][1];
-                        if (rope_ok) rope_pair_fast(x1, x2, rc[j], rs[j], x1, x2);
-                        qt[h * D + lane + 32 * j] = x1;
-                        qt[h * D + lane + 32 * j + D2] = x2;
-                        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float((uint32_t)x1 << 16)),
-                                                 fabsf(__uint_as_float((uint32_t)x2 << 16))));
+                    for (int g = 0; g < G; ++g) {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            uint16_t x1 = qx[h][g][j], x2 = qx[h][g][j + 2];
+                            if (rope_ok) rope_pair_fast(x1, x2, rc[j], rs[j], x1, x2);
+                            x[g][j] = __uint_as_float((uint32_t)x1 << 16);
+                            x[g][j + 2] = __uint_as_float((uint32_t)x2 << 16);
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(x[g][j]));
                     }
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                const float sq = amax > 0.f
-                                     ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
-                                     : 1.f;
-                __syncwarp();  // qt complete
-                const uint32_t qd = sQ + slot * Geo::kQ;
-                for (int e = lane; e < G * (D / 4); e += 32) {  // four dims per lane and step
-                    const int h = e / (D / 4), c = 4 * (e % (D / 4));
-                    const uint2 w = *reinterpret_cast<const uint2 *>(qt + h * D + c);
-                    uint32_t hi, lo;
-                    tc::split_e4m3x4(bf16lo(w.x) * sq, bf16hi(w.x) * sq, bf16lo(w.y) * sq, bf16hi(w.y) * sq, hi,
-                                     lo);
-                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(h, c)), "r"(hi) : "memory");
-                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd + sw_off(G + h, c)), "r"(lo) : "memory");
+                    for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                    const float sq = amax > 0.f
+                                         ? __int_as_float(__float_as_int(fminf(448.f / amax, 0x1p100f)) & 0x7F800000)
+                                         : 1.f;
+                    sqh[h] = sq;
+                    const uint32_t qh = qd + Geo::kQ1 * h;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        uint32_t hi, lo;
+                        tc::split_e4m3x4(x[g][0] * sq, x[g][1] * sq, x[g][2] * sq, x[g][3] * sq, hi, lo);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int c = lane + 32 * j;
+                            asm volatile("st.shared.u8 [%0], %1;" ::"r"(qh + sw_off(g, c)), "r"((hi >> (8 * j)) & 0xFFu)
+                                         : "memory");
+                            asm volatile("st.shared.u8 [%0], %1;" ::"r"(qh + sw_off(G + g, c)),
+                                         "r"((lo >> (8 * j)) & 0xFFu) : "memory");
+                        }
+                    }
                 }
                 int nt_row = -1;
                 if constexpr (STEP) {
                     if (nt_go && nt_e >= 0 && (long long)nt_e < p.num_blocks) {
-                        tc_store_new_token(static_cast<uint8_t *>(p.k_cache_w), static_cast<uint8_t *>(p.v_cache_w), p.Hkv,
-                                           ksc, vsc, p.rope != nullptr, kvh, nt_e * p.bs + pos % p.bs, nk, nv, rc, rs,
-                                           newcodes + slot * 256, lane);
+#pragma unroll 1
+                        for (int h = 0; h < kTcHP; ++h)
+                            tc_store_new_token(static_cast<uint8_t *>(p.k_cache_w), static_cast<uint8_t *>(p.v_cache_w),
+                                               p.Hkv, ksc[h], vsc[h], p.rope != nullptr, hp * kTcHP + h,
+                                               nt_e * p.bs + pos % p.bs, nk[h], nv[h], rc, rs,
+                                               newcodes + (slot * kTcHP + h) * 256, lane);
                         nt_row = pos % kTcTile;
                     }
                 }
@@ -771,16 +819,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     TcMeta &mt = meta[slot];
                     mt.nt_row = nt_row;
                     mt.b = b;
-                    mt.kvh = kvh;
+                    mt.hp = hp;
                     mt.tile = cur.tile;
                     mt.ntiles = cur.nt;
                     mt.piece_len = piece_len;
                     mt.L = L;
-                    mt.sc = p.scale_log2 * ksc / sq;
-                    mt.vs = vsc;
+#pragma unroll
+                    for (int h = 0; h < kTcHP; ++h) {
+                        mt.sc[h] = p.scale_log2 * ksc[h] / sqh[h];
+                        mt.vs[h] = vsc[h];
+                    }
                 }
                 fence_proxy_async_smem();
-                __syncwarp();  // (qt is rewritten by this warp's next piece)
+                __syncwarp();
                 if (lane == 0) mbar_arrive(bar_at(bars, kBQFull + slot));
                 Lraw = Lnext;
             }
@@ -790,8 +841,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp >= kTcEpiWarp && warp < kTcEpiWarp + 4) {
         // ---------------------------------------------------------------- epilogue
         // For each piece in turn, once its last PV has completed and the softmax has left the
-        // piece's description and (m, l): thread = dim d (TMEM lane d of O^T), the heads'
-        // columns h + 8+h -> the output rows (a whole segment) or the piece's partial slot,
+        // piece's description and (m, l): thread = dim d (TMEM lane d of O^T), each head's
+        // columns g + 8+g -> the output rows (a whole segment) or the piece's partial slots,
         // then O buffer free.
         const int quad = warp & 3;
         const int d = quad * 32 + lane;
@@ -807,51 +858,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             tc::tc_fence_after();
             const TcStats &st = stats[ob];
-            const int b = st.b, kvh = st.kvh, ntiles = st.ntiles, piece_len = st.piece_len;
+            const int b = st.b, hp = st.hp, ntiles = st.ntiles, piece_len = st.piece_len;
             const bool whole = st.whole != 0;
-            const float vs = st.vs;
-            float m[G], l[G];
+            float vs[kTcHP], m[kTcHP][G], l[kTcHP][G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                m[h] = st.m[h];
-                l[h] = st.l[h];
+            for (int h = 0; h < kTcHP; ++h) {
+                vs[h] = st.vs[h];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    m[h][g] = st.m[h][g];
+                    l[h][g] = st.l[h][g];
+                }
             }
-            uint32_t rr[16];
-            tc::tmem_ld16(tmem + lane_off + kTcO + 16u * (uint32_t)ob, rr);
+            uint32_t rr[32];
+            tc::tmem_ld32(tmem + lane_off + kTcO + kTcSCols * (uint32_t)ob, rr);
             tc::tc_wait_ld();
             tc::tc_fence_before();
             mbar_arrive(bar_at(bars, kBOFree + ob));  // O buffer and stats slot read
-            float o[G];
+            const int segu = b * Hu + hp;
 #pragma unroll
-            for (int h = 0; h < G; ++h) o[h] = __uint_as_float(rr[h]) + __uint_as_float(rr[8 + h]);
-            const int segu = b * Hu + kvh;
-            if (whole) {
+            for (int h = 0; h < kTcHP; ++h) {
+                float o[G];
 #pragma unroll
-                for (int h = 0; h < G; ++h)
-                    p.out[((size_t)b * p.Hq + kvh * G + h) * D + d] =
-                        __float2bfloat16_rn(l[h] > 0.f ? o[h] * (vs / l[h]) : 0.f);
-            } else {
-                float *slot = p.partials + (size_t)(segu + blockIdx.x) * (G * (D + 2));
+                for (int g = 0; g < G; ++g) o[g] = __uint_as_float(rr[16 * h + g]) + __uint_as_float(rr[16 * h + 8 + g]);
+                if (whole) {
 #pragma unroll
-                for (int h = 0; h < G; ++h) slot[h * D + d] = o[h];
-                if (quad == 0 && lane < G) {
-                    float mh = 0.f, lh = 0.f;
+                    for (int g = 0; g < G; ++g)
+                        p.out[((size_t)b * p.Hq + (hp * kTcHP + h) * G + g) * D + d] =
+                            __float2bfloat16_rn(l[h][g] > 0.f ? o[g] * (vs[h] / l[h][g]) : 0.f);
+                } else {
+                    float *slot = p.partials + (size_t)(kTcHP * (segu + blockIdx.x) + h) * (G * (D + 2));
 #pragma unroll
-                    for (int h = 0; h < G; ++h)
-                        if (lane == h) {
-                            mh = m[h];
-                            lh = l[h];
-                        }
-                    slot[G * D + lane] = mh;
-                    slot[G * D + G + lane] = lh;
+                    for (int g = 0; g < G; ++g) slot[g * D + d] = o[g];
+                    if (quad == 0 && lane < G) {
+                        float mh = 0.f, lh = 0.f;
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            if (lane == g) {
+                                mh = m[h][g];
+                                lh = l[h][g];
+                            }
+                        slot[G * D + lane] = mh;
+                        slot[G * D + G + lane] = lh;
+                    }
                 }
-                // every epilogue thread's part of the slot is written (and fenced) before the
+            }
+            if (!whole) {
+                // every epilogue thread's part of the slots is written (and fenced) before the
                 // first epilogue warp counts the CTA in
                 __threadfence();
                 named_bar(kTcEpiBar, 128);
                 if (quad == 0)
                     tc_merge_if_last<G, !STEP>(p.counters, p.ectr, p.epoch, p.err, p.partials, p.out, p.Hq, pfx, Hu,
-                                               start_of, p.nctas, b, kvh, ntiles, segu, vs, lane);
+                                               start_of, p.nctas, b, hp, ntiles, segu, vs[0], vs[1], lane);
             }
             k += piece_len;
         }
@@ -866,10 +925,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         int k = 0;
         TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
         for (int piece = 0; k < nunits; ++piece) {
-            const int b = cur.b, kvh = cur.kvh, tile = cur.tile, ntiles = cur.nt;
+            const int b = cur.b, hp = cur.hp, tile = cur.tile, ntiles = cur.nt;
             const int piece_len = min(ntiles - tile, nunits - k);
             const int qslot = piece % kTcQBufs;
-            const uint32_t tO = tmem + lane_off + kTcO + 16u * (uint32_t)(piece % kTcOBufs);  // this lane's dim
+            const uint32_t tO = tmem + lane_off + kTcO + kTcSCols * (uint32_t)(piece % kTcOBufs);  // this lane's dim
             // the piece's context length and scales (and q) from the stager
             const bool qok = alive && !*abort_flag &&
                              mbar_wait_bounded(bar_at(bars, kBQFull + qslot), (piece / kTcQBufs) & 1, p.err);
@@ -878,14 +937,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 *abort_flag = 1;
             }
             const int L = alive ? meta[qslot].L : 1;
-            const float sc = alive ? meta[qslot].sc : 0.f;
-            const float vsc = alive ? meta[qslot].vs : 0.f;
-            float mref[G], lsum[G];
+            float sc[kTcHP], vsc[kTcHP];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                mref[h] = -INFINITY;
-                lsum[h] = 0.f;
+            for (int h = 0; h < kTcHP; ++h) {
+                sc[h] = alive ? meta[qslot].sc[h] : 0.f;
+                vsc[h] = alive ? meta[qslot].vs[h] : 0.f;
             }
+            float mref[kTcHP][G], lsum[kTcHP][G];
+#pragma unroll
+            for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    mref[h][g] = -INFINITY;
+                    lsum[h][g] = 0.f;
+                }
             for (int j = 0; j < piece_len; ++j, ++k) {
                 const int sb = k % kTcSBufs, s = k % kTcStages;
                 bool got = alive && !*abort_flag &&
@@ -894,27 +959,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     alive = false;
                     *abort_flag = 1;
                 }
-                float sv[G];
+                float sv[kTcHP][G];
                 if (alive) {
                     tc::tc_fence_after();
-                    uint32_t c[16];
-                    tc::tmem_ld16(tmem + lane_off + 16 * sb, c);
+                    uint32_t c[32];
+                    tc::tmem_ld32(tmem + lane_off + kTcSCols * sb, c);
                     tc::tc_wait_ld();
                     const int valid = min(kTcTile, L - (tile + j) * kTcTile);
 #pragma unroll
-                    for (int h = 0; h < G; ++h)
-                        sv[h] = t < valid ? (__uint_as_float(c[h]) + __uint_as_float(c[G + h])) * sc : -INFINITY;
+                    for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            sv[h][g] = t < valid
+                                           ? (__uint_as_float(c[16 * h + g]) + __uint_as_float(c[16 * h + G + g])) * sc[h]
+                                           : -INFINITY;
                     if (t >= valid) {
                         // V rows past the context would multiply P = 0 by whatever they hold
-                        const uint32_t vrow = sStages + s * Geo::kStage + Geo::kKV + t * 128;
+                        // (the whole 128-byte row of each head: the swizzle only permutes its chunks)
+                        const uint32_t vrow = sStages + s * Geo::kStage + Geo::kKV + (t >> 3) * 2048 + (t & 7) * 128;
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + 16 * q), "r"(0u)
-                                         : "memory");
+                        for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + 1024 * h + 16 * q),
+                                             "r"(0u) : "memory");
                     }
                 } else {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) sv[h] = -INFINITY;
+                    for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                        for (int g = 0; g < G; ++g) sv[h][g] = -INFINITY;
                 }
                 tc::tc_fence_before();
                 mbar_arrive(bar_at(bars, kBSFree + sb));
@@ -925,36 +999,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // next tile's vote, which every thread reaches after its reads.)
                 bool grow = false;
 #pragma unroll
-                for (int h = 0; h < G; ++h) grow = grow || sv[h] > mref[h] + 8.0f;
-                float alpha[G];
+                for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                for (int h = 0; h < G; ++h) alpha[h] = 1.f;
+                    for (int g = 0; g < G; ++g) grow = grow || sv[h][g] > mref[h][g] + 8.0f;
+                float alpha[kTcHP][G];
+#pragma unroll
+                for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) alpha[h][g] = 1.f;
                 bool rescale = false;
                 if (named_bar_any(kTcBar, 128, grow)) {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        float m = sv[h];
+                    for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-                        if (lane == 0) red[8 * sw + h] = m;
-                    }
+                        for (int g = 0; g < G; ++g) {
+                            float m = sv[h][g];
+#pragma unroll
+                            for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                            if (lane == 0) red[16 * sw + 8 * h + g] = m;
+                        }
                     named_bar(kTcBar, 128);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float m = fmaxf(fmaxf(red[h], red[8 + h]), fmaxf(red[16 + h], red[24 + h]));
-                        if (m > mref[h] + 8.0f) {  // (token 0 of a tile is always valid: m is finite)
-                            alpha[h] = ex2(mref[h] - m);
-                            mref[h] = m;
-                            rescale = rescale || j > 0;
-                        }
-                    }
-                }
-                float pr[G];
+                    for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    pr[h] = ex2(sv[h] - mref[h]);
-                    lsum[h] = lsum[h] * alpha[h] + pr[h];
+                        for (int g = 0; g < G; ++g) {
+                            const int i = 8 * h + g;
+                            const float m = fmaxf(fmaxf(red[i], red[16 + i]), fmaxf(red[32 + i], red[48 + i]));
+                            if (m > mref[h][g] + 8.0f) {  // (token 0 of a tile is always valid: m is finite)
+                                alpha[h][g] = ex2(mref[h][g] - m);
+                                mref[h][g] = m;
+                                rescale = rescale || j > 0;
+                            }
+                        }
                 }
+                float pr[kTcHP][G];
+#pragma unroll
+                for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        pr[h][g] = ex2(sv[h][g] - mref[h][g]);
+                        lsum[h][g] = lsum[h][g] * alpha[h][g] + pr[h][g];
+                    }
                 // P buffer pb was last read by the PV of tile k - kTcPBufs
                 const int pb = k % kTcPBufs;
                 if (alive && k >= kTcPBufs &&
@@ -964,22 +1049,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 const uint32_t pd = sP + pb * Geo::kP;
 #pragma unroll
-                for (int h0 = 0; h0 < G; h0 += 4) {  // four heads per conversion (G = 2: two)
-                    uint32_t hi, lo;
-                    tc::split_e4m3x4(pr[h0], h0 + 1 < G ? pr[h0 + 1] : 0.f, h0 + 2 < G ? pr[h0 + 2] : 0.f,
-                                     h0 + 3 < G ? pr[h0 + 3] : 0.f, hi, lo);
+                for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                    for (int i = 0; i < 4 && h0 + i < G; ++i) {
-                        const int h = h0 + i;
-                        asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(h, t)), "r"((hi >> (8 * i)) & 0xFFu)
-                                     : "memory");
-                        asm volatile("st.shared.u8 [%0], %1;" ::"r"(pd + sw_off(8 + h, t)),
-                                     "r"((lo >> (8 * i)) & 0xFFu) : "memory");
+                    for (int g0 = 0; g0 < G; g0 += 4) {  // four heads per conversion (G = 2: two)
+                        uint32_t hi, lo;
+                        tc::split_e4m3x4(pr[h][g0], g0 + 1 < G ? pr[h][g0 + 1] : 0.f, g0 + 2 < G ? pr[h][g0 + 2] : 0.f,
+                                         g0 + 3 < G ? pr[h][g0 + 3] : 0.f, hi, lo);
+#pragma unroll
+                        for (int i = 0; i < 4 && g0 + i < G; ++i) {
+                            const uint32_t ph = pd + Geo::kP1 * h;
+                            asm volatile("st.shared.u8 [%0], %1;" ::"r"(ph + sw_off(g0 + i, t)),
+                                         "r"((hi >> (8 * i)) & 0xFFu) : "memory");
+                            asm volatile("st.shared.u8 [%0], %1;" ::"r"(ph + sw_off(8 + g0 + i, t)),
+                                         "r"((lo >> (8 * i)) & 0xFFu) : "memory");
+                        }
                     }
-                }
                 if (rescale && alive) {
-                    // O^T columns h and 8+h times alpha_h (each thread its dim's lane), once the
-                    // PV of the previous tile has finished
+                    // O^T columns g and 8+g of each head times alpha (each thread its dim's
+                    // lane), once the PV of the previous tile has finished
                     const int pj = (k - 1) % kTcPBufs;
                     if (!mbar_wait_bounded(bar_at(bars, kBPvDone + pj), ((k - 1) / kTcPBufs) & 1, p.err)) {
                         alive = false;
@@ -987,15 +1074,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     }
                     if (__all_sync(0xffffffffu, alive)) {
                         tc::tc_fence_after();
-                        uint32_t rr[16];
-                        tc::tmem_ld16(tO, rr);
+                        uint32_t rr[32];
+                        tc::tmem_ld32(tO, rr);
                         tc::tc_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < G; ++h) {
-                            rr[h] = __float_as_uint(__uint_as_float(rr[h]) * alpha[h]);
-                            rr[8 + h] = __float_as_uint(__uint_as_float(rr[8 + h]) * alpha[h]);
-                        }
-                        tc::tmem_st16(tO, rr);
+                        for (int h = 0; h < kTcHP; ++h)
+#pragma unroll
+                            for (int g = 0; g < G; ++g) {
+                                rr[16 * h + g] = __float_as_uint(__uint_as_float(rr[16 * h + g]) * alpha[h][g]);
+                                rr[16 * h + 8 + g] = __float_as_uint(__uint_as_float(rr[16 * h + 8 + g]) * alpha[h][g]);
+                            }
+                        tc::tmem_st32(tO, rr);
                         tc::tc_wait_st();
                     }
                 }
@@ -1005,14 +1094,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             // q buffer qslot is free: every S^T of the piece has completed (each SFull was waited)
             if (ct == 0) mbar_arrive(bar_at(bars, kBQEmpty + qslot));
-            // ---- end of the piece: its (m, l) per head for the epilogue warp
+            // ---- end of the piece: its (m, l) per head for the epilogue
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float l = lsum[h];
+            for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-                if (lane == 0) red[32 + 8 * sw + h] = l;
-            }
+                for (int g = 0; g < G; ++g) {
+                    float l = lsum[h][g];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+                    if (lane == 0) red[64 + 16 * sw + 8 * h + g] = l;
+                }
             named_bar(kTcBar, 128);
             if (quad == 0) {
                 // the stats slot was last read by the epilogue of piece - kTcOBufs
@@ -1023,21 +1114,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     *abort_flag = 1;
                 }
                 TcStats &st = stats[piece % kTcOBufs];
-                if (lane < G) {
+                if (lane < kTcHP * 8) {
+                    const int h = lane >> 3, g = lane & 7;
                     float m = -INFINITY;
 #pragma unroll
-                    for (int hh = 0; hh < G; ++hh)
-                        if (hh == lane) m = mref[hh];
-                    st.m[lane] = m;
-                    st.l[lane] = red[32 + lane] + red[40 + lane] + red[48 + lane] + red[56 + lane];
+                    for (int hh = 0; hh < kTcHP; ++hh)
+#pragma unroll
+                        for (int gg = 0; gg < G; ++gg)
+                            if (hh == h && gg == g) m = mref[hh][gg];
+                    const int i = 8 * h + g;
+                    st.m[h][g] = m;
+                    st.l[h][g] = red[64 + i] + red[80 + i] + red[96 + i] + red[112 + i];
                 }
                 if (lane == 0) {
                     st.b = b;
-                    st.kvh = kvh;
+                    st.hp = hp;
                     st.ntiles = ntiles;
                     st.whole = tile == 0 && piece_len == ntiles;
                     st.piece_len = piece_len;
-                    st.vs = vsc;
+#pragma unroll
+                    for (int h = 0; h < kTcHP; ++h) st.vs[h] = vsc[h];
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_at(bars, kBStats + piece % kTcOBufs));
@@ -1052,6 +1148,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc::tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTcCols));
     }
+}
+
+// Dynamic shared memory of a launch over B sequences on n CTAs, and whether it fits the
+// device (the prologue's second prefix borrows the stage ring, so B + 1 ints must fit there).
+size_t tc_smem_bytes(int B, int n) {
+    return (size_t)TcGeo<8>::kOffPfx + (size_t)tc_pfx_bytes(B) + (size_t)(n + 1) * 8 + 1024;
+}
+
+bool tc_fits(int B, int dev) {
+    return (size_t)(B + 1) * 4 <= (size_t)kTcStages * TcGeo<8>::kStage &&
+           tc_smem_bytes(B, device_sm_count(dev)) <= (size_t)max_optin_smem(dev) - 2048;
 }
 
 // A 48-bit tag per launch, never 0, starting from a per-process random point so that a
@@ -1072,10 +1179,8 @@ cudaError_t launch_tc_g(DecodeParams prm, const DecodeArgs &a, int dev, cudaStre
     using Geo = TcGeo<G>;
     auto kern = decode_tc_kernel<G, STEP>;
     const int nctas = device_sm_count(dev);  // one CTA per SM
-    const size_t smem = (size_t)Geo::kOffPfx + (size_t)tc_pfx_bytes(a.num_seqs) + (size_t)(nctas + 1) * 8 + 1024;
-    // the prologue's second prefix borrows the stage ring
-    if ((size_t)(a.num_seqs + 1) * 4 > (size_t)kTcStages * Geo::kStage) return cudaErrorNotSupported;
-    if (smem > (size_t)max_optin_smem(dev) - 2048) return cudaErrorNotSupported;
+    const size_t smem = tc_smem_bytes(a.num_seqs, nctas);
+    if (!tc_fits(a.num_seqs, dev)) return cudaErrorNotSupported;
     static std::atomic<int> attr_smem[kMaxDev];
     static std::mutex attr_mu;
     if ((size_t)attr_smem[dev].load(std::memory_order_acquire) < smem) {
@@ -1089,19 +1194,22 @@ cudaError_t launch_tc_g(DecodeParams prm, const DecodeArgs &a, int dev, cudaStre
     prm.nctas = nctas;
     if (!STEP) {
         // the call-tagged merge counters, past the partial slots the split can use (one per
-        // (sequence, kv head) plus one per CTA; the workspace holds one more per CTA)
-        const size_t used = (size_t)a.num_seqs * a.n_kv_heads + nctas;
+        // (sequence, kv head) plus kTcHP per CTA; the workspace holds at least as many more)
+        const size_t used = (size_t)a.num_seqs * a.n_kv_heads + (size_t)kTcHP * nctas;
         const size_t have = (size_t)a.num_seqs * a.n_kv_heads + 2 * (size_t)decode_grid_ctas(nctas);
         if ((have - used) * (size_t)(G * (128 + 2)) * sizeof(float) < (size_t)nctas * sizeof(unsigned long long))
             return cudaErrorNotSupported;
         prm.ectr = reinterpret_cast<unsigned long long *>(prm.partials + used * (size_t)(G * (128 + 2)));
         prm.epoch = next_call_tag();
     }
+    // (dim, slot % 8, head, slot / 8); a box is one block's tokens of two adjacent heads
     CUtensorMap tk, tv;
-    const uint64_t slots = (uint64_t)a.num_blocks * a.block_size;
-    const uint32_t box_rows = a.block_size == 8 ? 8u : 16u;
-    if (!encode_tensor_map_3d(&tk, a.k_cache, 1, 128, a.n_kv_heads, slots, 128, 1, box_rows, true) ||
-        !encode_tensor_map_3d(&tv, a.v_cache, 1, 128, a.n_kv_heads, slots, 128, 1, box_rows, true))
+    const uint64_t hk = (uint64_t)a.n_kv_heads;
+    const uint64_t dims[4] = {128, 8, hk, (uint64_t)a.num_blocks * a.block_size / 8};
+    const uint64_t strides[3] = {hk * 128, 128, 8 * hk * 128};
+    const uint32_t box[4] = {128, 8, (uint32_t)kTcHP, (uint32_t)a.block_size / 8};
+    if (!encode_tensor_map_4d_strided(&tk, a.k_cache, 1, dims, strides, box, true, 256) ||
+        !encode_tensor_map_4d_strided(&tv, a.v_cache, 1, dims, strides, box, true, 256))
         return cudaErrorUnknown;
     return launch_pdl(kern, dim3(prm.nctas), dim3(kTcThreads), smem, s, tk, tv, prm);
 }
@@ -1153,7 +1261,11 @@ cudaError_t dispatch_tc(const DecodeArgs &a, cudaStream_t s) {
 
 bool decode_tc_supported(const DecodeArgs &a) {
     const int G = a.n_q_heads / a.n_kv_heads;
-    return a.fp8 && a.head_dim == 128 && (G == 2 || G == 4 || G == 8);
+    if (!(a.fp8 && a.head_dim == 128 && (G == 2 || G == 4 || G == 8) && a.n_kv_heads % kTcHP == 0 &&
+          (a.block_size == 8 || a.block_size == 16 || a.block_size == 32)))
+        return false;
+    int dev = 0;
+    return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDev && tc_fits(a.num_seqs, dev);
 }
 
 cudaError_t launch_paged_decode_tc(const DecodeArgs &a, cudaStream_t s) { return dispatch_tc<false>(a, s); }

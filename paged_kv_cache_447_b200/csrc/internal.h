@@ -131,6 +131,11 @@ bool encode_tensor_map_3d_strided(CUtensorMap *map, const void *base, int esize,
                                   uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128,
                                   int promo_bytes);
 
+// 4-D tiled map with explicit byte strides of dims 1..3 (dims in any order) and L2 promotion.
+bool encode_tensor_map_4d_strided(CUtensorMap *map, const void *base, int esize, const uint64_t (&dim)[4],
+                                  const uint64_t (&stride)[3], const uint32_t (&boxdim)[4], bool swizzle128,
+                                  int promo_bytes);
+
 cudaError_t launch_kv_store(const StoreArgs &a, cudaStream_t s);
 cudaError_t launch_rope_apply(const RopeArgs &a, cudaStream_t s);
 // Returns cudaErrorInvalidValue if the workspace is too small.
