@@ -19,8 +19,10 @@
 // cache is read through a 4-D map (dim, slot % 8, head, slot / 8): a box lands as
 // [slot / 8][head][slot % 8][128 bytes], so each head's rows form 8-row, 1024-byte swizzle
 // atoms 2048 bytes apart -- a canonical K-major operand (K) and MN-major operand (V).
-//   warp 0      TMA producer: a tile's K and V boxes (one lane per box) into a 3-stage ring
-//               of 64 KB stages
+//   warp 0      TMA producer of K: a tile's K boxes (one lane per box) into a 2-slot ring of
+//               32 KB slots, each freed when its S^T MMAs complete
+//   warp 15     TMA producer of V: the same for V (3 slots), each freed when its PV completes
+//               (K's slots turn over long before V's, so neither waits for the other)
 //   warp 1      TMEM owner; lane 0 issues the S^T MMAs
 //   warps 2-5   128 softmax threads, thread t = token t of the tile = TMEM lane t
 //   warp 6      lane 0 issues the PV MMAs
@@ -39,8 +41,9 @@
 //   O^T += V^T P^T  M = 128 dims, N = 16, K = 128 tokens: A = head h's V rows read MN-major,
 //                 B = the P tile's 16 rows (K-major), so column g of O^T gathers the high
 //                 parts and column 8+g the low parts; the epilogue adds the two.
-// S^T and PV are issued by two threads, each waiting only for its own inputs, so a stage goes
-// back to the producer as soon as its PV completes and S^T of later tiles runs ahead.  TMEM:
+// S^T and PV are issued by two threads, each waiting only for its own inputs, so a K slot goes
+// back to its producer as soon as its S^T completes, a V slot as soon as its PV does, and S^T
+// of later tiles runs ahead.  TMEM:
 // S^T buffers of 32 columns (16 per head) at 0..127, O^T buffers of 32 columns at 128..223.
 #include <random>
 
@@ -50,18 +53,20 @@
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 480;
+constexpr int kTcThreads = 512;
+constexpr int kTcVWarp = 15;    // the V producer
 constexpr int kTcPvWarp = 6;    // the PV issuer
 constexpr int kTcStagers = 4;   // q stagers (warps 7, 12, 13, 14): stager i takes pieces i, i+4, ...
-__device__ __forceinline__ int tc_stager_index(int warp) { return warp == 7 ? 0 : (warp >= 12 ? warp - 11 : -1); }
+__device__ __forceinline__ int tc_stager_index(int warp) { return warp == 7 ? 0 : (warp >= 12 && warp <= 14 ? warp - 11 : -1); }
 constexpr int kTcEpiWarp = 8;   // the epilogue: warps 8-11, one per TMEM lane quarter (O^T rows = dims)
 constexpr int kTcEpiBar = 2;    // named barrier of the 128 epilogue threads
 constexpr int kTcHP = 2;        // kv heads per unit
 constexpr int kTcTile = 128;    // tokens per unit
-constexpr int kTcStages = 3;    // 64 KB stages
-constexpr int kTcQBufs = 4;     // q buffers: the stagers run up to this many pieces ahead
+constexpr int kTcKSlots = 2;    // K ring slots (32 KB each): a K slot is free once its S^T completes
+constexpr int kTcVSlots = 3;    // V ring slots (32 KB each): a V slot is held until its PV completes
+constexpr int kTcQBufs = 8;     // q buffers: the stagers run up to this many pieces ahead
 constexpr int kTcSBufs = 4;     // S^T buffers in TMEM
-constexpr int kTcPBufs = 2;     // P tiles in shared memory
+constexpr int kTcPBufs = 4;     // P tiles in shared memory
 constexpr int kTcSoftmax0 = 2;  // first softmax warp
 constexpr int kTcBar = 1;       // named barrier of the 128 softmax threads
 constexpr int kTcOBufs = 3;     // O buffers (and stats slots): the epilogue may lag two pieces
@@ -69,6 +74,7 @@ constexpr uint32_t kTcSCols = 16 * kTcHP;             // TMEM columns of one S^T
 constexpr uint32_t kTcO = kTcSCols * kTcSBufs;        // TMEM column of O^T buffer 0
 constexpr uint32_t kTcCols = 256;                     // TMEM columns allocated (a power of two)
 static_assert(kTcO + kTcSCols * kTcOBufs <= kTcCols, "TMEM plan");
+static_assert(kTcPBufs >= kTcVSlots, "the softmax's V wait reads PvDone of tile k - kTcVSlots");
 
 // What the q stager knows of a piece, for the softmax warps.
 struct TcMeta {
@@ -91,22 +97,22 @@ template <int G>
 struct TcGeo {
     static constexpr int D = 128;
     static constexpr int kHead = kTcTile * D;       // one head's E4M3 K (or V) tile: 16 KB
-    static constexpr int kKV = kTcHP * kHead;       // the pair's K (or V): 32 KB
-    static constexpr int kStage = 2 * kKV;
+    static constexpr int kKV = kTcHP * kHead;       // the pair's K (or V): 32 KB, one ring slot
+    static constexpr int kOffV = kTcKSlots * kKV;   // the V ring follows the K ring
     static constexpr int kQ1 = 16 * 128;            // B operand of one head's S^T: 16 rows x 128 codes
     static constexpr int kQ = kTcHP * kQ1;
     // B operand of one head's PV: p's high parts in rows 0..G-1, its low parts in rows
     // 8..8+G-1, zeros in the other rows; 16 rows x 128 tokens
     static constexpr int kP1 = 16 * 128;
     static constexpr int kP = kTcHP * kP1;
-    static constexpr int kOffQ = kTcStages * kStage;
+    static constexpr int kOffQ = (kTcKSlots + kTcVSlots) * kKV;
     static constexpr int kOffP = kOffQ + kTcQBufs * kQ;
     static constexpr int kOffRed = kOffP + kTcPBufs * kP;          // [4 warps][16] maxima, then sums
     static constexpr int kOffStats = kOffRed + 2 * 4 * 16 * 4;     // [kTcOBufs] TcStats
     static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);     // [q buffer][head][256] new-token codes
     static constexpr int kOffBar = kOffNew + kTcQBufs * kTcHP * 256;
-    static constexpr int kBars = 2 * kTcStages + 2 * kTcSBufs + 2 * kTcPBufs + 2 * kTcQBufs + 3 * kTcOBufs + 1;
+    static constexpr int kBars = 2 * kTcKSlots + 2 * kTcVSlots + 2 * kTcSBufs + 2 * kTcPBufs + 2 * kTcQBufs + 3 * kTcOBufs + 1;
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
     static_assert(kOffBar % 8 == 0 && kOffNew % 16 == 0, "mbarriers and code rows aligned");
@@ -117,9 +123,11 @@ struct TcGeo {
 __host__ __device__ constexpr int tc_pfx_bytes(int B) { return ((B + 1) * 4 + 7) & ~7; }
 
 // Barrier indices (8 bytes each after kOffBar)
-constexpr int kBFull = 0;                        // [kTcStages]  K/V landed (TMA bytes)
-constexpr int kBEmpty = kTcStages;               // [kTcStages]  K/V consumed (PV commit)
-constexpr int kBSFull = 2 * kTcStages;           // [kTcSBufs] S^T in TMEM (commit)
+constexpr int kBKFull = 0;                       // [kTcKSlots]  K landed (TMA bytes)
+constexpr int kBKEmpty = kTcKSlots;              // [kTcKSlots]  K consumed (S^T commit)
+constexpr int kBVFull = 2 * kTcKSlots;           // [kTcVSlots]  V landed (TMA bytes)
+constexpr int kBVEmpty = kBVFull + kTcVSlots;    // [kTcVSlots]  V consumed (PV commit)
+constexpr int kBSFull = kBVEmpty + kTcVSlots;    // [kTcSBufs] S^T in TMEM (commit)
 constexpr int kBSFree = kBSFull + kTcSBufs;      // [kTcSBufs] softmax has read S^T (128 arrivals)
 constexpr int kBPFull = kBSFree + kTcSBufs;      // [kTcPBufs] P tile written (128 arrivals)
 constexpr int kBPvDone = kBPFull + kTcPBufs;     // [kTcPBufs] PV done reading P buffer (commit)
@@ -166,13 +174,13 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
 }
 
 // Cost-balanced split.  A tile costs kTcUnitCost and a segment's first tile kTcPieceCost more
-// (the piece's q, its first tile's full maximum, its epilogue: measured at about two thirds
-// of a tile), so a CTA with many short sequences takes fewer tiles.  key(u) = kTcUnitCost * u
+// (the piece's q, its first tile's full maximum, its epilogue: measured at about one tile),
+// so a CTA with many short sequences takes fewer tiles.  key(u) = kTcUnitCost * u
 // + kTcPieceCost * (segments starting at or before u) rises by at most kTcUnitCost +
 // kTcPieceCost per unit; CTA c starts at the first unit with key(u) * n >= c * Ctot (Ctot =
 // key past the last unit), so with Ctot >= (kTcUnitCost + kTcPieceCost) * n every CTA gets
 // at least one unit.
-constexpr int kTcUnitCost = 3, kTcPieceCost = 2;
+constexpr int kTcUnitCost = 1, kTcPieceCost = 1;
 
 // The first unit whose key reaches thr (0 < thr, thr + kTcUnitCost <= Ctot); ne[b] counts the
 // sequences before b that hold at least one tile.
@@ -291,56 +299,75 @@ __device__ __noinline__ void tc_merge_if_last(int *counters, unsigned long long 
     __threadfence();
     // lane: dims 4*lane .. 4*lane+3 of every head g.  M_g = max m_c, o = sum e^(m_c - M) acc_c
     // / sum e^(m_c - M) l_c, accumulated over c in order (as the combine kernel does); the
-    // heads' loads of one CTA slot go out together.
+    // loads of one CTA slot go out together, for both kv heads at once where the registers
+    // allow (G <= 4).
     const int d = 4 * lane;
+    constexpr int NH = G <= 4 ? kTcHP : 1;  // kv heads per pass
 #pragma unroll 1
-    for (int h = 0; h < kTcHP; ++h) {
-        const float vs = h == 0 ? vs0 : vs1;
-        float M[G];
+    for (int h0 = 0; h0 < kTcHP; h0 += NH) {
+        float M[NH][G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) M[g] = -INFINITY;
+        for (int h = 0; h < NH; ++h)
+#pragma unroll
+            for (int g = 0; g < G; ++g) M[h][g] = -INFINITY;
         for (int cc = c0; cc <= c1; ++cc) {
-            const float *sl = partials + (size_t)(kTcHP * (segu + cc) + h) * (G * (D + 2)) + G * D;
-            float mk[G];
+            float mk[NH][G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) mk[g] = __ldcg(sl + g);
+            for (int h = 0; h < NH; ++h) {
+                const float *sl = partials + (size_t)(kTcHP * (segu + cc) + h0 + h) * (G * (D + 2)) + G * D;
 #pragma unroll
-            for (int g = 0; g < G; ++g) M[g] = fmaxf(M[g], mk[g]);
-        }
-        float4 acc[G];
-        float ls[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            acc[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-            ls[g] = 0.f;
-        }
-        for (int cc = c0; cc <= c1; ++cc) {
-            const float *sl = partials + (size_t)(kTcHP * (segu + cc) + h) * (G * (D + 2));
-            float mk[G], lk[G];
-            float4 x[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                mk[g] = __ldcg(sl + G * D + g);
-                lk[g] = __ldcg(sl + G * D + G + g);
-                x[g] = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
+                for (int g = 0; g < G; ++g) mk[h][g] = __ldcg(sl + g);
             }
 #pragma unroll
+            for (int h = 0; h < NH; ++h)
+#pragma unroll
+                for (int g = 0; g < G; ++g) M[h][g] = fmaxf(M[h][g], mk[h][g]);
+        }
+        float4 acc[NH][G];
+        float ls[NH][G];
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+#pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float f = (mk[g] == -INFINITY) ? 0.f : ex2(mk[g] - M[g]);
-                acc[g].x += f * x[g].x;
-                acc[g].y += f * x[g].y;
-                acc[g].z += f * x[g].z;
-                acc[g].w += f * x[g].w;
-                ls[g] += f * lk[g];
+                acc[h][g] = make_float4(0.f, 0.f, 0.f, 0.f);
+                ls[h][g] = 0.f;
             }
+        for (int cc = c0; cc <= c1; ++cc) {
+            float mk[NH][G], lk[NH][G];
+            float4 x[NH][G];
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                const float *sl = partials + (size_t)(kTcHP * (segu + cc) + h0 + h) * (G * (D + 2));
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    mk[h][g] = __ldcg(sl + G * D + g);
+                    lk[h][g] = __ldcg(sl + G * D + G + g);
+                    x[h][g] = __ldcg(reinterpret_cast<const float4 *>(sl + g * D + d));  // (G >= 2: aligned)
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float f = (mk[h][g] == -INFINITY) ? 0.f : ex2(mk[h][g] - M[h][g]);
+                    acc[h][g].x += f * x[h][g].x;
+                    acc[h][g].y += f * x[h][g].y;
+                    acc[h][g].z += f * x[h][g].z;
+                    acc[h][g].w += f * x[h][g].w;
+                    ls[h][g] += f * lk[h][g];
+                }
         }
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const bool any = ls[g] > 0.f;
-            uint2 w;
-            w.x = tc::pack_bf16x2(any ? acc[g].x / ls[g] * vs : 0.f, any ? acc[g].y / ls[g] * vs : 0.f);
-            w.y = tc::pack_bf16x2(any ? acc[g].z / ls[g] * vs : 0.f, any ? acc[g].w / ls[g] * vs : 0.f);
-            *reinterpret_cast<uint2 *>(out + ((size_t)b * Hq + (hp * kTcHP + h) * G + g) * D + d) = w;
+        for (int h = 0; h < NH; ++h) {
+            const float vs = h0 + h == 0 ? vs0 : vs1;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const bool any = ls[h][g] > 0.f;
+                uint2 w;
+                w.x = tc::pack_bf16x2(any ? acc[h][g].x / ls[h][g] * vs : 0.f, any ? acc[h][g].y / ls[h][g] * vs : 0.f);
+                w.y = tc::pack_bf16x2(any ? acc[h][g].z / ls[h][g] * vs : 0.f, any ? acc[h][g].w / ls[h][g] * vs : 0.f);
+                *reinterpret_cast<uint2 *>(out + ((size_t)b * Hq + (hp * kTcHP + h0 + h) * G + g) * D + d) = w;
+            }
         }
     }
     if (lane == 0) {
@@ -459,9 +486,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nunits = (int)(u1 - u0);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcStages; ++s) {
-            mbar_init(bar_at(bars, kBFull + s), 1);
-            mbar_init(bar_at(bars, kBEmpty + s), 1);
+        for (int s = 0; s < kTcKSlots; ++s) {
+            mbar_init(bar_at(bars, kBKFull + s), 1);
+            mbar_init(bar_at(bars, kBKEmpty + s), 1);
+        }
+        for (int s = 0; s < kTcVSlots; ++s) {
+            mbar_init(bar_at(bars, kBVFull + s), 1);
+            mbar_init(bar_at(bars, kBVEmpty + s), 1);
         }
         for (int i = 0; i < kTcSBufs; ++i) {
             mbar_init(bar_at(bars, kBSFull + i), 1);
@@ -508,12 +539,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
     };
 
-    if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-        }
+    if (warp == 0 || warp == kTcVWarp) {
+        // ---------------------------------------------------------------- TMA producers
+        // warp 0 fills the K ring, warp 15 the V ring, each walking every unit
+        const bool is_v = warp == kTcVWarp;
+        const CUtensorMap *tm = is_v ? &tm_v : &tm_k;
+        const uint32_t ring = sStages + (is_v ? Geo::kOffV : 0);
+        const int bfull = is_v ? kBVFull : kBKFull, bempty = is_v ? kBVEmpty : kBKEmpty;
+        const int nslots = is_v ? kTcVSlots : kTcKSlots;
+        if (lane == 0) prefetch_tmap(tm);
         // A box is one block's bs tokens (8, 16 or 32) of the pair's two heads; lanes cover a
         // batch of tiles: lane = tile of the batch * boxes + box.  One pass of block-table
         // loads serves the whole batch, and each box is issued by its own lane.
@@ -556,31 +590,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int t = 0; t < tpb; ++t) tc_next(cur, pfx, p.B, Hu);
             fetch(k0 + tpb, e_cur, L_cur);
             for (int t = 0; t < tpb && k0 + t < nunits; ++t) {
-                const int k = k0 + t, s = k % kTcStages;
-                const uint32_t fb = bar_at(bars, kBFull + s);
+                const int k = k0 + t, s = k % nslots;
+                const uint32_t fb = bar_at(bars, bfull + s);
                 if (lane == 0) {
                     if (*abort_flag ||
-                        !mbar_wait_bounded(bar_at(bars, kBEmpty + s), ((k / kTcStages) & 1) ^ 1, p.err)) {
+                        !mbar_wait_bounded(bar_at(bars, bempty + s), ((k / nslots) & 1) ^ 1, p.err)) {
                         ok = false;
                         *abort_flag = 1;
                     } else {
-                        mbar_arrive_expect_tx(fb, Geo::kStage);
+                        mbar_arrive_expect_tx(fb, Geo::kKV);
                         issued |= 1u << s;
-                        phases = (phases & ~(1u << s)) | ((uint32_t)((k / kTcStages) & 1) << s);
+                        phases = (phases & ~(1u << s)) | ((uint32_t)((k / nslots) & 1) << s);
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (!ok) break;
-                if (bt == t) {
-                    const uint32_t dk = sStages + s * Geo::kStage;
-                    tma_load_4d(dk + box_off, &tm_k, fb, 0, 0, kTcHP * hp, co);
-                    tma_load_4d(dk + Geo::kKV + box_off, &tm_v, fb, 0, 0, kTcHP * hp, co);
-                }
+                if (bt == t) tma_load_4d(ring + s * Geo::kKV + box_off, tm, fb, 0, 0, kTcHP * hp, co);
             }
         }
         if (lane == 0)  // never leave with a TMA copy landing in shared memory
-            for (int s = 0; s < kTcStages; ++s)
-                if ((issued >> s) & 1) mbar_wait_bounded(bar_at(bars, kBFull + s), (phases >> s) & 1, p.err);
+            for (int s = 0; s < nslots; ++s)
+                if ((issued >> s) & 1) mbar_wait_bounded(bar_at(bars, bfull + s), (phases >> s) & 1, p.err);
     } else if (warp == 1) {
         // ---------------------------------------------------------------- S^T issuer
         // Lane 0 alone walks the units and issues (with STEP it first stores the step's new
@@ -598,22 +628,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          mbar_wait_bounded(bar_at(bars, kBQFull + piece % kTcQBufs), (piece / kTcQBufs) & 1, p.err);
                 }
                 ok = ok && !*abort_flag &&
-                     mbar_wait_bounded(bar_at(bars, kBFull + k % kTcStages), (k / kTcStages) & 1, p.err) &&
+                     mbar_wait_bounded(bar_at(bars, kBKFull + k % kTcKSlots), (k / kTcKSlots) & 1, p.err) &&
                      (k < kTcSBufs ||
                       mbar_wait_bounded(bar_at(bars, kBSFree + k % kTcSBufs), ((k - kTcSBufs) / kTcSBufs) & 1, p.err));
                 if (!ok) break;
-                const uint32_t kd = sStages + (k % kTcStages) * Geo::kStage;
+                const uint32_t kd = sStages + (k % kTcKSlots) * Geo::kKV;
                 if constexpr (STEP) {
                     const int qs = piece % kTcQBufs, r = meta[qs].nt_row;
                     if (tile == ntiles - 1 && r >= 0) {
                         // the sequence's last tile holds its new token: the stager's codes
-                        // replace the slot's previous contents in both heads' K and V rows
+                        // replace the slot's previous contents in both heads' K rows (the
+                        // softmax patches V once it has landed)
 #pragma unroll 1
-                        for (int i = 0; i < 2 * kTcHP * 8; ++i) {
-                            const int h = i >> 4, kv = (i >> 3) & 1, c = 16 * (i & 7);
-                            const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + (qs * kTcHP + h) * 256 +
-                                                                             kv * D + c);
-                            const uint32_t dst = kd + kv * Geo::kKV + kv_off(r, h, c);
+                        for (int i = 0; i < kTcHP * 8; ++i) {
+                            const int h = i >> 3, c = 16 * (i & 7);
+                            const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + (qs * kTcHP + h) * 256 + c);
+                            const uint32_t dst = kd + kv_off(r, h, c);
                             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(x.x), "r"(x.y),
                                          "r"(x.z), "r"(x.w) : "memory");
                         }
@@ -630,6 +660,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                       tc::sw128_desc(kd + 1024 * h + 32 * kk, 16, 2048),
                                       tc::sw128_desc(qd + Geo::kQ1 * h + 32 * kk, 16, 1024), idS, kk > 0);
                 tc::mma_commit(bar_at(bars, kBSFull + k % kTcSBufs));
+                tc::mma_commit(bar_at(bars, kBKEmpty + k % kTcKSlots));
             }
             if (!ok) *abort_flag = 1;
             tc::mma_commit(bar_at(bars, kBDrain));  // (with the PV issuer's commit)
@@ -650,11 +681,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // must have read it
                 ok = !*abort_flag &&
                      mbar_wait_bounded(bar_at(bars, kBPFull + k % kTcPBufs), (k / kTcPBufs) & 1, p.err) &&
+                     mbar_wait_bounded(bar_at(bars, kBVFull + k % kTcVSlots), (k / kTcVSlots) & 1, p.err) &&
                      (!first || piece < kTcOBufs ||
                       mbar_wait_bounded(bar_at(bars, kBOFree + piece % kTcOBufs), (piece / kTcOBufs - 1) & 1, p.err));
                 if (!ok) break;
                 tc::tc_fence_after();
-                const uint32_t vd = sStages + (k % kTcStages) * Geo::kStage + Geo::kKV;
+                const uint32_t vd = sStages + Geo::kOffV + (k % kTcVSlots) * Geo::kKV;
                 const uint32_t pd = sP + (k % kTcPBufs) * Geo::kP;
                 const uint32_t tO = tmem + kTcO + kTcSCols * (uint32_t)(piece % kTcOBufs);
 #pragma unroll
@@ -664,7 +696,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         tc::mma_ss_f8(tO + 16 * h, tc::sw128_desc(vd + 1024 * h + 8192 * kk, 16384, 2048),
                                       tc::sw128_desc(pd + Geo::kP1 * h + 32 * kk, 16, 1024), idO,
                                       (first && kk == 0) ? 0u : 1u);
-                tc::mma_commit(bar_at(bars, kBEmpty + k % kTcStages));
+                tc::mma_commit(bar_at(bars, kBVEmpty + k % kTcVSlots));
                 tc::mma_commit(bar_at(bars, kBPvDone + k % kTcPBufs));
                 if (last) tc::mma_commit(bar_at(bars, kBOReady + piece % kTcOBufs));
             }
@@ -937,6 +969,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 *abort_flag = 1;
             }
             const int L = alive ? meta[qslot].L : 1;
+            const int nt_row = alive ? meta[qslot].nt_row : -1;  // (decode step) the new token's tile row
             float sc[kTcHP], vsc[kTcHP];
 #pragma unroll
             for (int h = 0; h < kTcHP; ++h) {
@@ -952,7 +985,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     lsum[h][g] = 0.f;
                 }
             for (int j = 0; j < piece_len; ++j, ++k) {
-                const int sb = k % kTcSBufs, s = k % kTcStages;
+                const int sb = k % kTcSBufs, s = k % kTcVSlots;  // (s: the tile's V slot)
                 bool got = alive && !*abort_flag &&
                            mbar_wait_bounded(bar_at(bars, kBSFull + sb), (k / kTcSBufs) & 1, p.err);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -973,16 +1006,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             sv[h][g] = t < valid
                                            ? (__uint_as_float(c[16 * h + g]) + __uint_as_float(c[16 * h + G + g])) * sc[h]
                                            : -INFINITY;
-                    if (t >= valid) {
-                        // V rows past the context would multiply P = 0 by whatever they hold
-                        // (the whole 128-byte row of each head: the swizzle only permutes its chunks)
-                        const uint32_t vrow = sStages + s * Geo::kStage + Geo::kKV + (t >> 3) * 2048 + (t & 7) * 128;
+                    // A tile that ends the context: its V rows past the context would multiply
+                    // P = 0 by whatever they hold, and (decode step) the new token's V codes
+                    // replace its slot's previous contents.  Both wait for the tile's V.
+                    const bool vpatch = STEP && nt_row >= 0 && tile + j == ntiles - 1;
+                    if (valid < kTcTile || vpatch) {
+                        // The softmax may run ahead of the PV MMAs, and V(k) shares its slot with
+                        // V(k - kTcVSlots): that tile's PV must be complete first, or the slot's
+                        // full barrier could still be in the earlier phase, whose parity the
+                        // wait below would take for this one.  (PvDone of that tile's P buffer
+                        // cannot alias either: this thread waited for its previous use at tile
+                        // k - kTcVSlots, and its next use needs a P tile not yet written, since
+                        // kTcPBufs >= kTcVSlots.)
+                        bool vok = !*abort_flag;
+                        if (vok && k >= kTcVSlots)
+                            vok = mbar_wait_bounded(bar_at(bars, kBPvDone + (k - kTcVSlots) % kTcPBufs),
+                                                    ((k - kTcVSlots) / kTcPBufs) & 1, p.err);
+                        vok = vok && mbar_wait_bounded(bar_at(bars, kBVFull + s), (k / kTcVSlots) & 1, p.err);
+                        if (!__all_sync(0xffffffffu, vok)) {
+                            alive = false;
+                            *abort_flag = 1;
+                        }
+                        const uint32_t vslot = sStages + Geo::kOffV + s * Geo::kKV;
+                        if (alive && t >= valid) {
+                            // (the whole 128-byte row of each head: the swizzle only permutes its chunks)
+                            const uint32_t vrow = vslot + (t >> 3) * 2048 + (t & 7) * 128;
 #pragma unroll
-                        for (int h = 0; h < kTcHP; ++h)
+                            for (int h = 0; h < kTcHP; ++h)
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + 1024 * h + 16 * q),
-                                             "r"(0u) : "memory");
+                                for (int q = 0; q < 8; ++q)
+                                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + 1024 * h + 16 * q),
+                                                 "r"(0u) : "memory");
+                        }
+                        if (alive && vpatch && t == nt_row) {
+#pragma unroll 1
+                            for (int i = 0; i < kTcHP * 8; ++i) {
+                                const int h = i >> 3, cc = 16 * (i & 7);
+                                const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + (qslot * kTcHP + h) * 256 +
+                                                                                 D + cc);
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vslot + kv_off(t, h, cc)),
+                                             "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w) : "memory");
+                            }
+                        }
                     }
                 } else {
 #pragma unroll
@@ -1157,7 +1222,7 @@ size_t tc_smem_bytes(int B, int n) {
 }
 
 bool tc_fits(int B, int dev) {
-    return (size_t)(B + 1) * 4 <= (size_t)kTcStages * TcGeo<8>::kStage &&
+    return (size_t)(B + 1) * 4 <= (size_t)TcGeo<8>::kOffQ &&
            tc_smem_bytes(B, device_sm_count(dev)) <= (size_t)max_optin_smem(dev) - 2048;
 }
 
