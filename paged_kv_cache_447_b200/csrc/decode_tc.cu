@@ -74,7 +74,6 @@ constexpr uint32_t kTcSCols = 16 * kTcHP;             // TMEM columns of one S^T
 constexpr uint32_t kTcO = kTcSCols * kTcSBufs;        // TMEM column of O^T buffer 0
 constexpr uint32_t kTcCols = 256;                     // TMEM columns allocated (a power of two)
 static_assert(kTcO + kTcSCols * kTcOBufs <= kTcCols, "TMEM plan");
-static_assert(kTcPBufs >= kTcVSlots, "the softmax's V wait reads PvDone of tile k - kTcVSlots");
 
 // What the q stager knows of a piece, for the softmax warps.
 struct TcMeta {
@@ -111,11 +110,15 @@ struct TcGeo {
     static constexpr int kOffStats = kOffRed + 2 * 4 * 16 * 4;     // [kTcOBufs] TcStats
     static constexpr int kOffMeta = kOffStats + kTcOBufs * (int)sizeof(TcStats);  // [kTcQBufs] TcMeta
     static constexpr int kOffNew = kOffMeta + kTcQBufs * (int)sizeof(TcMeta);     // [q buffer][head][256] new-token codes
-    static constexpr int kOffBar = kOffNew + kTcQBufs * kTcHP * 256;
+    // per P buffer: the tile's valid token count and (decode step) the new token's row, then
+    // its V codes for both heads, handed from the softmax to the PV warp with the P tile
+    static constexpr int kOffPvInfo = kOffNew + kTcQBufs * kTcHP * 256;            // [kTcPBufs] int2
+    static constexpr int kOffPvCodes = kOffPvInfo + kTcPBufs * 8;                   // [kTcPBufs][head][128]
+    static constexpr int kOffBar = kOffPvCodes + kTcPBufs * kTcHP * 128;
     static constexpr int kBars = 2 * kTcKSlots + 2 * kTcVSlots + 2 * kTcSBufs + 2 * kTcPBufs + 2 * kTcQBufs + 3 * kTcOBufs + 1;
     static constexpr int kOffPfx = kOffBar + 8 * kBars + 16;
     static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands on 1024-byte boundaries");
-    static_assert(kOffBar % 8 == 0 && kOffNew % 16 == 0, "mbarriers and code rows aligned");
+    static_assert(kOffBar % 8 == 0 && kOffNew % 16 == 0 && kOffPvCodes % 16 == 0, "mbarriers and code rows aligned");
     static_assert(2 * G <= 16, "q high and low rows fit the 16 rows of the B operand");
 };
 
@@ -174,13 +177,13 @@ __device__ __forceinline__ void tc_next(TcCursor &c, const int *pfx, int B, int 
 }
 
 // Cost-balanced split.  A tile costs kTcUnitCost and a segment's first tile kTcPieceCost more
-// (the piece's q, its first tile's full maximum, its epilogue: measured at about one tile),
+// (the piece's q, its first tile's full maximum, its epilogue: measured at about three tiles),
 // so a CTA with many short sequences takes fewer tiles.  key(u) = kTcUnitCost * u
 // + kTcPieceCost * (segments starting at or before u) rises by at most kTcUnitCost +
 // kTcPieceCost per unit; CTA c starts at the first unit with key(u) * n >= c * Ctot (Ctot =
 // key past the last unit), so with Ctot >= (kTcUnitCost + kTcPieceCost) * n every CTA gets
 // at least one unit.
-constexpr int kTcUnitCost = 1, kTcPieceCost = 1;
+constexpr int kTcUnitCost = 1, kTcPieceCost = 3;
 
 // The first unit whose key reaches thr (0 < thr, thr + kTcUnitCost <= Ctot); ne[b] counts the
 // sequences before b that hold at least one tile.
@@ -669,24 +672,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     } else if (warp == kTcPvWarp) {
         // ---------------------------------------------------------------- PV issuer
         constexpr uint32_t idO = tc::mma_idesc(128, 16, false, true) | tc::kIdescAMnMajor;  // A (V^T) MN-major
-        if (lane == 0) {
-            bool ok = true;
-            int piece = -1;
-            TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
-            for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
-                const bool first = k == 0 || cur.tile == 0;
-                const bool last = k == nunits - 1 || cur.tile == cur.nt - 1;
-                if (first) ++piece;
-                // a piece's first PV overwrites its O buffer: the epilogue of piece - kTcOBufs
-                // must have read it
+        // The warp walks the tiles; lane 0 waits and issues, and for a tile that ends its
+        // context the whole warp first fixes its V rows: the rows of the last block past the
+        // context (those past that block were filled with zeros by the copy engine) and
+        // (decode step) the new token's row.
+        bool ok = true;
+        int piece = -1;
+        TcCursor cur = tc_cursor(pfx, p.B, Hu, u0);
+        for (int k = 0; k < nunits && ok; ++k, tc_next(cur, pfx, p.B, Hu)) {
+            const bool first = k == 0 || cur.tile == 0;
+            const bool last = k == nunits - 1 || cur.tile == cur.nt - 1;
+            if (first) ++piece;
+            // a piece's first PV overwrites its O buffer: the epilogue of piece - kTcOBufs
+            // must have read it
+            if (lane == 0)
                 ok = !*abort_flag &&
                      mbar_wait_bounded(bar_at(bars, kBPFull + k % kTcPBufs), (k / kTcPBufs) & 1, p.err) &&
                      mbar_wait_bounded(bar_at(bars, kBVFull + k % kTcVSlots), (k / kTcVSlots) & 1, p.err) &&
                      (!first || piece < kTcOBufs ||
                       mbar_wait_bounded(bar_at(bars, kBOFree + piece % kTcOBufs), (piece / kTcOBufs - 1) & 1, p.err));
-                if (!ok) break;
+            __syncwarp();
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            const uint32_t vd = sStages + Geo::kOffV + (k % kTcVSlots) * Geo::kKV;
+            const int2 info = *reinterpret_cast<const int2 *>(smem + Geo::kOffPvInfo + 8 * (k % kTcPBufs));
+            if (info.x < kTcTile || info.y >= 0) {
+                const int zend = min(kTcTile, (info.x + p.bs - 1) / p.bs * p.bs);
+                for (int i = lane; i < (zend - info.x) * kTcHP * 8; i += 32) {  // 16 bytes per lane and step
+                    const int r = info.x + i / (kTcHP * 8), h = (i >> 3) % kTcHP, q = i & 7;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vd + (r >> 3) * 2048 + h * 1024 +
+                                                                                   (r & 7) * 128 + 16 * q),
+                                 "r"(0u) : "memory");
+                }
+                if (info.y >= 0 && lane < kTcHP * 8) {
+                    const int h = lane >> 3, cc = 16 * (lane & 7);
+                    const uint4 x = *reinterpret_cast<const uint4 *>(smem + Geo::kOffPvCodes +
+                                                                     (k % kTcPBufs) * (kTcHP * 128) + h * 128 + cc);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vd + kv_off(info.y, h, cc)), "r"(x.x),
+                                 "r"(x.y), "r"(x.z), "r"(x.w) : "memory");
+                }
+                fence_proxy_async_smem();  // the tensor cores read these rows next
+                __syncwarp();
+            }
+            if (lane == 0) {
                 tc::tc_fence_after();
-                const uint32_t vd = sStages + Geo::kOffV + (k % kTcVSlots) * Geo::kKV;
                 const uint32_t pd = sP + (k % kTcPBufs) * Geo::kP;
                 const uint32_t tO = tmem + kTcO + kTcSCols * (uint32_t)(piece % kTcOBufs);
 #pragma unroll
@@ -700,6 +729,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 tc::mma_commit(bar_at(bars, kBPvDone + k % kTcPBufs));
                 if (last) tc::mma_commit(bar_at(bars, kBOReady + piece % kTcOBufs));
             }
+            __syncwarp();
+        }
+        if (lane == 0) {
             if (!ok) *abort_flag = 1;
             // drain: no MMA of either issuer may still write TMEM when it is released
             tc::mma_commit(bar_at(bars, kBDrain));
@@ -993,6 +1025,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     *abort_flag = 1;
                 }
                 float sv[kTcHP][G];
+                int pv_valid = kTcTile, pv_row = -1;  // what the PV warp must fix in this tile's V
                 if (alive) {
                     tc::tc_fence_after();
                     uint32_t c[32];
@@ -1006,49 +1039,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             sv[h][g] = t < valid
                                            ? (__uint_as_float(c[16 * h + g]) + __uint_as_float(c[16 * h + G + g])) * sc[h]
                                            : -INFINITY;
-                    // A tile that ends the context: its V rows past the context would multiply
-                    // P = 0 by whatever they hold, and (decode step) the new token's V codes
-                    // replace its slot's previous contents.  Both wait for the tile's V.
-                    const bool vpatch = STEP && nt_row >= 0 && tile + j == ntiles - 1;
-                    if (valid < kTcTile || vpatch) {
-                        // The softmax may run ahead of the PV MMAs, and V(k) shares its slot with
-                        // V(k - kTcVSlots): that tile's PV must be complete first, or the slot's
-                        // full barrier could still be in the earlier phase, whose parity the
-                        // wait below would take for this one.  (PvDone of that tile's P buffer
-                        // cannot alias either: this thread waited for its previous use at tile
-                        // k - kTcVSlots, and its next use needs a P tile not yet written, since
-                        // kTcPBufs >= kTcVSlots.)
-                        bool vok = !*abort_flag;
-                        if (vok && k >= kTcVSlots)
-                            vok = mbar_wait_bounded(bar_at(bars, kBPvDone + (k - kTcVSlots) % kTcPBufs),
-                                                    ((k - kTcVSlots) / kTcPBufs) & 1, p.err);
-                        vok = vok && mbar_wait_bounded(bar_at(bars, kBVFull + s), (k / kTcVSlots) & 1, p.err);
-                        if (!__all_sync(0xffffffffu, vok)) {
-                            alive = false;
-                            *abort_flag = 1;
-                        }
-                        const uint32_t vslot = sStages + Geo::kOffV + s * Geo::kKV;
-                        if (alive && t >= valid) {
-                            // (the whole 128-byte row of each head: the swizzle only permutes its chunks)
-                            const uint32_t vrow = vslot + (t >> 3) * 2048 + (t & 7) * 128;
-#pragma unroll
-                            for (int h = 0; h < kTcHP; ++h)
-#pragma unroll
-                                for (int q = 0; q < 8; ++q)
-                                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + 1024 * h + 16 * q),
-                                                 "r"(0u) : "memory");
-                        }
-                        if (alive && vpatch && t == nt_row) {
-#pragma unroll 1
-                            for (int i = 0; i < kTcHP * 8; ++i) {
-                                const int h = i >> 3, cc = 16 * (i & 7);
-                                const uint4 x = *reinterpret_cast<const uint4 *>(newcodes + (qslot * kTcHP + h) * 256 +
-                                                                                 D + cc);
-                                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vslot + kv_off(t, h, cc)),
-                                             "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w) : "memory");
-                            }
-                        }
-                    }
+                    pv_valid = valid;
+                    pv_row = STEP && nt_row >= 0 && tile + j == ntiles - 1 ? nt_row : -1;
                 } else {
 #pragma unroll
                     for (int h = 0; h < kTcHP; ++h)
@@ -1113,6 +1105,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     *abort_flag = 1;
                 }
                 const uint32_t pd = sP + pb * Geo::kP;
+                // The PV warp fixes this tile's V once it has landed: rows past the context (which
+                // would multiply P = 0 by whatever they hold) and the decode step's new token.
+                // It learns what to fix here, with the P tile (buffer pb, free like the P tile).
+                if (ct == 0)
+                    *reinterpret_cast<int2 *>(smem + Geo::kOffPvInfo + 8 * pb) = make_int2(pv_valid, pv_row);
+                if (pv_row >= 0 && t == pv_row) {
+                    uint8_t *dst = smem + Geo::kOffPvCodes + pb * (kTcHP * 128);
+#pragma unroll
+                    for (int i = 0; i < kTcHP * 8; ++i) {
+                        const int h = i >> 3, cc = 16 * (i & 7);
+                        *reinterpret_cast<uint4 *>(dst + h * 128 + cc) =
+                            *reinterpret_cast<const uint4 *>(newcodes + (qslot * kTcHP + h) * 256 + D + cc);
+                    }
+                }
 #pragma unroll
                 for (int h = 0; h < kTcHP; ++h)
 #pragma unroll

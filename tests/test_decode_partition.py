@@ -9,7 +9,7 @@ segment's first interior boundary merges it.  Checked: every unit is covered exa
 each split segment gets exactly one partial per covering CTA and exactly one merging CTA;
 partial slots never collide and fit the workspace of B*Hkv + 2*CTAs slots.
 
-The tensor-core decode splits by cost instead: a unit costs 1 and a segment's first unit 1
+The tensor-core decode splits by cost instead: a unit costs 1 and a segment's first unit 3
 more, CTA c starts at the first unit whose running cost key(u) * CTAs reaches c * total cost
 (equal counts when the problem is too small for every CTA to get a unit).  Its closed form is
 checked against a brute-force walk over every unit, and the same invariants are checked for
@@ -80,7 +80,7 @@ def _model(blocks, hkv, hpu, nctas, starts=None):
     return total, covered, writes, whole, merged, starts, hu, pfx
 
 
-UNIT_COST, PIECE_COST = 1, 1
+UNIT_COST, PIECE_COST = 1, 3
 
 
 def _cost_starts(tiles, hu, nctas):
