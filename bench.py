@@ -116,10 +116,11 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def timed_region(fn, steps, warmup, stream, dist=None, sampler_index=0, on_timed=None):
+def timed_region(fn, steps, warmup, stream, dist=None, sampler_index=0, on_timed=None, on_end=None):
     """Run fn() warmup times, then time `steps` calls with CUDA events on `stream`,
     bracketed by a barrier and a device synchronisation; returns (ms total, clocks).
-    `on_timed` (if given) is called once between the warm-up and the timed calls."""
+    `on_timed` (if given) is called once between the warm-up and the timed calls; `on_end`
+    (if given) after the timed calls, before the end event (to join other streams' work)."""
     for _ in range(warmup):
         fn()
     if on_timed is not None:
@@ -135,6 +136,8 @@ def timed_region(fn, steps, warmup, stream, dist=None, sampler_index=0, on_timed
         start.record(stream)
         for _ in range(steps):
             fn()
+        if on_end is not None:
+            on_end()
         end.record(stream)
         torch.cuda.synchronize()
     if dist is not None:
@@ -248,10 +251,28 @@ class Runner:
         self.table = pkv.rope_build_table(wl.max_pos, wl.head_dim, wl.rope_base).cuda()
         self.k_scale = wl.k_scale.cuda() if wl.k_scale is not None else None
         self.v_scale = wl.v_scale.cuda() if wl.v_scale is not None else None
-        # per-step inputs (device copies) and pinned host copies for the end-to-end leg
+        # Per-step inputs: views into one flat pinned host buffer and one flat device buffer,
+        # so the end-to-end leg moves a step's inputs in one copy (plus one on-device copy).
         names = ["q", "k", "v", "slot_mapping", "cu_seqlens", "context_lens", "block_tables"]
-        self.host = {n: getattr(st, n).contiguous().pin_memory() for n in names}
-        self.dev = {n: t.cuda() for n, t in self.host.items()}
+        srcs = {n: getattr(st, n).contiguous() for n in names}
+        offs, total = {}, 0
+        for n, t in srcs.items():
+            offs[n] = total
+            total += (t.numel() * t.element_size() + 15) // 16 * 16
+        self.host_flat = torch.empty(total, dtype=torch.uint8).pin_memory()
+        self.dev_flat = torch.empty(total, dtype=torch.uint8, device="cuda")
+        self.stage_flat = [torch.empty_like(self.dev_flat) for _ in range(2)]
+
+        def view(buf, n):
+            t = srcs[n]
+            nb = t.numel() * t.element_size()
+            return buf[offs[n]:offs[n] + nb].view(t.dtype).view(t.shape)
+
+        self.host = {n: view(self.host_flat, n) for n in names}
+        self.dev = {n: view(self.dev_flat, n) for n in names}
+        for n in names:
+            self.host[n].copy_(srcs[n])
+            self.dev[n].copy_(srcs[n])
         B = st.decode_seqs
         self.B = B
         self.fused = fused
@@ -285,8 +306,18 @@ class Runner:
             self.pre_ctx = self.dev["context_lens"][B:].contiguous()
             self.pre_out = torch.empty_like(self.pre_q)
             self.max_new = int((st.cu_seqlens[B + 1:] - st.cu_seqlens[B:-1]).max())
-        self.host_out = torch.empty((st.num_tokens, wl.n_q_heads, wl.head_dim),
-                                    dtype=torch.bfloat16).pin_memory()
+        self.host_out = [torch.empty((st.num_tokens, wl.n_q_heads, wl.head_dim),
+                                     dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        # the end-to-end leg alternates two output sets (a step's result is read back while
+        # the next step computes into the other set)
+        self.out_sets = [(getattr(self, "dec_out", None), getattr(self, "pre_out", None))]
+        self.out_sets.append(tuple(None if t is None else torch.empty_like(t) for t in self.out_sets[0]))
+        # one stream per copy direction: on a single stream the read-back of step i would
+        # queue the inputs of step i+1 behind step i's compute
+        self.h2d_stream, self.d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+        self.e2e_i = 0
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        self.ev_loaded, self.ev_stage_free, self.ev_computed, self.ev_out_free = ev(), ev(), ev(), ev()
         self.ev_attn = []  # (start, end) event pairs around the dominant kernel
 
     def launches_per_step(self) -> int:
@@ -349,24 +380,42 @@ class Runner:
                     self.ev_attn.append((e0, e1))
 
     def e2e_step(self):
-        """Same step, with this step's inputs copied from pinned host memory first and the
-        attention output copied back (all on the current stream)."""
-        for n, h in self.host.items():
-            self.dev[n].copy_(h, non_blocking=True)
+        """The same step with its inputs copied from pinned host memory and its attention
+        output read back, pipelined as a serving loop would: on copy streams, step i's
+        inputs travel while step i-1 computes and step i's output returns while step i+1
+        computes.  On the compute stream the step waits for its inputs (then one on-device
+        copy puts them in place) and for the read-back of the output set it reuses."""
+        b = self.e2e_i & 1
+        self.e2e_i += 1
+        s, hs, ds = torch.cuda.current_stream(), self.h2d_stream, self.d2h_stream
+        hs.wait_event(self.ev_stage_free[b])        # the on-device copy of step i-2 read it
+        with torch.cuda.stream(hs):
+            self.stage_flat[b].copy_(self.host_flat, non_blocking=True)
+            self.ev_loaded[b].record(hs)
+        s.wait_event(self.ev_loaded[b])
+        self.dev_flat.copy_(self.stage_flat[b], non_blocking=True)
+        self.ev_stage_free[b].record(s)
+        s.wait_event(self.ev_out_free[b])            # step i-2's output has been read back
+        self.dec_out, self.pre_out = self.out_sets[b]
         self.step()
-        parts = []
-        if self.B:
-            parts.append(self.dec_out)
-        if self.P:
-            parts.append(self.pre_out)
-        off = 0
-        for p in parts:
-            self.host_out[off:off + p.shape[0]].copy_(p, non_blocking=True)
-            off += p.shape[0]
+        self.ev_computed[b].record(s)
+        ds.wait_event(self.ev_computed[b])
+        with torch.cuda.stream(ds):
+            off = 0
+            for t in self.out_sets[b]:
+                if t is not None:
+                    self.host_out[b][off:off + t.shape[0]].copy_(t, non_blocking=True)
+                    off += t.shape[0]
+            self.ev_out_free[b].record(ds)
+        self.dec_out, self.pre_out = self.out_sets[0]
+
+    def e2e_finish(self):
+        """The timed region ends once the last read-back has landed."""
+        torch.cuda.current_stream().wait_stream(self.d2h_stream)
 
     def e2e_bytes(self):
         h2d = sum(t.numel() * t.element_size() for t in self.host.values())
-        d2h = self.host_out.numel() * self.host_out.element_size()
+        d2h = self.host_out[0].numel() * self.host_out[0].element_size()
         return h2d, d2h
 
     def attn_ms(self) -> float:
@@ -453,7 +502,7 @@ def measure_ours(name, steps, warmup, dist=None, device_index=0, pk=None, e2e=Tr
         res["step_tflops"] = world * fl / (step_ms * 1e-3) / 1e12
     if e2e:
         ms_e, _ = timed_region(r.e2e_step, steps, warmup, torch.cuda.current_stream(), dist,
-                               device_index)
+                               device_index, on_end=r.e2e_finish)
         ms_e = max_over_ranks(ms_e, dist)
         h2d, d2h = r.e2e_bytes()
         res["e2e_step_ms"] = ms_e / steps
@@ -615,7 +664,10 @@ def main():
         else:
             ev = world * res["prefill_flops_per_step"] / (res["e2e_step_ms"] * 1e-3) / 1e12
         line["e2e"] = {"value": ev, "unit": unit, "h2d_bytes_per_step": res["e2e_h2d"],
-                       "d2h_bytes_per_step": res["e2e_d2h"], "ms_per_step": res["e2e_step_ms"]}
+                       "d2h_bytes_per_step": res["e2e_d2h"], "ms_per_step": res["e2e_step_ms"],
+                       "pipelining": "each step's inputs copied from pinned host memory and its "
+                                     "output read back on two copy streams, overlapping the "
+                                     "neighbouring steps' compute"}
     del runner
     torch.cuda.empty_cache()
 
