@@ -222,6 +222,11 @@ def recorded_traffic(kernel: str, workload: str):
         return None
 
 
+# Suite entries' minimum timed steps (each about 20 ms or more of device time).
+SUITE_MIN_STEPS = {"gqa_decode": 8, "shared_prefix": 8, "mix": 50, "mix_fp8": 50, "small_batch": 500,
+                   "qwen_decode": 100}
+
+
 def timed_kernel(wl, decode: bool) -> str:
     """Name of the kernel the bench's attention events bracket for this workload."""
     if not decode:
@@ -681,9 +686,12 @@ def main():
             key = name if fused else name + "_unfused"
             if name == args.workload and fused != args.unfused:
                 continue
+            # at least ~20 ms of timed work per entry, so that short steps are not measured
+            # over a handful of launches
+            n_steps = max(3, args.steps // 4, SUITE_MIN_STEPS.get(name, 3))
             try:
-                r, rr = measure_ours(name, max(3, args.steps // 4), 3, None, 0, pk, e2e=False,
-                                     fused=fused)
+                r, rr = measure_ours(name, n_steps, max(3, min(20, n_steps // 10)), None, 0, pk,
+                                     e2e=False, fused=fused)
                 del rr
                 torch.cuda.empty_cache()
                 keep = {k: v for k, v in r.items() if k not in ("clocks",)}
